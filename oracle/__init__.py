@@ -1,0 +1,176 @@
+"""CPU oracle for the SegQuant DualScale + SegLinear W8A8 linear layer.
+
+TEST INFRASTRUCTURE ONLY: imported by tests/, by the smoke check and by the
+benchmark's CPU-baseline leg; never by the library's product path.  It shares
+no code with the CUDA path.  The arithmetic lives in oracle.c (plain C, one
+obvious loop per formula); this module only marshals numpy arrays into it.
+
+Definitions followed (see oracle.c for the full list of readings):
+  "SegQuant" (papernotes.org), section DualScale: X+ = max(X,0), X- = min(X,0),
+  s+ = max/q_max, s- = |min|/|q_min|, Y = s+ s_w (X^+ W^) + s- s_w (X^- W^);
+  section SegLinear: output-segmented concatenation, input-segmented sum.
+  "SegQuant" author page, section 3: the case-wise quantizer Q_dual.
+
+Conventions: bf16 tensors travel as uint16 bit patterns; the segment table is
+(mode, offsets, G) with mode 0 = none, 1 = output-segmented, 2 = input-
+segmented.
+"""
+import ctypes
+
+import numpy as np
+
+from . import build as _build
+
+MODE_NONE, MODE_OUTPUT, MODE_INPUT = 0, 1, 2
+
+_lib = None
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        path = _build.build()
+        L = ctypes.CDLL(path)
+        p, i64, i32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int
+        L.orc_calibrate_act.argtypes = [p, i64, i64, i64, p, i32, i32, p, i32, i64, p]
+        L.orc_quantize_act.argtypes = [p, i64, i64, i64, p, p, i32, i32, p, i32, i64, p]
+        L.orc_quantize_weight.argtypes = [p, i64, i64, p, i32, i32, p, i32, p, p]
+        L.orc_gemm_s32.argtypes = [p, p, i64, i64, i64, i32, i32, p, i32, p, i64, p, i32]
+        L.orc_gemm.argtypes = [p, p, p, p, p, i64, i64, i64, i32, i32, p, i32, p, i64, p, i32]
+        L.orc_num_threads.argtypes = []
+        for f in (L.orc_calibrate_act, L.orc_quantize_act, L.orc_quantize_weight,
+                  L.orc_gemm_s32, L.orc_gemm, L.orc_num_threads):
+            f.restype = ctypes.c_int
+        _lib = L
+    return _lib
+
+
+def _ptr(a):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _c(a, dtype):
+    return None if a is None else np.ascontiguousarray(a, dtype=dtype)
+
+
+def _seg(mode, offsets, G, N, K):
+    if offsets is None:
+        offsets = [0, K if mode != MODE_OUTPUT else N]
+    off = np.ascontiguousarray(np.asarray(offsets, dtype=np.int32))
+    n_seg = len(off) - 1
+    S = n_seg if mode == MODE_INPUT else 1
+    return off, n_seg, S
+
+
+def _check(rc, what):
+    if rc != 0:
+        raise ValueError(f"oracle {what}: invalid arguments (rc={rc})")
+
+
+def num_threads():
+    return lib().orc_num_threads()
+
+
+def calibrate_act(x_bits, d=None, mode=MODE_NONE, offsets=None, G=1, N=0):
+    """AMax calibration: returns s_act float32 [G][S][2] = {s+, s-}."""
+    x = _c(x_bits, np.uint16)
+    M, K = x.shape
+    off, n_seg, S = _seg(mode, offsets, G, N, K)
+    d = _c(d, np.float32)
+    out = np.zeros((G, S, 2), np.float32)
+    _check(lib().orc_calibrate_act(_ptr(x), M, K, K, _ptr(d), mode, n_seg,
+                                   _ptr(off), G, N, _ptr(out)), "calibrate_act")
+    return out
+
+
+def quantize_act(x_bits, s_act, d=None, mode=MODE_NONE, offsets=None, G=1, N=0):
+    """Q_dual of X / d: returns planes int8 [G][2][M][K] (0 = X^+, 1 = X^-)."""
+    x = _c(x_bits, np.uint16)
+    M, K = x.shape
+    off, n_seg, S = _seg(mode, offsets, G, N, K)
+    s = _c(s_act, np.float32)
+    assert s.size == G * S * 2
+    d = _c(d, np.float32)
+    planes = np.zeros((G, 2, M, K), np.int8)
+    _check(lib().orc_quantize_act(_ptr(x), M, K, K, _ptr(d), _ptr(s), mode,
+                                  n_seg, _ptr(off), G, N, _ptr(planes)),
+           "quantize_act")
+    return planes
+
+
+def quantize_weight(w_bits, d=None, mode=MODE_NONE, offsets=None, G=1):
+    """Segment-wise AMax weight quantization: returns (wq int8 [N][K], s_w f32 [S][N])."""
+    w = _c(w_bits, np.uint16)
+    N, K = w.shape
+    off, n_seg, S = _seg(mode, offsets, G, N, K)
+    d = _c(d, np.float32)
+    wq = np.zeros((N, K), np.int8)
+    s_w = np.zeros((S, N), np.float32)
+    _check(lib().orc_quantize_weight(_ptr(w), N, K, _ptr(d), mode, n_seg,
+                                     _ptr(off), G, _ptr(wq), _ptr(s_w)),
+           "quantize_weight")
+    return wq, s_w
+
+
+def _rows(rows, M):
+    if rows is None:
+        return None, M
+    r = np.ascontiguousarray(np.asarray(rows, dtype=np.int64))
+    assert r.ndim == 1 and (r.size == 0 or (r.min() >= 0 and r.max() < M))
+    return r, r.size
+
+
+def gemm_s32(planes, wq, mode=MODE_NONE, offsets=None, rows=None, threads=1):
+    """Raw int32 accumulators [S][2][rows][N]."""
+    planes = _c(planes, np.int8)
+    wq = _c(wq, np.int8)
+    G, two, M, K = planes.shape
+    N = wq.shape[0]
+    assert two == 2 and wq.shape[1] == K
+    off, n_seg, S = _seg(mode, offsets, G, N, K)
+    r, nr = _rows(rows, M)
+    acc = np.zeros((S, 2, nr, N), np.int32)
+    _check(lib().orc_gemm_s32(_ptr(planes), _ptr(wq), M, N, K, mode, n_seg,
+                              _ptr(off), G, _ptr(r), nr, _ptr(acc), threads),
+           "gemm_s32")
+    return acc
+
+
+def gemm(planes, wq, s_w, s_act, bias_bits=None, mode=MODE_NONE, offsets=None,
+         rows=None, threads=1):
+    """Layer output, fp32 epilogue: float32 [rows][N]."""
+    planes = _c(planes, np.int8)
+    wq = _c(wq, np.int8)
+    G, two, M, K = planes.shape
+    N = wq.shape[0]
+    assert two == 2 and wq.shape[1] == K
+    off, n_seg, S = _seg(mode, offsets, G, N, K)
+    s_w = _c(s_w, np.float32)
+    s_act = _c(s_act, np.float32)
+    assert s_w.size == S * N and s_act.size == G * S * 2
+    b = _c(bias_bits, np.uint16)
+    r, nr = _rows(rows, M)
+    y = np.zeros((nr, N), np.float32)
+    _check(lib().orc_gemm(_ptr(planes), _ptr(wq), _ptr(s_w), _ptr(s_act),
+                          _ptr(b), M, N, K, mode, n_seg, _ptr(off), G, _ptr(r),
+                          nr, _ptr(y), threads), "gemm")
+    return y
+
+
+def layer(x_bits, w_bits, x_cal_bits, d=None, bias_bits=None, mode=MODE_NONE,
+          offsets=None, G=1, rows=None, threads=1):
+    """Whole static pipeline on the CPU: calibrate, quantize both sides, GEMM.
+
+    Returns a dict with s_act, planes, wq, s_w and y (fp32 rows)."""
+    w = _c(w_bits, np.uint16)
+    N = w.shape[0]
+    s_act = calibrate_act(x_cal_bits, d, mode, offsets, G, N)
+    planes = quantize_act(x_bits, s_act, d, mode, offsets, G, N)
+    wq, s_w = quantize_weight(w, d, mode, offsets, G)
+    y = gemm(planes, wq, s_w, s_act, bias_bits, mode, offsets, rows, threads)
+    return dict(s_act=s_act, planes=planes, wq=wq, s_w=s_w, y=y)
+
+
+__all__ = ["MODE_NONE", "MODE_OUTPUT", "MODE_INPUT", "calibrate_act",
+           "quantize_act", "quantize_weight", "gemm_s32", "gemm", "layer",
+           "num_threads", "lib"]

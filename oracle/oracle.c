@@ -1,0 +1,311 @@
+/*
+ * oracle.c -- plain CPU oracle for the SegQuant quantized linear layer
+ * (DualScale polarity split + SegLinear segmentation, W8A8).
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing in the library's product path may call,
+ * link or load this file; only the tests, the smoke check and the benchmark's
+ * CPU-baseline leg do.  It shares no code, header, table or helper with the
+ * CUDA path (w8a8_gemm_b200/csrc): its own structs, its own bf16 decoding, its
+ * own loops.  Every step is written the slow, obvious way so that it can be
+ * checked against the pages by eye.
+ *
+ * Sources (page title, section, formula):
+ *  - "SegQuant: A Semantics-Aware and Generalizable Quantization Framework for
+ *    Diffusion Models" (papernotes.org notes), section "DualScale":
+ *    X+ = max(X,0), X- = min(X,0); s- = |min(x)|/q_min, s+ = max(x)/q_max;
+ *    Y ~= s+ s_w (X^+ W^) + s- s_w (X^- W^).
+ *  - same page, section "SegLinear": output-segmented Y^ = [X^W^_1, ..., X^W^_N]
+ *    (W split by columns); input-segmented Y^ = sum_i X^_i W^_i (W split by rows).
+ *  - "SegQuant" author page (hliangzhao.me), section 3 "DualScale": the
+ *    case-wise quantizer Q_dual(x) = round(x/s-) for x < 0, round(x/s+) for
+ *    x >= 0, and the two-product reconstruction.
+ *  - papernotes.org page, "Loss function / training strategy": AMax (max-abs)
+ *    calibration is one of the two calibrators.
+ *
+ * Readings where the pages are silent or ambiguous (all stated again in the
+ * design notes):
+ *  - q_min: the pages divide |min| by q_min; with signed int8 q_min = -128 that
+ *    would give a negative step, so the magnitude 128 is used: s- = |min|/128,
+ *    s+ = max/127.  X^- lies in [-128, 0], X^+ in [0, 127].
+ *  - "round" is round-half-to-even, in fp32.
+ *  - The SmoothQuant divisor d (per group, per input channel, > 0) is an input.
+ *    Activations are quantized as x / d, weights as w * d.  The quantizer
+ *    multiplies by a folded reciprocal: t = fl(d * s), m = fl(1 / t),
+ *    v = fl(x * m), q = rne(clamp(v)).  Both sides take this decision in fp32.
+ *  - Out-of-range values saturate: q+ <= 127, q- >= -128.  NaN goes to 0 in
+ *    both planes (neither x < 0 nor x >= 0 holds); -0.0 goes to the + plane.
+ *  - Degenerate calibration: max <= 0 gives s+ = 1, min >= 0 gives s- = 1; an
+ *    all-zero weight column segment gives s_w = 1.
+ *  - Weights: symmetric AMax per output channel and per K-segment,
+ *    s_w = amax / 127, q = rne(clamp(w' / s_w, -127, 127)).
+ *  - Output-segmented layers may carry their own activation parameters per
+ *    output segment (a "group" g: its own d and s+/s-, hence its own planes).
+ *    G = 1 is the pages' formula with one shared X^.
+ *  - Epilogue in fp32, fixed order: for each K-segment i in ascending order,
+ *    t = s+_i * f(A+_i) + s-_i * f(A-_i), y = y + s_w[i][n] * t; bias last.
+ *    f is int32 -> fp32 round-to-nearest.
+ *
+ * Layouts (row-major, innermost last):
+ *  x      bf16 bits [M][ldx]          activations (nn.Linear input)
+ *  w      bf16 bits [N][K]            nn.Linear weight (the pages' W^T)
+ *  d      fp32 [G][K] or NULL (=1)    SmoothQuant divisor per group
+ *  s_act  fp32 [G][S][2]              {s+, s-} per group and K-segment
+ *  planes int8 [G][2][M][K]           plane 0 = X^+, plane 1 = X^-
+ *  wq     int8 [N][K]                 quantized weight
+ *  s_w    fp32 [S][N]                 weight scale per K-segment, per column
+ *  acc    int32 [S][2][M][N]          raw accumulators per segment, polarity
+ *  y      fp32 [rows][N]              layer output (fp32 epilogue)
+ *
+ * Segment description: mode 0 = none, 1 = output-segmented (offsets over N),
+ * 2 = input-segmented (offsets over K).  offsets has n_seg + 1 ascending
+ * entries from 0 to N (or K).  S = n_seg in input mode, else 1.  G is 1 or, in
+ * output mode, n_seg.
+ *
+ * Build: gcc -O2 -fopenmp -ffp-contract=off -fno-fast-math (no -ffast-math:
+ * the rounding of every fp32 operation is part of the definition).
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+#define ORC_MODE_NONE 0
+#define ORC_MODE_OUTPUT 1
+#define ORC_MODE_INPUT 2
+
+static float orc_bf16(uint16_t h) {
+  uint32_t u = ((uint32_t)h) << 16;
+  float f;
+  memcpy(&f, &u, sizeof f);
+  return f;
+}
+
+/* index i with off[i] <= p < off[i+1] */
+static int orc_seg_index(const int32_t *off, int n_seg, int64_t p) {
+  for (int i = 0; i < n_seg; ++i)
+    if (p < off[i + 1]) return i;
+  return n_seg - 1;
+}
+
+static int orc_check_seg(int mode, int n_seg, const int32_t *off, int G,
+                         int64_t N, int64_t K) {
+  if (mode == ORC_MODE_NONE) return (n_seg == 1 && G == 1) ? 0 : -1;
+  if (n_seg < 1 || off == NULL) return -1;
+  int64_t extent = (mode == ORC_MODE_OUTPUT) ? N : K;
+  if (off[0] != 0 || off[n_seg] != extent) return -1;
+  for (int i = 0; i < n_seg; ++i)
+    if (off[i + 1] <= off[i]) return -1;
+  if (mode == ORC_MODE_INPUT && G != 1) return -1;
+  if (mode == ORC_MODE_OUTPUT && G != 1 && G != n_seg) return -1;
+  return 0;
+}
+
+int orc_num_threads(void) {
+#ifdef _OPENMP
+  return omp_get_max_threads();
+#else
+  return 1;
+#endif
+}
+
+/* ---------------------------------------------------------------------------
+ * AMax calibration of the two activation scales (static, offline).
+ * For group g and K-segment i, over the calibration rows and the channels c of
+ * segment i: u = x / d[g][c]; hi = max(0, max u); lo = min(0, min u);
+ * s+ = hi / 127 (1 if hi == 0), s- = -lo / 128 (1 if lo == 0).
+ * In output mode N is unused; pass the layer's N anyway for the check.
+ * ------------------------------------------------------------------------- */
+int orc_calibrate_act(const uint16_t *x, int64_t M, int64_t K, int64_t ldx,
+                      const float *d, int mode, int n_seg,
+                      const int32_t *offsets, int G, int64_t N, float *s_act) {
+  if (orc_check_seg(mode, n_seg, offsets, G, N, K)) return -1;
+  int S = (mode == ORC_MODE_INPUT) ? n_seg : 1;
+  for (int g = 0; g < G; ++g) {
+    for (int i = 0; i < S; ++i) {
+      int64_t c0 = (S == 1) ? 0 : offsets[i];
+      int64_t c1 = (S == 1) ? K : offsets[i + 1];
+      float hi = 0.0f, lo = 0.0f;
+      for (int64_t m = 0; m < M; ++m) {
+        for (int64_t c = c0; c < c1; ++c) {
+          float xv = orc_bf16(x[m * ldx + c]);
+          float dv = d ? d[(int64_t)g * K + c] : 1.0f;
+          float u = xv / dv;
+          if (u > hi) hi = u; /* NaN compares false: ignored */
+          if (u < lo) lo = u;
+        }
+      }
+      float sp = (hi > 0.0f) ? hi / 127.0f : 1.0f;
+      float sm = (lo < 0.0f) ? (-lo) / 128.0f : 1.0f;
+      s_act[((int64_t)g * S + i) * 2 + 0] = sp;
+      s_act[((int64_t)g * S + i) * 2 + 1] = sm;
+    }
+  }
+  return 0;
+}
+
+/* ---------------------------------------------------------------------------
+ * DualScale activation quantization (Q_dual) with SmoothQuant divisor.
+ * ------------------------------------------------------------------------- */
+int orc_quantize_act(const uint16_t *x, int64_t M, int64_t K, int64_t ldx,
+                     const float *d, const float *s_act, int mode, int n_seg,
+                     const int32_t *offsets, int G, int64_t N, int8_t *planes) {
+  if (orc_check_seg(mode, n_seg, offsets, G, N, K)) return -1;
+  int S = (mode == ORC_MODE_INPUT) ? n_seg : 1;
+  for (int g = 0; g < G; ++g) {
+    int8_t *plus = planes + ((int64_t)g * 2 + 0) * M * K;
+    int8_t *minus = planes + ((int64_t)g * 2 + 1) * M * K;
+    for (int64_t m = 0; m < M; ++m) {
+      for (int64_t c = 0; c < K; ++c) {
+        int i = (S == 1) ? 0 : orc_seg_index(offsets, n_seg, c);
+        float sp = s_act[((int64_t)g * S + i) * 2 + 0];
+        float sm = s_act[((int64_t)g * S + i) * 2 + 1];
+        float dv = d ? d[(int64_t)g * K + c] : 1.0f;
+        float mp = 1.0f / (dv * sp); /* folded reciprocal, two fp32 ops */
+        float mm = 1.0f / (dv * sm);
+        float xv = orc_bf16(x[m * ldx + c]);
+        int qp = 0, qm = 0;
+        if (xv < 0.0f) { /* X- branch: round(x / s-) */
+          float v = xv * mm;
+          if (v < -128.0f) v = -128.0f;
+          qm = (int)rintf(v);
+        } else if (xv >= 0.0f) { /* X+ branch: round(x / s+) */
+          float v = xv * mp;
+          if (v > 127.0f) v = 127.0f;
+          qp = (int)rintf(v);
+        }
+        plus[m * K + c] = (int8_t)qp;
+        minus[m * K + c] = (int8_t)qm;
+      }
+    }
+  }
+  return 0;
+}
+
+/* ---------------------------------------------------------------------------
+ * Segment-wise symmetric AMax weight quantization.
+ * Column n of the pages' W (row n of the nn.Linear weight) is quantized
+ * independently on every K-segment i; in output mode each output segment j
+ * folds its own group's divisor d[j] when G > 1.
+ * ------------------------------------------------------------------------- */
+int orc_quantize_weight(const uint16_t *w, int64_t N, int64_t K, const float *d,
+                        int mode, int n_seg, const int32_t *offsets, int G,
+                        int8_t *wq, float *s_w) {
+  if (orc_check_seg(mode, n_seg, offsets, G, N, K)) return -1;
+  int S = (mode == ORC_MODE_INPUT) ? n_seg : 1;
+  for (int64_t n = 0; n < N; ++n) {
+    int g = (mode == ORC_MODE_OUTPUT && G > 1)
+                ? orc_seg_index(offsets, n_seg, n) : 0;
+    for (int i = 0; i < S; ++i) {
+      int64_t k0 = (S == 1) ? 0 : offsets[i];
+      int64_t k1 = (S == 1) ? K : offsets[i + 1];
+      float amax = 0.0f;
+      for (int64_t k = k0; k < k1; ++k) {
+        float dv = d ? d[(int64_t)g * K + k] : 1.0f;
+        float wv = orc_bf16(w[n * K + k]) * dv;
+        float a = fabsf(wv);
+        if (a > amax) amax = a;
+      }
+      float s = (amax > 0.0f) ? amax / 127.0f : 1.0f;
+      s_w[(int64_t)i * N + n] = s;
+      for (int64_t k = k0; k < k1; ++k) {
+        float dv = d ? d[(int64_t)g * K + k] : 1.0f;
+        float v = (orc_bf16(w[n * K + k]) * dv) / s;
+        if (v > 127.0f) v = 127.0f;
+        if (v < -127.0f) v = -127.0f;
+        wq[n * K + k] = (int8_t)(int)rintf(v);
+      }
+    }
+  }
+  return 0;
+}
+
+/* ---------------------------------------------------------------------------
+ * Integer products: A+-_i[m][n] = sum_{k in segment i} X^+-[g(n)][m][k] * W^[n][k]
+ * accumulated in int32 (the pages' fixed-width integer GEMM).  rows == NULL
+ * means all M rows; otherwise acc row r holds row rows[r].
+ * acc layout [S][2][n_rows][N].
+ * ------------------------------------------------------------------------- */
+int orc_gemm_s32(const int8_t *planes, const int8_t *wq, int64_t M, int64_t N,
+                 int64_t K, int mode, int n_seg, const int32_t *offsets, int G,
+                 const int64_t *rows, int64_t n_rows, int32_t *acc,
+                 int n_threads) {
+  if (orc_check_seg(mode, n_seg, offsets, G, N, K)) return -1;
+  int S = (mode == ORC_MODE_INPUT) ? n_seg : 1;
+  if (rows == NULL) n_rows = M;
+#ifdef _OPENMP
+  if (n_threads < 1) n_threads = 1;
+#pragma omp parallel for schedule(dynamic, 1) num_threads(n_threads)
+#endif
+  for (int64_t r = 0; r < n_rows; ++r) {
+    int64_t m = rows ? rows[r] : r;
+    for (int64_t n = 0; n < N; ++n) {
+      int g = (mode == ORC_MODE_OUTPUT && G > 1)
+                  ? orc_seg_index(offsets, n_seg, n) : 0;
+      const int8_t *xp = planes + (((int64_t)g * 2 + 0) * M + m) * K;
+      const int8_t *xm = planes + (((int64_t)g * 2 + 1) * M + m) * K;
+      const int8_t *wn = wq + n * K;
+      for (int i = 0; i < S; ++i) {
+        int64_t k0 = (S == 1) ? 0 : offsets[i];
+        int64_t k1 = (S == 1) ? K : offsets[i + 1];
+        int32_t ap = 0, am = 0;
+        for (int64_t k = k0; k < k1; ++k) {
+          ap += (int32_t)xp[k] * (int32_t)wn[k];
+          am += (int32_t)xm[k] * (int32_t)wn[k];
+        }
+        acc[(((int64_t)i * 2 + 0) * n_rows + r) * N + n] = ap;
+        acc[(((int64_t)i * 2 + 1) * n_rows + r) * N + n] = am;
+      }
+    }
+  }
+  return 0;
+}
+
+/* ---------------------------------------------------------------------------
+ * Full layer: integer products, then the DualScale reconstruction in fp32
+ *   y[m][n] = sum_i s_w[i][n] * (s+_i * f(A+_i) + s-_i * f(A-_i)) + bias[n]
+ * bias: bf16 bits [N] or NULL.  y layout [n_rows][N].
+ * ------------------------------------------------------------------------- */
+int orc_gemm(const int8_t *planes, const int8_t *wq, const float *s_w,
+             const float *s_act, const uint16_t *bias, int64_t M, int64_t N,
+             int64_t K, int mode, int n_seg, const int32_t *offsets, int G,
+             const int64_t *rows, int64_t n_rows, float *y, int n_threads) {
+  if (orc_check_seg(mode, n_seg, offsets, G, N, K)) return -1;
+  int S = (mode == ORC_MODE_INPUT) ? n_seg : 1;
+  if (rows == NULL) n_rows = M;
+#ifdef _OPENMP
+  if (n_threads < 1) n_threads = 1;
+#pragma omp parallel for schedule(dynamic, 1) num_threads(n_threads)
+#endif
+  for (int64_t r = 0; r < n_rows; ++r) {
+    int64_t m = rows ? rows[r] : r;
+    for (int64_t n = 0; n < N; ++n) {
+      int g = (mode == ORC_MODE_OUTPUT && G > 1)
+                  ? orc_seg_index(offsets, n_seg, n) : 0;
+      const int8_t *xp = planes + (((int64_t)g * 2 + 0) * M + m) * K;
+      const int8_t *xm = planes + (((int64_t)g * 2 + 1) * M + m) * K;
+      const int8_t *wn = wq + n * K;
+      float yv = 0.0f;
+      for (int i = 0; i < S; ++i) {
+        int64_t k0 = (S == 1) ? 0 : offsets[i];
+        int64_t k1 = (S == 1) ? K : offsets[i + 1];
+        int32_t ap = 0, am = 0;
+        for (int64_t k = k0; k < k1; ++k) {
+          ap += (int32_t)xp[k] * (int32_t)wn[k];
+          am += (int32_t)xm[k] * (int32_t)wn[k];
+        }
+        float sp = s_act[((int64_t)g * S + i) * 2 + 0];
+        float sm = s_act[((int64_t)g * S + i) * 2 + 1];
+        float tp = sp * (float)ap;
+        float tm = sm * (float)am;
+        float t = tp + tm;
+        yv = yv + s_w[(int64_t)i * N + n] * t;
+      }
+      if (bias) yv = yv + orc_bf16(bias[n]);
+      y[r * N + n] = yv;
+    }
+  }
+  return 0;
+}
