@@ -1,0 +1,205 @@
+/*
+ * segquant.h -- C ABI of the B200 (sm_100a) SegQuant quantized-linear library:
+ * DualScale polarity-split W8A8 GEMM with SegLinear segment-wise quantization.
+ *
+ * The method (SegQuant, arXiv 2507.14811), as described on the pages this
+ * library follows:
+ *  - "SegQuant" (papernotes.org notes), section "DualScale": the activation is
+ *    split by polarity, X+ = max(X,0) and X- = min(X,0); each part has its own
+ *    static step, s- = |min(x)|/q_min and s+ = max(x)/q_max; the layer output is
+ *    rebuilt as Y ~= s+ s_w (X^+ W^) + s- s_w (X^- W^).  The two integer
+ *    products run as one batched GEMM with a fused epilogue and no zero point.
+ *  - same page, section "SegLinear": an output-segmented layer splits W by
+ *    columns, Y^ = [X^W^_1, ..., X^W^_N]; an input-segmented layer splits X by
+ *    columns and W by rows, Y^ = sum_i X^_i W^_i; every segment is quantized
+ *    with its own parameters.
+ *  - "SegQuant" author page (hliangzhao.me), section 3: the case-wise
+ *    quantizer Q_dual(x) = round(x/s-) for x < 0, round(x/s+) for x >= 0.
+ *
+ * Readings taken where the pages are open (q_min magnitude 128, round half to
+ * even, saturation, SmoothQuant divisor folded as x/d and w*d, fp32 epilogue
+ * order) are spelled out per entry point below.
+ *
+ * Conventions for every call:
+ *  - Every pointer is a DEVICE pointer unless marked "host".  The caller owns
+ *    all buffers; the library allocates no device memory in any call.
+ *  - Calls are asynchronous on `stream` (0 = legacy default stream).  A return
+ *    of SQ_OK means the arguments were valid and the kernels were launched;
+ *    launch failures return SQ_ERR_CUDA.  Faults inside a kernel surface at
+ *    the caller's next synchronisation, as with any CUDA call.
+ *  - Arguments are validated on the host before anything is launched; an
+ *    invalid call launches nothing and leaves every output untouched.
+ *  - bf16 tensors are raw bfloat16 bit patterns (uint16) in row-major order.
+ *  - Layout of the stacked activation planes ("planes"): int8 [G][2][M][K],
+ *    row-major, K contiguous; plane [g][0] is X^+ (codes 0..127) and plane
+ *    [g][1] is X^- (codes -128..0) of activation group g.
+ */
+#ifndef SEGQUANT_H
+#define SEGQUANT_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Exported symbols (the library is built with hidden default visibility). */
+#if defined(__GNUC__)
+#define SQ_API __attribute__((visibility("default")))
+#else
+#define SQ_API
+#endif
+
+/* cudaStream_t without pulling in the CUDA headers. */
+typedef struct CUstream_st *sq_stream_t;
+
+typedef enum {
+  SQ_OK = 0,
+  SQ_ERR_INVALID_ARG = -1,   /* null pointer, bad size, bad segment table     */
+  SQ_ERR_UNSUPPORTED = -2,   /* valid request this build does not implement  */
+  SQ_ERR_ALIGNMENT = -3,     /* pointer / leading dimension misaligned       */
+  SQ_ERR_OVERFLOW = -4,      /* a K-segment could overflow the int32 sum     */
+  SQ_ERR_CUDA = -5,          /* a CUDA runtime call failed                    */
+  SQ_ERR_DEVICE_TIMEOUT = -6,/* a kernel gave up waiting (see status call)    */
+  SQ_ERR_NO_DEVICE = -7      /* no sm_100 device is current                   */
+} sq_status;
+
+typedef enum {
+  SQ_SEG_NONE = 0,   /* one segment over K and N                           */
+  SQ_SEG_OUTPUT = 1, /* segments over N (columns of the pages' W)          */
+  SQ_SEG_INPUT = 2   /* segments over K (rows of the pages' W)             */
+} sq_seg_mode;
+
+typedef enum { SQ_OUT_BF16 = 0, SQ_OUT_F32 = 1 } sq_out_dtype;
+
+/* Most segments a layer may have. */
+#define SQ_MAX_SEGMENTS 64
+
+/*
+ * Segment table (SegLinear).  `offsets` is a HOST array of n_seg + 1 strictly
+ * increasing int32 values from 0 to the segmented extent (N for SQ_SEG_OUTPUT,
+ * K for SQ_SEG_INPUT).  SQ_SEG_NONE takes n_seg = 1 and offsets may be NULL.
+ * n_groups (G) is the number of activation groups: 1, or, for SQ_SEG_OUTPUT
+ * only, n_seg, so that every output segment has its own SmoothQuant divisor,
+ * s+/s- and activation planes.  S, the number of K-segments, is n_seg for
+ * SQ_SEG_INPUT and 1 otherwise.
+ * Restrictions of this build: input-segment widths are multiples of 32 (the
+ * int8 MMA K step) and at most 132104 (so 128*127*width < 2^31); with G > 1
+ * output-segment widths are multiples of 128.
+ */
+typedef struct {
+  int32_t mode;            /* sq_seg_mode                        */
+  int32_t n_seg;           /* number of segments, 1..SQ_MAX_SEGMENTS */
+  const int32_t *offsets;  /* host, n_seg + 1 entries            */
+  int32_t n_groups;        /* G                                  */
+} sq_segments;
+
+/*
+ * sq_calibrate_act -- static AMax calibration of the two activation steps.
+ * Pages: papernotes.org "SegQuant", section DualScale (s- = |min|/q_min,
+ * s+ = max/q_max) and section "Loss function / training strategy" (AMax).
+ * For group g and K-segment i, over rows 0..M-1 and the channels c of segment
+ * i: u = x[m][c] / d[g][c] (fp32, IEEE division); hi = max(0, max u),
+ * lo = min(0, min u); s+ = hi/127 (1 if hi == 0), s- = -lo/128 (1 if lo == 0).
+ * NaN inputs are ignored.
+ *   x      bf16 [M][ldx]; M >= 1, K >= 16, K % 16 == 0, ldx >= K, ldx % 8 == 0,
+ *          x 16-byte aligned
+ *   d      fp32 [G][K] divisor (> 0, finite) or NULL for d = 1
+ *   s_act  fp32 [G][S][2] output, {s+, s-} per group and K-segment
+ * Launches three small kernels; no workspace.
+ */
+SQ_API sq_status sq_calibrate_act(const void *x, int64_t M, int64_t K, int64_t ldx,
+                           const float *d, const sq_segments *seg,
+                           float *s_act, sq_stream_t stream);
+
+/*
+ * sq_quantize_act -- DualScale activation quantization (the HBM-bound step).
+ * Pages: author page section 3 (Q_dual), papernotes.org section DualScale.
+ * For every element x (bf16, exact in fp32) of channel c in K-segment i and
+ * every group g:
+ *   m+ = 1/(d[g][c]*s+[g][i]), m- = 1/(d[g][c]*s-[g][i])   (fp32, each op RN)
+ *   x >= 0: X^+ = rne(min(x*m+, 127)),  X^- = 0
+ *   x <  0: X^- = rne(max(x*m-, -128)), X^+ = 0
+ *   NaN   : both 0.   (-0.0 counts as x >= 0; rne = round half to even.)
+ *   x      bf16 [M][ldx], constraints as in sq_calibrate_act
+ *   d      fp32 [G][K] or NULL;  s_act fp32 [G][S][2] (positive, finite, with
+ *          d*s a normal float)
+ *   planes int8 [G][2][M][K] output, 16-byte aligned
+ * M == 0 is a valid no-op.
+ */
+SQ_API sq_status sq_quantize_act(const void *x, int64_t M, int64_t K, int64_t ldx,
+                          const float *d, const float *s_act,
+                          const sq_segments *seg, int8_t *planes,
+                          sq_stream_t stream);
+
+/*
+ * sq_quantize_weight_seg -- segment-wise symmetric AMax weight quantization
+ * (offline, once per layer).  Pages: papernotes.org section SegLinear (each
+ * segment of W quantized independently) and AMax calibrator.
+ * w is the nn.Linear weight [N][K] (the pages' W transposed).  For output
+ * channel n in output segment j (group g = j when G > 1, else 0) and K-segment
+ * i:  w' = w[n][k]*d[g][k];  s_w[i][n] = max_k |w'| / 127 (1 if that is 0);
+ * W^[n][k] = rne(clamp(w'/s_w[i][n], -127, 127)).  Weights must be finite.
+ *   w   bf16 [N][K] (K % 16 == 0, 16-byte aligned);  d fp32 [G][K] or NULL
+ *   wq  int8 [N][K] output (16-byte aligned);  s_w fp32 [S][N] output
+ */
+SQ_API sq_status sq_quantize_weight_seg(const void *w, int64_t N, int64_t K,
+                                 const float *d, const sq_segments *seg,
+                                 int8_t *wq, float *s_w, sq_stream_t stream);
+
+/*
+ * sq_dualscale_seglinear_gemm -- the batched int8 GEMM with the fused DualScale
+ * reconstruction.  Pages: papernotes.org section DualScale (one BatchedGEMM
+ * launch over X^+ and X^-, results merged in a fused epilogue) and section
+ * SegLinear (output concatenation / input sum).
+ * Integer products, exact in int32, on the tensor cores (tcgen05 kind::i8):
+ *   A+_i[m][n] = sum_{k in segment i} X^+[g(n)][m][k] * W^[n][k]   (same for -)
+ * Epilogue in fp32, never leaving the chip:
+ *   y[m][n] = sum_i s_w[i][n] * (s+[g][i]*f(A+_i) + s-[g][i]*f(A-_i)) + bias[n]
+ * with f = int32 -> fp32 round-to-nearest.  With S == 1 the operations run in
+ * exactly this order; with S > 1 each segment's term is accumulated as
+ * (s_w s+) f(A+) + (s_w s-) f(A-) with fused multiply-adds (same value up to
+ * fp32 rounding).  Output rounds to bf16 (RN) or stays fp32.
+ *   planes int8 [G][2][M][K] from sq_quantize_act; wq int8 [N][K]
+ *   s_w fp32 [S][N]; s_act fp32 [G][S][2]; bias bf16 [N] or NULL
+ *   y      bf16 or fp32 [M][ldy] output, ldy >= N, ldy*elem % 16 == 0,
+ *          16-byte aligned
+ *   K % 16 == 0, K >= 16; N >= 1; M == 0 is a valid no-op.
+ * Returns SQ_ERR_OVERFLOW when a K-segment is wider than 132104.
+ */
+SQ_API sq_status sq_dualscale_seglinear_gemm(const int8_t *planes, const int8_t *wq,
+                                      const float *s_w, const float *s_act,
+                                      const void *bias, void *y,
+                                      sq_out_dtype out_dtype, int64_t M,
+                                      int64_t N, int64_t K, int64_t ldy,
+                                      const sq_segments *seg,
+                                      sq_stream_t stream);
+
+/*
+ * sq_debug_gemm_s32 -- the same tensor-core kernel, storing the raw int32
+ * accumulators instead of the epilogue, for bit-exact checks.
+ *   acc int32 [S][2][M][N] output (16-byte aligned), polarity 0 = A+, 1 = A-.
+ */
+SQ_API sq_status sq_debug_gemm_s32(const int8_t *planes, const int8_t *wq, int64_t M,
+                            int64_t N, int64_t K, const sq_segments *seg,
+                            int32_t *acc, sq_stream_t stream);
+
+/*
+ * sq_get_device_status -- synchronises the current device, then returns and
+ * clears the library's device-side error word: SQ_OK, or
+ * SQ_ERR_DEVICE_TIMEOUT if a kernel's bounded wait on a barrier ran out (the
+ * kernel then abandoned its tile and left its outputs incomplete).
+ */
+SQ_API sq_status sq_get_device_status(void);
+
+/* Static, human-readable name of a status code (never NULL). */
+SQ_API const char *sq_status_string(sq_status status);
+
+/* Library ABI version (major * 100 + minor). */
+SQ_API int32_t sq_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* SEGQUANT_H */

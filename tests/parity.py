@@ -1,0 +1,99 @@
+"""Shared helpers of the parity tests: run one synthetic layer through the CUDA
+path (C ABI via the binding) and through the CPU oracle, on the same seeded
+inputs, and compare."""
+import numpy as np
+import torch
+
+import oracle
+from w8a8_gemm_b200 import binding as B
+from w8a8_gemm_b200 import workloads as wl
+
+
+def segments(layer: wl.Layer) -> B.Segments:
+    if layer.mode == wl.MODE_NONE:
+        return B.Segments(B.SQ_SEG_NONE, None, 1)
+    return B.Segments(layer.mode, list(layer.offsets), layer.G)
+
+
+def oracle_offsets(layer: wl.Layer):
+    return None if layer.mode == wl.MODE_NONE else list(layer.offsets)
+
+
+def gpu_run(layer: wl.Layer, out_dtype=torch.float32, with_bias=True, s32=False):
+    """CUDA path: weight quantization, calibration, activation quantization and
+    the fused GEMM, all through the library."""
+    dev = torch.device("cuda")
+    seg = segments(layer)
+    x = layer.x.to(dev)
+    w = layer.w.to(dev)
+    xc = layer.x_cal.to(dev)
+    d = None if layer.d is None else layer.d.to(dev)
+    bias = layer.bias.to(dev) if (with_bias and layer.bias is not None) else None
+    M, K, N, G, S = layer.M, layer.K, layer.N, layer.G, layer.S
+    wq = torch.empty(N, K, dtype=torch.int8, device=dev)
+    s_w = torch.empty(S, N, dtype=torch.float32, device=dev)
+    B.sq_quantize_weight_seg(w, d, seg, wq, s_w)
+    s_act = torch.empty(G, S, 2, dtype=torch.float32, device=dev)
+    B.sq_calibrate_act(xc, d, seg, s_act)
+    planes = torch.empty(G, 2, M, K, dtype=torch.int8, device=dev)
+    B.sq_quantize_act(x, d, s_act, seg, planes)
+    ldy = (N + 7) // 8 * 8   # rows start 16-byte aligned for either dtype
+    y = torch.empty(M, ldy, dtype=out_dtype, device=dev)[:, :N]
+    B.sq_dualscale_seglinear_gemm(planes, wq, s_w, s_act, bias, y, seg)
+    out = dict(wq=wq, s_w=s_w, s_act=s_act, planes=planes, y=y)
+    if s32:
+        acc = torch.empty(S, 2, M, N, dtype=torch.int32, device=dev)
+        B.sq_debug_gemm_s32(planes, wq, seg, acc)
+        out["acc"] = acc
+    torch.cuda.synchronize()
+    assert B.sq_get_device_status() == 0
+    return out
+
+
+def oracle_prep(layer: wl.Layer):
+    """Oracle calibration and quantization of both operands."""
+    off = oracle_offsets(layer)
+    d = None if layer.d is None else layer.d.numpy()
+    s_act = oracle.calibrate_act(wl.bits(layer.x_cal), d, layer.mode, off, layer.G, layer.N)
+    planes = oracle.quantize_act(wl.bits(layer.x), s_act, d, layer.mode, off, layer.G, layer.N)
+    wq, s_w = oracle.quantize_weight(wl.bits(layer.w), d, layer.mode, off, layer.G)
+    return dict(s_act=s_act, planes=planes, wq=wq, s_w=s_w)
+
+
+def oracle_y(layer, prep, rows=None, with_bias=True, threads=None):
+    bias = wl.bits(layer.bias) if (with_bias and layer.bias is not None) else None
+    return oracle.gemm(prep["planes"], prep["wq"], prep["s_w"], prep["s_act"], bias, layer.mode,
+                       oracle_offsets(layer), rows=rows,
+                       threads=threads or oracle.num_threads())
+
+
+def oracle_acc(layer, prep, rows=None, threads=None):
+    return oracle.gemm_s32(prep["planes"], prep["wq"], layer.mode, oracle_offsets(layer),
+                           rows=rows, threads=threads or oracle.num_threads())
+
+
+def rel_err_floor(y: np.ndarray, r: np.ndarray) -> float:
+    """max |y - r| / (|r| + 1e-3 rms(r)): relative error with a floor near 0."""
+    r = r.astype(np.float64)
+    rms = float(np.sqrt(np.mean(r * r))) if r.size else 0.0
+    den = np.abs(r) + 1e-3 * rms + 1e-30
+    return float(np.max(np.abs(y.astype(np.float64) - r) / den)) if r.size else 0.0
+
+
+def bf16_ulp_diff(y_bf16: torch.Tensor, r_f32: np.ndarray) -> int:
+    """Largest distance, in bf16 ulps, between y and RNE_bf16(r)."""
+    ref = torch.from_numpy(np.ascontiguousarray(r_f32)).to(torch.bfloat16)
+    a = y_bf16.cpu().view(torch.int16).to(torch.int32)
+    b = ref.view(torch.int16).to(torch.int32)
+    # map sign-magnitude bf16 bit patterns onto a monotone integer line
+    a = torch.where(a < 0, -(a & 0x7FFF), a)
+    b = torch.where(b < 0, -(b & 0x7FFF), b)
+    return int((a - b).abs().max()) if a.numel() else 0
+
+
+def sample_rows(M: int, bm: int = 128, stride: int = 97):
+    """Every row of the first and last 128-row tile plus a strided subsample."""
+    rows = set(range(min(bm, M)))
+    rows |= set(range(max(0, M - bm), M))
+    rows |= set(range(0, M, stride))
+    return np.array(sorted(rows), dtype=np.int64)

@@ -1,0 +1,141 @@
+"""Host-side checks that need no GPU: the C-ABI library loads, exports every
+entry point include/segquant.h declares, and rejects invalid arguments on the
+host before touching CUDA (so these calls are safe without a device)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from w8a8_gemm_b200 import binding as B
+from w8a8_gemm_b200 import build as sqbuild
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "segquant.h")
+
+SQ_ERR_INVALID_ARG, SQ_ERR_UNSUPPORTED, SQ_ERR_ALIGNMENT, SQ_ERR_OVERFLOW = -1, -2, -3, -4
+
+
+@pytest.fixture(scope="module")
+def L():
+    sqbuild.build()
+    return B.lib()
+
+
+def declared_entry_points():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"SQ_API\s+[\w\s\*]+?\b(sq_\w+)\s*\(", text)))
+
+
+def test_header_declares_expected_calls():
+    names = declared_entry_points()
+    for n in ("sq_quantize_act", "sq_quantize_weight_seg", "sq_dualscale_seglinear_gemm"):
+        assert n in names
+    assert set(names) == set(B.EXPORTED)
+
+
+def test_library_exports_every_declared_symbol(L):
+    for name in declared_entry_points():
+        assert hasattr(L, name), name
+
+
+def test_status_strings(L):
+    assert B.status_string(0) == "SQ_OK"
+    for code in range(-7, 0):
+        assert B.status_string(code).startswith("SQ_ERR_")
+    assert B.lib().sq_version() == 100
+
+
+def _seg(mode, offsets, groups=1):
+    s = B.Segments(mode, offsets, groups)
+    c, keep = s._c()
+    return c, keep
+
+
+FAKE = 0x10000  # 16-byte aligned, never dereferenced: validation fails first
+
+
+def test_quantize_act_rejects_bad_shapes(L):
+    p = ctypes.c_void_p
+    c, keep = _seg(B.SQ_SEG_NONE, None)
+    # K not a multiple of 16
+    assert L.sq_quantize_act(p(FAKE), 4, 24, 24, None, p(FAKE), ctypes.byref(c), p(FAKE),
+                             None) == SQ_ERR_INVALID_ARG
+    # ldx < K
+    assert L.sq_quantize_act(p(FAKE), 4, 32, 16, None, p(FAKE), ctypes.byref(c), p(FAKE),
+                             None) == SQ_ERR_INVALID_ARG
+    # misaligned x
+    assert L.sq_quantize_act(p(FAKE + 2), 4, 32, 32, None, p(FAKE), ctypes.byref(c), p(FAKE),
+                             None) == SQ_ERR_ALIGNMENT
+    # ldx not a multiple of 8 elements
+    assert L.sq_quantize_act(p(FAKE), 4, 32, 36, None, p(FAKE), ctypes.byref(c), p(FAKE),
+                             None) == SQ_ERR_ALIGNMENT
+
+
+def test_segment_table_validation(L):
+    p = ctypes.c_void_p
+    # input segments must end at K and be multiples of 32 wide
+    c, keep = _seg(B.SQ_SEG_INPUT, [0, 32, 48])
+    assert L.sq_quantize_act(p(FAKE), 4, 48, 48, None, p(FAKE), ctypes.byref(c), p(FAKE),
+                             None) == SQ_ERR_UNSUPPORTED
+    c, keep = _seg(B.SQ_SEG_INPUT, [0, 32, 32, 64])
+    assert L.sq_quantize_act(p(FAKE), 4, 64, 64, None, p(FAKE), ctypes.byref(c), p(FAKE),
+                             None) == SQ_ERR_INVALID_ARG
+    c, keep = _seg(B.SQ_SEG_INPUT, [0, 32, 64])
+    assert L.sq_quantize_act(p(FAKE), 4, 96, 96, None, p(FAKE), ctypes.byref(c), p(FAKE),
+                             None) == SQ_ERR_INVALID_ARG
+    # input mode has one activation group
+    c, keep = _seg(B.SQ_SEG_INPUT, [0, 32, 64], groups=2)
+    assert L.sq_quantize_act(p(FAKE), 4, 64, 64, None, p(FAKE), ctypes.byref(c), p(FAKE),
+                             None) == SQ_ERR_INVALID_ARG
+    # output mode: G must be 1 or n_seg; with G > 1 widths are multiples of 128
+    c, keep = _seg(B.SQ_SEG_OUTPUT, [0, 128, 256, 384], groups=2)
+    assert L.sq_quantize_weight_seg(p(FAKE), 384, 64, None, ctypes.byref(c), p(FAKE), p(FAKE),
+                                    None) == SQ_ERR_INVALID_ARG
+    c, keep = _seg(B.SQ_SEG_OUTPUT, [0, 64, 192], groups=2)
+    assert L.sq_quantize_weight_seg(p(FAKE), 192, 64, None, ctypes.byref(c), p(FAKE), p(FAKE),
+                                    None) == SQ_ERR_UNSUPPORTED
+    # output offsets must end at N
+    c, keep = _seg(B.SQ_SEG_OUTPUT, [0, 128, 256], groups=1)
+    assert L.sq_quantize_weight_seg(p(FAKE), 300, 64, None, ctypes.byref(c), p(FAKE), p(FAKE),
+                                    None) == SQ_ERR_INVALID_ARG
+    # too many segments
+    offs = list(range(0, 32 * 66, 32))
+    c, keep = _seg(B.SQ_SEG_INPUT, offs)
+    K = offs[-1]
+    assert L.sq_quantize_act(p(FAKE), 4, K, K, None, p(FAKE), ctypes.byref(c), p(FAKE),
+                             None) == SQ_ERR_INVALID_ARG
+
+
+def test_gemm_overflow_and_layout_checks(L):
+    p = ctypes.c_void_p
+    c, keep = _seg(B.SQ_SEG_NONE, None)
+    # one K-segment wider than 132104 could overflow int32
+    K = 132112
+    assert L.sq_dualscale_seglinear_gemm(p(FAKE), p(FAKE), p(FAKE), p(FAKE), None, p(FAKE), 0,
+                                         8, 8, K, 8, ctypes.byref(c), None) == SQ_ERR_OVERFLOW
+    # ldy < N
+    assert L.sq_dualscale_seglinear_gemm(p(FAKE), p(FAKE), p(FAKE), p(FAKE), None, p(FAKE), 0,
+                                         8, 16, 64, 8, ctypes.byref(c), None) == SQ_ERR_INVALID_ARG
+    # bf16 output rows must start 16-byte aligned (ldy multiple of 8)
+    assert L.sq_dualscale_seglinear_gemm(p(FAKE), p(FAKE), p(FAKE), p(FAKE), None, p(FAKE), 0,
+                                         8, 20, 64, 20, ctypes.byref(c), None) == SQ_ERR_ALIGNMENT
+    # bad output dtype
+    assert L.sq_dualscale_seglinear_gemm(p(FAKE), p(FAKE), p(FAKE), p(FAKE), None, p(FAKE), 7,
+                                         8, 16, 64, 16, ctypes.byref(c), None) == SQ_ERR_INVALID_ARG
+    # misaligned planes
+    assert L.sq_dualscale_seglinear_gemm(p(FAKE + 8), p(FAKE), p(FAKE), p(FAKE), None, p(FAKE), 0,
+                                         8, 16, 64, 16, ctypes.byref(c), None) == SQ_ERR_ALIGNMENT
+    # null scales
+    assert L.sq_dualscale_seglinear_gemm(p(FAKE), p(FAKE), None, p(FAKE), None, p(FAKE), 0,
+                                         8, 16, 64, 16, ctypes.byref(c), None) == SQ_ERR_INVALID_ARG
+    # M == 0 is a valid no-op that never touches CUDA
+    assert L.sq_dualscale_seglinear_gemm(None, None, None, None, None, None, 0,
+                                         0, 16, 64, 16, ctypes.byref(c), None) == 0
+
+
+def test_binding_without_library_fails_loudly(monkeypatch, tmp_path):
+    monkeypatch.setattr(B, "LIB_PATH", str(tmp_path / "missing.so"))
+    monkeypatch.setattr(B, "_lib", None)
+    with pytest.raises(RuntimeError, match="missing"):
+        B.lib()

@@ -1,0 +1,155 @@
+"""Parity of the CUDA path against the CPU oracle on the same seeded inputs.
+
+Bar (as fixed for this method): int8 planes, int8 weights, the scales that
+come out of calibration and the int32 accumulators are bit-exact; fp32 output
+within max |y - r| / (|r| + 1e-3 rms(r)) <= 1e-3 (and, for one K-segment, the
+epilogue runs the oracle's fp32 operations in the oracle's order, so it is
+bit-exact); bf16 output within 1 bf16 ulp of RNE_bf16(oracle fp32).
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from w8a8_gemm_b200 import binding as B
+from w8a8_gemm_b200 import workloads as wl
+
+from parity import (bf16_ulp_diff, gpu_run, oracle_acc, oracle_prep, oracle_y, rel_err_floor,
+                    sample_rows, segments)
+
+pytestmark = pytest.mark.gpu
+FP32_TOL = 1e-3
+
+
+def _input_layer_mixed():
+    L = wl.outproj_layer("mixed", 300, 416, 264, 32, seed=11)
+    L.offsets = [0, 64, 96, 224, 416]   # widths 64, 32, 128, 192
+    return L
+
+
+SMALL = {
+    "none_tails": lambda: wl.gelu_layer("none", 300, 416, 520, seed=1, bias=True),
+    "none_tiny": lambda: wl.gelu_layer("tiny", 1, 16, 8, seed=2, bias=True),
+    "none_ragged": lambda: wl.gelu_layer("rag", 5, 48, 13, seed=3, bias=True),
+    "none_k_tail": lambda: wl.gelu_layer("ktail", 129, 144, 300, seed=4, bias=True),
+    "input_heads": lambda: wl.outproj_layer("heads", 300, 448, 264, 64, seed=5),
+    "input_mixed": _input_layer_mixed,
+    "input_wide": lambda: wl.outproj_layer("wide", 130, 1024, 136, 512, seed=6),
+    "output_g1": lambda: wl.adanorm_layer("o1", 200, 256, 768, 3, seed=7, G=1),
+    "output_g3": lambda: wl.adanorm_layer("o3", 200, 256, 768, 3, seed=8, G=3),
+    "output_g2_bn128": lambda: wl.adanorm_layer("o2", 130, 128, 256, 2, seed=9, G=2),
+    "qkv_g3": lambda: wl.qkv_layer("qkv", 257, 192, 384, 3, seed=10, G=3),
+}
+
+
+def _check_layer(L, full_rows=True):
+    prep = oracle_prep(L)
+    g = gpu_run(L, out_dtype=torch.float32, s32=True)
+    assert np.array_equal(g["s_act"].cpu().numpy(), prep["s_act"])
+    assert np.array_equal(g["wq"].cpu().numpy(), prep["wq"])
+    assert np.array_equal(g["s_w"].cpu().numpy(), prep["s_w"])
+    assert np.array_equal(g["planes"].cpu().numpy(), prep["planes"])
+    acc = oracle_acc(L, prep)
+    assert np.array_equal(g["acc"].cpu().numpy(), acc)
+    r = oracle_y(L, prep)
+    y = g["y"].cpu().numpy()
+    assert rel_err_floor(y, r) <= FP32_TOL
+    if L.S == 1:
+        assert np.array_equal(y, r)          # same fp32 operations, same order
+    gb = gpu_run(L, out_dtype=torch.bfloat16)
+    assert bf16_ulp_diff(gb["y"], r) <= 1
+
+
+@pytest.mark.parametrize("name", sorted(SMALL))
+def test_small_layers_bitexact(name):
+    _check_layer(SMALL[name]())
+
+
+def test_every_bf16_value_quantizes_like_oracle():
+    allbits = np.arange(65536, dtype=np.uint32).astype(np.uint16).reshape(256, 256)
+    s_act = np.array([[[1 / 64, 1 / 512]]], np.float32)
+    ref = oracle.quantize_act(allbits, s_act)
+    x = torch.from_numpy(allbits.view(np.int16)).view(torch.bfloat16).cuda()
+    planes = torch.empty(1, 2, 256, 256, dtype=torch.int8, device="cuda")
+    B.sq_quantize_act(x, None, torch.from_numpy(s_act).cuda(), B.Segments(), planes)
+    assert np.array_equal(planes.cpu().numpy(), ref)
+
+
+def test_strided_activation_rows():
+    """ldx > K: the activation is a column slice of a wider tensor."""
+    L = wl.gelu_layer("ld", 70, 96, 40, seed=12, bias=True)
+    wide = torch.zeros(70, 160, dtype=torch.bfloat16)
+    wide[:, 32:128] = L.x
+    xg = wide.cuda()[:, 32:128]
+    s_act = oracle.calibrate_act(wl.bits(L.x_cal))
+    ref = oracle.quantize_act(wl.bits(L.x), s_act)
+    planes = torch.empty(1, 2, 70, 96, dtype=torch.int8, device="cuda")
+    B.sq_quantize_act(xg, None, torch.from_numpy(s_act).cuda(), B.Segments(), planes)
+    assert np.array_equal(planes.cpu().numpy(), ref)
+
+
+def test_empty_batch_is_noop():
+    L = wl.gelu_layer("e", 4, 32, 16, seed=13)
+    seg = B.Segments()
+    planes = torch.empty(1, 2, 0, 32, dtype=torch.int8, device="cuda")
+    x = torch.empty(0, 32, dtype=torch.bfloat16, device="cuda")
+    s_act = torch.ones(1, 1, 2, device="cuda")
+    B.sq_quantize_act(x, None, s_act, seg, planes)
+    y = torch.empty(0, 16, dtype=torch.bfloat16, device="cuda")
+    wq = torch.zeros(16, 32, dtype=torch.int8, device="cuda")
+    B.sq_dualscale_seglinear_gemm(planes, wq, torch.ones(1, 16, device="cuda"), s_act, None, y,
+                                  seg)
+    torch.cuda.synchronize()
+
+
+def test_output_segments_equal_separate_calls_on_gpu():
+    """SegLinear output identity on the device: one G = 3 call equals three
+    single-segment calls on the same planes and weights, bit for bit."""
+    L = wl.adanorm_layer("o3", 260, 256, 768, 3, seed=14, G=3)
+    g = gpu_run(L, out_dtype=torch.float32)
+    for j in range(3):
+        n0, n1 = L.offsets[j], L.offsets[j + 1]
+        y = torch.empty(L.M, n1 - n0, dtype=torch.float32, device="cuda")
+        B.sq_dualscale_seglinear_gemm(g["planes"][j:j + 1].contiguous(),
+                                      g["wq"][n0:n1].contiguous(),
+                                      g["s_w"][:, n0:n1].contiguous(),
+                                      g["s_act"][j:j + 1].contiguous(),
+                                      L.bias[n0:n1].cuda(), y, B.Segments())
+        assert torch.equal(y, g["y"][:, n0:n1])
+
+
+def test_input_segments_sum_on_gpu():
+    """SegLinear input identity on the device: the int32 partials of each
+    K-segment equal a standalone one-segment call on that slice."""
+    L = wl.outproj_layer("heads", 200, 256, 136, 64, seed=15)
+    g = gpu_run(L, out_dtype=torch.float32, s32=True)
+    for i in range(4):
+        k0, k1 = L.offsets[i], L.offsets[i + 1]
+        acc = torch.empty(1, 2, L.M, L.N, dtype=torch.int32, device="cuda")
+        B.sq_debug_gemm_s32(g["planes"][:, :, :, k0:k1].contiguous(),
+                            g["wq"][:, k0:k1].contiguous(), B.Segments(), acc)
+        assert torch.equal(acc[0], g["acc"][i])
+
+
+FULL = ["c1_tiny_dualscale", "c2_sd35_adanorm", "c3_sd35_attn_out", "c4_sd35_ffn"]
+
+
+@pytest.mark.parametrize("cfg", FULL)
+def test_full_size_configs_sampled_rows(cfg):
+    """BASELINE-sized layers: planes, weights and scales compared in full,
+    outputs on every row of the first and last M tile plus a strided sample."""
+    for L in wl.config_layers(cfg, seed=0):
+        prep = oracle_prep(L)
+        g = gpu_run(L, out_dtype=torch.bfloat16)
+        assert np.array_equal(g["s_act"].cpu().numpy(), prep["s_act"])
+        assert np.array_equal(g["wq"].cpu().numpy(), prep["wq"])
+        assert np.array_equal(g["s_w"].cpu().numpy(), prep["s_w"])
+        assert np.array_equal(g["planes"].cpu().numpy(), prep["planes"])
+        rows = sample_rows(L.M)
+        r = oracle_y(L, prep, rows=rows)
+        yb = g["y"][torch.from_numpy(rows).cuda()]
+        assert bf16_ulp_diff(yb, r) <= 1
+        gf = gpu_run(L, out_dtype=torch.float32)
+        assert rel_err_floor(gf["y"][torch.from_numpy(rows).cuda()].cpu().numpy(), r) <= FP32_TOL
+        del g, gf
+        torch.cuda.empty_cache()

@@ -1,0 +1,227 @@
+"""Thin Python binding of libsegquant.so: the same entry points as
+include/segquant.h, taking torch tensors.  Argument marshalling only -- every
+step of the computation runs in the library's CUDA kernels; there is no CPU or
+PyTorch fallback.  A missing library raises at the first call.
+
+All tensors must be CUDA tensors on the current device; calls are enqueued on
+torch's current CUDA stream.  Every call raises SegQuantError unless the
+library returned SQ_OK.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+from typing import Optional, Sequence
+
+import torch
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libsegquant.so")
+
+SQ_OK = 0
+SQ_SEG_NONE, SQ_SEG_OUTPUT, SQ_SEG_INPUT = 0, 1, 2
+SQ_OUT_BF16, SQ_OUT_F32 = 0, 1
+SQ_MAX_SEGMENTS = 64
+
+EXPORTED = ("sq_calibrate_act", "sq_quantize_act", "sq_quantize_weight_seg",
+            "sq_dualscale_seglinear_gemm", "sq_debug_gemm_s32", "sq_get_device_status",
+            "sq_status_string", "sq_version")
+
+
+class SegQuantError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        self.code = code
+        super().__init__(f"{where}: {status_string(code)} ({code})")
+
+
+class _Segments(ctypes.Structure):
+    _fields_ = [("mode", ctypes.c_int32), ("n_seg", ctypes.c_int32),
+                ("offsets", ctypes.POINTER(ctypes.c_int32)), ("n_groups", ctypes.c_int32)]
+
+
+@dataclass
+class Segments:
+    """SegLinear segment table: mode, boundaries (over N for output mode, over
+    K for input mode) and the number of activation groups G."""
+    mode: int = SQ_SEG_NONE
+    offsets: Optional[Sequence[int]] = None
+    n_groups: int = 1
+
+    @property
+    def n_seg(self) -> int:
+        return 1 if self.offsets is None else len(self.offsets) - 1
+
+    @property
+    def S(self) -> int:
+        return self.n_seg if self.mode == SQ_SEG_INPUT else 1
+
+    def _c(self):
+        if self.offsets is None:
+            arr = None
+            ptr = ctypes.POINTER(ctypes.c_int32)()
+        else:
+            arr = (ctypes.c_int32 * len(self.offsets))(*[int(v) for v in self.offsets])
+            ptr = ctypes.cast(arr, ctypes.POINTER(ctypes.c_int32))
+        s = _Segments(self.mode, self.n_seg, ptr, self.n_groups)
+        return s, arr  # keep the array alive for the call
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load libsegquant.so (built in-tree by w8a8_gemm_b200.build)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(
+                f"{LIB_PATH} is missing: build it with `python -m w8a8_gemm_b200.build` "
+                "(there is no fallback implementation)")
+        L = ctypes.CDLL(LIB_PATH)
+        p, i64 = ctypes.c_void_p, ctypes.c_int64
+        seg = ctypes.POINTER(_Segments)
+        L.sq_calibrate_act.argtypes = [p, i64, i64, i64, p, seg, p, p]
+        L.sq_quantize_act.argtypes = [p, i64, i64, i64, p, p, seg, p, p]
+        L.sq_quantize_weight_seg.argtypes = [p, i64, i64, p, seg, p, p, p]
+        L.sq_dualscale_seglinear_gemm.argtypes = [p, p, p, p, p, p, ctypes.c_int, i64, i64, i64,
+                                                  i64, seg, p]
+        L.sq_debug_gemm_s32.argtypes = [p, p, i64, i64, i64, seg, p, p]
+        L.sq_get_device_status.argtypes = []
+        L.sq_status_string.argtypes = [ctypes.c_int]
+        L.sq_status_string.restype = ctypes.c_char_p
+        L.sq_version.argtypes = []
+        for f in (L.sq_calibrate_act, L.sq_quantize_act, L.sq_quantize_weight_seg,
+                  L.sq_dualscale_seglinear_gemm, L.sq_debug_gemm_s32, L.sq_get_device_status,
+                  L.sq_version):
+            f.restype = ctypes.c_int
+        _lib = L
+    return _lib
+
+
+def status_string(code: int) -> str:
+    return lib().sq_status_string(int(code)).decode()
+
+
+def _check(code: int, where: str):
+    if code != SQ_OK:
+        raise SegQuantError(code, where)
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream():
+    return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+
+def _need(t: Optional[torch.Tensor], dtype, name: str, optional=False):
+    if t is None:
+        if optional:
+            return
+        raise ValueError(f"{name} is required")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+
+
+def _rows(x: torch.Tensor):
+    if x.dim() != 2 or x.stride(1) != 1:
+        raise ValueError("expected a 2-D tensor with unit column stride")
+    return x.shape[0], x.shape[1], x.stride(0)
+
+
+# --------------------------------------------------------------------- calls
+def sq_calibrate_act(x: torch.Tensor, d: Optional[torch.Tensor], seg: Segments,
+                     s_act: torch.Tensor) -> torch.Tensor:
+    """AMax calibration into s_act fp32 [G][S][2]."""
+    _need(x, torch.bfloat16, "x")
+    _need(d, torch.float32, "d", optional=True)
+    _need(s_act, torch.float32, "s_act")
+    M, K, ldx = _rows(x)
+    cs, keep = seg._c()
+    _check(lib().sq_calibrate_act(_ptr(x), M, K, ldx, _ptr(d), ctypes.byref(cs), _ptr(s_act),
+                                  _stream()), "sq_calibrate_act")
+    return s_act
+
+
+def sq_quantize_act(x: torch.Tensor, d: Optional[torch.Tensor], s_act: torch.Tensor,
+                    seg: Segments, planes: torch.Tensor) -> torch.Tensor:
+    """DualScale quantization of X / d into planes int8 [G][2][M][K]."""
+    _need(x, torch.bfloat16, "x")
+    _need(d, torch.float32, "d", optional=True)
+    _need(s_act, torch.float32, "s_act")
+    _need(planes, torch.int8, "planes")
+    M, K, ldx = _rows(x)
+    if tuple(planes.shape) != (seg.n_groups, 2, M, K) or not planes.is_contiguous():
+        raise ValueError(f"planes must be contiguous [{seg.n_groups}, 2, {M}, {K}]")
+    cs, keep = seg._c()
+    _check(lib().sq_quantize_act(_ptr(x), M, K, ldx, _ptr(d), _ptr(s_act), ctypes.byref(cs),
+                                 _ptr(planes), _stream()), "sq_quantize_act")
+    return planes
+
+
+def sq_quantize_weight_seg(w: torch.Tensor, d: Optional[torch.Tensor], seg: Segments,
+                           wq: torch.Tensor, s_w: torch.Tensor):
+    """Segment-wise AMax weight quantization: wq int8 [N][K], s_w fp32 [S][N]."""
+    _need(w, torch.bfloat16, "w")
+    _need(d, torch.float32, "d", optional=True)
+    _need(wq, torch.int8, "wq")
+    _need(s_w, torch.float32, "s_w")
+    if not (w.is_contiguous() and wq.is_contiguous() and s_w.is_contiguous()):
+        raise ValueError("w, wq and s_w must be contiguous")
+    N, K = w.shape
+    cs, keep = seg._c()
+    _check(lib().sq_quantize_weight_seg(_ptr(w), N, K, _ptr(d), ctypes.byref(cs), _ptr(wq),
+                                        _ptr(s_w), _stream()), "sq_quantize_weight_seg")
+    return wq, s_w
+
+
+def sq_dualscale_seglinear_gemm(planes: torch.Tensor, wq: torch.Tensor, s_w: torch.Tensor,
+                                s_act: torch.Tensor, bias: Optional[torch.Tensor],
+                                y: torch.Tensor, seg: Segments) -> torch.Tensor:
+    """Y = sum_i s_w (s+ X^+_i W^_i + s- X^-_i W^_i) + bias into y (bf16 or fp32 [M][N])."""
+    _need(planes, torch.int8, "planes")
+    _need(wq, torch.int8, "wq")
+    _need(s_w, torch.float32, "s_w")
+    _need(s_act, torch.float32, "s_act")
+    _need(bias, torch.bfloat16, "bias", optional=True)
+    if y.dtype not in (torch.bfloat16, torch.float32) or not y.is_cuda:
+        raise ValueError("y must be a CUDA bf16 or fp32 tensor")
+    G, two, M, K = planes.shape
+    N = wq.shape[0]
+    if two != 2 or wq.shape[1] != K or y.shape[0] != M or y.shape[1] != N or y.stride(1) != 1:
+        raise ValueError("shape mismatch between planes [G,2,M,K], wq [N,K] and y [M,N]")
+    out = SQ_OUT_BF16 if y.dtype == torch.bfloat16 else SQ_OUT_F32
+    cs, keep = seg._c()
+    _check(lib().sq_dualscale_seglinear_gemm(_ptr(planes), _ptr(wq), _ptr(s_w), _ptr(s_act),
+                                             _ptr(bias), _ptr(y), out, M, N, K, y.stride(0),
+                                             ctypes.byref(cs), _stream()),
+           "sq_dualscale_seglinear_gemm")
+    return y
+
+
+def sq_debug_gemm_s32(planes: torch.Tensor, wq: torch.Tensor, seg: Segments,
+                      acc: torch.Tensor) -> torch.Tensor:
+    """Raw int32 accumulators [S][2][M][N] of the same tensor-core kernel."""
+    _need(planes, torch.int8, "planes")
+    _need(wq, torch.int8, "wq")
+    _need(acc, torch.int32, "acc")
+    G, two, M, K = planes.shape
+    N = wq.shape[0]
+    if tuple(acc.shape) != (seg.S, 2, M, N) or not acc.is_contiguous():
+        raise ValueError(f"acc must be contiguous [{seg.S}, 2, {M}, {N}]")
+    cs, keep = seg._c()
+    _check(lib().sq_debug_gemm_s32(_ptr(planes), _ptr(wq), M, N, K, ctypes.byref(cs), _ptr(acc),
+                                   _stream()), "sq_debug_gemm_s32")
+    return acc
+
+
+def sq_get_device_status() -> int:
+    """Synchronise and return (and clear) the device error word."""
+    return lib().sq_get_device_status()
+
+
+def sq_version() -> int:
+    return lib().sq_version()

@@ -1,0 +1,274 @@
+// api.cu -- the C ABI declared in include/segquant.h: argument validation on
+// the host, the device error word, and dispatch to the kernels.  Nothing here
+// allocates device memory.
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <mutex>
+
+#include "sq_internal.h"
+
+namespace sq {
+namespace {
+
+// Error word written by kernels whose bounded waits ran out.
+__device__ int g_device_status = 0;
+
+constexpr int64_t kMaxSegWidth = 132104;   // 128 * 127 * 132104 < 2^31
+constexpr int kMaxDevices = 64;
+
+bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// Current device must be sm_100 (the kernels are built for sm_100a only).
+sq_status check_device() {
+  static int checked[kMaxDevices] = {};  // 0 unknown, 1 ok, -1 unsupported
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+    cudaGetLastError();
+    return SQ_ERR_NO_DEVICE;
+  }
+  if (checked[dev] == 0) {
+    int major = 0, minor = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess) {
+      cudaGetLastError();
+      return SQ_ERR_NO_DEVICE;
+    }
+    checked[dev] = (major == 10 && minor == 0) ? 1 : -1;
+  }
+  return checked[dev] == 1 ? SQ_OK : SQ_ERR_NO_DEVICE;
+}
+
+// Validates a segment table.  extent_n < 0 means N is not known to the call
+// (activation-side calls), in which case the output offsets end is not checked.
+sq_status parse_segments(const sq_segments *seg, int64_t K, int64_t extent_n, SegParams *out) {
+  SegParams p{};
+  if (seg == nullptr) {
+    p.mode = SQ_SEG_NONE;
+    p.n_seg = 1;
+    p.G = 1;
+    p.S = 1;
+    p.off[0] = 0;
+    p.off[1] = static_cast<int32_t>(K);
+    *out = p;
+    return SQ_OK;
+  }
+  if (seg->mode < SQ_SEG_NONE || seg->mode > SQ_SEG_INPUT) return SQ_ERR_INVALID_ARG;
+  if (seg->n_seg < 1 || seg->n_seg > SQ_MAX_SEGMENTS || seg->n_groups < 1)
+    return SQ_ERR_INVALID_ARG;
+  p.mode = seg->mode;
+  p.n_seg = seg->n_seg;
+  p.G = seg->n_groups;
+  if (seg->mode == SQ_SEG_NONE) {
+    if (seg->n_seg != 1 || seg->n_groups != 1) return SQ_ERR_INVALID_ARG;
+    p.S = 1;
+    p.off[0] = 0;
+    p.off[1] = static_cast<int32_t>(K);
+    *out = p;
+    return SQ_OK;
+  }
+  if (seg->offsets == nullptr || seg->offsets[0] != 0) return SQ_ERR_INVALID_ARG;
+  for (int i = 0; i < seg->n_seg; ++i) {
+    if (seg->offsets[i + 1] <= seg->offsets[i]) return SQ_ERR_INVALID_ARG;
+    p.off[i] = seg->offsets[i];
+  }
+  p.off[seg->n_seg] = seg->offsets[seg->n_seg];
+  if (seg->mode == SQ_SEG_INPUT) {
+    if (seg->n_groups != 1) return SQ_ERR_INVALID_ARG;
+    if (p.off[p.n_seg] != K) return SQ_ERR_INVALID_ARG;
+    for (int i = 0; i < p.n_seg; ++i) {
+      const int64_t w = p.off[i + 1] - p.off[i];
+      if (w % 32 != 0) return SQ_ERR_UNSUPPORTED;
+      if (w > kMaxSegWidth) return SQ_ERR_OVERFLOW;
+    }
+    p.S = p.n_seg;
+  } else {
+    if (seg->n_groups != 1 && seg->n_groups != seg->n_seg) return SQ_ERR_INVALID_ARG;
+    if (extent_n >= 0 && p.off[p.n_seg] != extent_n) return SQ_ERR_INVALID_ARG;
+    if (seg->n_groups > 1)
+      for (int i = 0; i < p.n_seg; ++i)
+        if ((p.off[i + 1] - p.off[i]) % 128 != 0) return SQ_ERR_UNSUPPORTED;
+    p.S = 1;
+  }
+  *out = p;
+  return SQ_OK;
+}
+
+sq_status check_k(int64_t K) {
+  if (K < 16 || K % 16 != 0 || K > INT32_MAX) return SQ_ERR_INVALID_ARG;
+  return SQ_OK;
+}
+
+sq_status check_act(const void *x, int64_t M, int64_t K, int64_t ldx) {
+  if (M < 0 || M > INT32_MAX) return SQ_ERR_INVALID_ARG;
+  sq_status st = check_k(K);
+  if (st != SQ_OK) return st;
+  if (ldx < K) return SQ_ERR_INVALID_ARG;
+  if (M > 0 && x == nullptr) return SQ_ERR_INVALID_ARG;
+  if (ldx % 8 != 0 || !aligned(x, 16)) return SQ_ERR_ALIGNMENT;
+  return SQ_OK;
+}
+
+sq_status from_cuda(cudaError_t e) { return e == cudaSuccess ? SQ_OK : SQ_ERR_CUDA; }
+
+#define SQ_TRY(expr)               \
+  do {                             \
+    const sq_status _s = (expr);   \
+    if (_s != SQ_OK) return _s;    \
+  } while (0)
+
+sq_status gemm_common(const int8_t *planes, const int8_t *wq, const float *s_w,
+                      const float *s_act, const void *bias, void *y, int out_kind, int64_t M,
+                      int64_t N, int64_t K, int64_t ldy, const sq_segments *seg,
+                      cudaStream_t stream) {
+  if (M < 0 || M > INT32_MAX || N < 1 || N > INT32_MAX) return SQ_ERR_INVALID_ARG;
+  SQ_TRY(check_k(K));
+  SegParams sp;
+  SQ_TRY(parse_segments(seg, K, N, &sp));
+  if (sp.S == 1 && K > kMaxSegWidth) return SQ_ERR_OVERFLOW;
+  if (M == 0) return SQ_OK;
+  if (planes == nullptr || wq == nullptr || y == nullptr) return SQ_ERR_INVALID_ARG;
+  if (out_kind != OUT_S32 && (s_w == nullptr || s_act == nullptr)) return SQ_ERR_INVALID_ARG;
+  if (!aligned(planes, 16) || !aligned(wq, 16) || !aligned(y, 16)) return SQ_ERR_ALIGNMENT;
+  if (s_w && !aligned(s_w, 4)) return SQ_ERR_ALIGNMENT;
+  if (s_act && !aligned(s_act, 4)) return SQ_ERR_ALIGNMENT;
+  if (bias && !aligned(bias, 2)) return SQ_ERR_ALIGNMENT;
+  if (out_kind != OUT_S32) {
+    const int64_t elem = (out_kind == OUT_BF16) ? 2 : 4;
+    if (ldy < N) return SQ_ERR_INVALID_ARG;
+    if ((ldy * elem) % 16 != 0) return SQ_ERR_ALIGNMENT;
+  }
+  SQ_TRY(check_device());
+  GemmRequest r;
+  r.planes = planes;
+  r.wq = wq;
+  r.s_w = s_w;
+  r.s_act = s_act;
+  r.bias = static_cast<const uint16_t *>(bias);
+  r.y = y;
+  r.ldy = ldy;
+  r.out_kind = out_kind;
+  r.M = M;
+  r.N = N;
+  r.K = K;
+  r.seg = sp;
+  r.status = device_status_word();
+  if (r.status == nullptr) return SQ_ERR_CUDA;
+  return launch_gemm(r, stream);
+}
+
+}  // namespace
+
+int *device_status_word() {
+  static int *addr[kMaxDevices] = {};
+  static std::mutex mu;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lock(mu);
+  if (addr[dev] == nullptr) {
+    void *p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_device_status) != cudaSuccess) {
+      cudaGetLastError();
+      return nullptr;
+    }
+    addr[dev] = static_cast<int *>(p);
+  }
+  return addr[dev];
+}
+
+}  // namespace sq
+
+using namespace sq;
+
+extern "C" {
+
+sq_status sq_calibrate_act(const void *x, int64_t M, int64_t K, int64_t ldx, const float *d,
+                           const sq_segments *seg, float *s_act, sq_stream_t stream) {
+  if (M < 1) return SQ_ERR_INVALID_ARG;
+  SQ_TRY(check_act(x, M, K, ldx));
+  SegParams sp;
+  SQ_TRY(parse_segments(seg, K, -1, &sp));
+  if (s_act == nullptr || !aligned(s_act, 4)) return SQ_ERR_INVALID_ARG;
+  if (d && !aligned(d, 4)) return SQ_ERR_ALIGNMENT;
+  SQ_TRY(check_device());
+  return from_cuda(launch_calibrate_act(static_cast<const uint16_t *>(x), M, K, ldx, d, sp,
+                                        s_act, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+sq_status sq_quantize_act(const void *x, int64_t M, int64_t K, int64_t ldx, const float *d,
+                          const float *s_act, const sq_segments *seg, int8_t *planes,
+                          sq_stream_t stream) {
+  SQ_TRY(check_act(x, M, K, ldx));
+  SegParams sp;
+  SQ_TRY(parse_segments(seg, K, -1, &sp));
+  if (M == 0) return SQ_OK;
+  if (s_act == nullptr || planes == nullptr) return SQ_ERR_INVALID_ARG;
+  if (!aligned(s_act, 4) || (d && !aligned(d, 4)) || !aligned(planes, 16))
+    return SQ_ERR_ALIGNMENT;
+  SQ_TRY(check_device());
+  return from_cuda(launch_quantize_act(static_cast<const uint16_t *>(x), M, K, ldx, d, s_act, sp,
+                                       planes, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+sq_status sq_quantize_weight_seg(const void *w, int64_t N, int64_t K, const float *d,
+                                 const sq_segments *seg, int8_t *wq, float *s_w,
+                                 sq_stream_t stream) {
+  if (N < 1 || N > INT32_MAX) return SQ_ERR_INVALID_ARG;
+  SQ_TRY(check_k(K));
+  SegParams sp;
+  SQ_TRY(parse_segments(seg, K, N, &sp));
+  if (w == nullptr || wq == nullptr || s_w == nullptr) return SQ_ERR_INVALID_ARG;
+  if (!aligned(w, 16) || !aligned(wq, 16) || !aligned(s_w, 4) || (d && !aligned(d, 4)))
+    return SQ_ERR_ALIGNMENT;
+  SQ_TRY(check_device());
+  return from_cuda(launch_quantize_weight(static_cast<const uint16_t *>(w), N, K, d, sp, wq, s_w,
+                                          reinterpret_cast<cudaStream_t>(stream)));
+}
+
+sq_status sq_dualscale_seglinear_gemm(const int8_t *planes, const int8_t *wq, const float *s_w,
+                                      const float *s_act, const void *bias, void *y,
+                                      sq_out_dtype out_dtype, int64_t M, int64_t N, int64_t K,
+                                      int64_t ldy, const sq_segments *seg, sq_stream_t stream) {
+  if (out_dtype != SQ_OUT_BF16 && out_dtype != SQ_OUT_F32) return SQ_ERR_INVALID_ARG;
+  return gemm_common(planes, wq, s_w, s_act, bias, y,
+                     out_dtype == SQ_OUT_BF16 ? OUT_BF16 : OUT_F32, M, N, K, ldy, seg,
+                     reinterpret_cast<cudaStream_t>(stream));
+}
+
+sq_status sq_debug_gemm_s32(const int8_t *planes, const int8_t *wq, int64_t M, int64_t N,
+                            int64_t K, const sq_segments *seg, int32_t *acc,
+                            sq_stream_t stream) {
+  return gemm_common(planes, wq, nullptr, nullptr, nullptr, acc, OUT_S32, M, N, K, N, seg,
+                     reinterpret_cast<cudaStream_t>(stream));
+}
+
+sq_status sq_get_device_status(void) {
+  SQ_TRY(check_device());
+  if (cudaDeviceSynchronize() != cudaSuccess) return SQ_ERR_CUDA;
+  int *word = device_status_word();
+  if (word == nullptr) return SQ_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpy(&v, word, sizeof v, cudaMemcpyDeviceToHost) != cudaSuccess) return SQ_ERR_CUDA;
+  const int zero = 0;
+  if (cudaMemcpy(word, &zero, sizeof zero, cudaMemcpyHostToDevice) != cudaSuccess)
+    return SQ_ERR_CUDA;
+  return v == 0 ? SQ_OK : static_cast<sq_status>(v);
+}
+
+const char *sq_status_string(sq_status s) {
+  switch (s) {
+    case SQ_OK: return "SQ_OK";
+    case SQ_ERR_INVALID_ARG: return "SQ_ERR_INVALID_ARG: invalid argument";
+    case SQ_ERR_UNSUPPORTED: return "SQ_ERR_UNSUPPORTED: valid request this build does not implement";
+    case SQ_ERR_ALIGNMENT: return "SQ_ERR_ALIGNMENT: pointer or leading dimension misaligned";
+    case SQ_ERR_OVERFLOW: return "SQ_ERR_OVERFLOW: K-segment too wide for int32 accumulation";
+    case SQ_ERR_CUDA: return "SQ_ERR_CUDA: a CUDA runtime call failed";
+    case SQ_ERR_DEVICE_TIMEOUT: return "SQ_ERR_DEVICE_TIMEOUT: a kernel gave up waiting on a barrier";
+    case SQ_ERR_NO_DEVICE: return "SQ_ERR_NO_DEVICE: no sm_100 device is current";
+  }
+  return "unknown sq_status";
+}
+
+int32_t sq_version(void) { return 100; }
+
+}  // extern "C"

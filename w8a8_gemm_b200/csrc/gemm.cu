@@ -1,0 +1,531 @@
+// gemm.cu -- DualScale + SegLinear W8A8 GEMM for sm_100a.
+//
+// What it computes ("SegQuant", papernotes.org, sections DualScale and
+// SegLinear): for every output element
+//   y[m][n] = sum_i s_w[i][n] * (s+_i * A+_i[m][n] + s-_i * A-_i[m][n]) + bias[n]
+// where A+-_i are the exact int32 products of the X^+ / X^- planes with the
+// shared int8 weight over K-segment i.  The pages run the two products as one
+// batched GEMM with a fused epilogue; here both polarities of a 128-row tile
+// share every weight tile staged in shared memory and accumulate side by side
+// in tensor memory, so the X^- product never reaches HBM.
+//
+// Structure (one persistent CTA per SM, 320 threads):
+//   warp 0      TMA producer: per 128-byte k-block, one 3D box {128 B, 128
+//               rows, 2 planes} of [X^+; X^-] and one box {128 B, BN rows} of
+//               W^, into a STAGES-deep ring guarded by mbarriers;
+//   warp 1      TMEM owner and MMA issuer (one thread): tcgen05.mma kind::i8,
+//               M = 128, N = BN, K = 32, two per k-step (X^+ and X^-);
+//   warps 2-9   epilogue: tcgen05.ld of both accumulators, fp32 reconstruction,
+//               bias, bf16/fp32 stores.  Input-segmented layers drain one
+//               accumulator pair per K-segment into fp32 running sums held in
+//               registers while the MMA warp fills the other TMEM buffer.
+// TMEM holds 512 columns: BN = 256 gives one buffer (+ and - of 256 columns);
+// BN = 128 gives two, so drains overlap the next segment's MMAs.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <mutex>
+
+#include "sm100.cuh"
+#include "sq_internal.h"
+
+namespace sq {
+namespace {
+
+constexpr int BM = 128;              // rows of M per tile (TMEM lanes)
+constexpr int BK = 128;              // int8 K elements per stage = one 128-B swizzle row
+constexpr int MMA_K = 32;            // K of one kind::i8 MMA
+constexpr int NUM_EPI_WARPS = 8;
+constexpr int NUM_THREADS = 64 + 32 * NUM_EPI_WARPS;
+constexpr uint64_t kWaitLimitNs = 2000000000ull;   // 2 s: far above any tile's latency
+
+struct GemmParams {
+  int32_t M, N, K;
+  int32_t num_n_tiles, num_tiles, num_kb;
+  int32_t G, S;
+  int32_t n_seg_out;                // output segments mapped to groups (G > 1)
+  int32_t exact_small_acc;          // every K-segment <= 256 wide: |acc| < 2^22
+  int32_t k_off[SQ_MAX_SEGMENTS + 1];
+  int32_t n_off[SQ_MAX_SEGMENTS + 1];
+  const float *s_w;
+  const float *s_act;
+  const uint16_t *bias;
+  void *y;
+  int64_t ldy;
+  int *status;
+};
+
+template <int BN, int STAGES>
+struct Smem {
+  static constexpr int A_BYTES = 2 * BM * BK;   // X^+ tile, then X^- tile
+  static constexpr int B_BYTES = BN * BK;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int NBUF = 512 / (2 * BN);   // TMEM accumulator buffers
+  static constexpr int BAR_OFFSET = STAGES * STAGE_BYTES;
+  static constexpr int NUM_BARS = 2 * STAGES + 2 * NBUF + 1;
+  static constexpr int BYTES = BAR_OFFSET + NUM_BARS * 8 + 16 + 1024;  // + 1 KB alignment slack
+};
+
+__device__ __forceinline__ int group_of_tile(const GemmParams &p, int nt, int BN) {
+  if (p.G == 1) return 0;
+  return seg_index(p.n_off, p.n_seg_out, static_cast<int64_t>(nt) * BN);
+}
+
+// Bounded wait that also gives up when another role has already aborted.
+__device__ __forceinline__ bool wait_bar(uint64_t *bar, uint32_t parity, volatile int *abort_flag,
+                                         int *status) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  while (true) {
+#pragma unroll 1
+    for (int i = 0; i < 64; ++i)
+      if (mbar_try_wait(bar, parity)) return true;
+    if (*abort_flag) return false;
+    if (globaltimer_ns() - t0 > kWaitLimitNs) {
+      *abort_flag = 1;
+      atomicExch(status, static_cast<int>(SQ_ERR_DEVICE_TIMEOUT));
+      return false;
+    }
+  }
+}
+
+// int32 -> fp32.  When |a| < 2^22 the bit pattern 0x4B400000 + a is the float
+// 1.5 * 2^23 + a exactly, so one integer add and one float subtract give the
+// exact value (the same as round-to-nearest conversion, which is exact there).
+__device__ __forceinline__ float i2f_small(int32_t a) {
+  return __int_as_float(0x4B400000 + a) - 12582912.0f;
+}
+
+__device__ __forceinline__ float bf16_to_f32(uint16_t h) {
+  return __uint_as_float(static_cast<uint32_t>(h) << 16);
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t *>(&v);
+}
+
+template <int OUT>
+__device__ __forceinline__ void store_row_chunk(const GemmParams &p, int64_t m, int64_t n0,
+                                                const float (&v)[32]) {
+  if (OUT == OUT_BF16) {
+    uint16_t *row = reinterpret_cast<uint16_t *>(p.y) + m * p.ldy;
+    if (n0 + 32 <= p.N) {
+      uint4 *dst = reinterpret_cast<uint4 *>(row + n0);
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+        dst[q] = make_uint4(pack_bf16x2(v[8 * q + 0], v[8 * q + 1]),
+                            pack_bf16x2(v[8 * q + 2], v[8 * q + 3]),
+                            pack_bf16x2(v[8 * q + 4], v[8 * q + 5]),
+                            pack_bf16x2(v[8 * q + 6], v[8 * q + 7]));
+    } else {
+#pragma unroll
+      for (int j = 0; j < 32; ++j)
+        if (n0 + j < p.N) {
+          const __nv_bfloat16 b = __float2bfloat16_rn(v[j]);
+          row[n0 + j] = *reinterpret_cast<const uint16_t *>(&b);
+        }
+    }
+  } else {
+    float *row = reinterpret_cast<float *>(p.y) + m * p.ldy;
+    if (n0 + 32 <= p.N) {
+      float4 *dst = reinterpret_cast<float4 *>(row + n0);
+#pragma unroll
+      for (int q = 0; q < 8; ++q)
+        dst[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+    } else {
+#pragma unroll
+      for (int j = 0; j < 32; ++j)
+        if (n0 + j < p.N) row[n0 + j] = v[j];
+    }
+  }
+}
+
+template <int BN, int STAGES, int OUT, bool SEGK>
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+    dualscale_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
+                          const __grid_constant__ CUtensorMap tmB,
+                          const __grid_constant__ GemmParams p) {
+  using L = Smem<BN, STAGES>;
+  constexpr int NBUF = L::NBUF;
+  constexpr int HALF = BN / 2;       // columns per epilogue warp
+  constexpr int CHUNKS = HALF / 32;  // 32-column TMEM loads per warp per unit
+  static_assert(NBUF >= 1, "BN too large for TMEM");
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint64_t *full = reinterpret_cast<uint64_t *>(smem + L::BAR_OFFSET);
+  uint64_t *empty = full + STAGES;
+  uint64_t *acc_full = empty + STAGES;
+  uint64_t *acc_empty = acc_full + NBUF;
+  uint64_t *mma_done = acc_empty + NBUF;
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(mma_done + 1);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < NBUF; ++b) {
+      mbar_init(&acc_full[b], 1);
+      mbar_init(&acc_empty[b], NUM_EPI_WARPS);
+    }
+    mbar_init(mma_done, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+    prefetch_tmap(&tmA);
+    prefetch_tmap(&tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t armed = 0, armed_parity = 0;  // per stage: has a load, its phase
+      for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x) {
+        const int mt = tile / p.num_n_tiles, nt = tile % p.num_n_tiles;
+        const int g = group_of_tile(p, nt, BN);
+        for (int kb = 0; kb < p.num_kb; ++kb) {
+          if (!wait_bar(&empty[stage], phase ^ 1, abort_flag, p.status)) goto producer_done;
+          uint8_t *sa = smem + stage * L::STAGE_BYTES;
+          mbar_arrive_expect_tx(&full[stage], L::STAGE_BYTES);
+          tma_load_3d(sa, &tmA, &full[stage], kb * BK, mt * BM, 2 * g);
+          tma_load_2d(sa + L::A_BYTES, &tmB, &full[stage], kb * BK, nt * BN);
+          armed |= 1u << stage;
+          armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+      }
+    producer_done:
+      // Never leave with a copy in flight into this CTA's shared memory.
+      for (int s = 0; s < STAGES; ++s)
+        if (armed & (1u << s)) mbar_wait(&full[s], (armed_parity >> s) & 1u, kWaitLimitNs);
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_i8(BM, BN);
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t acc_iter = 0;
+      for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x) {
+        int seg = 0;
+        int seg_end = SEGK ? p.k_off[1] : p.K;
+        uint32_t buf = acc_iter % NBUF;
+        if (!wait_bar(&acc_empty[buf], ((acc_iter / NBUF) & 1) ^ 1, abort_flag, p.status))
+          goto mma_exit;
+        tc_fence_after();
+        uint32_t d_plus = tmem_base + buf * 2 * BN;
+        uint32_t accumulate = 0;
+        for (int kb = 0; kb < p.num_kb; ++kb) {
+          if (!wait_bar(&full[stage], phase, abort_flag, p.status)) goto mma_exit;
+          tc_fence_after();
+          const uint32_t sa = smem_u32(smem + stage * L::STAGE_BYTES);
+          const uint32_t sb = sa + L::A_BYTES;
+#pragma unroll
+          for (int kk = 0; kk < BK / MMA_K; ++kk) {
+            const int k = kb * BK + kk * MMA_K;
+            if (k >= p.K) break;
+            if (SEGK && k == seg_end) {
+              // K-segment boundary: hand this accumulator pair to the epilogue
+              // and continue in the next TMEM buffer.
+              mma_commit(&acc_full[buf]);
+              ++acc_iter;
+              buf = acc_iter % NBUF;
+              if (!wait_bar(&acc_empty[buf], ((acc_iter / NBUF) & 1) ^ 1, abort_flag, p.status))
+                goto mma_exit;
+              tc_fence_after();
+              d_plus = tmem_base + buf * 2 * BN;
+              accumulate = 0;
+              ++seg;
+              seg_end = p.k_off[seg + 1];
+            }
+            const uint64_t b_desc = sdesc_kmajor_sw128(sb + kk * MMA_K);
+            mma_i8(d_plus, sdesc_kmajor_sw128(sa + kk * MMA_K), b_desc, idesc, accumulate);
+            mma_i8(d_plus + BN, sdesc_kmajor_sw128(sa + BM * BK + kk * MMA_K), b_desc, idesc,
+                   accumulate);
+            accumulate = 1;
+          }
+          mma_commit(&empty[stage]);  // frees the stage once these MMAs finish
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+        mma_commit(&acc_full[buf]);
+        ++acc_iter;
+      }
+    mma_exit:
+      // Wait for every MMA this thread issued before TMEM can be released.
+      mma_commit(mma_done);
+      mbar_wait(mma_done, 0, kWaitLimitNs);
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int ew = warp - 2;
+    const int quarter = warp & 3;       // TMEM lanes this warp may read
+    const int half = ew >> 2;           // which half of the BN columns
+    const int row = quarter * 32 + lane;
+    const uint32_t lane_addr = static_cast<uint32_t>(quarter * 32) << 16;
+    uint32_t acc_iter = 0;
+    for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x) {
+      const int mt = tile / p.num_n_tiles, nt = tile % p.num_n_tiles;
+      const int g = group_of_tile(p, nt, BN);
+      const int64_t m = static_cast<int64_t>(mt) * BM + row;
+      const int64_t nb = static_cast<int64_t>(nt) * BN + half * HALF;
+      float run[SEGK ? HALF : 1];
+      if (SEGK) {
+#pragma unroll
+        for (int j = 0; j < (SEGK ? HALF : 1); ++j) run[j] = 0.0f;
+      }
+      const int units = SEGK ? p.S : 1;
+      for (int u = 0; u < units; ++u) {
+        const uint32_t buf = acc_iter % NBUF;
+        if (!wait_bar(&acc_full[buf], (acc_iter / NBUF) & 1, abort_flag, p.status))
+          goto epilogue_exit;
+        tc_fence_after();
+        const uint32_t t_plus = tmem_base + lane_addr + buf * 2 * BN + half * HALF;
+        const float sp = p.s_act[(g * p.S + u) * 2 + 0];
+        const float sm = p.s_act[(g * p.S + u) * 2 + 1];
+#pragma unroll
+        for (int c = 0; c < CHUNKS; ++c) {
+          uint32_t ap[32], am[32];
+          tmem_ld_32x32b_x32(t_plus + c * 32, ap);
+          tmem_ld_32x32b_x32(t_plus + BN + c * 32, am);
+          tmem_ld_wait();
+          const int64_t n0 = nb + c * 32;
+          if constexpr (OUT == OUT_S32) {
+            if (m < p.M) {
+              int32_t *accp = reinterpret_cast<int32_t *>(p.y) +
+                              ((static_cast<int64_t>(u) * 2) * p.M + m) * p.N;
+              int32_t *accm = accp + static_cast<int64_t>(p.M) * p.N;
+#pragma unroll
+              for (int j = 0; j < 32; ++j)
+                if (n0 + j < p.N) {
+                  accp[n0 + j] = static_cast<int32_t>(ap[j]);
+                  accm[n0 + j] = static_cast<int32_t>(am[j]);
+                }
+            }
+          } else if constexpr (!SEGK) {
+            // One K-segment: the fp32 operations in the reference order
+            //   t = s+ f(A+) + s- f(A-);  y = s_w t + bias.
+            if (m < p.M) {
+              float v[32];
+#pragma unroll
+              for (int j = 0; j < 32; ++j) {
+                const int64_t n = n0 + j;
+                const bool ok = n < p.N;
+                const float sw = ok ? __ldg(p.s_w + n) : 0.0f;
+                const float tp = __fmul_rn(sp, __int2float_rn(static_cast<int32_t>(ap[j])));
+                const float tm = __fmul_rn(sm, __int2float_rn(static_cast<int32_t>(am[j])));
+                float yv = __fmul_rn(sw, __fadd_rn(tp, tm));
+                if (p.bias != nullptr && ok) yv = __fadd_rn(yv, bf16_to_f32(__ldg(p.bias + n)));
+                v[j] = yv;
+              }
+              store_row_chunk<OUT>(p, m, n0, v);
+            }
+          } else {
+            // Several K-segments: y += (s_w s+) f(A+) + (s_w s-) f(A-).
+            const float *swu = p.s_w + static_cast<int64_t>(u) * p.N;
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              const int64_t n = n0 + j;
+              const float sw = (n < p.N) ? __ldg(swu + n) : 0.0f;
+              const int32_t a1 = static_cast<int32_t>(ap[j]), a2 = static_cast<int32_t>(am[j]);
+              const float f1 = p.exact_small_acc ? i2f_small(a1) : __int2float_rn(a1);
+              const float f2 = p.exact_small_acc ? i2f_small(a2) : __int2float_rn(a2);
+              run[c * 32 + j] = fmaf(sw * sp, f1, run[c * 32 + j]);
+              run[c * 32 + j] = fmaf(sw * sm, f2, run[c * 32 + j]);
+            }
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&acc_empty[buf]);
+        ++acc_iter;
+      }
+      if constexpr (SEGK && OUT != OUT_S32) {
+        if (m < p.M) {
+#pragma unroll
+        for (int c = 0; c < CHUNKS; ++c) {
+          const int64_t n0 = nb + c * 32;
+          float v[32];
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            const int64_t n = n0 + j;
+            float yv = run[c * 32 + j];
+            if (p.bias != nullptr && n < p.N) yv = __fadd_rn(yv, bf16_to_f32(__ldg(p.bias + n)));
+            v[j] = yv;
+          }
+          store_row_chunk<OUT>(p, m, n0, v);
+        }
+        }
+      }
+    }
+  epilogue_exit:;
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem_base, 512);
+  }
+}
+
+// ------------------------------------------------------------------ host side
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                  const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                  const cuuint32_t *, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion,
+                                  CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void *ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  });
+  return fn;
+}
+
+int device_sm_count() {
+  int dev = 0, sms = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  return sms > 0 ? sms : 148;
+}
+
+template <int BN, int STAGES, int OUT, bool SEGK>
+sq_status run_gemm(const GemmRequest &r, const GemmParams &p, cudaStream_t stream) {
+  using L = Smem<BN, STAGES>;
+  EncodeTiledFn enc = encode_fn();
+  if (enc == nullptr) return SQ_ERR_CUDA;
+  const int G = r.seg.G;
+  CUtensorMap tmA, tmB;
+  {
+    // planes viewed as 3D: x = K (bytes), y = M rows, z = 2G planes.
+    const cuuint64_t dims[3] = {static_cast<cuuint64_t>(r.K), static_cast<cuuint64_t>(r.M),
+                                static_cast<cuuint64_t>(2 * G)};
+    const cuuint64_t strides[2] = {static_cast<cuuint64_t>(r.K),
+                                   static_cast<cuuint64_t>(r.K) * static_cast<cuuint64_t>(r.M)};
+    const cuuint32_t box[3] = {BK, BM, 2};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    if (enc(&tmA, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<int8_t *>(r.planes), dims, strides,
+            box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return SQ_ERR_CUDA;
+  }
+  {
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(r.K), static_cast<cuuint64_t>(r.N)};
+    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(r.K)};
+    const cuuint32_t box[2] = {BK, BN};
+    const cuuint32_t estr[2] = {1, 1};
+    if (enc(&tmB, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<int8_t *>(r.wq), dims, strides,
+            box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return SQ_ERR_CUDA;
+  }
+  auto kernel = dualscale_gemm_kernel<BN, STAGES, OUT, SEGK>;
+  static bool attr_set[64] = {};  // per instantiation and device
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64) return SQ_ERR_CUDA;
+  if (!attr_set[dev]) {
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, L::BYTES) !=
+        cudaSuccess)
+      return SQ_ERR_CUDA;
+    attr_set[dev] = true;
+  }
+  const int grid = p.num_tiles < device_sm_count() ? p.num_tiles : device_sm_count();
+  kernel<<<grid, NUM_THREADS, L::BYTES, stream>>>(tmA, tmB, p);
+  return cudaGetLastError() == cudaSuccess ? SQ_OK : SQ_ERR_CUDA;
+}
+
+}  // namespace
+
+sq_status launch_gemm(const GemmRequest &r, cudaStream_t stream) {
+  if (r.M == 0) return SQ_OK;
+  const bool segk = r.seg.mode == SQ_SEG_INPUT && r.seg.S > 1;
+  int BN = segk ? 128 : 256;
+  if (r.seg.G > 1) {
+    for (int j = 0; j < r.seg.n_seg; ++j)
+      if ((r.seg.off[j + 1] - r.seg.off[j]) % 256 != 0) BN = 128;
+  }
+  GemmParams p;
+  p.M = static_cast<int32_t>(r.M);
+  p.N = static_cast<int32_t>(r.N);
+  p.K = static_cast<int32_t>(r.K);
+  p.num_n_tiles = static_cast<int32_t>((r.N + BN - 1) / BN);
+  const int32_t num_m_tiles = static_cast<int32_t>((r.M + BM - 1) / BM);
+  p.num_tiles = num_m_tiles * p.num_n_tiles;
+  p.num_kb = static_cast<int32_t>((r.K + BK - 1) / BK);
+  p.G = r.seg.G;
+  p.S = r.seg.S;
+  p.n_seg_out = (r.seg.mode == SQ_SEG_OUTPUT) ? r.seg.n_seg : 1;
+  p.exact_small_acc = 1;
+  for (int i = 0; i <= SQ_MAX_SEGMENTS; ++i) {
+    p.k_off[i] = 0;
+    p.n_off[i] = 0;
+  }
+  if (r.seg.mode == SQ_SEG_INPUT) {
+    for (int i = 0; i <= r.seg.n_seg; ++i) p.k_off[i] = r.seg.off[i];
+    for (int i = 0; i < r.seg.n_seg; ++i)
+      if (r.seg.off[i + 1] - r.seg.off[i] > 256) p.exact_small_acc = 0;
+  } else {
+    p.k_off[0] = 0;
+    p.k_off[1] = p.K;
+    p.exact_small_acc = p.K <= 256;
+  }
+  if (r.seg.mode == SQ_SEG_OUTPUT)
+    for (int i = 0; i <= r.seg.n_seg; ++i) p.n_off[i] = r.seg.off[i];
+  p.s_w = r.s_w;
+  p.s_act = r.s_act;
+  p.bias = r.bias;
+  p.y = r.y;
+  p.ldy = r.ldy;
+  p.status = r.status;
+
+  if (r.out_kind == OUT_S32) {
+    if (segk) return run_gemm<128, 4, OUT_S32, true>(r, p, stream);
+    return BN == 256 ? run_gemm<256, 3, OUT_S32, false>(r, p, stream)
+                     : run_gemm<128, 4, OUT_S32, false>(r, p, stream);
+  }
+  if (r.out_kind == OUT_F32) {
+    if (segk) return run_gemm<128, 4, OUT_F32, true>(r, p, stream);
+    return BN == 256 ? run_gemm<256, 3, OUT_F32, false>(r, p, stream)
+                     : run_gemm<128, 4, OUT_F32, false>(r, p, stream);
+  }
+  if (segk) return run_gemm<128, 4, OUT_BF16, true>(r, p, stream);
+  return BN == 256 ? run_gemm<256, 3, OUT_BF16, false>(r, p, stream)
+                   : run_gemm<128, 4, OUT_BF16, false>(r, p, stream);
+}
+
+}  // namespace sq

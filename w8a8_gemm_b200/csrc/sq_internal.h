@@ -1,0 +1,60 @@
+// sq_internal.h -- declarations shared by the library's own translation units
+// (kernels and the C-ABI layer).  Not installed; not used by anything else.
+#pragma once
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/segquant.h"
+
+namespace sq {
+
+// Segment table as the kernels see it (passed by value as a kernel argument).
+struct SegParams {
+  int32_t mode;   // sq_seg_mode
+  int32_t n_seg;  // segments
+  int32_t G;      // activation groups
+  int32_t S;      // K-segments (n_seg in input mode, else 1)
+  int32_t off[SQ_MAX_SEGMENTS + 1];
+};
+
+// Index i with off[i] <= p < off[i + 1] (tables are short: a linear scan).
+__host__ __device__ inline int seg_index(const int32_t *off, int n_seg, int64_t p) {
+  int i = 0;
+  while (i + 1 < n_seg && p >= off[i + 1]) ++i;
+  return i;
+}
+
+// ---- launchers (quant.cu) --------------------------------------------------
+cudaError_t launch_calibrate_act(const uint16_t *x, int64_t M, int64_t K, int64_t ldx,
+                                 const float *d, const SegParams &seg, float *s_act,
+                                 cudaStream_t stream);
+cudaError_t launch_quantize_act(const uint16_t *x, int64_t M, int64_t K, int64_t ldx,
+                                const float *d, const float *s_act, const SegParams &seg,
+                                int8_t *planes, cudaStream_t stream);
+cudaError_t launch_quantize_weight(const uint16_t *w, int64_t N, int64_t K, const float *d,
+                                   const SegParams &seg, int8_t *wq, float *s_w,
+                                   cudaStream_t stream);
+
+// ---- launcher (gemm.cu) ----------------------------------------------------
+enum OutKind { OUT_BF16 = 0, OUT_F32 = 1, OUT_S32 = 2 };
+
+struct GemmRequest {
+  const int8_t *planes;
+  const int8_t *wq;
+  const float *s_w;
+  const float *s_act;
+  const uint16_t *bias;
+  void *y;
+  int64_t ldy;
+  int out_kind;
+  int64_t M, N, K;
+  SegParams seg;
+  int *status;  // device error word
+};
+
+sq_status launch_gemm(const GemmRequest &req, cudaStream_t stream);
+
+// Device address of the library's error word on the current device.
+int *device_status_word();
+
+}  // namespace sq

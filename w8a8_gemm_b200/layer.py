@@ -1,0 +1,60 @@
+"""Layer-level use of the library: one DualScale + SegLinear quantized linear.
+
+Offline (once): quantize the weight segment-wise and calibrate s+ / s- on a
+calibration slice -- both on the GPU through the C ABI.  Online (per call):
+quantize the activation into the stacked planes, then run the fused GEMM.
+"""
+from __future__ import annotations
+
+from typing import Optional
+
+import torch
+
+from . import binding as B
+
+
+class DualScaleSegLinear:
+    """W8A8 DualScale linear with SegLinear segments.
+
+    w      bf16 [N][K] nn.Linear weight (CUDA)
+    bias   bf16 [N] or None
+    d      fp32 [G][K] SmoothQuant divisor or None
+    seg    binding.Segments
+    x_cal  bf16 [rows][K] calibration activations
+    """
+
+    def __init__(self, w: torch.Tensor, bias: Optional[torch.Tensor], d: Optional[torch.Tensor],
+                 seg: B.Segments, x_cal: torch.Tensor, out_dtype=torch.bfloat16):
+        self.N, self.K = w.shape
+        self.seg = seg
+        self.G, self.S = seg.n_groups, seg.S
+        self.d = d
+        self.bias = bias
+        self.out_dtype = out_dtype
+        dev = w.device
+        self.wq = torch.empty(self.N, self.K, dtype=torch.int8, device=dev)
+        self.s_w = torch.empty(self.S, self.N, dtype=torch.float32, device=dev)
+        B.sq_quantize_weight_seg(w, d, seg, self.wq, self.s_w)
+        self.s_act = torch.empty(self.G, self.S, 2, dtype=torch.float32, device=dev)
+        B.sq_calibrate_act(x_cal, d, seg, self.s_act)
+        self._planes = None
+
+    def planes_for(self, M: int, device) -> torch.Tensor:
+        if self._planes is None or self._planes.shape[2] != M:
+            self._planes = torch.empty(self.G, 2, M, self.K, dtype=torch.int8, device=device)
+        return self._planes
+
+    def quantize(self, x: torch.Tensor, planes: Optional[torch.Tensor] = None) -> torch.Tensor:
+        if planes is None:
+            planes = self.planes_for(x.shape[0], x.device)
+        return B.sq_quantize_act(x, self.d, self.s_act, self.seg, planes)
+
+    def gemm(self, planes: torch.Tensor, y: Optional[torch.Tensor] = None) -> torch.Tensor:
+        M = planes.shape[2]
+        if y is None:
+            y = torch.empty(M, self.N, dtype=self.out_dtype, device=planes.device)
+        return B.sq_dualscale_seglinear_gemm(planes, self.wq, self.s_w, self.s_act, self.bias,
+                                             y, self.seg)
+
+    def __call__(self, x: torch.Tensor, y: Optional[torch.Tensor] = None) -> torch.Tensor:
+        return self.gemm(self.quantize(x), y)
