@@ -1,0 +1,473 @@
+#!/usr/bin/env python
+"""Benchmark of the SegQuant DualScale + SegLinear W8A8 linear path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME] [--impl ours|reference]
+
+One step = one pass of the whole hot path over one batch: for every layer of
+the configuration, the DualScale activation quantization (bf16 X -> stacked
+int8 planes) and the fused DualScale/SegLinear GEMM (planes x int8 W -> bf16 Y),
+inputs already resident in HBM.  The default workload is the SD3.5-medium FFN
+pair (fc1 [8858x1536]x[1536x6144], fc2 [8858x6144]x[6144x1536]), the shape the
+throughput target is set on.
+
+Metric: effective TOPS = sum over layers of 2*M*N*K / step time.  Also reported:
+executed TOPS (the doubled 2M rows of X^+ and X^-), their fraction of the B200's
+dense INT8 peak, and the activation-quantize kernel's GB/s against HBM.
+
+Timing: CUDA events on the launching stream around every kernel, L2 flushed
+(512 MiB write) between steps outside the timed events, W warm-up steps, then K
+timed steps; across N GPUs (one process each, replicas of the same workload,
+no collective on the data path) the step time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from w8a8_gemm_b200 import workloads as wl  # noqa: E402
+
+DEFAULT_CONFIG = "c4_sd35_ffn"
+METRIC = "DualScale-SegLinear W8A8 GEMM effective TOPS & % of B200 INT8 peak; quant GB/s"
+# Peaks measured on this machine (copy bandwidth and cuBLAS bf16); used when the
+# generated MEASURED_PEAKS.json is absent.
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+INT8_OVER_BF16 = 4.5 / 2.25   # dense INT8 / dense bf16, nominal B200 ratio
+FLUSH_BYTES = 512 << 20
+SMI_FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+
+# ----------------------------------------------------------------- helpers
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            pk = json.load(f)
+        return pk, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def layer_units(L):
+    eff = 2.0 * L.M * L.N * L.K
+    quant_bytes = 2.0 * L.M * L.K + 2.0 * L.G * L.M * L.K
+    return eff, 2.0 * eff, quant_bytes
+
+
+def dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+def aggregate_over_ranks(local_value: float, op: str = "max", device=None) -> float:
+    """Reduce one float over the process group (max for times)."""
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return local_value
+    t = torch.tensor([local_value], dtype=torch.float64, device=device or "cpu")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX if op == "max" else dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons during a region."""
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        fd, self.path = tempfile.mkstemp(prefix="sq_clocks_", suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={SMI_FIELDS}", "--format=csv",
+                 "-lms", "100", "-f", self.path], stdout=subprocess.DEVNULL,
+                stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            time.sleep(0.2)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        out = {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        if not self.path or not os.path.exists(self.path):
+            return out
+        rows = []
+        with open(self.path) as f:
+            for ln in f:
+                parts = [p.strip() for p in ln.split(",")]
+                if len(parts) < 9 or not parts[1].split()[0].isdigit():
+                    continue
+                rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return out
+        sm = [int(r[1].split()[0]) for r in rows]
+        mx = [int(r[2].split()[0]) for r in rows]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = set()
+        for r in rows:
+            for nm, v in zip(names, r[5:9]):
+                if v.lower() == "active":
+                    reasons.add(nm)
+        loaded = [s for s in sm if s > 0.5 * max(mx)] or sm
+        out.update(sm_mhz=int(statistics.median(loaded)), sm_max_mhz=max(mx),
+                   reasons=sorted(reasons), samples=len(rows),
+                   power_w_max=max(float(r[3].split()[0]) for r in rows if r[3][0].isdigit())
+                   if any(r[3][0].isdigit() for r in rows) else None)
+        return out
+
+
+def traffic_from_profile():
+    """Per-launch DRAM bytes of the GEMM from the committed ncu summary, valid
+    only while the kernel source is the one that was profiled."""
+    import hashlib
+    prof = os.path.join(ROOT, "profiles", "gemm_c4_sd35_ffn_traffic.txt")
+    src = os.path.join(ROOT, "w8a8_gemm_b200", "csrc", "gemm.cu")
+    if not (os.path.exists(prof) and os.path.exists(src)):
+        return None, None
+    h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+    vals = {}
+    for ln in open(prof):
+        if ":" in ln and not ln.startswith("#"):
+            k, v = ln.split(":", 1)
+            vals[k.strip()] = v.strip()
+    if vals.get("gemm_cu_sha256_16") != h:
+        return None, "kernel changed since the counters were taken"
+    try:
+        return float(vals["dram_bytes_per_launch"]), vals.get("note")
+    except (KeyError, ValueError):
+        return None, None
+
+
+# ------------------------------------------------------------- our path
+class GpuLayer:
+    def __init__(self, L, dev):
+        from w8a8_gemm_b200 import binding as B
+        from w8a8_gemm_b200.layer import DualScaleSegLinear
+        self.L = L
+        seg = (B.Segments() if L.mode == wl.MODE_NONE
+               else B.Segments(L.mode, list(L.offsets), L.G))
+        d = None if L.d is None else L.d.to(dev)
+        bias = None if L.bias is None else L.bias.to(dev)
+        self.lin = DualScaleSegLinear(L.w.to(dev), bias, d, seg, L.x_cal.to(dev))
+        self.x = L.x.to(dev)
+        self.planes = torch.empty(L.G, 2, L.M, L.K, dtype=torch.int8, device=dev)
+        self.y = torch.empty(L.M, L.N, dtype=torch.bfloat16, device=dev)
+
+    def quantize(self):
+        self.lin.quantize(self.x, self.planes)
+
+    def gemm(self):
+        self.lin.gemm(self.planes, self.y)
+
+
+def run_ours(args, ws, rank, local):
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    from w8a8_gemm_b200 import binding as B
+    B.lib()  # fail loudly now if the library is missing
+    layers_cpu = wl.config_layers(args.config, seed=0)
+    glayers = [GpuLayer(L, dev) for L in layers_cpu]
+    torch.cuda.synchronize()
+    eff_ops = sum(layer_units(g.L)[0] for g in glayers)
+    exe_ops = sum(layer_units(g.L)[1] for g in glayers)
+    qbytes = sum(layer_units(g.L)[2] for g in glayers)
+    flush = torch.empty(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream()
+    nl = len(glayers)
+
+    def one_step(ev):
+        ev[0].record(stream)
+        for i, g in enumerate(glayers):
+            g.quantize()
+            ev[2 * i + 1].record(stream)
+            g.gemm()
+            ev[2 * i + 2].record(stream)
+
+    mk = lambda: [torch.cuda.Event(enable_timing=True) for _ in range(2 * nl + 1)]
+    for _ in range(args.warmup):
+        flush.zero_()
+        one_step(mk())
+    torch.cuda.synchronize()
+    if ws > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    torch.cuda.synchronize()
+    events = [mk() for _ in range(args.steps)]
+    with ClockSampler(local) as clocks:
+        t_wall = time.perf_counter()
+        for k in range(args.steps):
+            flush.zero_()
+            one_step(events[k])
+        torch.cuda.synchronize()
+        t_wall = time.perf_counter() - t_wall
+    if ws > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    torch.cuda.synchronize()
+    step_ms, q_ms, g_ms = [], [0.0] * nl, [0.0] * nl
+    for ev in events:
+        step_ms.append(ev[0].elapsed_time(ev[-1]))
+        for i in range(nl):
+            q_ms[i] += (ev[0] if i == 0 else ev[2 * i]).elapsed_time(ev[2 * i + 1])
+            g_ms[i] += ev[2 * i + 1].elapsed_time(ev[2 * i + 2])
+    total_ms = sum(step_ms)
+    total_ms = aggregate_over_ranks(total_ms, "max", device=dev)
+    ms_step = total_ms / args.steps
+    gemm_ms = sum(g_ms) / args.steps
+    quant_ms = sum(q_ms) / args.steps
+    res = dict(eff_ops=eff_ops, exe_ops=exe_ops, qbytes=qbytes, ms_step=ms_step,
+               gemm_ms=gemm_ms, quant_ms=quant_ms, wall_s=t_wall, clocks=clocks.summary(),
+               per_layer=[dict(name=g.L.name, M=g.L.M, N=g.L.N, K=g.L.K, G=g.L.G, S=g.L.S,
+                               quant_us=1e3 * q_ms[i] / args.steps,
+                               gemm_us=1e3 * g_ms[i] / args.steps)
+                          for i, g in enumerate(glayers)],
+               launches=2 * nl * args.steps)
+
+    # end to end through the library with host buffers: H2D of the step's
+    # activations from pinned memory, the kernels, D2H of the outputs.
+    hx = [g.x.cpu().pin_memory() for g in glayers]
+    hy = [torch.empty(g.L.M, g.L.N, dtype=torch.bfloat16).pin_memory() for g in glayers]
+    e2e_steps = max(3, min(args.steps, args.e2e_steps))
+    for _ in range(2):
+        for i, g in enumerate(glayers):
+            g.x.copy_(hx[i], non_blocking=True)
+            g.quantize()
+            g.gemm()
+            hy[i].copy_(g.y, non_blocking=True)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        for i, g in enumerate(glayers):
+            g.x.copy_(hx[i], non_blocking=True)
+            g.quantize()
+            g.gemm()
+            hy[i].copy_(g.y, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = aggregate_over_ranks(e0.elapsed_time(e1), "max", device=dev) / e2e_steps
+    res["e2e_ms"] = e2e_ms
+    res["h2d"] = sum(t.numel() * t.element_size() for t in hx)
+    res["d2h"] = sum(t.numel() * t.element_size() for t in hy)
+    return res, layers_cpu
+
+
+# --------------------------------------------------------- oracle (CPU) leg
+def prepare_oracle(layers):
+    """Oracle calibration and weight quantization (offline work, untimed)."""
+    import oracle
+    prepared = []
+    for L in layers:
+        off = None if L.mode == wl.MODE_NONE else list(L.offsets)
+        d = None if L.d is None else L.d.numpy()
+        s_act = oracle.calibrate_act(wl.bits(L.x_cal), d, L.mode, off, L.G, L.N)
+        wq, s_w = oracle.quantize_weight(wl.bits(L.w), d, L.mode, off, L.G)
+        bias = None if L.bias is None else wl.bits(L.bias)
+        prepared.append((L, off, d, s_act, wq, s_w, bias))
+    return prepared
+
+
+def oracle_rows(prepared, rows: int, threads: int):
+    """One pass of the oracle's per-batch work (activation quantization and the
+    DualScale GEMM) over the first `rows` rows of every layer; returns
+    (seconds, effective ops)."""
+    import oracle
+    t0 = time.perf_counter()
+    ops = 0.0
+    for L, off, d, s_act, wq, s_w, bias in prepared:
+        planes = oracle.quantize_act(wl.bits(L.x[:rows]), s_act, d, L.mode, off, L.G, L.N)
+        oracle.gemm(planes, wq, s_w, s_act, bias, L.mode, off, threads=threads)
+        ops += 2.0 * rows * L.N * L.K
+    return time.perf_counter() - t0, ops
+
+
+def oracle_sample(layers, target_s: float, threads: int, prepared=None):
+    """Times the CPU oracle on a row sample of every layer, sized so that the
+    timed work takes about target_s seconds."""
+    prepared = prepared or prepare_oracle(layers)
+    max_rows = min(L.M for L in layers)
+    rows = 4
+    while True:
+        dt, ops = oracle_rows(prepared, rows, threads)
+        if dt >= 0.5 * target_s or rows >= max_rows:
+            return dict(rows=rows, seconds=dt, eff_ops=ops, tops=ops / dt / 1e12)
+        rows = min(max_rows, max(rows * 2, int(rows * target_s / max(dt, 1e-3))))
+
+
+# ---------------------------------------------------------------------- main
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--config", default=DEFAULT_CONFIG, choices=sorted(wl.CONFIGS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--e2e-steps", type=int, default=40)
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    ws, rank, local = dist_env()
+    n_gpus = max(args.gpus, ws)
+
+    if args.impl == "reference":
+        return main_reference(args, ws, rank)
+
+    pg = False
+    if ws > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+        pg = True
+    try:
+        res, layers = run_ours(args, ws, rank, local)
+    finally:
+        if pg:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+    if rank != 0:
+        return 0
+
+    peaks, peak_src = load_peaks()
+    int8_peak_burst = peaks["bf16_tflops"] * INT8_OVER_BF16
+    int8_peak_sust = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]) * INT8_OVER_BF16
+    hbm = peaks["hbm_gbs"]
+    ms = res["ms_step"]
+    eff_tops = n_gpus * res["eff_ops"] / (ms * 1e-3) / 1e12
+    exe_tops_step = res["exe_ops"] / (ms * 1e-3) / 1e12
+    gemm_tops = res["exe_ops"] / (res["gemm_ms"] * 1e-3) / 1e12
+    quant_gbs = res["qbytes"] / (res["quant_ms"] * 1e-3) / 1e9
+    traffic, traffic_note = traffic_from_profile()
+    cpu = None
+    if n_gpus == 1 and not args.no_cpu_baseline:
+        import oracle
+        thr = oracle.num_threads()
+        s = oracle_sample(layers, args.cpu_seconds, thr)
+        cpu = {"value": s["tops"], "unit": "TOPS", "cores": thr, "kind": "oracle",
+               "sample": f"first {s['rows']} rows of every layer of {args.config} "
+                         f"(quantize + GEMM, calibration and weights prepared untimed), "
+                         f"{s['seconds']:.1f} s"}
+    e2e_tops = n_gpus * res["eff_ops"] / (res["e2e_ms"] * 1e-3) / 1e12
+    out = {
+        "metric": METRIC,
+        "value": round(eff_tops, 2),
+        "unit": "TOPS",
+        "n_gpus": n_gpus,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms, 5),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "s8",
+        "data": "synthetic (seeded SD3.5/FLUX-shaped activations and weights)",
+        "config": {"workload": f"{args.config}: {wl.CONFIGS[args.config]}",
+                   "layers": [{k: v for k, v in p.items() if k in ("name", "M", "N", "K", "G", "S")}
+                              for p in res["per_layer"]],
+                   "output": "bf16", "l2": "flushed between steps (512 MiB write, untimed)",
+                   "parallelism": f"replicas x{n_gpus}"},
+        "executed_tops": round(n_gpus * exe_tops_step, 2),
+        "executed_frac_int8_peak": round(exe_tops_step / int8_peak_burst, 4),
+        "gemm_executed_tops": round(gemm_tops, 2),
+        "quant_gbs": round(quant_gbs, 1),
+        "quant_frac_hbm": round(quant_gbs / hbm, 4),
+        "per_layer_us": [{"name": p["name"], "quant": round(p["quant_us"], 2),
+                          "gemm": round(p["gemm_us"], 2)} for p in res["per_layer"]],
+        "roofline": {"bound": "tensor", "achieved": round(gemm_tops, 2),
+                     "peak": round(int8_peak_burst, 1), "unit": "TOPS",
+                     "frac": round(gemm_tops / int8_peak_burst, 4),
+                     "traffic": traffic,
+                     "kernel": "dualscale_gemm_kernel (tcgen05 kind::i8)",
+                     "peak_source": f"{peak_src}: bf16 burst {peaks['bf16_tflops']} TF/s x 2 "
+                                    f"(nominal INT8/bf16 ratio); sustained-based INT8 peak "
+                                    f"{round(int8_peak_sust, 1)}",
+                     "traffic_note": traffic_note},
+        "quant_roofline": {"bound": "hbm", "achieved": round(quant_gbs, 1), "peak": hbm,
+                           "unit": "GB/s", "frac": round(quant_gbs / hbm, 4)},
+        "cpu_baseline": cpu,
+        "e2e": {"value": round(e2e_tops, 3), "unit": "TOPS",
+                "h2d_bytes_per_step": res["h2d"], "d2h_bytes_per_step": res["d2h"],
+                "ms_per_step": round(res["e2e_ms"], 4)},
+        "gpu_launches": res["launches"],
+        "clocks": res["clocks"],
+        "wall_s_timed_region": round(res["wall_s"], 3),
+    }
+    print(json.dumps(out))
+    return 0
+
+
+def main_reference(args, ws, rank):
+    """Reference arm: the CPU oracle as it stands, on this machine's host cores, on
+    a bounded row sample of the same workload per step."""
+    if rank != 0:
+        return 0
+    import oracle
+    layers = wl.config_layers(args.config, seed=0)
+    thr = oracle.num_threads()
+    prepared = prepare_oracle(layers)
+    total_budget_s = 120.0
+    probe = oracle_sample(layers, 1.0, thr, prepared)
+    per_row_s = probe["seconds"] / probe["rows"]
+    rows = max(1, int(total_budget_s / (args.steps + args.warmup) / per_row_s))
+    rows = min(rows, min(L.M for L in layers))
+
+    def step():
+        oracle_rows(prepared, rows, thr)
+
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    dt = time.perf_counter() - t0
+    ops = sum(2.0 * rows * L.N * L.K for L in layers)
+    tops = ops * args.steps / dt / 1e12
+    out = {"metric": METRIC, "value": round(tops, 6), "unit": "TOPS", "impl": "reference",
+           "n_gpus": max(args.gpus, ws), "steps": args.steps, "warmup": args.warmup,
+           "ms_per_step": round(1e3 * dt / args.steps, 3), "higher_is_better": True,
+           "scaling": "weak", "vs_baseline": None, "dtype": "s8",
+           "data": "synthetic (seeded SD3.5/FLUX-shaped activations and weights)",
+           "config": {"workload": f"{args.config}: {wl.CONFIGS[args.config]}",
+                      "sample_rows_per_layer": rows},
+           "cpu_baseline": {"value": round(tops, 6), "unit": "TOPS", "cores": thr,
+                            "kind": "oracle",
+                            "sample": f"first {rows} rows of every layer per step"},
+           "e2e": {"value": round(tops, 6), "unit": "TOPS", "h2d_bytes_per_step": 0,
+                   "d2h_bytes_per_step": 0}}
+    print(json.dumps(out))
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

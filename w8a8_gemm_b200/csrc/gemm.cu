@@ -63,7 +63,9 @@ struct Smem {
   static constexpr int B_BYTES = BN * BK;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr int NBUF = 512 / (2 * BN);   // TMEM accumulator buffers
-  static constexpr int BAR_OFFSET = STAGES * STAGE_BYTES;
+  static constexpr int EPI_OFFSET = STAGES * STAGE_BYTES;  // per-warp column constants
+  static constexpr int EPI_BYTES = NUM_EPI_WARPS * 2 * (BN / 2) * 4;
+  static constexpr int BAR_OFFSET = EPI_OFFSET + EPI_BYTES;
   static constexpr int NUM_BARS = 2 * STAGES + 2 * NBUF + 1;
   static constexpr int BYTES = BAR_OFFSET + NUM_BARS * 8 + 16 + 1024;  // + 1 KB alignment slack
 };
@@ -286,26 +288,51 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const int half = ew >> 2;           // which half of the BN columns
     const int row = quarter * 32 + lane;
     const uint32_t lane_addr = static_cast<uint32_t>(quarter * 32) << 16;
+    // Warp-private column constants in shared memory, read back as broadcast
+    // float4s: [0, HALF) and [HALF, 2*HALF).
+    float *cst = reinterpret_cast<float *>(smem + L::EPI_OFFSET) + ew * 2 * HALF;
     uint32_t acc_iter = 0;
     for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x) {
       const int mt = tile / p.num_n_tiles, nt = tile % p.num_n_tiles;
       const int g = group_of_tile(p, nt, BN);
       const int64_t m = static_cast<int64_t>(mt) * BM + row;
       const int64_t nb = static_cast<int64_t>(nt) * BN + half * HALF;
+      if constexpr (!SEGK && OUT != OUT_S32) {
+        // s_w and bias of this warp's columns, staged while the MMAs run.
+        __syncwarp();
+        for (int j = lane; j < HALF; j += 32) {
+          const int64_t n = nb + j;
+          cst[j] = n < p.N ? p.s_w[n] : 0.0f;
+          cst[HALF + j] = (p.bias != nullptr && n < p.N) ? bf16_to_f32(p.bias[n]) : 0.0f;
+        }
+        __syncwarp();
+      }
       float run[SEGK ? HALF : 1];
-      if (SEGK) {
+      if constexpr (SEGK) {
 #pragma unroll
         for (int j = 0; j < (SEGK ? HALF : 1); ++j) run[j] = 0.0f;
       }
       const int units = SEGK ? p.S : 1;
       for (int u = 0; u < units; ++u) {
+        const float sp = p.s_act[(g * p.S + u) * 2 + 0];
+        const float sm = p.s_act[(g * p.S + u) * 2 + 1];
+        if constexpr (SEGK && OUT != OUT_S32) {
+          // Folded coefficients of this K-segment: c+- = s_w[u][n] * s+-[u].
+          __syncwarp();
+          const float *swu = p.s_w + static_cast<int64_t>(u) * p.N;
+          for (int j = lane; j < HALF; j += 32) {
+            const int64_t n = nb + j;
+            const float sw = n < p.N ? swu[n] : 0.0f;
+            cst[j] = sw * sp;
+            cst[HALF + j] = sw * sm;
+          }
+          __syncwarp();
+        }
         const uint32_t buf = acc_iter % NBUF;
         if (!wait_bar(&acc_full[buf], (acc_iter / NBUF) & 1, abort_flag, p.status))
           goto epilogue_exit;
         tc_fence_after();
         const uint32_t t_plus = tmem_base + lane_addr + buf * 2 * BN + half * HALF;
-        const float sp = p.s_act[(g * p.S + u) * 2 + 0];
-        const float sm = p.s_act[(g * p.S + u) * 2 + 1];
 #pragma unroll
         for (int c = 0; c < CHUNKS; ++c) {
           uint32_t ap[32], am[32];
@@ -329,32 +356,40 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             // One K-segment: the fp32 operations in the reference order
             //   t = s+ f(A+) + s- f(A-);  y = s_w t + bias.
             if (m < p.M) {
+              const float4 *sw4 = reinterpret_cast<const float4 *>(cst + c * 32);
+              const float4 *b4 = reinterpret_cast<const float4 *>(cst + HALF + c * 32);
               float v[32];
 #pragma unroll
-              for (int j = 0; j < 32; ++j) {
-                const int64_t n = n0 + j;
-                const bool ok = n < p.N;
-                const float sw = ok ? __ldg(p.s_w + n) : 0.0f;
-                const float tp = __fmul_rn(sp, __int2float_rn(static_cast<int32_t>(ap[j])));
-                const float tm = __fmul_rn(sm, __int2float_rn(static_cast<int32_t>(am[j])));
-                float yv = __fmul_rn(sw, __fadd_rn(tp, tm));
-                if (p.bias != nullptr && ok) yv = __fadd_rn(yv, bf16_to_f32(__ldg(p.bias + n)));
-                v[j] = yv;
+              for (int q = 0; q < 8; ++q) {
+                const float4 w = sw4[q], b = b4[q];
+                const float wv[4] = {w.x, w.y, w.z, w.w}, bv[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                  const int j = 4 * q + e;
+                  const float tp = __fmul_rn(sp, __int2float_rn(static_cast<int32_t>(ap[j])));
+                  const float tm = __fmul_rn(sm, __int2float_rn(static_cast<int32_t>(am[j])));
+                  v[j] = __fadd_rn(__fmul_rn(wv[e], __fadd_rn(tp, tm)), bv[e]);
+                }
               }
               store_row_chunk<OUT>(p, m, n0, v);
             }
           } else {
-            // Several K-segments: y += (s_w s+) f(A+) + (s_w s-) f(A-).
-            const float *swu = p.s_w + static_cast<int64_t>(u) * p.N;
+            // Several K-segments: y += c+ f(A+) + c- f(A-).
+            const float4 *cp4 = reinterpret_cast<const float4 *>(cst + c * 32);
+            const float4 *cm4 = reinterpret_cast<const float4 *>(cst + HALF + c * 32);
 #pragma unroll
-            for (int j = 0; j < 32; ++j) {
-              const int64_t n = n0 + j;
-              const float sw = (n < p.N) ? __ldg(swu + n) : 0.0f;
-              const int32_t a1 = static_cast<int32_t>(ap[j]), a2 = static_cast<int32_t>(am[j]);
-              const float f1 = p.exact_small_acc ? i2f_small(a1) : __int2float_rn(a1);
-              const float f2 = p.exact_small_acc ? i2f_small(a2) : __int2float_rn(a2);
-              run[c * 32 + j] = fmaf(sw * sp, f1, run[c * 32 + j]);
-              run[c * 32 + j] = fmaf(sw * sm, f2, run[c * 32 + j]);
+            for (int q = 0; q < 8; ++q) {
+              const float4 a = cp4[q], b = cm4[q];
+              const float cpv[4] = {a.x, a.y, a.z, a.w}, cmv[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                const int j = 4 * q + e;
+                const int32_t a1 = static_cast<int32_t>(ap[j]), a2 = static_cast<int32_t>(am[j]);
+                const float f1 = p.exact_small_acc ? i2f_small(a1) : __int2float_rn(a1);
+                const float f2 = p.exact_small_acc ? i2f_small(a2) : __int2float_rn(a2);
+                run[c * 32 + j] = fmaf(cpv[e], f1, run[c * 32 + j]);
+                run[c * 32 + j] = fmaf(cmv[e], f2, run[c * 32 + j]);
+              }
             }
           }
         }
@@ -364,20 +399,27 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         ++acc_iter;
       }
       if constexpr (SEGK && OUT != OUT_S32) {
+        __syncwarp();
+        for (int j = lane; j < HALF; j += 32) {
+          const int64_t n = nb + j;
+          cst[j] = (p.bias != nullptr && n < p.N) ? bf16_to_f32(p.bias[n]) : 0.0f;
+        }
+        __syncwarp();
         if (m < p.M) {
 #pragma unroll
-        for (int c = 0; c < CHUNKS; ++c) {
-          const int64_t n0 = nb + c * 32;
-          float v[32];
+          for (int c = 0; c < CHUNKS; ++c) {
+            const float4 *b4 = reinterpret_cast<const float4 *>(cst + c * 32);
+            float v[32];
 #pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            const int64_t n = n0 + j;
-            float yv = run[c * 32 + j];
-            if (p.bias != nullptr && n < p.N) yv = __fadd_rn(yv, bf16_to_f32(__ldg(p.bias + n)));
-            v[j] = yv;
+            for (int q = 0; q < 8; ++q) {
+              const float4 b = b4[q];
+              v[4 * q + 0] = __fadd_rn(run[c * 32 + 4 * q + 0], b.x);
+              v[4 * q + 1] = __fadd_rn(run[c * 32 + 4 * q + 1], b.y);
+              v[4 * q + 2] = __fadd_rn(run[c * 32 + 4 * q + 2], b.z);
+              v[4 * q + 3] = __fadd_rn(run[c * 32 + 4 * q + 3], b.w);
+            }
+            store_row_chunk<OUT>(p, m, nb + c * 32, v);
           }
-          store_row_chunk<OUT>(p, m, n0, v);
-        }
         }
       }
     }

@@ -18,7 +18,7 @@ namespace {
 constexpr int kColsPerThread = 8;                     // one 16-byte bf16 load
 constexpr int kWarpCols = 32 * kColsPerThread;        // 256 channels per warp row
 constexpr int kRowsPerBlock = 8;                      // warps per block
-constexpr int kUnroll = 4;                            // rows in flight per thread
+constexpr int kUnroll = 3;                            // rows in flight per thread
 
 __device__ __forceinline__ float bf16_bits_to_f32(uint32_t h) {
   return __uint_as_float(h << 16);
@@ -34,9 +34,9 @@ __device__ __forceinline__ void unpack8(const uint4 &v, float (&x)[8]) {
 }
 
 // ------------------------------------------------------------- calibration
-// Pass 1: per-thread max of u = x / d and of -u over its rows, then one
-// atomicMax per thread into s_act (which holds raw maxima, non-negative
-// floats, whose bit patterns order like unsigned integers).
+// Pass 1: per-thread max of u = x / d and of -u over its rows, combined across
+// the lanes of one K-segment, then atomicMax into s_act, which holds the raw
+// maxima until pass 2 (non-negative floats order like their bit patterns).
 __global__ void __launch_bounds__(256) calib_reduce_kernel(const uint16_t *__restrict__ x,
                                                            int64_t M, int64_t K, int64_t ldx,
                                                            const float *__restrict__ d,
@@ -83,37 +83,79 @@ __global__ void calib_finalize_kernel(float *s_act, int n) {
 }
 
 // ---------------------------------------------------- activation quantize
+// q = rne(v) saturated to [-128, 127] (cvt.rni.sat.s8.f32; NaN gives 0).
+__device__ __forceinline__ uint32_t f2s8_rn_sat(float v) {
+  uint32_t r;
+  asm("cvt.rni.sat.s8.f32 %0, %1;" : "=r"(r) : "f"(v));
+  return r;
+}
+
+// Packs the low bytes of four codes into one word (byte j = code j).
+__device__ __forceinline__ uint32_t pack4(uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+  return __byte_perm(__byte_perm(a, b, 0x0040), __byte_perm(c, d, 0x0040), 0x5410);
+}
+
+// Eight channels x of one row -> X^+ and X^- codes, 8 bytes each.  One signed
+// code per element, q = sat(rne(x * (x >= 0 ? m+ : m-))): its sign is the
+// sign of x, so X^+ = max(q, 0) and X^- = min(q, 0) byte-wise.  This is the
+// case-wise Q_dual with the clamps of the reference: x >= 0 (including -0.0)
+// gives a code in [0, 127], x < 0 a code in [-128, 0], NaN gives 0 in both.
+__device__ __forceinline__ void dualscale8(const float (&x)[8], const float (&mp)[8],
+                                           const float (&mm)[8], uint2 &plus, uint2 &minus) {
+  uint32_t q[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) q[j] = f2s8_rn_sat(__fmul_rn(x[j], x[j] >= 0.0f ? mp[j] : mm[j]));
+  const uint32_t w0 = pack4(q[0], q[1], q[2], q[3]);
+  const uint32_t w1 = pack4(q[4], q[5], q[6], q[7]);
+  plus = make_uint2(__vmaxs4(w0, 0u), __vmaxs4(w1, 0u));
+  minus = make_uint2(__vmins4(w0, 0u), __vmins4(w1, 0u));
+}
+
 // Block: 32 x 8 threads.  blockIdx.x owns 256 consecutive channels; every
 // warp streams whole rows of them (512 contiguous bytes per row), kUnroll rows
-// in flight per thread.  The folded multipliers m+- = 1/(d*s+-) of the block's
-// channels, for every group, sit in shared memory: [G][2][256] floats.
-__global__ void __launch_bounds__(256) quant_act_kernel(const uint16_t *__restrict__ x,
+// in flight per thread.  With one activation group the folded multipliers
+// m+- = 1/(d*s+-) of the thread's eight channels live in registers; with G
+// groups they sit in shared memory, [G][2][256] floats.
+template <bool kOneGroup>
+__global__ void __launch_bounds__(256, 4) quant_act_kernel(const uint16_t *__restrict__ x,
                                                         int64_t M, int64_t K, int64_t ldx,
                                                         const float *__restrict__ d,
                                                         const float *__restrict__ s_act,
                                                         SegParams seg,
                                                         int8_t *__restrict__ planes) {
-  extern __shared__ float mtab[];  // [G][2][kWarpCols]
-  const int G = seg.G;
-  const int tid = threadIdx.y * 32 + threadIdx.x;
+  extern __shared__ float mtab[];  // [G][2][kWarpCols] when G > 1
+  const int G = kOneGroup ? 1 : seg.G;
   const int64_t cblk = static_cast<int64_t>(blockIdx.x) * kWarpCols;
-  for (int t = tid; t < G * kWarpCols; t += 256) {
-    const int g = t / kWarpCols, cl = t % kWarpCols;
-    const int64_t c = cblk + cl;
-    float mp = 0.0f, mm = 0.0f;
-    if (c < K) {
-      const int i = (seg.mode == SQ_SEG_INPUT) ? seg_index(seg.off, seg.n_seg, c) : 0;
-      const float dv = d ? d[g * K + c] : 1.0f;
-      const float sp = s_act[(g * seg.S + i) * 2 + 0];
-      const float sm = s_act[(g * seg.S + i) * 2 + 1];
-      mp = __fdiv_rn(1.0f, __fmul_rn(dv, sp));
-      mm = __fdiv_rn(1.0f, __fmul_rn(dv, sm));
-    }
-    mtab[(g * 2 + 0) * kWarpCols + cl] = mp;
-    mtab[(g * 2 + 1) * kWarpCols + cl] = mm;
-  }
-  __syncthreads();
   const int64_t c0 = cblk + threadIdx.x * kColsPerThread;
+  float mp_r[8], mm_r[8];
+  if (kOneGroup) {
+    if (c0 < K) {
+      const int i = (seg.mode == SQ_SEG_INPUT) ? seg_index(seg.off, seg.n_seg, c0) : 0;
+      const float sp = s_act[i * 2 + 0], sm = s_act[i * 2 + 1];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const float dv = d ? d[c0 + j] : 1.0f;
+        mp_r[j] = __fdiv_rn(1.0f, __fmul_rn(dv, sp));
+        mm_r[j] = __fdiv_rn(1.0f, __fmul_rn(dv, sm));
+      }
+    }
+  } else {
+    const int tid = threadIdx.y * 32 + threadIdx.x;
+    for (int t = tid; t < G * kWarpCols; t += 256) {
+      const int g = t / kWarpCols, cl = t % kWarpCols;
+      const int64_t c = cblk + cl;
+      float mp = 0.0f, mm = 0.0f;
+      if (c < K) {
+        const int i = (seg.mode == SQ_SEG_INPUT) ? seg_index(seg.off, seg.n_seg, c) : 0;
+        const float dv = d ? d[g * K + c] : 1.0f;
+        mp = __fdiv_rn(1.0f, __fmul_rn(dv, s_act[(g * seg.S + i) * 2 + 0]));
+        mm = __fdiv_rn(1.0f, __fmul_rn(dv, s_act[(g * seg.S + i) * 2 + 1]));
+      }
+      mtab[(g * 2 + 0) * kWarpCols + cl] = mp;
+      mtab[(g * 2 + 1) * kWarpCols + cl] = mm;
+    }
+    __syncthreads();
+  }
   if (c0 >= K) return;
   const int64_t plane_stride = M * K;
   const int64_t row_step = static_cast<int64_t>(gridDim.y) * kRowsPerBlock * kUnroll;
@@ -132,21 +174,22 @@ __global__ void __launch_bounds__(256) quant_act_kernel(const uint16_t *__restri
       float xv[8];
       unpack8(v[u], xv);
       for (int g = 0; g < G; ++g) {
-        const float *mp = mtab + (g * 2 + 0) * kWarpCols + threadIdx.x * kColsPerThread;
-        const float *mm = mtab + (g * 2 + 1) * kWarpCols + threadIdx.x * kColsPerThread;
-        uint32_t pk[2] = {0u, 0u}, nk[2] = {0u, 0u};
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const float xj = xv[j];
-          int qp = 0, qm = 0;
-          if (xj >= 0.0f) qp = __float2int_rn(fminf(__fmul_rn(xj, mp[j]), 127.0f));
-          if (xj < 0.0f) qm = __float2int_rn(fmaxf(__fmul_rn(xj, mm[j]), -128.0f));
-          pk[j >> 2] |= (static_cast<uint32_t>(qp) & 0xFFu) << (8 * (j & 3));
-          nk[j >> 2] |= (static_cast<uint32_t>(qm) & 0xFFu) << (8 * (j & 3));
+        if (!kOneGroup) {
+          const float4 *mp4 = reinterpret_cast<const float4 *>(
+              mtab + (g * 2 + 0) * kWarpCols + threadIdx.x * kColsPerThread);
+          const float4 *mm4 = reinterpret_cast<const float4 *>(
+              mtab + (g * 2 + 1) * kWarpCols + threadIdx.x * kColsPerThread);
+          const float4 a = mp4[0], b = mp4[1], c = mm4[0], e = mm4[1];
+          mp_r[0] = a.x; mp_r[1] = a.y; mp_r[2] = a.z; mp_r[3] = a.w;
+          mp_r[4] = b.x; mp_r[5] = b.y; mp_r[6] = b.z; mp_r[7] = b.w;
+          mm_r[0] = c.x; mm_r[1] = c.y; mm_r[2] = c.z; mm_r[3] = c.w;
+          mm_r[4] = e.x; mm_r[5] = e.y; mm_r[6] = e.z; mm_r[7] = e.w;
         }
+        uint2 pk, nk;
+        dualscale8(xv, mp_r, mm_r, pk, nk);
         int8_t *dst = planes + (static_cast<int64_t>(g) * 2) * plane_stride + r * K + c0;
-        *reinterpret_cast<uint2 *>(dst) = make_uint2(pk[0], pk[1]);
-        *reinterpret_cast<uint2 *>(dst + plane_stride) = make_uint2(nk[0], nk[1]);
+        __stcs(reinterpret_cast<uint2 *>(dst), pk);
+        __stcs(reinterpret_cast<uint2 *>(dst + plane_stride), nk);
       }
     }
   }
@@ -240,15 +283,19 @@ cudaError_t launch_quantize_act(const uint16_t *x, int64_t M, int64_t K, int64_t
   int64_t gy = (static_cast<int64_t>(num_sms()) * 8 + gx - 1) / gx;
   if (gy > row_groups) gy = row_groups;
   if (gy < 1) gy = 1;
+  const dim3 grid(gx, static_cast<unsigned>(gy)), block(32, kRowsPerBlock);
+  if (seg.G == 1) {
+    quant_act_kernel<true><<<grid, block, 0, stream>>>(x, M, K, ldx, d, s_act, seg, planes);
+    return cudaGetLastError();
+  }
   const size_t smem = sizeof(float) * 2 * kWarpCols * seg.G;
   if (smem > 48 * 1024) {
-    cudaError_t e = cudaFuncSetAttribute(quant_act_kernel,
+    cudaError_t e = cudaFuncSetAttribute(quant_act_kernel<false>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem));
     if (e != cudaSuccess) return e;
   }
-  quant_act_kernel<<<dim3(gx, static_cast<unsigned>(gy)), dim3(32, kRowsPerBlock), smem,
-                     stream>>>(x, M, K, ldx, d, s_act, seg, planes);
+  quant_act_kernel<false><<<grid, block, smem, stream>>>(x, M, K, ldx, d, s_act, seg, planes);
   return cudaGetLastError();
 }
 
