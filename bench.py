@@ -14,10 +14,13 @@ Metric: effective TOPS = sum over layers of 2*M*N*K / step time.  Also reported:
 executed TOPS (the doubled 2M rows of X^+ and X^-), their fraction of the B200's
 dense INT8 peak, and the activation-quantize kernel's GB/s against HBM.
 
-Timing: CUDA events on the launching stream around every kernel, L2 flushed
-(512 MiB write) between steps outside the timed events, W warm-up steps, then K
-timed steps; across N GPUs (one process each, replicas of the same workload,
-no collective on the data path) the step time is the max over ranks.
+Timing: CUDA events on the launching stream around every kernel; between steps,
+outside the timed events, the L2 is flushed (512 MiB written, then 256 MiB of
+another buffer read so that the flush's dirty lines are written back before the
+step starts); W warm-up steps, then K timed steps; across N GPUs (one process
+each, replicas of the same workload, no collective on the data path) the step
+time is the max over ranks.  Each quantize launch is also timed alone after a
+flush (its own HBM roofline).
 """
 from __future__ import annotations
 
@@ -45,7 +48,8 @@ METRIC = "DualScale-SegLinear W8A8 GEMM effective TOPS & % of B200 INT8 peak; qu
 # generated MEASURED_PEAKS.json is absent.
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 INT8_OVER_BF16 = 4.5 / 2.25   # dense INT8 / dense bf16, nominal B200 ratio
-FLUSH_BYTES = 512 << 20
+FLUSH_BYTES = 512 << 20       # written between steps (4x the 126 MB L2) ...
+SWEEP_BYTES = 256 << 20       # ... then a second buffer is read, so the L2 holds clean lines
 SMI_FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
@@ -200,6 +204,16 @@ def run_ours(args, ws, rank, local):
     exe_ops = sum(layer_units(g.L)[1] for g in glayers)
     qbytes = sum(layer_units(g.L)[2] for g in glayers)
     flush = torch.empty(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    sweep = torch.ones(SWEEP_BYTES // 4, dtype=torch.float32, device=dev)
+    sink = torch.empty((), dtype=torch.float32, device=dev)
+
+    def flush_l2():
+        # Evict everything: write a buffer larger than L2, then read another
+        # one, so that the dirty lines of the write are written back here
+        # (untimed) and not by the first timed kernel.
+        flush.zero_()
+        torch.sum(sweep, dim=0, out=sink)
+
     stream = torch.cuda.current_stream()
     nl = len(glayers)
 
@@ -213,7 +227,7 @@ def run_ours(args, ws, rank, local):
 
     mk = lambda: [torch.cuda.Event(enable_timing=True) for _ in range(2 * nl + 1)]
     for _ in range(args.warmup):
-        flush.zero_()
+        flush_l2()
         one_step(mk())
     torch.cuda.synchronize()
     if ws > 1:
@@ -224,7 +238,7 @@ def run_ours(args, ws, rank, local):
     with ClockSampler(local) as clocks:
         t_wall = time.perf_counter()
         for k in range(args.steps):
-            flush.zero_()
+            flush_l2()
             one_step(events[k])
         torch.cuda.synchronize()
         t_wall = time.perf_counter() - t_wall
@@ -250,6 +264,23 @@ def run_ours(args, ws, rank, local):
                                gemm_us=1e3 * g_ms[i] / args.steps)
                           for i, g in enumerate(glayers)],
                launches=2 * nl * args.steps)
+
+    # Each activation-quantize launch alone after an L2 flush: the kernel's own
+    # HBM roofline, free of the write-back left in L2 by the previous kernel of
+    # the step.
+    iso_steps = max(3, min(args.steps, 200))
+    iso_ms = [0.0] * nl
+    for i, g in enumerate(glayers):
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(iso_steps)]
+        for k in range(iso_steps):
+            flush_l2()
+            ev[k][0].record(stream)
+            g.quantize()
+            ev[k][1].record(stream)
+        torch.cuda.synchronize()
+        iso_ms[i] = sum(a.elapsed_time(b) for a, b in ev) / iso_steps
+    res["quant_isolated_ms"] = iso_ms
 
     # end to end through the library with host buffers: H2D of the step's
     # activations from pinned memory, the kernels, D2H of the outputs.
@@ -368,6 +399,7 @@ def main(argv=None):
     exe_tops_step = res["exe_ops"] / (ms * 1e-3) / 1e12
     gemm_tops = res["exe_ops"] / (res["gemm_ms"] * 1e-3) / 1e12
     quant_gbs = res["qbytes"] / (res["quant_ms"] * 1e-3) / 1e9
+    quant_iso_gbs = res["qbytes"] / (sum(res["quant_isolated_ms"]) * 1e-3) / 1e9
     traffic, traffic_note = traffic_from_profile()
     cpu = None
     if n_gpus == 1 and not args.no_cpu_baseline:
@@ -395,7 +427,8 @@ def main(argv=None):
         "config": {"workload": f"{args.config}: {wl.CONFIGS[args.config]}",
                    "layers": [{k: v for k, v in p.items() if k in ("name", "M", "N", "K", "G", "S")}
                               for p in res["per_layer"]],
-                   "output": "bf16", "l2": "flushed between steps (512 MiB write, untimed)",
+                   "output": "bf16",
+                   "l2": "flushed between steps, untimed: 512 MiB written, then 256 MiB read",
                    "parallelism": f"replicas x{n_gpus}"},
         "executed_tops": round(n_gpus * exe_tops_step, 2),
         "executed_frac_int8_peak": round(exe_tops_step / int8_peak_burst, 4),
@@ -413,8 +446,12 @@ def main(argv=None):
                                     f"(nominal INT8/bf16 ratio); sustained-based INT8 peak "
                                     f"{round(int8_peak_sust, 1)}",
                      "traffic_note": traffic_note},
-        "quant_roofline": {"bound": "hbm", "achieved": round(quant_gbs, 1), "peak": hbm,
-                           "unit": "GB/s", "frac": round(quant_gbs / hbm, 4)},
+        "quant_roofline": {"bound": "hbm", "achieved": round(quant_iso_gbs, 1), "peak": hbm,
+                           "unit": "GB/s", "frac": round(quant_iso_gbs / hbm, 4),
+                           "measured": "each quantize launch alone after an L2 flush",
+                           "in_step_achieved": round(quant_gbs, 1),
+                           "in_step_frac": round(quant_gbs / hbm, 4),
+                           "isolated_us": [round(1e3 * t, 2) for t in res["quant_isolated_ms"]]},
         "cpu_baseline": cpu,
         "e2e": {"value": round(e2e_tops, 3), "unit": "TOPS",
                 "h2d_bytes_per_step": res["h2d"], "d2h_bytes_per_step": res["d2h"],

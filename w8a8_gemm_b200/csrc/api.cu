@@ -159,6 +159,20 @@ sq_status gemm_common(const int8_t *planes, const int8_t *wq, const float *s_w,
 
 }  // namespace
 
+EncodeTiledFn tensor_map_encoder() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void *ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  });
+  return fn;
+}
+
 int *device_status_word() {
   static int *addr[kMaxDevices] = {};
   static std::mutex mu;
@@ -206,8 +220,10 @@ sq_status sq_quantize_act(const void *x, int64_t M, int64_t K, int64_t ldx, cons
   if (!aligned(s_act, 4) || (d && !aligned(d, 4)) || !aligned(planes, 16))
     return SQ_ERR_ALIGNMENT;
   SQ_TRY(check_device());
-  return from_cuda(launch_quantize_act(static_cast<const uint16_t *>(x), M, K, ldx, d, s_act, sp,
-                                       planes, reinterpret_cast<cudaStream_t>(stream)));
+  int *status = device_status_word();
+  if (status == nullptr) return SQ_ERR_CUDA;
+  return launch_quantize_act(static_cast<const uint16_t *>(x), M, K, ldx, d, s_act, sp, planes,
+                             status, reinterpret_cast<cudaStream_t>(stream));
 }
 
 sq_status sq_quantize_weight_seg(const void *w, int64_t N, int64_t K, const float *d,

@@ -34,11 +34,18 @@
 namespace sq {
 namespace {
 
+// Column tile of one-segment layers: 256 (one TMEM buffer, the epilogue runs
+// between tiles) or 128 (two buffers, the epilogue overlaps the next tile).
+#ifndef SQ_GEMM_BN_ONE_SEG
+#define SQ_GEMM_BN_ONE_SEG 256
+#endif
+
 constexpr int BM = 128;              // rows of M per tile (TMEM lanes)
 constexpr int BK = 128;              // int8 K elements per stage = one 128-B swizzle row
 constexpr int MMA_K = 32;            // K of one kind::i8 MMA
-constexpr int NUM_EPI_WARPS = 8;
-constexpr int NUM_THREADS = 64 + 32 * NUM_EPI_WARPS;
+// Epilogue warps: 8 for one-segment layers (register-heavy final epilogue), 16
+// for input-segmented layers (latency-bound per-segment drains).
+constexpr int threads_for(int epi_warps) { return 64 + 32 * epi_warps; }
 constexpr uint64_t kWaitLimitNs = 2000000000ull;   // 2 s: far above any tile's latency
 
 struct GemmParams {
@@ -57,14 +64,15 @@ struct GemmParams {
   int *status;
 };
 
-template <int BN, int STAGES>
+template <int BN, int STAGES, int EPI_WARPS>
 struct Smem {
   static constexpr int A_BYTES = 2 * BM * BK;   // X^+ tile, then X^- tile
   static constexpr int B_BYTES = BN * BK;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr int NBUF = 512 / (2 * BN);   // TMEM accumulator buffers
   static constexpr int EPI_OFFSET = STAGES * STAGE_BYTES;  // per-warp column constants
-  static constexpr int EPI_BYTES = NUM_EPI_WARPS * 2 * (BN / 2) * 4;
+  static constexpr int COLS = BN / (EPI_WARPS / 4);  // columns per epilogue warp
+  static constexpr int EPI_BYTES = EPI_WARPS * 4 * COLS * 4;  // 2 buffers x 2 arrays
   static constexpr int BAR_OFFSET = EPI_OFFSET + EPI_BYTES;
   static constexpr int NUM_BARS = 2 * STAGES + 2 * NBUF + 1;
   static constexpr int BYTES = BAR_OFFSET + NUM_BARS * 8 + 16 + 1024;  // + 1 KB alignment slack
@@ -81,9 +89,7 @@ __device__ __forceinline__ bool wait_bar(uint64_t *bar, uint32_t parity, volatil
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   while (true) {
-#pragma unroll 1
-    for (int i = 0; i < 64; ++i)
-      if (mbar_try_wait(bar, parity)) return true;
+    if (mbar_try_wait_sleep(bar, parity, kSleepHintNs)) return true;
     if (*abort_flag) return false;
     if (globaltimer_ns() - t0 > kWaitLimitNs) {
       *abort_flag = 1;
@@ -93,11 +99,30 @@ __device__ __forceinline__ bool wait_bar(uint64_t *bar, uint32_t parity, volatil
   }
 }
 
-// int32 -> fp32.  When |a| < 2^22 the bit pattern 0x4B400000 + a is the float
-// 1.5 * 2^23 + a exactly, so one integer add and one float subtract give the
-// exact value (the same as round-to-nearest conversion, which is exact there).
-__device__ __forceinline__ float i2f_small(int32_t a) {
-  return __int_as_float(0x4B400000 + a) - 12582912.0f;
+// Packed pairs of fp32 (sm_100 f32x2 arithmetic): two lanes of work per instruction.
+__device__ __forceinline__ uint64_t f2pack(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void f2unpack(uint64_t v, float &lo, float &hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t ffma2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t fadd2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+// Two accumulators (|a| < 2^22) to exact fp32, packed: 0x4B400000 + a is the
+// float 1.5 * 2^23 + a, and one packed subtract removes the offset.
+__device__ __forceinline__ uint64_t i2f_small2(uint32_t a, uint32_t b) {
+  return fadd2(f2pack(__uint_as_float(a + 0x4B400000u), __uint_as_float(b + 0x4B400000u)),
+               f2pack(-12582912.0f, -12582912.0f));
 }
 
 __device__ __forceinline__ float bf16_to_f32(uint16_t h) {
@@ -145,15 +170,19 @@ __device__ __forceinline__ void store_row_chunk(const GemmParams &p, int64_t m, 
   }
 }
 
-template <int BN, int STAGES, int OUT, bool SEGK>
-__global__ void __launch_bounds__(NUM_THREADS, 1)
+// One CTA per SM (shared memory allows no more).  Its warps spread over the four
+// 16K-register sub-partitions (10 warps: 3/3/2/2, a thread at most 168
+// registers; 18 warps: 5/5/4/4, at most 96).
+template <int BN, int STAGES, int OUT, bool SEGK, int EPI_WARPS>
+__global__ void __launch_bounds__(threads_for(EPI_WARPS), 1)
     dualscale_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                           const __grid_constant__ CUtensorMap tmB,
                           const __grid_constant__ GemmParams p) {
-  using L = Smem<BN, STAGES>;
+  using L = Smem<BN, STAGES, EPI_WARPS>;
   constexpr int NBUF = L::NBUF;
-  constexpr int HALF = BN / 2;       // columns per epilogue warp
+  constexpr int HALF = L::COLS;      // columns per epilogue warp
   constexpr int CHUNKS = HALF / 32;  // 32-column TMEM loads per warp per unit
+  static_assert(EPI_WARPS % 4 == 0 && HALF % 32 == 0, "epilogue split");
   static_assert(NBUF >= 1, "BN too large for TMEM");
 
   extern __shared__ uint8_t smem_raw[];
@@ -177,7 +206,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
     for (int b = 0; b < NBUF; ++b) {
       mbar_init(&acc_full[b], 1);
-      mbar_init(&acc_empty[b], NUM_EPI_WARPS);
+      mbar_init(&acc_empty[b], EPI_WARPS);
     }
     mbar_init(mma_done, 1);
     *abort_flag = 0;
@@ -285,12 +314,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     // ------------------------------------------------------------ epilogue
     const int ew = warp - 2;
     const int quarter = warp & 3;       // TMEM lanes this warp may read
-    const int half = ew >> 2;           // which half of the BN columns
+    const int half = ew >> 2;           // which column part of the tile
     const int row = quarter * 32 + lane;
     const uint32_t lane_addr = static_cast<uint32_t>(quarter * 32) << 16;
     // Warp-private column constants in shared memory, read back as broadcast
-    // float4s: [0, HALF) and [HALF, 2*HALF).
-    float *cst = reinterpret_cast<float *>(smem + L::EPI_OFFSET) + ew * 2 * HALF;
+    // float4s: two buffers of [HALF] + [HALF] floats.
+    float *cst_base = reinterpret_cast<float *>(smem + L::EPI_OFFSET) + ew * 4 * HALF;
     uint32_t acc_iter = 0;
     for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x) {
       const int mt = tile / p.num_n_tiles, nt = tile % p.num_n_tiles;
@@ -302,29 +331,46 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         __syncwarp();
         for (int j = lane; j < HALF; j += 32) {
           const int64_t n = nb + j;
-          cst[j] = n < p.N ? p.s_w[n] : 0.0f;
-          cst[HALF + j] = (p.bias != nullptr && n < p.N) ? bf16_to_f32(p.bias[n]) : 0.0f;
+          cst_base[j] = n < p.N ? p.s_w[n] : 0.0f;
+          cst_base[HALF + j] = (p.bias != nullptr && n < p.N) ? bf16_to_f32(p.bias[n]) : 0.0f;
         }
         __syncwarp();
       }
-      float run[SEGK ? HALF : 1];
-      if constexpr (SEGK) {
+      // Multi-segment state: packed running sums (column pairs) and the next
+      // K-segment's weight scales, loaded one segment ahead.
+      uint64_t run2[SEGK ? HALF / 2 : 1];
+      float sw_next[SEGK ? HALF / 32 : 1];
+      if constexpr (SEGK && OUT != OUT_S32) {
 #pragma unroll
-        for (int j = 0; j < (SEGK ? HALF : 1); ++j) run[j] = 0.0f;
+        for (int j = 0; j < HALF / 2; ++j) run2[j] = 0ull;
+#pragma unroll
+        for (int q = 0; q < HALF / 32; ++q) {
+          const int64_t n = nb + q * 32 + lane;
+          sw_next[q] = n < p.N ? p.s_w[n] : 0.0f;
+        }
       }
       const int units = SEGK ? p.S : 1;
       for (int u = 0; u < units; ++u) {
         const float sp = p.s_act[(g * p.S + u) * 2 + 0];
         const float sm = p.s_act[(g * p.S + u) * 2 + 1];
+        float *cst = cst_base;
         if constexpr (SEGK && OUT != OUT_S32) {
-          // Folded coefficients of this K-segment: c+- = s_w[u][n] * s+-[u].
-          __syncwarp();
-          const float *swu = p.s_w + static_cast<int64_t>(u) * p.N;
-          for (int j = lane; j < HALF; j += 32) {
-            const int64_t n = nb + j;
-            const float sw = n < p.N ? swu[n] : 0.0f;
-            cst[j] = sw * sp;
-            cst[HALF + j] = sw * sm;
+          // Folded coefficients of K-segment u: c+- = s_w[u][n] * s+-[u], into
+          // buffer u & 1 (the other buffer may still be read by segment u - 1
+          // only in program order of this warp, so no wait is needed).
+          cst = cst_base + (u & 1) * 2 * HALF;
+#pragma unroll
+          for (int q = 0; q < HALF / 32; ++q) {
+            cst[q * 32 + lane] = sw_next[q] * sp;
+            cst[HALF + q * 32 + lane] = sw_next[q] * sm;
+          }
+          if (u + 1 < units) {
+            const float *swn = p.s_w + static_cast<int64_t>(u + 1) * p.N;
+#pragma unroll
+            for (int q = 0; q < HALF / 32; ++q) {
+              const int64_t n = nb + q * 32 + lane;
+              sw_next[q] = n < p.N ? swn[n] : 0.0f;
+            }
           }
           __syncwarp();
         }
@@ -334,7 +380,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         tc_fence_after();
         const uint32_t t_plus = tmem_base + lane_addr + buf * 2 * BN + half * HALF;
 #pragma unroll
-        for (int c = 0; c < CHUNKS; ++c) {
+        for (int c = 0; c < ((SEGK && OUT != OUT_S32) ? 0 : CHUNKS); ++c) {
           uint32_t ap[32], am[32];
           tmem_ld_32x32b_x32(t_plus + c * 32, ap);
           tmem_ld_32x32b_x32(t_plus + BN + c * 32, am);
@@ -373,22 +419,38 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
               }
               store_row_chunk<OUT>(p, m, n0, v);
             }
-          } else {
-            // Several K-segments: y += c+ f(A+) + c- f(A-).
-            const float4 *cp4 = reinterpret_cast<const float4 *>(cst + c * 32);
-            const float4 *cm4 = reinterpret_cast<const float4 *>(cst + HALF + c * 32);
+          }
+        }
+        if constexpr (SEGK && OUT != OUT_S32) {
+          // Several K-segments: y += c+ f(A+) + c- f(A-), two columns per packed
+          // instruction, 16 columns per TMEM load to keep register pressure low.
 #pragma unroll
-            for (int q = 0; q < 8; ++q) {
+          for (int c = 0; c < HALF / 16; ++c) {
+            uint32_t ap[16], am[16];
+            tmem_ld_32x32b_x16(t_plus + c * 16, ap);
+            tmem_ld_32x32b_x16(t_plus + BN + c * 16, am);
+            tmem_ld_wait();
+            const float4 *cp4 = reinterpret_cast<const float4 *>(cst + c * 16);
+            const float4 *cm4 = reinterpret_cast<const float4 *>(cst + HALF + c * 16);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
               const float4 a = cp4[q], b = cm4[q];
-              const float cpv[4] = {a.x, a.y, a.z, a.w}, cmv[4] = {b.x, b.y, b.z, b.w};
-#pragma unroll
-              for (int e = 0; e < 4; ++e) {
-                const int j = 4 * q + e;
-                const int32_t a1 = static_cast<int32_t>(ap[j]), a2 = static_cast<int32_t>(am[j]);
-                const float f1 = p.exact_small_acc ? i2f_small(a1) : __int2float_rn(a1);
-                const float f2 = p.exact_small_acc ? i2f_small(a2) : __int2float_rn(a2);
-                run[c * 32 + j] = fmaf(cpv[e], f1, run[c * 32 + j]);
-                run[c * 32 + j] = fmaf(cmv[e], f2, run[c * 32 + j]);
+              const int j = 4 * q;
+              uint64_t &r0 = run2[c * 8 + 2 * q], &r1 = run2[c * 8 + 2 * q + 1];
+              if (p.exact_small_acc) {
+                r0 = ffma2(f2pack(a.x, a.y), i2f_small2(ap[j], ap[j + 1]), r0);
+                r1 = ffma2(f2pack(a.z, a.w), i2f_small2(ap[j + 2], ap[j + 3]), r1);
+                r0 = ffma2(f2pack(b.x, b.y), i2f_small2(am[j], am[j + 1]), r0);
+                r1 = ffma2(f2pack(b.z, b.w), i2f_small2(am[j + 2], am[j + 3]), r1);
+              } else {
+                const auto cvt2 = [](uint32_t x, uint32_t y) {
+                  return f2pack(__int2float_rn(static_cast<int32_t>(x)),
+                                __int2float_rn(static_cast<int32_t>(y)));
+                };
+                r0 = ffma2(f2pack(a.x, a.y), cvt2(ap[j], ap[j + 1]), r0);
+                r1 = ffma2(f2pack(a.z, a.w), cvt2(ap[j + 2], ap[j + 3]), r1);
+                r0 = ffma2(f2pack(b.x, b.y), cvt2(am[j], am[j + 1]), r0);
+                r1 = ffma2(f2pack(b.z, b.w), cvt2(am[j + 2], am[j + 3]), r1);
               }
             }
           }
@@ -399,28 +461,32 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         ++acc_iter;
       }
       if constexpr (SEGK && OUT != OUT_S32) {
-        __syncwarp();
+        float *bst = cst_base + (units & 1) * 2 * HALF;  // buffer not read by the last segment
         for (int j = lane; j < HALF; j += 32) {
           const int64_t n = nb + j;
-          cst[j] = (p.bias != nullptr && n < p.N) ? bf16_to_f32(p.bias[n]) : 0.0f;
+          bst[j] = (p.bias != nullptr && n < p.N) ? bf16_to_f32(p.bias[n]) : 0.0f;
         }
         __syncwarp();
         if (m < p.M) {
 #pragma unroll
           for (int c = 0; c < CHUNKS; ++c) {
-            const float4 *b4 = reinterpret_cast<const float4 *>(cst + c * 32);
+            const float4 *b4 = reinterpret_cast<const float4 *>(bst + c * 32);
             float v[32];
 #pragma unroll
             for (int q = 0; q < 8; ++q) {
               const float4 b = b4[q];
-              v[4 * q + 0] = __fadd_rn(run[c * 32 + 4 * q + 0], b.x);
-              v[4 * q + 1] = __fadd_rn(run[c * 32 + 4 * q + 1], b.y);
-              v[4 * q + 2] = __fadd_rn(run[c * 32 + 4 * q + 2], b.z);
-              v[4 * q + 3] = __fadd_rn(run[c * 32 + 4 * q + 3], b.w);
+              float r0, r1, r2, r3;
+              f2unpack(run2[c * 16 + 2 * q], r0, r1);
+              f2unpack(run2[c * 16 + 2 * q + 1], r2, r3);
+              v[4 * q + 0] = __fadd_rn(r0, b.x);
+              v[4 * q + 1] = __fadd_rn(r1, b.y);
+              v[4 * q + 2] = __fadd_rn(r2, b.z);
+              v[4 * q + 3] = __fadd_rn(r3, b.w);
             }
             store_row_chunk<OUT>(p, m, nb + c * 32, v);
           }
         }
+        __syncwarp();
       }
     }
   epilogue_exit:;
@@ -436,26 +502,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 }
 
 // ------------------------------------------------------------------ host side
-typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
-                                  const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
-                                  const cuuint32_t *, CUtensorMapInterleave,
-                                  CUtensorMapSwizzle, CUtensorMapL2promotion,
-                                  CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_fn() {
-  static EncodeTiledFn fn = nullptr;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    void *ptr = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
-            cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiledFn>(ptr);
-  });
-  return fn;
-}
-
 int device_sm_count() {
   int dev = 0, sms = 0;
   cudaGetDevice(&dev);
@@ -463,10 +509,10 @@ int device_sm_count() {
   return sms > 0 ? sms : 148;
 }
 
-template <int BN, int STAGES, int OUT, bool SEGK>
+template <int BN, int STAGES, int OUT, bool SEGK, int EPI_WARPS>
 sq_status run_gemm(const GemmRequest &r, const GemmParams &p, cudaStream_t stream) {
-  using L = Smem<BN, STAGES>;
-  EncodeTiledFn enc = encode_fn();
+  using L = Smem<BN, STAGES, EPI_WARPS>;
+  EncodeTiledFn enc = tensor_map_encoder();
   if (enc == nullptr) return SQ_ERR_CUDA;
   const int G = r.seg.G;
   CUtensorMap tmA, tmB;
@@ -495,7 +541,7 @@ sq_status run_gemm(const GemmRequest &r, const GemmParams &p, cudaStream_t strea
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
       return SQ_ERR_CUDA;
   }
-  auto kernel = dualscale_gemm_kernel<BN, STAGES, OUT, SEGK>;
+  auto kernel = dualscale_gemm_kernel<BN, STAGES, OUT, SEGK, EPI_WARPS>;
   static bool attr_set[64] = {};  // per instantiation and device
   int dev = 0;
   cudaGetDevice(&dev);
@@ -507,7 +553,7 @@ sq_status run_gemm(const GemmRequest &r, const GemmParams &p, cudaStream_t strea
     attr_set[dev] = true;
   }
   const int grid = p.num_tiles < device_sm_count() ? p.num_tiles : device_sm_count();
-  kernel<<<grid, NUM_THREADS, L::BYTES, stream>>>(tmA, tmB, p);
+  kernel<<<grid, threads_for(EPI_WARPS), L::BYTES, stream>>>(tmA, tmB, p);
   return cudaGetLastError() == cudaSuccess ? SQ_OK : SQ_ERR_CUDA;
 }
 
@@ -516,7 +562,7 @@ sq_status run_gemm(const GemmRequest &r, const GemmParams &p, cudaStream_t strea
 sq_status launch_gemm(const GemmRequest &r, cudaStream_t stream) {
   if (r.M == 0) return SQ_OK;
   const bool segk = r.seg.mode == SQ_SEG_INPUT && r.seg.S > 1;
-  int BN = segk ? 128 : 256;
+  int BN = segk ? 128 : SQ_GEMM_BN_ONE_SEG;
   if (r.seg.G > 1) {
     for (int j = 0; j < r.seg.n_seg; ++j)
       if ((r.seg.off[j + 1] - r.seg.off[j]) % 256 != 0) BN = 128;
@@ -556,18 +602,18 @@ sq_status launch_gemm(const GemmRequest &r, cudaStream_t stream) {
   p.status = r.status;
 
   if (r.out_kind == OUT_S32) {
-    if (segk) return run_gemm<128, 4, OUT_S32, true>(r, p, stream);
-    return BN == 256 ? run_gemm<256, 3, OUT_S32, false>(r, p, stream)
-                     : run_gemm<128, 4, OUT_S32, false>(r, p, stream);
+    if (segk) return run_gemm<128, 4, OUT_S32, true, 16>(r, p, stream);
+    return BN == 256 ? run_gemm<256, 3, OUT_S32, false, 8>(r, p, stream)
+                     : run_gemm<128, 4, OUT_S32, false, 8>(r, p, stream);
   }
   if (r.out_kind == OUT_F32) {
-    if (segk) return run_gemm<128, 4, OUT_F32, true>(r, p, stream);
-    return BN == 256 ? run_gemm<256, 3, OUT_F32, false>(r, p, stream)
-                     : run_gemm<128, 4, OUT_F32, false>(r, p, stream);
+    if (segk) return run_gemm<128, 4, OUT_F32, true, 16>(r, p, stream);
+    return BN == 256 ? run_gemm<256, 3, OUT_F32, false, 8>(r, p, stream)
+                     : run_gemm<128, 4, OUT_F32, false, 8>(r, p, stream);
   }
-  if (segk) return run_gemm<128, 4, OUT_BF16, true>(r, p, stream);
-  return BN == 256 ? run_gemm<256, 3, OUT_BF16, false>(r, p, stream)
-                   : run_gemm<128, 4, OUT_BF16, false>(r, p, stream);
+  if (segk) return run_gemm<128, 4, OUT_BF16, true, 16>(r, p, stream);
+  return BN == 256 ? run_gemm<256, 3, OUT_BF16, false, 8>(r, p, stream)
+                   : run_gemm<128, 4, OUT_BF16, false, 8>(r, p, stream);
 }
 
 }  // namespace sq

@@ -10,6 +10,7 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include "sm100.cuh"
 #include "sq_internal.h"
 
 namespace sq {
@@ -18,7 +19,10 @@ namespace {
 constexpr int kColsPerThread = 8;                     // one 16-byte bf16 load
 constexpr int kWarpCols = 32 * kColsPerThread;        // 256 channels per warp row
 constexpr int kRowsPerBlock = 8;                      // warps per block
-constexpr int kUnroll = 3;                            // rows in flight per thread
+constexpr int kQRows = 32;                            // rows per staged tile
+constexpr int kQStages = 4;                           // tiles in flight per block
+constexpr int kQTileBytes = kQRows * kWarpCols * 2;   // 16 KB of bf16
+constexpr uint64_t kQuantWaitNs = 2000000000ull;      // bounded wait on a tile: 2 s
 
 __device__ __forceinline__ float bf16_bits_to_f32(uint32_t h) {
   return __uint_as_float(h << 16);
@@ -83,114 +87,183 @@ __global__ void calib_finalize_kernel(float *s_act, int n) {
 }
 
 // ---------------------------------------------------- activation quantize
-// q = rne(v) saturated to [-128, 127] (cvt.rni.sat.s8.f32; NaN gives 0).
-__device__ __forceinline__ uint32_t f2s8_rn_sat(float v) {
-  uint32_t r;
-  asm("cvt.rni.sat.s8.f32 %0, %1;" : "=r"(r) : "f"(v));
+// sat(a * b) clamped to [0, 1]; NaN gives +0.
+__device__ __forceinline__ float mul_sat(float a, float b) {
+  float r;
+  asm("fma.rn.sat.f32 %0, %1, %2, 0f00000000;" : "=f"(r) : "f"(a), "f"(b));
   return r;
 }
 
-// Packs the low bytes of four codes into one word (byte j = code j).
-__device__ __forceinline__ uint32_t pack4(uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+// Packs the low bytes of four words into one word (byte j = low byte of word j).
+__device__ __forceinline__ uint32_t pack4_lo(uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
   return __byte_perm(__byte_perm(a, b, 0x0040), __byte_perm(c, d, 0x0040), 0x5410);
 }
 
-// Eight channels x of one row -> X^+ and X^- codes, 8 bytes each.  One signed
-// code per element, q = sat(rne(x * (x >= 0 ? m+ : m-))): its sign is the
-// sign of x, so X^+ = max(q, 0) and X^- = min(q, 0) byte-wise.  This is the
-// case-wise Q_dual with the clamps of the reference: x >= 0 (including -0.0)
-// gives a code in [0, 127], x < 0 a code in [-128, 0], NaN gives 0 in both.
-__device__ __forceinline__ void dualscale8(const float (&x)[8], const float (&mp)[8],
-                                           const float (&mm)[8], uint2 &plus, uint2 &minus) {
-  uint32_t q[8];
-#pragma unroll
-  for (int j = 0; j < 8; ++j) q[j] = f2s8_rn_sat(__fmul_rn(x[j], x[j] >= 0.0f ? mp[j] : mm[j]));
-  const uint32_t w0 = pack4(q[0], q[1], q[2], q[3]);
-  const uint32_t w1 = pack4(q[4], q[5], q[6], q[7]);
-  plus = make_uint2(__vmaxs4(w0, 0u), __vmaxs4(w1, 0u));
-  minus = make_uint2(__vmins4(w0, 0u), __vmins4(w1, 0u));
+// Bit patterns of fl(1.5 * 2^23 + k * u0) and fl(1.5 * 2^23 + k * u1), one packed
+// FMA (f32x2) for both; the low byte of each is rne(k * u) for |k u| <= 128.
+__device__ __forceinline__ void round2(float u0, float u1, float k, uint32_t &r0, uint32_t &r1) {
+  uint64_t a, b, c, d;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(a) : "f"(u0), "f"(u1));
+  asm("mov.b64 %0, {%1, %1};" : "=l"(b) : "f"(k));
+  asm("mov.b64 %0, {%1, %1};" : "=l"(c) : "f"(12582912.0f));
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  asm("mov.b64 {%0, %1}, %2;" : "=r"(r0), "=r"(r1) : "l"(d));
 }
 
-// Block: 32 x 8 threads.  blockIdx.x owns 256 consecutive channels; every
-// warp streams whole rows of them (512 contiguous bytes per row), kUnroll rows
-// in flight per thread.  With one activation group the folded multipliers
-// m+- = 1/(d*s+-) of the thread's eight channels live in registers; with G
-// groups they sit in shared memory, [G][2][256] floats.
+// Eight channels x of one row -> X^+ and X^- codes, 8 bytes each, with the
+// multipliers pre-scaled by 2^-7: p7 = m+ / 128, n7 = -m- / 128.
+//   u+ = sat(x * p7) = clamp(fl(x * m+), 0, 128) / 128   (power-of-two scaling
+//        commutes with rounding, so this is exact; x < 0 and NaN give 0)
+//   q+ = rne(128 u+): the FP add of 1.5 * 2^23 rounds to nearest even and the
+//        code is the low byte of the sum's bits; 128 is then lowered to 127.
+//   u- = sat(x * n7) = clamp(-fl(x * m-), 0, 128) / 128, q- = -rne(128 u-).
+// This is the case-wise Q_dual with the reference's clamps: x >= 0 (including
+// -0.0) gives a code in [0, 127] and none in X^-, x < 0 the reverse, NaN 0.
+__device__ __forceinline__ void dualscale8(const float (&x)[8], const float (&p7)[8],
+                                           const float (&n7)[8], uint2 &plus, uint2 &minus) {
+  uint32_t qp[8], qm[8];
+#pragma unroll
+  for (int j = 0; j < 8; j += 2) {
+    // rne(128 u) + 1.5 * 2^23 for two channels per packed FMA
+    round2(mul_sat(x[j], p7[j]), mul_sat(x[j + 1], p7[j + 1]), 128.0f, qp[j], qp[j + 1]);
+    round2(mul_sat(x[j], n7[j]), mul_sat(x[j + 1], n7[j + 1]), -128.0f, qm[j], qm[j + 1]);
+  }
+  plus = make_uint2(__vminu4(pack4_lo(qp[0], qp[1], qp[2], qp[3]), 0x7F7F7F7Fu),
+                    __vminu4(pack4_lo(qp[4], qp[5], qp[6], qp[7]), 0x7F7F7F7Fu));
+  minus = make_uint2(pack4_lo(qm[0], qm[1], qm[2], qm[3]), pack4_lo(qm[4], qm[5], qm[6], qm[7]));
+}
+
+// Work unit = one tile of 32 rows x 256 channels.  Units are numbered column
+// block major and every block takes one contiguous range of them, so the grid
+// is balanced to within one unit and a block changes column block (and
+// recomputes its folded multipliers m+- = 1/(d*s+-)) at most a few times.
+// Thread 0 keeps kQStages tiles in flight with 2D TMA copies into shared
+// memory; every warp then takes whole rows of the staged tile (lane = 8
+// channels, one conflict-free 16-byte shared load) and writes 8 bytes per plane
+// per row, 256 contiguous bytes per warp.  With one activation group a thread's
+// multipliers live in registers; with G groups they sit in shared memory,
+// [G][2][256] floats.  Multipliers are kept as m+/128 and -m-/128 (see
+// dualscale8).
 template <bool kOneGroup>
-__global__ void __launch_bounds__(256, 4) quant_act_kernel(const uint16_t *__restrict__ x,
-                                                        int64_t M, int64_t K, int64_t ldx,
-                                                        const float *__restrict__ d,
-                                                        const float *__restrict__ s_act,
-                                                        SegParams seg,
-                                                        int8_t *__restrict__ planes) {
-  extern __shared__ float mtab[];  // [G][2][kWarpCols] when G > 1
-  const int G = kOneGroup ? 1 : seg.G;
-  const int64_t cblk = static_cast<int64_t>(blockIdx.x) * kWarpCols;
-  const int64_t c0 = cblk + threadIdx.x * kColsPerThread;
-  float mp_r[8], mm_r[8];
+__device__ __forceinline__ void load_multipliers(int64_t cblk, int64_t K, const float *d,
+                                                 const float *s_act, const SegParams &seg,
+                                                 float (&mp_r)[8], float (&mm_r)[8],
+                                                 float *mtab) {
+  const int lane = threadIdx.x & 31;
   if (kOneGroup) {
+    const int64_t c0 = cblk + lane * kColsPerThread;
     if (c0 < K) {
       const int i = (seg.mode == SQ_SEG_INPUT) ? seg_index(seg.off, seg.n_seg, c0) : 0;
       const float sp = s_act[i * 2 + 0], sm = s_act[i * 2 + 1];
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
         const float dv = d ? d[c0 + j] : 1.0f;
-        mp_r[j] = __fdiv_rn(1.0f, __fmul_rn(dv, sp));
-        mm_r[j] = __fdiv_rn(1.0f, __fmul_rn(dv, sm));
+        mp_r[j] = __fdiv_rn(1.0f, __fmul_rn(dv, sp)) * 0.0078125f;
+        mm_r[j] = __fdiv_rn(1.0f, __fmul_rn(dv, sm)) * -0.0078125f;
       }
     }
   } else {
-    const int tid = threadIdx.y * 32 + threadIdx.x;
-    for (int t = tid; t < G * kWarpCols; t += 256) {
+    for (int t = threadIdx.x; t < seg.G * kWarpCols; t += blockDim.x) {
       const int g = t / kWarpCols, cl = t % kWarpCols;
       const int64_t c = cblk + cl;
       float mp = 0.0f, mm = 0.0f;
       if (c < K) {
         const int i = (seg.mode == SQ_SEG_INPUT) ? seg_index(seg.off, seg.n_seg, c) : 0;
         const float dv = d ? d[g * K + c] : 1.0f;
-        mp = __fdiv_rn(1.0f, __fmul_rn(dv, s_act[(g * seg.S + i) * 2 + 0]));
-        mm = __fdiv_rn(1.0f, __fmul_rn(dv, s_act[(g * seg.S + i) * 2 + 1]));
+        mp = __fdiv_rn(1.0f, __fmul_rn(dv, s_act[(g * seg.S + i) * 2 + 0])) * 0.0078125f;
+        mm = __fdiv_rn(1.0f, __fmul_rn(dv, s_act[(g * seg.S + i) * 2 + 1])) * -0.0078125f;
       }
       mtab[(g * 2 + 0) * kWarpCols + cl] = mp;
       mtab[(g * 2 + 1) * kWarpCols + cl] = mm;
     }
-    __syncthreads();
   }
-  if (c0 >= K) return;
-  const int64_t plane_stride = M * K;
-  const int64_t row_step = static_cast<int64_t>(gridDim.y) * kRowsPerBlock * kUnroll;
-  for (int64_t base = static_cast<int64_t>(blockIdx.y) * kRowsPerBlock * kUnroll + threadIdx.y;
-       base < M; base += row_step) {
-    uint4 v[kUnroll];
-#pragma unroll
-    for (int u = 0; u < kUnroll; ++u) {
-      const int64_t r = base + u * kRowsPerBlock;
-      if (r < M) v[u] = __ldcs(reinterpret_cast<const uint4 *>(x + r * ldx + c0));
+}
+
+template <bool kOneGroup>
+__global__ void __launch_bounds__(256, 3) quant_act_kernel(const __grid_constant__ CUtensorMap tmX,
+                                                           int64_t M, int64_t K,
+                                                           const float *__restrict__ d,
+                                                           const float *__restrict__ s_act,
+                                                           SegParams seg,
+                                                           int8_t *__restrict__ planes,
+                                                           int *status) {
+  extern __shared__ __align__(128) uint8_t qsmem[];
+  uint64_t *full = reinterpret_cast<uint64_t *>(qsmem + kQStages * kQTileBytes);
+  float *mtab = reinterpret_cast<float *>(full + kQStages);
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int G = kOneGroup ? 1 : seg.G;
+  const int64_t n_rt = (M + kQRows - 1) / kQRows;                 // row tiles
+  const int64_t n_units = n_rt * ((K + kWarpCols - 1) / kWarpCols);
+  const int64_t u_begin = n_units * blockIdx.x / gridDim.x;
+  const int64_t u_end = n_units * (blockIdx.x + 1) / gridDim.x;
+
+  if (tid == 0) {
+    for (int st = 0; st < kQStages; ++st) mbar_init(&full[st], 1);
+    fence_mbar_init();
+    prefetch_tmap(&tmX);
+    for (int st = 0; st < kQStages && u_begin + st < u_end; ++st) {
+      const int64_t u = u_begin + st;
+      mbar_arrive_expect_tx(&full[st], kQTileBytes);
+      tma_load_2d(qsmem + st * kQTileBytes, &tmX, &full[st],
+                  static_cast<int32_t>((u / n_rt) * kWarpCols),
+                  static_cast<int32_t>((u % n_rt) * kQRows));
     }
-#pragma unroll
-    for (int u = 0; u < kUnroll; ++u) {
-      const int64_t r = base + u * kRowsPerBlock;
-      if (r >= M) break;
-      float xv[8];
-      unpack8(v[u], xv);
-      for (int g = 0; g < G; ++g) {
-        if (!kOneGroup) {
-          const float4 *mp4 = reinterpret_cast<const float4 *>(
-              mtab + (g * 2 + 0) * kWarpCols + threadIdx.x * kColsPerThread);
-          const float4 *mm4 = reinterpret_cast<const float4 *>(
-              mtab + (g * 2 + 1) * kWarpCols + threadIdx.x * kColsPerThread);
-          const float4 a = mp4[0], b = mp4[1], c = mm4[0], e = mm4[1];
-          mp_r[0] = a.x; mp_r[1] = a.y; mp_r[2] = a.z; mp_r[3] = a.w;
-          mp_r[4] = b.x; mp_r[5] = b.y; mp_r[6] = b.z; mp_r[7] = b.w;
-          mm_r[0] = c.x; mm_r[1] = c.y; mm_r[2] = c.z; mm_r[3] = c.w;
-          mm_r[4] = e.x; mm_r[5] = e.y; mm_r[6] = e.z; mm_r[7] = e.w;
+  }
+  float mp_r[8], mm_r[8];
+  int64_t cb = -1;
+  const int64_t plane_stride = M * K;
+  int it = 0;
+  for (int64_t u = u_begin; u < u_end; ++u, ++it) {
+    const int64_t ucb = u / n_rt;
+    if (ucb != cb) {
+      if (!kOneGroup) __syncthreads();  // nobody reads the previous table any more
+      cb = ucb;
+      load_multipliers<kOneGroup>(cb * kWarpCols, K, d, s_act, seg, mp_r, mm_r, mtab);
+      __syncthreads();  // barriers initialised, table written
+    }
+    const int st = it % kQStages;
+    if (!mbar_wait(&full[st], (it / kQStages) & 1, kQuantWaitNs)) {
+      atomicExch(status, static_cast<int>(SQ_ERR_DEVICE_TIMEOUT));
+      return;
+    }
+    const uint16_t *tile = reinterpret_cast<const uint16_t *>(qsmem + st * kQTileBytes);
+    const int64_t c0 = cb * kWarpCols + lane * kColsPerThread;
+    const int64_t r_base = (u % n_rt) * kQRows;
+    if (c0 < K) {
+#pragma unroll 2
+      for (int rr = warp; rr < kQRows; rr += 8) {
+        const int64_t r = r_base + rr;
+        if (r >= M) break;
+        const uint4 v = *reinterpret_cast<const uint4 *>(tile + rr * kWarpCols + lane * kColsPerThread);
+        float xv[8];
+        unpack8(v, xv);
+        for (int g = 0; g < G; ++g) {
+          if (!kOneGroup) {
+            const float4 *mp4 = reinterpret_cast<const float4 *>(
+                mtab + (g * 2 + 0) * kWarpCols + lane * kColsPerThread);
+            const float4 *mm4 = reinterpret_cast<const float4 *>(
+                mtab + (g * 2 + 1) * kWarpCols + lane * kColsPerThread);
+            const float4 a = mp4[0], b = mp4[1], c = mm4[0], e = mm4[1];
+            mp_r[0] = a.x; mp_r[1] = a.y; mp_r[2] = a.z; mp_r[3] = a.w;
+            mp_r[4] = b.x; mp_r[5] = b.y; mp_r[6] = b.z; mp_r[7] = b.w;
+            mm_r[0] = c.x; mm_r[1] = c.y; mm_r[2] = c.z; mm_r[3] = c.w;
+            mm_r[4] = e.x; mm_r[5] = e.y; mm_r[6] = e.z; mm_r[7] = e.w;
+          }
+          uint2 pk, nk;
+          dualscale8(xv, mp_r, mm_r, pk, nk);
+          int8_t *dst = planes + (static_cast<int64_t>(g) * 2) * plane_stride + r * K + c0;
+          *reinterpret_cast<uint2 *>(dst) = pk;
+          *reinterpret_cast<uint2 *>(dst + plane_stride) = nk;
         }
-        uint2 pk, nk;
-        dualscale8(xv, mp_r, mm_r, pk, nk);
-        int8_t *dst = planes + (static_cast<int64_t>(g) * 2) * plane_stride + r * K + c0;
-        __stcs(reinterpret_cast<uint2 *>(dst), pk);
-        __stcs(reinterpret_cast<uint2 *>(dst + plane_stride), nk);
       }
+    }
+    __syncthreads();  // every warp is done with stage st
+    if (tid == 0 && u + kQStages < u_end) {
+      const int64_t un = u + kQStages;
+      mbar_arrive_expect_tx(&full[st], kQTileBytes);
+      tma_load_2d(qsmem + st * kQTileBytes, &tmX, &full[st],
+                  static_cast<int32_t>((un / n_rt) * kWarpCols),
+                  static_cast<int32_t>((un % n_rt) * kQRows));
     }
   }
 }
@@ -273,30 +346,42 @@ cudaError_t launch_calibrate_act(const uint16_t *x, int64_t M, int64_t K, int64_
   return cudaGetLastError();
 }
 
-cudaError_t launch_quantize_act(const uint16_t *x, int64_t M, int64_t K, int64_t ldx,
-                                const float *d, const float *s_act, const SegParams &seg,
-                                int8_t *planes, cudaStream_t stream) {
-  if (M == 0) return cudaSuccess;
-  const int gx = static_cast<int>((K + kWarpCols - 1) / kWarpCols);
-  const int64_t row_groups = (M + kRowsPerBlock * kUnroll - 1) / (kRowsPerBlock * kUnroll);
-  // 8 resident blocks of 256 threads per SM fill its 2048 thread slots.
-  int64_t gy = (static_cast<int64_t>(num_sms()) * 8 + gx - 1) / gx;
-  if (gy > row_groups) gy = row_groups;
-  if (gy < 1) gy = 1;
-  const dim3 grid(gx, static_cast<unsigned>(gy)), block(32, kRowsPerBlock);
+sq_status launch_quantize_act(const uint16_t *x, int64_t M, int64_t K, int64_t ldx,
+                              const float *d, const float *s_act, const SegParams &seg,
+                              int8_t *planes, int *status, cudaStream_t stream) {
+  if (M == 0) return SQ_OK;
+  EncodeTiledFn enc = tensor_map_encoder();
+  if (enc == nullptr) return SQ_ERR_CUDA;
+  CUtensorMap tmX;
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(M)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(ldx) * 2};
+  const cuuint32_t box[2] = {kWarpCols, kQRows};
+  const cuuint32_t estr[2] = {1, 1};
+  if (enc(&tmX, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t *>(x), dims, strides,
+          box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return SQ_ERR_CUDA;
+  const int64_t n_units = ((M + kQRows - 1) / kQRows) * ((K + kWarpCols - 1) / kWarpCols);
+  // Three resident blocks per SM, each keeping kQStages tiles in flight; the
+  // units are split evenly over exactly that many blocks.
+  int64_t nblk = static_cast<int64_t>(num_sms()) * 3;
+  if (nblk > n_units) nblk = n_units;
+  const size_t smem = kQStages * kQTileBytes + kQStages * sizeof(uint64_t) +
+                      (seg.G > 1 ? sizeof(float) * 2 * kWarpCols * seg.G : 0);
+  const dim3 grid(static_cast<unsigned>(nblk));
+  cudaError_t e;
   if (seg.G == 1) {
-    quant_act_kernel<true><<<grid, block, 0, stream>>>(x, M, K, ldx, d, s_act, seg, planes);
-    return cudaGetLastError();
+    e = cudaFuncSetAttribute(quant_act_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(smem));
+    if (e != cudaSuccess) return SQ_ERR_CUDA;
+    quant_act_kernel<true><<<grid, 256, smem, stream>>>(tmX, M, K, d, s_act, seg, planes, status);
+  } else {
+    e = cudaFuncSetAttribute(quant_act_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(smem));
+    if (e != cudaSuccess) return SQ_ERR_CUDA;
+    quant_act_kernel<false><<<grid, 256, smem, stream>>>(tmX, M, K, d, s_act, seg, planes, status);
   }
-  const size_t smem = sizeof(float) * 2 * kWarpCols * seg.G;
-  if (smem > 48 * 1024) {
-    cudaError_t e = cudaFuncSetAttribute(quant_act_kernel<false>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(smem));
-    if (e != cudaSuccess) return e;
-  }
-  quant_act_kernel<false><<<grid, block, smem, stream>>>(x, M, K, ldx, d, s_act, seg, planes);
-  return cudaGetLastError();
+  return cudaGetLastError() == cudaSuccess ? SQ_OK : SQ_ERR_CUDA;
 }
 
 cudaError_t launch_quantize_weight(const uint16_t *w, int64_t N, int64_t K, const float *d,

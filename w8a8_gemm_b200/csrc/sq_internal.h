@@ -1,6 +1,7 @@
 // sq_internal.h -- declarations shared by the library's own translation units
 // (kernels and the C-ABI layer).  Not installed; not used by anything else.
 #pragma once
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -28,9 +29,9 @@ __host__ __device__ inline int seg_index(const int32_t *off, int n_seg, int64_t 
 cudaError_t launch_calibrate_act(const uint16_t *x, int64_t M, int64_t K, int64_t ldx,
                                  const float *d, const SegParams &seg, float *s_act,
                                  cudaStream_t stream);
-cudaError_t launch_quantize_act(const uint16_t *x, int64_t M, int64_t K, int64_t ldx,
-                                const float *d, const float *s_act, const SegParams &seg,
-                                int8_t *planes, cudaStream_t stream);
+sq_status launch_quantize_act(const uint16_t *x, int64_t M, int64_t K, int64_t ldx,
+                              const float *d, const float *s_act, const SegParams &seg,
+                              int8_t *planes, int *status, cudaStream_t stream);
 cudaError_t launch_quantize_weight(const uint16_t *w, int64_t N, int64_t K, const float *d,
                                    const SegParams &seg, int8_t *wq, float *s_w,
                                    cudaStream_t stream);
@@ -56,5 +57,13 @@ sq_status launch_gemm(const GemmRequest &req, cudaStream_t stream);
 
 // Device address of the library's error word on the current device.
 int *device_status_word();
+
+// cuTensorMapEncodeTiled, resolved through the runtime (no link-time libcuda).
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                  const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                  const cuuint32_t *, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion,
+                                  CUtensorMapFloatOOBfill);
+EncodeTiledFn tensor_map_encoder();  // nullptr if the driver lacks it
 
 }  // namespace sq
