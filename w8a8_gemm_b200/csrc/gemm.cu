@@ -400,21 +400,32 @@ __global__ void __launch_bounds__(threads_for(EPI_WARPS), 1)
             }
           } else if constexpr (!SEGK) {
             // One K-segment: the fp32 operations in the reference order
-            //   t = s+ f(A+) + s- f(A-);  y = s_w t + bias.
+            //   t = s+ f(A+) + s- f(A-);  y = s_w t + bias,
+            // two columns per packed instruction (each lane rounds once per
+            // operation, exactly as the scalar sequence does).
             if (m < p.M) {
               const float4 *sw4 = reinterpret_cast<const float4 *>(cst + c * 32);
               const float4 *b4 = reinterpret_cast<const float4 *>(cst + HALF + c * 32);
+              const uint64_t sp2 = f2pack(sp, sp), sm2 = f2pack(sm, sm);
+              const uint64_t zero2 = f2pack(0.0f, 0.0f), one2 = f2pack(1.0f, 1.0f);
               float v[32];
 #pragma unroll
               for (int q = 0; q < 8; ++q) {
                 const float4 w = sw4[q], b = b4[q];
-                const float wv[4] = {w.x, w.y, w.z, w.w}, bv[4] = {b.x, b.y, b.z, b.w};
 #pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                  const int j = 4 * q + e;
-                  const float tp = __fmul_rn(sp, __int2float_rn(static_cast<int32_t>(ap[j])));
-                  const float tm = __fmul_rn(sm, __int2float_rn(static_cast<int32_t>(am[j])));
-                  v[j] = __fadd_rn(__fmul_rn(wv[e], __fadd_rn(tp, tm)), bv[e]);
+                for (int h = 0; h < 2; ++h) {
+                  const int j = 4 * q + 2 * h;
+                  const uint64_t fp = f2pack(__int2float_rn(static_cast<int32_t>(ap[j])),
+                                             __int2float_rn(static_cast<int32_t>(ap[j + 1])));
+                  const uint64_t fm = f2pack(__int2float_rn(static_cast<int32_t>(am[j])),
+                                             __int2float_rn(static_cast<int32_t>(am[j + 1])));
+                  // Each step is one packed FMA with a zero addend or a unit
+                  // factor, i.e. exactly one rounding of the scalar product
+                  // or sum, and nothing the compiler could contract further.
+                  const uint64_t t = ffma2(one2, ffma2(sp2, fp, zero2), ffma2(sm2, fm, zero2));
+                  const uint64_t u = ffma2(h ? f2pack(w.z, w.w) : f2pack(w.x, w.y), t, zero2);
+                  const uint64_t y = ffma2(one2, u, h ? f2pack(b.z, b.w) : f2pack(b.x, b.y));
+                  f2unpack(y, v[j], v[j + 1]);
                 }
               }
               store_row_chunk<OUT>(p, m, n0, v);
