@@ -53,7 +53,6 @@ struct GemmParams {
   int32_t num_n_tiles, num_tiles, num_kb;
   int32_t G, S;
   int32_t n_seg_out;                // output segments mapped to groups (G > 1)
-  int32_t exact_small_acc;          // every K-segment <= 256 wide: |acc| < 2^22
   int32_t k_off[SQ_MAX_SEGMENTS + 1];
   int32_t n_off[SQ_MAX_SEGMENTS + 1];
   const float *s_w;
@@ -113,18 +112,6 @@ __device__ __forceinline__ uint64_t ffma2(uint64_t a, uint64_t b, uint64_t c) {
   asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
   return d;
 }
-__device__ __forceinline__ uint64_t fadd2(uint64_t a, uint64_t b) {
-  uint64_t d;
-  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-  return d;
-}
-// Two accumulators (|a| < 2^22) to exact fp32, packed: 0x4B400000 + a is the
-// float 1.5 * 2^23 + a, and one packed subtract removes the offset.
-__device__ __forceinline__ uint64_t i2f_small2(uint32_t a, uint32_t b) {
-  return fadd2(f2pack(__uint_as_float(a + 0x4B400000u), __uint_as_float(b + 0x4B400000u)),
-               f2pack(-12582912.0f, -12582912.0f));
-}
-
 __device__ __forceinline__ float bf16_to_f32(uint16_t h) {
   return __uint_as_float(static_cast<uint32_t>(h) << 16);
 }
@@ -448,21 +435,14 @@ __global__ void __launch_bounds__(threads_for(EPI_WARPS), 1)
               const float4 a = cp4[q], b = cm4[q];
               const int j = 4 * q;
               uint64_t &r0 = run2[c * 8 + 2 * q], &r1 = run2[c * 8 + 2 * q + 1];
-              if (p.exact_small_acc) {
-                r0 = ffma2(f2pack(a.x, a.y), i2f_small2(ap[j], ap[j + 1]), r0);
-                r1 = ffma2(f2pack(a.z, a.w), i2f_small2(ap[j + 2], ap[j + 3]), r1);
-                r0 = ffma2(f2pack(b.x, b.y), i2f_small2(am[j], am[j + 1]), r0);
-                r1 = ffma2(f2pack(b.z, b.w), i2f_small2(am[j + 2], am[j + 3]), r1);
-              } else {
-                const auto cvt2 = [](uint32_t x, uint32_t y) {
-                  return f2pack(__int2float_rn(static_cast<int32_t>(x)),
-                                __int2float_rn(static_cast<int32_t>(y)));
-                };
-                r0 = ffma2(f2pack(a.x, a.y), cvt2(ap[j], ap[j + 1]), r0);
-                r1 = ffma2(f2pack(a.z, a.w), cvt2(ap[j + 2], ap[j + 3]), r1);
-                r0 = ffma2(f2pack(b.x, b.y), cvt2(am[j], am[j + 1]), r0);
-                r1 = ffma2(f2pack(b.z, b.w), cvt2(am[j + 2], am[j + 3]), r1);
-              }
+              const auto cvt2 = [](uint32_t x, uint32_t y) {
+                return f2pack(__int2float_rn(static_cast<int32_t>(x)),
+                              __int2float_rn(static_cast<int32_t>(y)));
+              };
+              r0 = ffma2(f2pack(a.x, a.y), cvt2(ap[j], ap[j + 1]), r0);
+              r1 = ffma2(f2pack(a.z, a.w), cvt2(ap[j + 2], ap[j + 3]), r1);
+              r0 = ffma2(f2pack(b.x, b.y), cvt2(am[j], am[j + 1]), r0);
+              r1 = ffma2(f2pack(b.z, b.w), cvt2(am[j + 2], am[j + 3]), r1);
             }
           }
         }
@@ -589,19 +569,15 @@ sq_status launch_gemm(const GemmRequest &r, cudaStream_t stream) {
   p.G = r.seg.G;
   p.S = r.seg.S;
   p.n_seg_out = (r.seg.mode == SQ_SEG_OUTPUT) ? r.seg.n_seg : 1;
-  p.exact_small_acc = 1;
   for (int i = 0; i <= SQ_MAX_SEGMENTS; ++i) {
     p.k_off[i] = 0;
     p.n_off[i] = 0;
   }
   if (r.seg.mode == SQ_SEG_INPUT) {
     for (int i = 0; i <= r.seg.n_seg; ++i) p.k_off[i] = r.seg.off[i];
-    for (int i = 0; i < r.seg.n_seg; ++i)
-      if (r.seg.off[i + 1] - r.seg.off[i] > 256) p.exact_small_acc = 0;
   } else {
     p.k_off[0] = 0;
     p.k_off[1] = p.K;
-    p.exact_small_acc = p.K <= 256;
   }
   if (r.seg.mode == SQ_SEG_OUTPUT)
     for (int i = 0; i <= r.seg.n_seg; ++i) p.n_off[i] = r.seg.off[i];

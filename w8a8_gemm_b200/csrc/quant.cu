@@ -133,53 +133,52 @@ __device__ __forceinline__ void dualscale8(const float (&x)[8], const float (&p7
   minus = make_uint2(pack4_lo(qm[0], qm[1], qm[2], qm[3]), pack4_lo(qm[4], qm[5], qm[6], qm[7]));
 }
 
-// Work unit = one tile of 32 rows x 256 channels.  Units are numbered column
-// block major and every block takes one contiguous range of them, so the grid
-// is balanced to within one unit and a block changes column block (and
-// recomputes its folded multipliers m+- = 1/(d*s+-)) at most a few times.
+// Work unit = one activation group g and one tile of 32 rows x 256 channels.
+// Units are numbered group-major, then column block, then row tile, and every
+// block takes one contiguous range of them: the grid is balanced to within one
+// unit, and a block changes (group, column block) -- and recomputes its eight
+// channels' folded multipliers m+- = 1/(d*s+-), kept in registers as m+/128 and
+// -m-/128 (see dualscale8) -- at most a few times.  With G > 1 every group
+// re-reads the same X tiles, which stay resident in L2 between the passes.
 // Thread 0 keeps kQStages tiles in flight with 2D TMA copies into shared
 // memory; every warp then takes whole rows of the staged tile (lane = 8
 // channels, one conflict-free 16-byte shared load) and writes 8 bytes per plane
-// per row, 256 contiguous bytes per warp.  With one activation group a thread's
-// multipliers live in registers; with G groups they sit in shared memory,
-// [G][2][256] floats.  Multipliers are kept as m+/128 and -m-/128 (see
-// dualscale8).
-template <bool kOneGroup>
-__device__ __forceinline__ void load_multipliers(int64_t cblk, int64_t K, const float *d,
+// per row, 256 contiguous bytes per warp.
+__device__ __forceinline__ void load_multipliers(int g, int64_t c0, int64_t K, const float *d,
                                                  const float *s_act, const SegParams &seg,
-                                                 float (&mp_r)[8], float (&mm_r)[8],
-                                                 float *mtab) {
-  const int lane = threadIdx.x & 31;
-  if (kOneGroup) {
-    const int64_t c0 = cblk + lane * kColsPerThread;
-    if (c0 < K) {
-      const int i = (seg.mode == SQ_SEG_INPUT) ? seg_index(seg.off, seg.n_seg, c0) : 0;
-      const float sp = s_act[i * 2 + 0], sm = s_act[i * 2 + 1];
+                                                 float (&p7)[8], float (&n7)[8]) {
+  if (c0 >= K) return;
+  const int i = (seg.mode == SQ_SEG_INPUT) ? seg_index(seg.off, seg.n_seg, c0) : 0;
+  const float sp = s_act[(g * seg.S + i) * 2 + 0], sm = s_act[(g * seg.S + i) * 2 + 1];
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const float dv = d ? d[c0 + j] : 1.0f;
-        mp_r[j] = __fdiv_rn(1.0f, __fmul_rn(dv, sp)) * 0.0078125f;
-        mm_r[j] = __fdiv_rn(1.0f, __fmul_rn(dv, sm)) * -0.0078125f;
-      }
-    }
-  } else {
-    for (int t = threadIdx.x; t < seg.G * kWarpCols; t += blockDim.x) {
-      const int g = t / kWarpCols, cl = t % kWarpCols;
-      const int64_t c = cblk + cl;
-      float mp = 0.0f, mm = 0.0f;
-      if (c < K) {
-        const int i = (seg.mode == SQ_SEG_INPUT) ? seg_index(seg.off, seg.n_seg, c) : 0;
-        const float dv = d ? d[g * K + c] : 1.0f;
-        mp = __fdiv_rn(1.0f, __fmul_rn(dv, s_act[(g * seg.S + i) * 2 + 0])) * 0.0078125f;
-        mm = __fdiv_rn(1.0f, __fmul_rn(dv, s_act[(g * seg.S + i) * 2 + 1])) * -0.0078125f;
-      }
-      mtab[(g * 2 + 0) * kWarpCols + cl] = mp;
-      mtab[(g * 2 + 1) * kWarpCols + cl] = mm;
-    }
+  for (int j = 0; j < 8; ++j) {
+    const float dv = d ? d[g * K + c0 + j] : 1.0f;
+    p7[j] = __fdiv_rn(1.0f, __fmul_rn(dv, sp)) * 0.0078125f;
+    n7[j] = __fdiv_rn(1.0f, __fmul_rn(dv, sm)) * -0.0078125f;
   }
 }
 
-template <bool kOneGroup>
+// Position of a work unit: group, column block, row tile (row tiles vary fastest).
+struct UnitCursor {
+  int g, cb, rt;
+  __device__ void set(int64_t u, int n_cb, int n_rt) {
+    const int64_t per_group = static_cast<int64_t>(n_cb) * n_rt;
+    g = static_cast<int>(u / per_group);
+    const int64_t rem = u - g * per_group;
+    cb = static_cast<int>(rem / n_rt);
+    rt = static_cast<int>(rem - static_cast<int64_t>(cb) * n_rt);
+  }
+  __device__ void next(int n_cb, int n_rt) {
+    if (++rt == n_rt) {
+      rt = 0;
+      if (++cb == n_cb) {
+        cb = 0;
+        ++g;
+      }
+    }
+  }
+};
+
 __global__ void __launch_bounds__(256, 3) quant_act_kernel(const __grid_constant__ CUtensorMap tmX,
                                                            int64_t M, int64_t K,
                                                            const float *__restrict__ d,
@@ -189,37 +188,39 @@ __global__ void __launch_bounds__(256, 3) quant_act_kernel(const __grid_constant
                                                            int *status) {
   extern __shared__ __align__(128) uint8_t qsmem[];
   uint64_t *full = reinterpret_cast<uint64_t *>(qsmem + kQStages * kQTileBytes);
-  float *mtab = reinterpret_cast<float *>(full + kQStages);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int G = kOneGroup ? 1 : seg.G;
-  const int64_t n_rt = (M + kQRows - 1) / kQRows;                 // row tiles
-  const int64_t n_units = n_rt * ((K + kWarpCols - 1) / kWarpCols);
+  const int n_rt = static_cast<int>((M + kQRows - 1) / kQRows);      // row tiles
+  const int n_cb = static_cast<int>((K + kWarpCols - 1) / kWarpCols);  // column blocks
+  const int64_t n_units = static_cast<int64_t>(n_rt) * n_cb * seg.G;
   const int64_t u_begin = n_units * blockIdx.x / gridDim.x;
   const int64_t u_end = n_units * (blockIdx.x + 1) / gridDim.x;
+  const int n_mine = static_cast<int>(u_end - u_begin);
 
+  UnitCursor fetch;  // next unit to bring in (thread 0 only)
   if (tid == 0) {
     for (int st = 0; st < kQStages; ++st) mbar_init(&full[st], 1);
     fence_mbar_init();
     prefetch_tmap(&tmX);
-    for (int st = 0; st < kQStages && u_begin + st < u_end; ++st) {
-      const int64_t u = u_begin + st;
+    fetch.set(u_begin, n_cb, n_rt);
+    for (int st = 0; st < kQStages && st < n_mine; ++st) {
       mbar_arrive_expect_tx(&full[st], kQTileBytes);
-      tma_load_2d(qsmem + st * kQTileBytes, &tmX, &full[st],
-                  static_cast<int32_t>((u / n_rt) * kWarpCols),
-                  static_cast<int32_t>((u % n_rt) * kQRows));
+      tma_load_2d(qsmem + st * kQTileBytes, &tmX, &full[st], fetch.cb * kWarpCols,
+                  fetch.rt * kQRows);
+      fetch.next(n_cb, n_rt);
     }
   }
-  float mp_r[8], mm_r[8];
-  int64_t cb = -1;
+  __syncthreads();  // barriers initialised
+  UnitCursor cur;
+  cur.set(u_begin, n_cb, n_rt);
+  float p7[8], n7[8];
+  int key_g = -1, key_cb = -1;  // (group, column block) of the multipliers held
   const int64_t plane_stride = M * K;
-  int it = 0;
-  for (int64_t u = u_begin; u < u_end; ++u, ++it) {
-    const int64_t ucb = u / n_rt;
-    if (ucb != cb) {
-      if (!kOneGroup) __syncthreads();  // nobody reads the previous table any more
-      cb = ucb;
-      load_multipliers<kOneGroup>(cb * kWarpCols, K, d, s_act, seg, mp_r, mm_r, mtab);
-      __syncthreads();  // barriers initialised, table written
+  for (int it = 0; it < n_mine; ++it, cur.next(n_cb, n_rt)) {
+    const int64_t c0 = static_cast<int64_t>(cur.cb) * kWarpCols + lane * kColsPerThread;
+    if (cur.g != key_g || cur.cb != key_cb) {
+      key_g = cur.g;
+      key_cb = cur.cb;
+      load_multipliers(cur.g, c0, K, d, s_act, seg, p7, n7);
     }
     const int st = it % kQStages;
     if (!mbar_wait(&full[st], (it / kQStages) & 1, kQuantWaitNs)) {
@@ -227,9 +228,9 @@ __global__ void __launch_bounds__(256, 3) quant_act_kernel(const __grid_constant
       return;
     }
     const uint16_t *tile = reinterpret_cast<const uint16_t *>(qsmem + st * kQTileBytes);
-    const int64_t c0 = cb * kWarpCols + lane * kColsPerThread;
-    const int64_t r_base = (u % n_rt) * kQRows;
+    const int64_t r_base = static_cast<int64_t>(cur.rt) * kQRows;
     if (c0 < K) {
+      int8_t *plus = planes + (static_cast<int64_t>(cur.g) * 2) * plane_stride + c0;
 #pragma unroll 2
       for (int rr = warp; rr < kQRows; rr += 8) {
         const int64_t r = r_base + rr;
@@ -237,33 +238,18 @@ __global__ void __launch_bounds__(256, 3) quant_act_kernel(const __grid_constant
         const uint4 v = *reinterpret_cast<const uint4 *>(tile + rr * kWarpCols + lane * kColsPerThread);
         float xv[8];
         unpack8(v, xv);
-        for (int g = 0; g < G; ++g) {
-          if (!kOneGroup) {
-            const float4 *mp4 = reinterpret_cast<const float4 *>(
-                mtab + (g * 2 + 0) * kWarpCols + lane * kColsPerThread);
-            const float4 *mm4 = reinterpret_cast<const float4 *>(
-                mtab + (g * 2 + 1) * kWarpCols + lane * kColsPerThread);
-            const float4 a = mp4[0], b = mp4[1], c = mm4[0], e = mm4[1];
-            mp_r[0] = a.x; mp_r[1] = a.y; mp_r[2] = a.z; mp_r[3] = a.w;
-            mp_r[4] = b.x; mp_r[5] = b.y; mp_r[6] = b.z; mp_r[7] = b.w;
-            mm_r[0] = c.x; mm_r[1] = c.y; mm_r[2] = c.z; mm_r[3] = c.w;
-            mm_r[4] = e.x; mm_r[5] = e.y; mm_r[6] = e.z; mm_r[7] = e.w;
-          }
-          uint2 pk, nk;
-          dualscale8(xv, mp_r, mm_r, pk, nk);
-          int8_t *dst = planes + (static_cast<int64_t>(g) * 2) * plane_stride + r * K + c0;
-          *reinterpret_cast<uint2 *>(dst) = pk;
-          *reinterpret_cast<uint2 *>(dst + plane_stride) = nk;
-        }
+        uint2 pk, nk;
+        dualscale8(xv, p7, n7, pk, nk);
+        *reinterpret_cast<uint2 *>(plus + r * K) = pk;
+        *reinterpret_cast<uint2 *>(plus + plane_stride + r * K) = nk;
       }
     }
     __syncthreads();  // every warp is done with stage st
-    if (tid == 0 && u + kQStages < u_end) {
-      const int64_t un = u + kQStages;
+    if (tid == 0 && it + kQStages < n_mine) {
       mbar_arrive_expect_tx(&full[st], kQTileBytes);
-      tma_load_2d(qsmem + st * kQTileBytes, &tmX, &full[st],
-                  static_cast<int32_t>((un / n_rt) * kWarpCols),
-                  static_cast<int32_t>((un % n_rt) * kQRows));
+      tma_load_2d(qsmem + st * kQTileBytes, &tmX, &full[st], fetch.cb * kWarpCols,
+                  fetch.rt * kQRows);
+      fetch.next(n_cb, n_rt);
     }
   }
 }
@@ -361,26 +347,18 @@ sq_status launch_quantize_act(const uint16_t *x, int64_t M, int64_t K, int64_t l
           box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
     return SQ_ERR_CUDA;
-  const int64_t n_units = ((M + kQRows - 1) / kQRows) * ((K + kWarpCols - 1) / kWarpCols);
+  const int64_t n_units =
+      ((M + kQRows - 1) / kQRows) * ((K + kWarpCols - 1) / kWarpCols) * seg.G;
   // Three resident blocks per SM, each keeping kQStages tiles in flight; the
   // units are split evenly over exactly that many blocks.
   int64_t nblk = static_cast<int64_t>(num_sms()) * 3;
   if (nblk > n_units) nblk = n_units;
-  const size_t smem = kQStages * kQTileBytes + kQStages * sizeof(uint64_t) +
-                      (seg.G > 1 ? sizeof(float) * 2 * kWarpCols * seg.G : 0);
-  const dim3 grid(static_cast<unsigned>(nblk));
-  cudaError_t e;
-  if (seg.G == 1) {
-    e = cudaFuncSetAttribute(quant_act_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(smem));
-    if (e != cudaSuccess) return SQ_ERR_CUDA;
-    quant_act_kernel<true><<<grid, 256, smem, stream>>>(tmX, M, K, d, s_act, seg, planes, status);
-  } else {
-    e = cudaFuncSetAttribute(quant_act_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(smem));
-    if (e != cudaSuccess) return SQ_ERR_CUDA;
-    quant_act_kernel<false><<<grid, 256, smem, stream>>>(tmX, M, K, d, s_act, seg, planes, status);
-  }
+  const size_t smem = kQStages * kQTileBytes + kQStages * sizeof(uint64_t);
+  if (cudaFuncSetAttribute(quant_act_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(smem)) != cudaSuccess)
+    return SQ_ERR_CUDA;
+  quant_act_kernel<<<static_cast<unsigned>(nblk), 256, smem, stream>>>(tmX, M, K, d, s_act, seg,
+                                                                       planes, status);
   return cudaGetLastError() == cudaSuccess ? SQ_OK : SQ_ERR_CUDA;
 }
 
