@@ -186,6 +186,18 @@ SQ_API sq_status sq_debug_gemm_s32(const int8_t *planes, const int8_t *wq, int64
                             int32_t *acc, sq_stream_t stream);
 
 /*
+ * sq_debug_timeout_probe -- test only: launches one small kernel that waits on
+ * a barrier nothing ever signals, with the library's bounded wait and a limit
+ * of `limit_us` microseconds (1..100000), so that the wait runs out and the
+ * kernel records SQ_ERR_DEVICE_TIMEOUT in the device error word, exactly as a
+ * stalled GEMM or quantize kernel would.  Nothing faults or hangs; the
+ * context stays usable.  Read the result with sq_get_device_status().  (A
+ * verification aid for the failure reporting; it has no counterpart in the
+ * pages.)
+ */
+SQ_API sq_status sq_debug_timeout_probe(uint32_t limit_us, sq_stream_t stream);
+
+/*
  * sq_get_device_status -- synchronises the current device, then returns and
  * clears the library's device-side error word: SQ_OK, or
  * SQ_ERR_DEVICE_TIMEOUT if a kernel's bounded wait on a barrier ran out (the

@@ -80,6 +80,34 @@ def test_every_bf16_value_quantizes_like_oracle():
     assert np.array_equal(planes.cpu().numpy(), ref)
 
 
+@pytest.mark.parametrize("kind", ["positive", "negative", "zero", "nan_and_inf", "mixed"])
+def test_calibration_degenerate_slices_on_gpu(kind):
+    """AMax calibration on the GPU equals the oracle's, bit for bit, including
+    one-sided, all-zero and NaN/Inf slices (R5, R6)."""
+    rng = np.random.default_rng(17)
+    x = rng.standard_normal((5, 64)).astype(np.float32)
+    if kind == "positive":
+        x = np.abs(x)
+    elif kind == "negative":
+        x = -np.abs(x)
+    elif kind == "zero":
+        x = np.zeros_like(x)
+    elif kind == "nan_and_inf":
+        x[0, 3] = np.nan
+        x[2, 7] = np.inf
+        x[4, 9] = -np.inf
+    xt = torch.from_numpy(x).to(torch.bfloat16)
+    bits = xt.view(torch.int16).numpy().view(np.uint16)
+    d = rng.uniform(0.5, 2.0, (1, 64)).astype(np.float32)
+    for seg, mode, off in ((B.Segments(), oracle.MODE_NONE, None),
+                           (B.Segments(B.SQ_SEG_INPUT, [0, 32, 64], 1), oracle.MODE_INPUT,
+                            [0, 32, 64])):
+        ref = oracle.calibrate_act(bits, d, mode, off, 1, 0)
+        s_act = torch.empty(1, seg.S, 2, device="cuda")
+        B.sq_calibrate_act(xt.cuda(), torch.from_numpy(d).cuda(), seg, s_act)
+        assert np.array_equal(s_act.cpu().numpy(), ref)
+
+
 def test_strided_activation_rows():
     """ldx > K: the activation is a column slice of a wider tensor."""
     L = wl.gelu_layer("ld", 70, 96, 40, seed=12, bias=True)
@@ -136,7 +164,8 @@ def test_input_segments_sum_on_gpu():
         assert torch.equal(acc[0], g["acc"][i])
 
 
-FULL = ["c1_tiny_dualscale", "c2_sd35_adanorm", "c3_sd35_attn_out", "c4_sd35_ffn"]
+FULL = ["c1_tiny_dualscale", "c2_sd35_adanorm", "c3_sd35_attn_out", "c4_sd35_ffn",
+        "c5_flux_block"]
 
 
 @pytest.mark.parametrize("cfg", FULL)

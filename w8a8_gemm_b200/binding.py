@@ -25,7 +25,7 @@ SQ_MAX_SEGMENTS = 64
 
 EXPORTED = ("sq_calibrate_act", "sq_quantize_act", "sq_quantize_weight_seg",
             "sq_dualscale_seglinear_gemm", "sq_debug_gemm_s32", "sq_get_device_status",
-            "sq_status_string", "sq_version")
+            "sq_status_string", "sq_version", "sq_debug_timeout_probe")
 
 
 class SegQuantError(RuntimeError):
@@ -87,12 +87,13 @@ def lib() -> ctypes.CDLL:
                                                   i64, seg, p]
         L.sq_debug_gemm_s32.argtypes = [p, p, i64, i64, i64, seg, p, p]
         L.sq_get_device_status.argtypes = []
+        L.sq_debug_timeout_probe.argtypes = [ctypes.c_uint32, p]
         L.sq_status_string.argtypes = [ctypes.c_int]
         L.sq_status_string.restype = ctypes.c_char_p
         L.sq_version.argtypes = []
         for f in (L.sq_calibrate_act, L.sq_quantize_act, L.sq_quantize_weight_seg,
                   L.sq_dualscale_seglinear_gemm, L.sq_debug_gemm_s32, L.sq_get_device_status,
-                  L.sq_version):
+                  L.sq_version, L.sq_debug_timeout_probe):
             f.restype = ctypes.c_int
         _lib = L
     return _lib
@@ -221,6 +222,12 @@ def sq_debug_gemm_s32(planes: torch.Tensor, wq: torch.Tensor, seg: Segments,
 def sq_get_device_status() -> int:
     """Synchronise and return (and clear) the device error word."""
     return lib().sq_get_device_status()
+
+
+def sq_debug_timeout_probe(limit_us: int) -> None:
+    """Test only: a kernel whose bounded barrier wait runs out after limit_us;
+    the timeout lands in the device error word (see sq_get_device_status)."""
+    _check(lib().sq_debug_timeout_probe(int(limit_us), _stream()), "sq_debug_timeout_probe")
 
 
 def sq_version() -> int:

@@ -258,6 +258,14 @@ sq_status sq_debug_gemm_s32(const int8_t *planes, const int8_t *wq, int64_t M, i
                      reinterpret_cast<cudaStream_t>(stream));
 }
 
+sq_status sq_debug_timeout_probe(uint32_t limit_us, sq_stream_t stream) {
+  if (limit_us < 1 || limit_us > 100000) return SQ_ERR_INVALID_ARG;
+  SQ_TRY(check_device());
+  int *status = device_status_word();
+  if (status == nullptr) return SQ_ERR_CUDA;
+  return from_cuda(launch_timeout_probe(limit_us, status, reinterpret_cast<cudaStream_t>(stream)));
+}
+
 sq_status sq_get_device_status(void) {
   SQ_TRY(check_device());
   if (cudaDeviceSynchronize() != cudaSuccess) return SQ_ERR_CUDA;

@@ -55,6 +55,9 @@ struct GemmRequest {
 
 sq_status launch_gemm(const GemmRequest &req, cudaStream_t stream);
 
+// ---- test-only probe (probe.cu) --------------------------------------------
+cudaError_t launch_timeout_probe(uint32_t limit_us, int *status, cudaStream_t stream);
+
 // Device address of the library's error word on the current device.
 int *device_status_word();
 
