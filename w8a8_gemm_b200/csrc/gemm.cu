@@ -36,6 +36,11 @@ namespace {
 
 // Column tile of one-segment layers: 256 (one TMEM buffer, the epilogue runs
 // between tiles) or 128 (two buffers, the epilogue overlaps the next tile).
+// Epilogue warps of one-segment layers (multiple of 4).
+#ifndef SQ_ONESEG_EPI_WARPS
+#define SQ_ONESEG_EPI_WARPS 8
+#endif
+
 #ifndef SQ_GEMM_BN_ONE_SEG
 #define SQ_GEMM_BN_ONE_SEG 256
 #endif
@@ -121,22 +126,22 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<const uint32_t *>(&v);
 }
 
-template <int OUT>
+template <int OUT, int W = 32>
 __device__ __forceinline__ void store_row_chunk(const GemmParams &p, int64_t m, int64_t n0,
-                                                const float (&v)[32]) {
+                                                const float (&v)[W]) {
   if (OUT == OUT_BF16) {
     uint16_t *row = reinterpret_cast<uint16_t *>(p.y) + m * p.ldy;
-    if (n0 + 32 <= p.N) {
+    if (n0 + W <= p.N) {
       uint4 *dst = reinterpret_cast<uint4 *>(row + n0);
 #pragma unroll
-      for (int q = 0; q < 4; ++q)
+      for (int q = 0; q < W / 8; ++q)
         dst[q] = make_uint4(pack_bf16x2(v[8 * q + 0], v[8 * q + 1]),
                             pack_bf16x2(v[8 * q + 2], v[8 * q + 3]),
                             pack_bf16x2(v[8 * q + 4], v[8 * q + 5]),
                             pack_bf16x2(v[8 * q + 6], v[8 * q + 7]));
     } else {
 #pragma unroll
-      for (int j = 0; j < 32; ++j)
+      for (int j = 0; j < W; ++j)
         if (n0 + j < p.N) {
           const __nv_bfloat16 b = __float2bfloat16_rn(v[j]);
           row[n0 + j] = *reinterpret_cast<const uint16_t *>(&b);
@@ -144,17 +149,26 @@ __device__ __forceinline__ void store_row_chunk(const GemmParams &p, int64_t m, 
     }
   } else {
     float *row = reinterpret_cast<float *>(p.y) + m * p.ldy;
-    if (n0 + 32 <= p.N) {
+    if (n0 + W <= p.N) {
       float4 *dst = reinterpret_cast<float4 *>(row + n0);
 #pragma unroll
-      for (int q = 0; q < 8; ++q)
+      for (int q = 0; q < W / 4; ++q)
         dst[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
     } else {
 #pragma unroll
-      for (int j = 0; j < 32; ++j)
+      for (int j = 0; j < W; ++j)
         if (n0 + j < p.N) row[n0 + j] = v[j];
     }
   }
+}
+
+// TMEM columns of one chunk: 16 or 32 per lane.
+template <int CW>
+__device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, uint32_t (&r)[CW]) {
+  if constexpr (CW == 32)
+    tmem_ld_32x32b_x32(taddr, r);
+  else
+    tmem_ld_32x32b_x16(taddr, r);
 }
 
 // One CTA per SM (shared memory allows no more).  Its warps spread over the four
@@ -168,7 +182,10 @@ __global__ void __launch_bounds__(threads_for(EPI_WARPS), 1)
   using L = Smem<BN, STAGES, EPI_WARPS>;
   constexpr int NBUF = L::NBUF;
   constexpr int HALF = L::COLS;      // columns per epilogue warp
-  constexpr int CHUNKS = HALF / 32;  // 32-column TMEM loads per warp per unit
+  constexpr int CHUNKS = HALF / 32;  // 32-column groups (final multi-segment stores)
+  // TMEM chunk of the one-segment epilogue: 32 columns with 8 warps, 16 with
+  // more warps (their register budget is smaller).
+  constexpr int CW = EPI_WARPS >= 16 ? 16 : 32;
   static_assert(EPI_WARPS % 4 == 0 && HALF % 32 == 0, "epilogue split");
   static_assert(NBUF >= 1, "BN too large for TMEM");
 
@@ -367,19 +384,19 @@ __global__ void __launch_bounds__(threads_for(EPI_WARPS), 1)
         tc_fence_after();
         const uint32_t t_plus = tmem_base + lane_addr + buf * 2 * BN + half * HALF;
 #pragma unroll
-        for (int c = 0; c < ((SEGK && OUT != OUT_S32) ? 0 : CHUNKS); ++c) {
-          uint32_t ap[32], am[32];
-          tmem_ld_32x32b_x32(t_plus + c * 32, ap);
-          tmem_ld_32x32b_x32(t_plus + BN + c * 32, am);
+        for (int c = 0; c < ((SEGK && OUT != OUT_S32) ? 0 : HALF / CW); ++c) {
+          uint32_t ap[CW], am[CW];
+          tmem_ld_cols<CW>(t_plus + c * CW, ap);
+          tmem_ld_cols<CW>(t_plus + BN + c * CW, am);
           tmem_ld_wait();
-          const int64_t n0 = nb + c * 32;
+          const int64_t n0 = nb + c * CW;
           if constexpr (OUT == OUT_S32) {
             if (m < p.M) {
               int32_t *accp = reinterpret_cast<int32_t *>(p.y) +
                               ((static_cast<int64_t>(u) * 2) * p.M + m) * p.N;
               int32_t *accm = accp + static_cast<int64_t>(p.M) * p.N;
 #pragma unroll
-              for (int j = 0; j < 32; ++j)
+              for (int j = 0; j < CW; ++j)
                 if (n0 + j < p.N) {
                   accp[n0 + j] = static_cast<int32_t>(ap[j]);
                   accm[n0 + j] = static_cast<int32_t>(am[j]);
@@ -391,13 +408,13 @@ __global__ void __launch_bounds__(threads_for(EPI_WARPS), 1)
             // two columns per packed instruction (each lane rounds once per
             // operation, exactly as the scalar sequence does).
             if (m < p.M) {
-              const float4 *sw4 = reinterpret_cast<const float4 *>(cst + c * 32);
-              const float4 *b4 = reinterpret_cast<const float4 *>(cst + HALF + c * 32);
+              const float4 *sw4 = reinterpret_cast<const float4 *>(cst + c * CW);
+              const float4 *b4 = reinterpret_cast<const float4 *>(cst + HALF + c * CW);
               const uint64_t sp2 = f2pack(sp, sp), sm2 = f2pack(sm, sm);
               const uint64_t zero2 = f2pack(0.0f, 0.0f), one2 = f2pack(1.0f, 1.0f);
-              float v[32];
+              float v[CW];
 #pragma unroll
-              for (int q = 0; q < 8; ++q) {
+              for (int q = 0; q < CW / 4; ++q) {
                 const float4 w = sw4[q], b = b4[q];
 #pragma unroll
                 for (int h = 0; h < 2; ++h) {
@@ -415,7 +432,7 @@ __global__ void __launch_bounds__(threads_for(EPI_WARPS), 1)
                   f2unpack(y, v[j], v[j + 1]);
                 }
               }
-              store_row_chunk<OUT>(p, m, n0, v);
+              store_row_chunk<OUT, CW>(p, m, n0, v);
             }
           }
         }
@@ -590,17 +607,17 @@ sq_status launch_gemm(const GemmRequest &r, cudaStream_t stream) {
 
   if (r.out_kind == OUT_S32) {
     if (segk) return run_gemm<128, 4, OUT_S32, true, 16>(r, p, stream);
-    return BN == 256 ? run_gemm<256, 3, OUT_S32, false, 8>(r, p, stream)
-                     : run_gemm<128, 4, OUT_S32, false, 8>(r, p, stream);
+    return BN == 256 ? run_gemm<256, 3, OUT_S32, false, SQ_ONESEG_EPI_WARPS>(r, p, stream)
+                     : run_gemm<128, 4, OUT_S32, false, SQ_ONESEG_EPI_WARPS>(r, p, stream);
   }
   if (r.out_kind == OUT_F32) {
     if (segk) return run_gemm<128, 4, OUT_F32, true, 16>(r, p, stream);
-    return BN == 256 ? run_gemm<256, 3, OUT_F32, false, 8>(r, p, stream)
-                     : run_gemm<128, 4, OUT_F32, false, 8>(r, p, stream);
+    return BN == 256 ? run_gemm<256, 3, OUT_F32, false, SQ_ONESEG_EPI_WARPS>(r, p, stream)
+                     : run_gemm<128, 4, OUT_F32, false, SQ_ONESEG_EPI_WARPS>(r, p, stream);
   }
   if (segk) return run_gemm<128, 4, OUT_BF16, true, 16>(r, p, stream);
-  return BN == 256 ? run_gemm<256, 3, OUT_BF16, false, 8>(r, p, stream)
-                   : run_gemm<128, 4, OUT_BF16, false, 8>(r, p, stream);
+  return BN == 256 ? run_gemm<256, 3, OUT_BF16, false, SQ_ONESEG_EPI_WARPS>(r, p, stream)
+                   : run_gemm<128, 4, OUT_BF16, false, SQ_ONESEG_EPI_WARPS>(r, p, stream);
 }
 
 }  // namespace sq
