@@ -32,11 +32,12 @@ def lib():
         path = _build.build()
         L = ctypes.CDLL(path)
         p, i64, i32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int
-        L.orc_calibrate_act.argtypes = [p, i64, i64, i64, p, i32, i32, p, i32, i64, p]
-        L.orc_quantize_act.argtypes = [p, i64, i64, i64, p, p, i32, i32, p, i32, i64, p]
+        L.orc_calibrate_act.argtypes = [p, i64, i64, i64, p, i32, i32, p, i32, i64, i32, p]
+        L.orc_quantize_act.argtypes = [p, i64, i64, i64, p, p, i32, i32, p, i32, i64, i32, p]
         L.orc_quantize_weight.argtypes = [p, i64, i64, p, i32, i32, p, i32, p, p]
-        L.orc_gemm_s32.argtypes = [p, p, i64, i64, i64, i32, i32, p, i32, p, i64, p, i32]
-        L.orc_gemm.argtypes = [p, p, p, p, p, i64, i64, i64, i32, i32, p, i32, p, i64, p, i32]
+        L.orc_gemm_s32.argtypes = [p, p, i64, i64, i64, i32, i32, p, i32, i32, p, i64, p, i32]
+        L.orc_gemm.argtypes = [p, p, p, p, p, i64, i64, i64, i32, i32, p, i32, i32, p, i64, p,
+                               i32]
         L.orc_num_threads.argtypes = []
         for f in (L.orc_calibrate_act, L.orc_quantize_act, L.orc_quantize_weight,
                   L.orc_gemm_s32, L.orc_gemm, L.orc_num_threads):
@@ -71,29 +72,32 @@ def num_threads():
     return lib().orc_num_threads()
 
 
-def calibrate_act(x_bits, d=None, mode=MODE_NONE, offsets=None, G=1, N=0):
-    """AMax calibration: returns s_act float32 [G][S][2] = {s+, s-}."""
+def calibrate_act(x_bits, d=None, mode=MODE_NONE, offsets=None, G=1, N=0, single=False):
+    """AMax calibration: returns s_act float32 [G][S][2] = {s+, s-} (equal in
+    single-scale mode)."""
     x = _c(x_bits, np.uint16)
     M, K = x.shape
     off, n_seg, S = _seg(mode, offsets, G, N, K)
     d = _c(d, np.float32)
     out = np.zeros((G, S, 2), np.float32)
     _check(lib().orc_calibrate_act(_ptr(x), M, K, K, _ptr(d), mode, n_seg,
-                                   _ptr(off), G, N, _ptr(out)), "calibrate_act")
+                                   _ptr(off), G, N, int(single), _ptr(out)), "calibrate_act")
     return out
 
 
-def quantize_act(x_bits, s_act, d=None, mode=MODE_NONE, offsets=None, G=1, N=0):
-    """Q_dual of X / d: returns planes int8 [G][2][M][K] (0 = X^+, 1 = X^-)."""
+def quantize_act(x_bits, s_act, d=None, mode=MODE_NONE, offsets=None, G=1, N=0,
+                 single=False):
+    """Q_dual of X / d: returns planes int8 [G][2][M][K] (0 = X^+, 1 = X^-), or
+    [G][1][M][K] holding X^+ + X^- in single-scale mode."""
     x = _c(x_bits, np.uint16)
     M, K = x.shape
     off, n_seg, S = _seg(mode, offsets, G, N, K)
     s = _c(s_act, np.float32)
     assert s.size == G * S * 2
     d = _c(d, np.float32)
-    planes = np.zeros((G, 2, M, K), np.int8)
+    planes = np.zeros((G, 1 if single else 2, M, K), np.int8)
     _check(lib().orc_quantize_act(_ptr(x), M, K, K, _ptr(d), _ptr(s), mode,
-                                  n_seg, _ptr(off), G, N, _ptr(planes)),
+                                  n_seg, _ptr(off), G, N, int(single), _ptr(planes)),
            "quantize_act")
     return planes
 
@@ -121,17 +125,17 @@ def _rows(rows, M):
 
 
 def gemm_s32(planes, wq, mode=MODE_NONE, offsets=None, rows=None, threads=1):
-    """Raw int32 accumulators [S][2][rows][N]."""
+    """Raw int32 accumulators [S][P][rows][N] (P = planes per group)."""
     planes = _c(planes, np.int8)
     wq = _c(wq, np.int8)
-    G, two, M, K = planes.shape
+    G, P, M, K = planes.shape
     N = wq.shape[0]
-    assert two == 2 and wq.shape[1] == K
+    assert P in (1, 2) and wq.shape[1] == K
     off, n_seg, S = _seg(mode, offsets, G, N, K)
     r, nr = _rows(rows, M)
-    acc = np.zeros((S, 2, nr, N), np.int32)
+    acc = np.zeros((S, P, nr, N), np.int32)
     _check(lib().orc_gemm_s32(_ptr(planes), _ptr(wq), M, N, K, mode, n_seg,
-                              _ptr(off), G, _ptr(r), nr, _ptr(acc), threads),
+                              _ptr(off), G, P, _ptr(r), nr, _ptr(acc), threads),
            "gemm_s32")
     return acc
 
@@ -141,9 +145,9 @@ def gemm(planes, wq, s_w, s_act, bias_bits=None, mode=MODE_NONE, offsets=None,
     """Layer output, fp32 epilogue: float32 [rows][N]."""
     planes = _c(planes, np.int8)
     wq = _c(wq, np.int8)
-    G, two, M, K = planes.shape
+    G, P, M, K = planes.shape
     N = wq.shape[0]
-    assert two == 2 and wq.shape[1] == K
+    assert P in (1, 2) and wq.shape[1] == K
     off, n_seg, S = _seg(mode, offsets, G, N, K)
     s_w = _c(s_w, np.float32)
     s_act = _c(s_act, np.float32)
@@ -152,20 +156,20 @@ def gemm(planes, wq, s_w, s_act, bias_bits=None, mode=MODE_NONE, offsets=None,
     r, nr = _rows(rows, M)
     y = np.zeros((nr, N), np.float32)
     _check(lib().orc_gemm(_ptr(planes), _ptr(wq), _ptr(s_w), _ptr(s_act),
-                          _ptr(b), M, N, K, mode, n_seg, _ptr(off), G, _ptr(r),
+                          _ptr(b), M, N, K, mode, n_seg, _ptr(off), G, P, _ptr(r),
                           nr, _ptr(y), threads), "gemm")
     return y
 
 
 def layer(x_bits, w_bits, x_cal_bits, d=None, bias_bits=None, mode=MODE_NONE,
-          offsets=None, G=1, rows=None, threads=1):
+          offsets=None, G=1, rows=None, threads=1, single=False):
     """Whole static pipeline on the CPU: calibrate, quantize both sides, GEMM.
 
     Returns a dict with s_act, planes, wq, s_w and y (fp32 rows)."""
     w = _c(w_bits, np.uint16)
     N = w.shape[0]
-    s_act = calibrate_act(x_cal_bits, d, mode, offsets, G, N)
-    planes = quantize_act(x_bits, s_act, d, mode, offsets, G, N)
+    s_act = calibrate_act(x_cal_bits, d, mode, offsets, G, N, single)
+    planes = quantize_act(x_bits, s_act, d, mode, offsets, G, N, single)
     wq, s_w = quantize_weight(w, d, mode, offsets, G)
     y = gemm(planes, wq, s_w, s_act, bias_bits, mode, offsets, rows, threads)
     return dict(s_act=s_act, planes=planes, wq=wq, s_w=s_w, y=y)

@@ -41,6 +41,11 @@
  *  - Output-segmented layers may carry their own activation parameters per
  *    output segment (a "group" g: its own d and s+/s-, hence its own planes).
  *    G = 1 is the pages' formula with one shared X^.
+ *  - Single-scale mode (the adaptive variant the papernotes page names under
+ *    "Limitations": DualScale only on polarity-asymmetric layers): one step
+ *    s = max(max u, -min u) / 127 for both signs, i.e. the DualScale quantizer
+ *    with s+ = s-, whose two planes are then one: q = q+ + q- in [-128, 127],
+ *    and one integer product A = sum q w.  Planes [G][1][M][K].
  *  - Epilogue in fp32, fixed order: for each K-segment i in ascending order,
  *    t = s+_i * f(A+_i) + s-_i * f(A-_i), y = y + s_w[i][n] * t; bias last.
  *    f is int32 -> fp32 round-to-nearest.
@@ -50,10 +55,11 @@
  *  w      bf16 bits [N][K]            nn.Linear weight (the pages' W^T)
  *  d      fp32 [G][K] or NULL (=1)    SmoothQuant divisor per group
  *  s_act  fp32 [G][S][2]              {s+, s-} per group and K-segment
- *  planes int8 [G][2][M][K]           plane 0 = X^+, plane 1 = X^-
+ *  planes int8 [G][P][M][K]           P = 2: plane 0 = X^+, plane 1 = X^-;
+ *                                     P = 1 (single scale): q = X^+ + X^-
  *  wq     int8 [N][K]                 quantized weight
  *  s_w    fp32 [S][N]                 weight scale per K-segment, per column
- *  acc    int32 [S][2][M][N]          raw accumulators per segment, polarity
+ *  acc    int32 [S][P][M][N]          raw accumulators per segment, polarity
  *  y      fp32 [rows][N]              layer output (fp32 epilogue)
  *
  * Segment description: mode 0 = none, 1 = output-segmented (offsets over N),
@@ -120,7 +126,8 @@ int orc_num_threads(void) {
  * ------------------------------------------------------------------------- */
 int orc_calibrate_act(const uint16_t *x, int64_t M, int64_t K, int64_t ldx,
                       const float *d, int mode, int n_seg,
-                      const int32_t *offsets, int G, int64_t N, float *s_act) {
+                      const int32_t *offsets, int G, int64_t N, int single,
+                      float *s_act) {
   if (orc_check_seg(mode, n_seg, offsets, G, N, K)) return -1;
   int S = (mode == ORC_MODE_INPUT) ? n_seg : 1;
   for (int g = 0; g < G; ++g) {
@@ -139,6 +146,11 @@ int orc_calibrate_act(const uint16_t *x, int64_t M, int64_t K, int64_t ldx,
       }
       float sp = (hi > 0.0f) ? hi / 127.0f : 1.0f;
       float sm = (lo < 0.0f) ? (-lo) / 128.0f : 1.0f;
+      if (single) { /* one symmetric step: the larger side over 127 */
+        float amax = (hi > -lo) ? hi : -lo;
+        sp = (amax > 0.0f) ? amax / 127.0f : 1.0f;
+        sm = sp;
+      }
       s_act[((int64_t)g * S + i) * 2 + 0] = sp;
       s_act[((int64_t)g * S + i) * 2 + 1] = sm;
     }
@@ -151,12 +163,14 @@ int orc_calibrate_act(const uint16_t *x, int64_t M, int64_t K, int64_t ldx,
  * ------------------------------------------------------------------------- */
 int orc_quantize_act(const uint16_t *x, int64_t M, int64_t K, int64_t ldx,
                      const float *d, const float *s_act, int mode, int n_seg,
-                     const int32_t *offsets, int G, int64_t N, int8_t *planes) {
+                     const int32_t *offsets, int G, int64_t N, int single,
+                     int8_t *planes) {
   if (orc_check_seg(mode, n_seg, offsets, G, N, K)) return -1;
   int S = (mode == ORC_MODE_INPUT) ? n_seg : 1;
+  int P = single ? 1 : 2;
   for (int g = 0; g < G; ++g) {
-    int8_t *plus = planes + ((int64_t)g * 2 + 0) * M * K;
-    int8_t *minus = planes + ((int64_t)g * 2 + 1) * M * K;
+    int8_t *plus = planes + ((int64_t)g * P + 0) * M * K;
+    int8_t *minus = single ? plus : planes + ((int64_t)g * P + 1) * M * K;
     for (int64_t m = 0; m < M; ++m) {
       for (int64_t c = 0; c < K; ++c) {
         int i = (S == 1) ? 0 : orc_seg_index(offsets, n_seg, c);
@@ -176,8 +190,12 @@ int orc_quantize_act(const uint16_t *x, int64_t M, int64_t K, int64_t ldx,
           if (v > 127.0f) v = 127.0f;
           qp = (int)rintf(v);
         }
-        plus[m * K + c] = (int8_t)qp;
-        minus[m * K + c] = (int8_t)qm;
+        if (single) {
+          plus[m * K + c] = (int8_t)(qp + qm); /* one of the two is 0 */
+        } else {
+          plus[m * K + c] = (int8_t)qp;
+          minus[m * K + c] = (int8_t)qm;
+        }
       }
     }
   }
@@ -230,9 +248,10 @@ int orc_quantize_weight(const uint16_t *w, int64_t N, int64_t K, const float *d,
  * ------------------------------------------------------------------------- */
 int orc_gemm_s32(const int8_t *planes, const int8_t *wq, int64_t M, int64_t N,
                  int64_t K, int mode, int n_seg, const int32_t *offsets, int G,
-                 const int64_t *rows, int64_t n_rows, int32_t *acc,
+                 int P, const int64_t *rows, int64_t n_rows, int32_t *acc,
                  int n_threads) {
   if (orc_check_seg(mode, n_seg, offsets, G, N, K)) return -1;
+  if (P != 1 && P != 2) return -1;
   int S = (mode == ORC_MODE_INPUT) ? n_seg : 1;
   if (rows == NULL) n_rows = M;
 #ifdef _OPENMP
@@ -244,19 +263,16 @@ int orc_gemm_s32(const int8_t *planes, const int8_t *wq, int64_t M, int64_t N,
     for (int64_t n = 0; n < N; ++n) {
       int g = (mode == ORC_MODE_OUTPUT && G > 1)
                   ? orc_seg_index(offsets, n_seg, n) : 0;
-      const int8_t *xp = planes + (((int64_t)g * 2 + 0) * M + m) * K;
-      const int8_t *xm = planes + (((int64_t)g * 2 + 1) * M + m) * K;
       const int8_t *wn = wq + n * K;
       for (int i = 0; i < S; ++i) {
         int64_t k0 = (S == 1) ? 0 : offsets[i];
         int64_t k1 = (S == 1) ? K : offsets[i + 1];
-        int32_t ap = 0, am = 0;
-        for (int64_t k = k0; k < k1; ++k) {
-          ap += (int32_t)xp[k] * (int32_t)wn[k];
-          am += (int32_t)xm[k] * (int32_t)wn[k];
+        for (int pl = 0; pl < P; ++pl) {
+          const int8_t *xq = planes + (((int64_t)g * P + pl) * M + m) * K;
+          int32_t a = 0;
+          for (int64_t k = k0; k < k1; ++k) a += (int32_t)xq[k] * (int32_t)wn[k];
+          acc[(((int64_t)i * P + pl) * n_rows + r) * N + n] = a;
         }
-        acc[(((int64_t)i * 2 + 0) * n_rows + r) * N + n] = ap;
-        acc[(((int64_t)i * 2 + 1) * n_rows + r) * N + n] = am;
       }
     }
   }
@@ -271,8 +287,10 @@ int orc_gemm_s32(const int8_t *planes, const int8_t *wq, int64_t M, int64_t N,
 int orc_gemm(const int8_t *planes, const int8_t *wq, const float *s_w,
              const float *s_act, const uint16_t *bias, int64_t M, int64_t N,
              int64_t K, int mode, int n_seg, const int32_t *offsets, int G,
-             const int64_t *rows, int64_t n_rows, float *y, int n_threads) {
+             int P, const int64_t *rows, int64_t n_rows, float *y,
+             int n_threads) {
   if (orc_check_seg(mode, n_seg, offsets, G, N, K)) return -1;
+  if (P != 1 && P != 2) return -1;
   int S = (mode == ORC_MODE_INPUT) ? n_seg : 1;
   if (rows == NULL) n_rows = M;
 #ifdef _OPENMP
@@ -284,23 +302,30 @@ int orc_gemm(const int8_t *planes, const int8_t *wq, const float *s_w,
     for (int64_t n = 0; n < N; ++n) {
       int g = (mode == ORC_MODE_OUTPUT && G > 1)
                   ? orc_seg_index(offsets, n_seg, n) : 0;
-      const int8_t *xp = planes + (((int64_t)g * 2 + 0) * M + m) * K;
-      const int8_t *xm = planes + (((int64_t)g * 2 + 1) * M + m) * K;
+      const int8_t *xp = planes + (((int64_t)g * P + 0) * M + m) * K;
+      const int8_t *xm = planes + (((int64_t)g * P + (P - 1)) * M + m) * K;
       const int8_t *wn = wq + n * K;
       float yv = 0.0f;
       for (int i = 0; i < S; ++i) {
         int64_t k0 = (S == 1) ? 0 : offsets[i];
         int64_t k1 = (S == 1) ? K : offsets[i + 1];
-        int32_t ap = 0, am = 0;
-        for (int64_t k = k0; k < k1; ++k) {
-          ap += (int32_t)xp[k] * (int32_t)wn[k];
-          am += (int32_t)xm[k] * (int32_t)wn[k];
-        }
         float sp = s_act[((int64_t)g * S + i) * 2 + 0];
         float sm = s_act[((int64_t)g * S + i) * 2 + 1];
-        float tp = sp * (float)ap;
-        float tm = sm * (float)am;
-        float t = tp + tm;
+        float t;
+        if (P == 2) { /* DualScale: t = s+ f(A+) + s- f(A-) */
+          int32_t ap = 0, am = 0;
+          for (int64_t k = k0; k < k1; ++k) {
+            ap += (int32_t)xp[k] * (int32_t)wn[k];
+            am += (int32_t)xm[k] * (int32_t)wn[k];
+          }
+          float tp = sp * (float)ap;
+          float tm = sm * (float)am;
+          t = tp + tm;
+        } else { /* single scale: t = s f(A) */
+          int32_t a = 0;
+          for (int64_t k = k0; k < k1; ++k) a += (int32_t)xp[k] * (int32_t)wn[k];
+          t = sp * (float)a;
+        }
         yv = yv + s_w[(int64_t)i * N + n] * t;
       }
       if (bias) yv = yv + orc_bf16(bias[n]);

@@ -447,3 +447,87 @@ def test_invalid_segments_rejected():
         oracle.calibrate_act(x, None, MODE_INPUT, [0, 40, 30, 64])
     with pytest.raises(ValueError):
         oracle.calibrate_act(x, None, MODE_INPUT, [0, 32, 60])
+
+
+# ------------------------------------------------ single-scale (adaptive) mode
+def test_worked_single_scale(golden_dir):
+    fx = read_fixture(golden_dir, "single_scale_worked.txt")
+    kv = dict((k, v) for k, v in fx if k != "case")
+    s = oracle.calibrate_act(bf16_bits(np.array([parse_floats(kv["calib"])], np.float32)),
+                             single=True)
+    assert s[0, 0].tolist() == [float(kv["s"])] * 2
+    s2 = oracle.calibrate_act(bf16_bits(np.array([parse_floats(kv["calib2"])], np.float32)),
+                              single=True)
+    assert s2[0, 0].tolist() == [float(kv["s2"])] * 2
+    cases = [v.split() for k, v in fx if k == "case"]
+    xs = np.array([float(c[0]) for c in cases], np.float32)[None]
+    planes = oracle.quantize_act(bf16_bits(xs), s, single=True)
+    assert planes.shape[1] == 1
+    assert planes[0, 0, 0].tolist() == [int(c[1]) for c in cases]
+
+
+def test_single_scale_every_bf16_value():
+    allbits = np.arange(65536, dtype=np.uint32).astype(np.uint16).reshape(256, 256)
+    s_act = np.array([[[1 / 64, 1 / 64]]], np.float32)
+    planes = oracle.quantize_act(allbits, s_act, single=True)
+    xs = bits_to_f32(allbits.reshape(-1))
+    exp = []
+    for x in xs:
+        x = float(x)
+        if math.isnan(x):
+            exp.append(0)
+        elif math.isinf(x):
+            exp.append(127 if x > 0 else -128)
+        else:
+            exp.append(max(-128, min(127, rne_fraction(Fraction(x) * 64))))
+    assert planes[0, 0].reshape(-1).tolist() == exp
+
+
+def test_single_scale_is_dualscale_with_equal_steps():
+    """Single-scale planes are X^+ + X^- of the DualScale quantizer run with
+    s+ = s- = s, and its accumulator is A+ + A- (bit-exact)."""
+    L = wl.outproj_layer("t", 57, 192, 70, 64, seed=21)
+    d = L.d.numpy()
+    xb, wb = wl.bits(L.x), wl.bits(L.w)
+    s1 = oracle.calibrate_act(wl.bits(L.x_cal), d, MODE_INPUT, L.offsets, single=True)
+    assert np.array_equal(s1[..., 0], s1[..., 1])
+    p1 = oracle.quantize_act(xb, s1, d, MODE_INPUT, L.offsets, single=True)
+    p2 = oracle.quantize_act(xb, s1, d, MODE_INPUT, L.offsets)
+    assert np.array_equal(p1[:, 0].astype(np.int16), p2[:, 0].astype(np.int16) + p2[:, 1])
+    wq, _ = oracle.quantize_weight(wb, d, MODE_INPUT, L.offsets)
+    a1 = oracle.gemm_s32(p1, wq, MODE_INPUT, L.offsets)
+    a2 = oracle.gemm_s32(p2, wq, MODE_INPUT, L.offsets)
+    assert np.array_equal(a1[:, 0].astype(np.int64), a2[:, 0].astype(np.int64) + a2[:, 1])
+
+
+@pytest.mark.parametrize("mode,G", [(MODE_NONE, 1), (MODE_INPUT, 1), (MODE_OUTPUT, 3)])
+def test_single_scale_dequantized_matmul(mode, G):
+    rng = np.random.default_rng(31 + mode)
+    M, K, N = 13, 96, 15
+    offsets = {MODE_NONE: None, MODE_INPUT: [0, 32, 64, 96], MODE_OUTPUT: [0, 5, 10, 15]}[mode]
+    x = (rng.standard_normal((M, K)) * rng.uniform(0.1, 3, K)).astype(np.float32)
+    xb = bf16_bits(x)
+    wb = bf16_bits((rng.standard_normal((N, K)) * 0.05).astype(np.float32))
+    bb = bf16_bits((rng.standard_normal(N) * 0.1).astype(np.float32))
+    d = rng.uniform(0.5, 2.0, (G, K)).astype(np.float32)
+    out = oracle.layer(xb, wb, xb, d, bb, mode, offsets, G, single=True)
+    planes, wq, s_w, s_act = out["planes"], out["wq"], out["s_w"], out["s_act"]
+    assert planes.shape[1] == 1
+    koff = offsets if mode == MODE_INPUT else [0, K]
+    noff = offsets if mode == MODE_OUTPUT else [0, N]
+    S = len(koff) - 1
+    y_bf = np.zeros((M, N))
+    mag = np.zeros((M, N))
+    for gi in range(len(noff) - 1):
+        n0, n1 = noff[gi], noff[gi + 1]
+        gg = gi if G > 1 else 0
+        for i in range(S):
+            k0, k1 = koff[i], koff[i + 1]
+            xq = float(s_act[gg, i, 0]) * planes[gg, 0][:, k0:k1].astype(np.float64)
+            wt = s_w[i, n0:n1].astype(np.float64)[:, None] * wq[n0:n1, k0:k1].astype(np.float64)
+            y_bf[:, n0:n1] += xq @ wt.T
+            mag[:, n0:n1] += np.abs(xq @ wt.T)
+    b = bits_to_f32(bb).astype(np.float64)[None]
+    y_bf += b
+    mag += np.abs(b) + 1e-30
+    assert np.all(np.abs(out["y"] - y_bf) <= 1e-6 * mag)
