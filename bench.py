@@ -65,10 +65,12 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
-def layer_units(L):
+def layer_units(L, P=2):
+    """Effective ops 2MNK, executed ops (P products: the X^+ and X^- planes, or
+    one merged plane on the single-scale path) and quantize bytes."""
     eff = 2.0 * L.M * L.N * L.K
-    quant_bytes = 2.0 * L.M * L.K + 2.0 * L.G * L.M * L.K
-    return eff, 2.0 * eff, quant_bytes
+    quant_bytes = 2.0 * L.M * L.K + P * L.G * L.M * L.K
+    return eff, P * eff, quant_bytes
 
 
 def dist_env():
@@ -172,7 +174,7 @@ def traffic_from_profile():
 
 # ------------------------------------------------------------- our path
 class GpuLayer:
-    def __init__(self, L, dev):
+    def __init__(self, L, dev, adaptive=False):
         from w8a8_gemm_b200 import binding as B
         from w8a8_gemm_b200.layer import DualScaleSegLinear
         self.L = L
@@ -180,9 +182,10 @@ class GpuLayer:
                else B.Segments(L.mode, list(L.offsets), L.G))
         d = None if L.d is None else L.d.to(dev)
         bias = None if L.bias is None else L.bias.to(dev)
-        self.lin = DualScaleSegLinear(L.w.to(dev), bias, d, seg, L.x_cal.to(dev))
+        self.lin = DualScaleSegLinear(L.w.to(dev), bias, d, seg, L.x_cal.to(dev),
+                                      adaptive=adaptive)
         self.x = L.x.to(dev)
-        self.planes = torch.empty(L.G, 2, L.M, L.K, dtype=torch.int8, device=dev)
+        self.planes = torch.empty(L.G, self.lin.seg.P, L.M, L.K, dtype=torch.int8, device=dev)
         self.y = torch.empty(L.M, L.N, dtype=torch.bfloat16, device=dev)
 
     def quantize(self):
@@ -198,11 +201,11 @@ def run_ours(args, ws, rank, local):
     from w8a8_gemm_b200 import binding as B
     B.lib()  # fail loudly now if the library is missing
     layers_cpu = wl.config_layers(args.config, seed=0)
-    glayers = [GpuLayer(L, dev) for L in layers_cpu]
+    glayers = [GpuLayer(L, dev, adaptive=args.adaptive) for L in layers_cpu]
     torch.cuda.synchronize()
-    eff_ops = sum(layer_units(g.L)[0] for g in glayers)
-    exe_ops = sum(layer_units(g.L)[1] for g in glayers)
-    qbytes = sum(layer_units(g.L)[2] for g in glayers)
+    eff_ops = sum(layer_units(g.L, g.lin.seg.P)[0] for g in glayers)
+    exe_ops = sum(layer_units(g.L, g.lin.seg.P)[1] for g in glayers)
+    qbytes = sum(layer_units(g.L, g.lin.seg.P)[2] for g in glayers)
     flush = torch.empty(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
     sweep = torch.ones(SWEEP_BYTES // 4, dtype=torch.float32, device=dev)
     sink = torch.empty((), dtype=torch.float32, device=dev)
@@ -260,6 +263,7 @@ def run_ours(args, ws, rank, local):
     res = dict(eff_ops=eff_ops, exe_ops=exe_ops, qbytes=qbytes, ms_step=ms_step,
                gemm_ms=gemm_ms, quant_ms=quant_ms, wall_s=t_wall, clocks=clocks.summary(),
                per_layer=[dict(name=g.L.name, M=g.L.M, N=g.L.N, K=g.L.K, G=g.L.G, S=g.L.S,
+                               P=g.lin.seg.P,
                                quant_us=1e3 * q_ms[i] / args.steps,
                                gemm_us=1e3 * g_ms[i] / args.steps)
                           for i, g in enumerate(glayers)],
@@ -364,6 +368,8 @@ def main(argv=None):
     ap.add_argument("--e2e-steps", type=int, default=40)
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--adaptive", action="store_true",
+                    help="single-scale path on layers whose calibrated sides differ by < 2x")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -425,8 +431,11 @@ def main(argv=None):
         "dtype": "s8",
         "data": "synthetic (seeded SD3.5/FLUX-shaped activations and weights)",
         "config": {"workload": f"{args.config}: {wl.CONFIGS[args.config]}",
-                   "layers": [{k: v for k, v in p.items() if k in ("name", "M", "N", "K", "G", "S")}
+                   "layers": [{k: v for k, v in p.items()
+                               if k in ("name", "M", "N", "K", "G", "S", "P")}
                               for p in res["per_layer"]],
+                   "path": ("adaptive: single-scale where calibrated sides differ < 2x"
+                            if args.adaptive else "DualScale on every layer"),
                    "output": "bf16",
                    "l2": "flushed between steps, untimed: 512 MiB written, then 256 MiB read",
                    "parallelism": f"replicas x{n_gpus}"},

@@ -77,6 +77,19 @@ typedef enum { SQ_OUT_BF16 = 0, SQ_OUT_F32 = 1 } sq_out_dtype;
 #define SQ_MAX_SEGMENTS 64
 
 /*
+ * Flags of a segment table.  SQ_FLAG_SINGLE_SCALE selects the single-scale
+ * (non-DualScale) path for a layer, for the adaptive use the papernotes page
+ * proposes under "Limitations" (DualScale only where activations are strongly
+ * polarity-asymmetric): one step s per group and K-segment serves both signs,
+ * s = max(max u, -min u)/127; the code is the DualScale code with s+ = s- = s,
+ * so X^+ and X^- collapse into one plane q = X^+ + X^- in [-128, 127]; the GEMM
+ * runs one integer product per k-step instead of two, y = sum_i s_w s f(A_i) + b.
+ * Layouts become planes [G][1][M][K] and accumulators [S][1][M][N]; s_act keeps
+ * its [G][S][2] shape with both entries equal.
+ */
+#define SQ_FLAG_SINGLE_SCALE 1
+
+/*
  * Segment table (SegLinear).  `offsets` is a HOST array of n_seg + 1 strictly
  * increasing int32 values from 0 to the segmented extent (N for SQ_SEG_OUTPUT,
  * K for SQ_SEG_INPUT).  SQ_SEG_NONE takes n_seg = 1 and offsets may be NULL.
@@ -93,6 +106,7 @@ typedef struct {
   int32_t n_seg;           /* number of segments, 1..SQ_MAX_SEGMENTS */
   const int32_t *offsets;  /* host, n_seg + 1 entries            */
   int32_t n_groups;        /* G                                  */
+  int32_t flags;           /* 0 (DualScale) or SQ_FLAG_SINGLE_SCALE */
 } sq_segments;
 
 /*
@@ -107,6 +121,7 @@ typedef struct {
  *          x 16-byte aligned
  *   d      fp32 [G][K] divisor (> 0, finite) or NULL for d = 1
  *   s_act  fp32 [G][S][2] output, {s+, s-} per group and K-segment
+ * With SQ_FLAG_SINGLE_SCALE: s+ = s- = max(hi, -lo)/127 (1 if both are 0).
  * Launches three small kernels; no workspace.
  */
 SQ_API sq_status sq_calibrate_act(const void *x, int64_t M, int64_t K, int64_t ldx,
@@ -126,6 +141,8 @@ SQ_API sq_status sq_calibrate_act(const void *x, int64_t M, int64_t K, int64_t l
  *   d      fp32 [G][K] or NULL;  s_act fp32 [G][S][2] (positive, finite, with
  *          d*s a normal float)
  *   planes int8 [G][2][M][K] output, 16-byte aligned
+ * With SQ_FLAG_SINGLE_SCALE the two codes of an element are written as their
+ * sum, one plane per group: planes int8 [G][1][M][K].
  * M == 0 is a valid no-op.
  */
 SQ_API sq_status sq_quantize_act(const void *x, int64_t M, int64_t K, int64_t ldx,
@@ -161,7 +178,9 @@ SQ_API sq_status sq_quantize_weight_seg(const void *w, int64_t N, int64_t K,
  * exactly this order; with S > 1 each segment's term is accumulated as
  * (s_w s+) f(A+) + (s_w s-) f(A-) with fused multiply-adds (same value up to
  * fp32 rounding).  Output rounds to bf16 (RN) or stays fp32.
- *   planes int8 [G][2][M][K] from sq_quantize_act; wq int8 [N][K]
+ *   planes int8 [G][P][M][K] from sq_quantize_act (P = 1 with
+ *          SQ_FLAG_SINGLE_SCALE: one product, y = sum_i s_w[i][n] s[g][i] f(A_i)
+ *          + bias, s = s_act[g][i][0]); wq int8 [N][K]
  *   s_w fp32 [S][N]; s_act fp32 [G][S][2]; bias bf16 [N] or NULL
  *   y      bf16 or fp32 [M][ldy] output, ldy >= N, ldy*elem % 16 == 0,
  *          16-byte aligned
@@ -179,7 +198,8 @@ SQ_API sq_status sq_dualscale_seglinear_gemm(const int8_t *planes, const int8_t 
 /*
  * sq_debug_gemm_s32 -- the same tensor-core kernel, storing the raw int32
  * accumulators instead of the epilogue, for bit-exact checks.
- *   acc int32 [S][2][M][N] output (16-byte aligned), polarity 0 = A+, 1 = A-.
+ *   acc int32 [S][P][M][N] output (16-byte aligned), polarity 0 = A+, 1 = A-;
+ *   P = 1 (one product of the merged plane) with SQ_FLAG_SINGLE_SCALE.
  */
 SQ_API sq_status sq_debug_gemm_s32(const int8_t *planes, const int8_t *wq, int64_t M,
                             int64_t N, int64_t K, const sq_segments *seg,

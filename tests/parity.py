@@ -9,21 +9,23 @@ from w8a8_gemm_b200 import binding as B
 from w8a8_gemm_b200 import workloads as wl
 
 
-def segments(layer: wl.Layer) -> B.Segments:
+def segments(layer: wl.Layer, single=False) -> B.Segments:
+    flags = B.SQ_FLAG_SINGLE_SCALE if single else 0
     if layer.mode == wl.MODE_NONE:
-        return B.Segments(B.SQ_SEG_NONE, None, 1)
-    return B.Segments(layer.mode, list(layer.offsets), layer.G)
+        return B.Segments(B.SQ_SEG_NONE, None, 1, flags)
+    return B.Segments(layer.mode, list(layer.offsets), layer.G, flags)
 
 
 def oracle_offsets(layer: wl.Layer):
     return None if layer.mode == wl.MODE_NONE else list(layer.offsets)
 
 
-def gpu_run(layer: wl.Layer, out_dtype=torch.float32, with_bias=True, s32=False):
+def gpu_run(layer: wl.Layer, out_dtype=torch.float32, with_bias=True, s32=False,
+            single=False):
     """CUDA path: weight quantization, calibration, activation quantization and
     the fused GEMM, all through the library."""
     dev = torch.device("cuda")
-    seg = segments(layer)
+    seg = segments(layer, single)
     x = layer.x.to(dev)
     w = layer.w.to(dev)
     xc = layer.x_cal.to(dev)
@@ -35,14 +37,14 @@ def gpu_run(layer: wl.Layer, out_dtype=torch.float32, with_bias=True, s32=False)
     B.sq_quantize_weight_seg(w, d, seg, wq, s_w)
     s_act = torch.empty(G, S, 2, dtype=torch.float32, device=dev)
     B.sq_calibrate_act(xc, d, seg, s_act)
-    planes = torch.empty(G, 2, M, K, dtype=torch.int8, device=dev)
+    planes = torch.empty(G, seg.P, M, K, dtype=torch.int8, device=dev)
     B.sq_quantize_act(x, d, s_act, seg, planes)
     ldy = (N + 7) // 8 * 8   # rows start 16-byte aligned for either dtype
     y = torch.empty(M, ldy, dtype=out_dtype, device=dev)[:, :N]
     B.sq_dualscale_seglinear_gemm(planes, wq, s_w, s_act, bias, y, seg)
     out = dict(wq=wq, s_w=s_w, s_act=s_act, planes=planes, y=y)
     if s32:
-        acc = torch.empty(S, 2, M, N, dtype=torch.int32, device=dev)
+        acc = torch.empty(S, seg.P, M, N, dtype=torch.int32, device=dev)
         B.sq_debug_gemm_s32(planes, wq, seg, acc)
         out["acc"] = acc
     torch.cuda.synchronize()
@@ -50,12 +52,14 @@ def gpu_run(layer: wl.Layer, out_dtype=torch.float32, with_bias=True, s32=False)
     return out
 
 
-def oracle_prep(layer: wl.Layer):
+def oracle_prep(layer: wl.Layer, single=False):
     """Oracle calibration and quantization of both operands."""
     off = oracle_offsets(layer)
     d = None if layer.d is None else layer.d.numpy()
-    s_act = oracle.calibrate_act(wl.bits(layer.x_cal), d, layer.mode, off, layer.G, layer.N)
-    planes = oracle.quantize_act(wl.bits(layer.x), s_act, d, layer.mode, off, layer.G, layer.N)
+    s_act = oracle.calibrate_act(wl.bits(layer.x_cal), d, layer.mode, off, layer.G, layer.N,
+                                 single)
+    planes = oracle.quantize_act(wl.bits(layer.x), s_act, d, layer.mode, off, layer.G, layer.N,
+                                 single)
     wq, s_w = oracle.quantize_weight(wl.bits(layer.w), d, layer.mode, off, layer.G)
     return dict(s_act=s_act, planes=planes, wq=wq, s_w=s_w)
 

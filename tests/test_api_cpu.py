@@ -43,7 +43,7 @@ def test_status_strings(L):
     assert B.status_string(0) == "SQ_OK"
     for code in range(-7, 0):
         assert B.status_string(code).startswith("SQ_ERR_")
-    assert B.lib().sq_version() == 100
+    assert B.lib().sq_version() == 101
 
 
 def _seg(mode, offsets, groups=1):
@@ -105,6 +105,19 @@ def test_segment_table_validation(L):
     K = offs[-1]
     assert L.sq_quantize_act(p(FAKE), 4, K, K, None, p(FAKE), ctypes.byref(c), p(FAKE),
                              None) == SQ_ERR_INVALID_ARG
+
+
+def test_unknown_flags_rejected(L):
+    p = ctypes.c_void_p
+    s = B.Segments(B.SQ_SEG_NONE, None, 1, flags=2)
+    c, keep = s._c()
+    assert L.sq_quantize_act(p(FAKE), 4, 32, 32, None, p(FAKE), ctypes.byref(c), p(FAKE),
+                             None) == SQ_ERR_INVALID_ARG
+    s = B.Segments(B.SQ_SEG_NONE, None, 1, flags=B.SQ_FLAG_SINGLE_SCALE)
+    c, keep = s._c()
+    # a valid single-scale table gets past validation (M == 0: no-op, no CUDA)
+    assert L.sq_quantize_act(p(FAKE), 0, 32, 32, None, p(FAKE), ctypes.byref(c), p(FAKE),
+                             None) == 0
 
 
 def test_gemm_overflow_and_layout_checks(L):

@@ -22,6 +22,7 @@ SQ_OK = 0
 SQ_SEG_NONE, SQ_SEG_OUTPUT, SQ_SEG_INPUT = 0, 1, 2
 SQ_OUT_BF16, SQ_OUT_F32 = 0, 1
 SQ_MAX_SEGMENTS = 64
+SQ_FLAG_SINGLE_SCALE = 1
 
 EXPORTED = ("sq_calibrate_act", "sq_quantize_act", "sq_quantize_weight_seg",
             "sq_dualscale_seglinear_gemm", "sq_debug_gemm_s32", "sq_get_device_status",
@@ -36,16 +37,24 @@ class SegQuantError(RuntimeError):
 
 class _Segments(ctypes.Structure):
     _fields_ = [("mode", ctypes.c_int32), ("n_seg", ctypes.c_int32),
-                ("offsets", ctypes.POINTER(ctypes.c_int32)), ("n_groups", ctypes.c_int32)]
+                ("offsets", ctypes.POINTER(ctypes.c_int32)), ("n_groups", ctypes.c_int32),
+                ("flags", ctypes.c_int32)]
 
 
 @dataclass
 class Segments:
     """SegLinear segment table: mode, boundaries (over N for output mode, over
-    K for input mode) and the number of activation groups G."""
+    K for input mode), the number of activation groups G, and flags
+    (SQ_FLAG_SINGLE_SCALE for the single-scale path)."""
     mode: int = SQ_SEG_NONE
     offsets: Optional[Sequence[int]] = None
     n_groups: int = 1
+    flags: int = 0
+
+    @property
+    def P(self) -> int:
+        """Activation planes per group: 2 (X^+, X^-), or 1 in single-scale mode."""
+        return 1 if self.flags & SQ_FLAG_SINGLE_SCALE else 2
 
     @property
     def n_seg(self) -> int:
@@ -62,7 +71,7 @@ class Segments:
         else:
             arr = (ctypes.c_int32 * len(self.offsets))(*[int(v) for v in self.offsets])
             ptr = ctypes.cast(arr, ctypes.POINTER(ctypes.c_int32))
-        s = _Segments(self.mode, self.n_seg, ptr, self.n_groups)
+        s = _Segments(self.mode, self.n_seg, ptr, self.n_groups, self.flags)
         return s, arr  # keep the array alive for the call
 
 
@@ -149,14 +158,14 @@ def sq_calibrate_act(x: torch.Tensor, d: Optional[torch.Tensor], seg: Segments,
 
 def sq_quantize_act(x: torch.Tensor, d: Optional[torch.Tensor], s_act: torch.Tensor,
                     seg: Segments, planes: torch.Tensor) -> torch.Tensor:
-    """DualScale quantization of X / d into planes int8 [G][2][M][K]."""
+    """DualScale quantization of X / d into planes int8 [G][P][M][K]."""
     _need(x, torch.bfloat16, "x")
     _need(d, torch.float32, "d", optional=True)
     _need(s_act, torch.float32, "s_act")
     _need(planes, torch.int8, "planes")
     M, K, ldx = _rows(x)
-    if tuple(planes.shape) != (seg.n_groups, 2, M, K) or not planes.is_contiguous():
-        raise ValueError(f"planes must be contiguous [{seg.n_groups}, 2, {M}, {K}]")
+    if tuple(planes.shape) != (seg.n_groups, seg.P, M, K) or not planes.is_contiguous():
+        raise ValueError(f"planes must be contiguous [{seg.n_groups}, {seg.P}, {M}, {K}]")
     cs, keep = seg._c()
     _check(lib().sq_quantize_act(_ptr(x), M, K, ldx, _ptr(d), _ptr(s_act), ctypes.byref(cs),
                                  _ptr(planes), _stream()), "sq_quantize_act")
@@ -190,10 +199,10 @@ def sq_dualscale_seglinear_gemm(planes: torch.Tensor, wq: torch.Tensor, s_w: tor
     _need(bias, torch.bfloat16, "bias", optional=True)
     if y.dtype not in (torch.bfloat16, torch.float32) or not y.is_cuda:
         raise ValueError("y must be a CUDA bf16 or fp32 tensor")
-    G, two, M, K = planes.shape
+    G, P, M, K = planes.shape
     N = wq.shape[0]
-    if two != 2 or wq.shape[1] != K or y.shape[0] != M or y.shape[1] != N or y.stride(1) != 1:
-        raise ValueError("shape mismatch between planes [G,2,M,K], wq [N,K] and y [M,N]")
+    if P != seg.P or wq.shape[1] != K or y.shape[0] != M or y.shape[1] != N or y.stride(1) != 1:
+        raise ValueError("shape mismatch between planes [G,P,M,K], wq [N,K] and y [M,N]")
     out = SQ_OUT_BF16 if y.dtype == torch.bfloat16 else SQ_OUT_F32
     cs, keep = seg._c()
     _check(lib().sq_dualscale_seglinear_gemm(_ptr(planes), _ptr(wq), _ptr(s_w), _ptr(s_act),
@@ -205,14 +214,14 @@ def sq_dualscale_seglinear_gemm(planes: torch.Tensor, wq: torch.Tensor, s_w: tor
 
 def sq_debug_gemm_s32(planes: torch.Tensor, wq: torch.Tensor, seg: Segments,
                       acc: torch.Tensor) -> torch.Tensor:
-    """Raw int32 accumulators [S][2][M][N] of the same tensor-core kernel."""
+    """Raw int32 accumulators [S][P][M][N] of the same tensor-core kernel."""
     _need(planes, torch.int8, "planes")
     _need(wq, torch.int8, "wq")
     _need(acc, torch.int32, "acc")
-    G, two, M, K = planes.shape
+    G, P, M, K = planes.shape
     N = wq.shape[0]
-    if tuple(acc.shape) != (seg.S, 2, M, N) or not acc.is_contiguous():
-        raise ValueError(f"acc must be contiguous [{seg.S}, 2, {M}, {N}]")
+    if tuple(acc.shape) != (seg.S, seg.P, M, N) or not acc.is_contiguous():
+        raise ValueError(f"acc must be contiguous [{seg.S}, {seg.P}, {M}, {N}]")
     cs, keep = seg._c()
     _check(lib().sq_debug_gemm_s32(_ptr(planes), _ptr(wq), M, N, K, ctypes.byref(cs), _ptr(acc),
                                    _stream()), "sq_debug_gemm_s32")

@@ -48,6 +48,7 @@ sq_status parse_segments(const sq_segments *seg, int64_t K, int64_t extent_n, Se
     p.n_seg = 1;
     p.G = 1;
     p.S = 1;
+    p.P = 2;
     p.off[0] = 0;
     p.off[1] = static_cast<int32_t>(K);
     *out = p;
@@ -56,6 +57,8 @@ sq_status parse_segments(const sq_segments *seg, int64_t K, int64_t extent_n, Se
   if (seg->mode < SQ_SEG_NONE || seg->mode > SQ_SEG_INPUT) return SQ_ERR_INVALID_ARG;
   if (seg->n_seg < 1 || seg->n_seg > SQ_MAX_SEGMENTS || seg->n_groups < 1)
     return SQ_ERR_INVALID_ARG;
+  if (seg->flags != 0 && seg->flags != SQ_FLAG_SINGLE_SCALE) return SQ_ERR_INVALID_ARG;
+  p.P = (seg->flags & SQ_FLAG_SINGLE_SCALE) ? 1 : 2;
   p.mode = seg->mode;
   p.n_seg = seg->n_seg;
   p.G = seg->n_groups;
@@ -293,6 +296,6 @@ const char *sq_status_string(sq_status s) {
   return "unknown sq_status";
 }
 
-int32_t sq_version(void) { return 100; }
+int32_t sq_version(void) { return 101; }
 
 }  // extern "C"

@@ -36,11 +36,6 @@ namespace {
 
 // Column tile of one-segment layers: 256 (one TMEM buffer, the epilogue runs
 // between tiles) or 128 (two buffers, the epilogue overlaps the next tile).
-// Epilogue warps of one-segment layers (multiple of 4).
-#ifndef SQ_ONESEG_EPI_WARPS
-#define SQ_ONESEG_EPI_WARPS 8
-#endif
-
 #ifndef SQ_GEMM_BN_ONE_SEG
 #define SQ_GEMM_BN_ONE_SEG 256
 #endif
@@ -68,12 +63,14 @@ struct GemmParams {
   int *status;
 };
 
-template <int BN, int STAGES, int EPI_WARPS>
+// POL = activation planes per group: 2 for DualScale (X^+ and X^-), 1 for the
+// single-scale path (one merged plane).
+template <int BN, int STAGES, int EPI_WARPS, int POL>
 struct Smem {
-  static constexpr int A_BYTES = 2 * BM * BK;   // X^+ tile, then X^- tile
+  static constexpr int A_BYTES = POL * BM * BK;  // X^+ tile, then X^- tile
   static constexpr int B_BYTES = BN * BK;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-  static constexpr int NBUF = 512 / (2 * BN);   // TMEM accumulator buffers
+  static constexpr int NBUF = 512 / (POL * BN);  // TMEM accumulator buffers
   static constexpr int EPI_OFFSET = STAGES * STAGE_BYTES;  // per-warp column constants
   static constexpr int COLS = BN / (EPI_WARPS / 4);  // columns per epilogue warp
   static constexpr int EPI_BYTES = EPI_WARPS * 4 * COLS * 4;  // 2 buffers x 2 arrays
@@ -174,13 +171,14 @@ __device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, uint32_t (&r)[CW]) 
 // One CTA per SM (shared memory allows no more).  Its warps spread over the four
 // 16K-register sub-partitions (10 warps: 3/3/2/2, a thread at most 168
 // registers; 18 warps: 5/5/4/4, at most 96).
-template <int BN, int STAGES, int OUT, bool SEGK, int EPI_WARPS>
+template <int BN, int STAGES, int OUT, bool SEGK, int EPI_WARPS, int POL>
 __global__ void __launch_bounds__(threads_for(EPI_WARPS), 1)
     dualscale_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                           const __grid_constant__ CUtensorMap tmB,
                           const __grid_constant__ GemmParams p) {
-  using L = Smem<BN, STAGES, EPI_WARPS>;
+  using L = Smem<BN, STAGES, EPI_WARPS, POL>;
   constexpr int NBUF = L::NBUF;
+  constexpr int ACC_COLS = POL * BN;  // TMEM columns of one accumulator buffer
   constexpr int HALF = L::COLS;      // columns per epilogue warp
   constexpr int CHUNKS = HALF / 32;  // 32-column groups (final multi-segment stores)
   // TMEM chunk of the one-segment epilogue: 32 columns with 8 warps, 16 with
@@ -240,7 +238,7 @@ __global__ void __launch_bounds__(threads_for(EPI_WARPS), 1)
           if (!wait_bar(&empty[stage], phase ^ 1, abort_flag, p.status)) goto producer_done;
           uint8_t *sa = smem + stage * L::STAGE_BYTES;
           mbar_arrive_expect_tx(&full[stage], L::STAGE_BYTES);
-          tma_load_3d(sa, &tmA, &full[stage], kb * BK, mt * BM, 2 * g);
+          tma_load_3d(sa, &tmA, &full[stage], kb * BK, mt * BM, POL * g);
           tma_load_2d(sa + L::A_BYTES, &tmB, &full[stage], kb * BK, nt * BN);
           armed |= 1u << stage;
           armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
@@ -269,7 +267,7 @@ __global__ void __launch_bounds__(threads_for(EPI_WARPS), 1)
         if (!wait_bar(&acc_empty[buf], ((acc_iter / NBUF) & 1) ^ 1, abort_flag, p.status))
           goto mma_exit;
         tc_fence_after();
-        uint32_t d_plus = tmem_base + buf * 2 * BN;
+        uint32_t d_plus = tmem_base + buf * ACC_COLS;
         uint32_t accumulate = 0;
         for (int kb = 0; kb < p.num_kb; ++kb) {
           if (!wait_bar(&full[stage], phase, abort_flag, p.status)) goto mma_exit;
@@ -289,15 +287,16 @@ __global__ void __launch_bounds__(threads_for(EPI_WARPS), 1)
               if (!wait_bar(&acc_empty[buf], ((acc_iter / NBUF) & 1) ^ 1, abort_flag, p.status))
                 goto mma_exit;
               tc_fence_after();
-              d_plus = tmem_base + buf * 2 * BN;
+              d_plus = tmem_base + buf * ACC_COLS;
               accumulate = 0;
               ++seg;
               seg_end = p.k_off[seg + 1];
             }
             const uint64_t b_desc = sdesc_kmajor_sw128(sb + kk * MMA_K);
             mma_i8(d_plus, sdesc_kmajor_sw128(sa + kk * MMA_K), b_desc, idesc, accumulate);
-            mma_i8(d_plus + BN, sdesc_kmajor_sw128(sa + BM * BK + kk * MMA_K), b_desc, idesc,
-                   accumulate);
+            if (POL == 2)
+              mma_i8(d_plus + BN, sdesc_kmajor_sw128(sa + BM * BK + kk * MMA_K), b_desc, idesc,
+                     accumulate);
             accumulate = 1;
           }
           mma_commit(&empty[stage]);  // frees the stage once these MMAs finish
@@ -382,24 +381,24 @@ __global__ void __launch_bounds__(threads_for(EPI_WARPS), 1)
         if (!wait_bar(&acc_full[buf], (acc_iter / NBUF) & 1, abort_flag, p.status))
           goto epilogue_exit;
         tc_fence_after();
-        const uint32_t t_plus = tmem_base + lane_addr + buf * 2 * BN + half * HALF;
+        const uint32_t t_plus = tmem_base + lane_addr + buf * ACC_COLS + half * HALF;
 #pragma unroll
         for (int c = 0; c < ((SEGK && OUT != OUT_S32) ? 0 : HALF / CW); ++c) {
           uint32_t ap[CW], am[CW];
           tmem_ld_cols<CW>(t_plus + c * CW, ap);
-          tmem_ld_cols<CW>(t_plus + BN + c * CW, am);
+          if constexpr (POL == 2) tmem_ld_cols<CW>(t_plus + BN + c * CW, am);
           tmem_ld_wait();
           const int64_t n0 = nb + c * CW;
           if constexpr (OUT == OUT_S32) {
             if (m < p.M) {
               int32_t *accp = reinterpret_cast<int32_t *>(p.y) +
-                              ((static_cast<int64_t>(u) * 2) * p.M + m) * p.N;
+                              ((static_cast<int64_t>(u) * POL) * p.M + m) * p.N;
               int32_t *accm = accp + static_cast<int64_t>(p.M) * p.N;
 #pragma unroll
               for (int j = 0; j < CW; ++j)
                 if (n0 + j < p.N) {
                   accp[n0 + j] = static_cast<int32_t>(ap[j]);
-                  accm[n0 + j] = static_cast<int32_t>(am[j]);
+                  if constexpr (POL == 2) accm[n0 + j] = static_cast<int32_t>(am[j]);
                 }
             }
           } else if constexpr (!SEGK) {
@@ -421,12 +420,17 @@ __global__ void __launch_bounds__(threads_for(EPI_WARPS), 1)
                   const int j = 4 * q + 2 * h;
                   const uint64_t fp = f2pack(__int2float_rn(static_cast<int32_t>(ap[j])),
                                              __int2float_rn(static_cast<int32_t>(ap[j + 1])));
-                  const uint64_t fm = f2pack(__int2float_rn(static_cast<int32_t>(am[j])),
-                                             __int2float_rn(static_cast<int32_t>(am[j + 1])));
                   // Each step is one packed FMA with a zero addend or a unit
                   // factor, i.e. exactly one rounding of the scalar product
                   // or sum, and nothing the compiler could contract further.
-                  const uint64_t t = ffma2(one2, ffma2(sp2, fp, zero2), ffma2(sm2, fm, zero2));
+                  uint64_t t;
+                  if constexpr (POL == 2) {
+                    const uint64_t fm = f2pack(__int2float_rn(static_cast<int32_t>(am[j])),
+                                               __int2float_rn(static_cast<int32_t>(am[j + 1])));
+                    t = ffma2(one2, ffma2(sp2, fp, zero2), ffma2(sm2, fm, zero2));
+                  } else {
+                    t = ffma2(sp2, fp, zero2);  // single scale: t = s f(A)
+                  }
                   const uint64_t u = ffma2(h ? f2pack(w.z, w.w) : f2pack(w.x, w.y), t, zero2);
                   const uint64_t y = ffma2(one2, u, h ? f2pack(b.z, b.w) : f2pack(b.x, b.y));
                   f2unpack(y, v[j], v[j + 1]);
@@ -443,7 +447,7 @@ __global__ void __launch_bounds__(threads_for(EPI_WARPS), 1)
           for (int c = 0; c < HALF / 16; ++c) {
             uint32_t ap[16], am[16];
             tmem_ld_32x32b_x16(t_plus + c * 16, ap);
-            tmem_ld_32x32b_x16(t_plus + BN + c * 16, am);
+            if constexpr (POL == 2) tmem_ld_32x32b_x16(t_plus + BN + c * 16, am);
             tmem_ld_wait();
             const float4 *cp4 = reinterpret_cast<const float4 *>(cst + c * 16);
             const float4 *cm4 = reinterpret_cast<const float4 *>(cst + HALF + c * 16);
@@ -458,8 +462,10 @@ __global__ void __launch_bounds__(threads_for(EPI_WARPS), 1)
               };
               r0 = ffma2(f2pack(a.x, a.y), cvt2(ap[j], ap[j + 1]), r0);
               r1 = ffma2(f2pack(a.z, a.w), cvt2(ap[j + 2], ap[j + 3]), r1);
-              r0 = ffma2(f2pack(b.x, b.y), cvt2(am[j], am[j + 1]), r0);
-              r1 = ffma2(f2pack(b.z, b.w), cvt2(am[j + 2], am[j + 3]), r1);
+              if constexpr (POL == 2) {
+                r0 = ffma2(f2pack(b.x, b.y), cvt2(am[j], am[j + 1]), r0);
+                r1 = ffma2(f2pack(b.z, b.w), cvt2(am[j + 2], am[j + 3]), r1);
+              }
             }
           }
         }
@@ -517,20 +523,20 @@ int device_sm_count() {
   return sms > 0 ? sms : 148;
 }
 
-template <int BN, int STAGES, int OUT, bool SEGK, int EPI_WARPS>
+template <int BN, int STAGES, int OUT, bool SEGK, int EPI_WARPS, int POL>
 sq_status run_gemm(const GemmRequest &r, const GemmParams &p, cudaStream_t stream) {
-  using L = Smem<BN, STAGES, EPI_WARPS>;
+  using L = Smem<BN, STAGES, EPI_WARPS, POL>;
   EncodeTiledFn enc = tensor_map_encoder();
   if (enc == nullptr) return SQ_ERR_CUDA;
   const int G = r.seg.G;
   CUtensorMap tmA, tmB;
   {
-    // planes viewed as 3D: x = K (bytes), y = M rows, z = 2G planes.
+    // planes viewed as 3D: x = K (bytes), y = M rows, z = POL * G planes.
     const cuuint64_t dims[3] = {static_cast<cuuint64_t>(r.K), static_cast<cuuint64_t>(r.M),
-                                static_cast<cuuint64_t>(2 * G)};
+                                static_cast<cuuint64_t>(POL * G)};
     const cuuint64_t strides[2] = {static_cast<cuuint64_t>(r.K),
                                    static_cast<cuuint64_t>(r.K) * static_cast<cuuint64_t>(r.M)};
-    const cuuint32_t box[3] = {BK, BM, 2};
+    const cuuint32_t box[3] = {BK, BM, POL};
     const cuuint32_t estr[3] = {1, 1, 1};
     if (enc(&tmA, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<int8_t *>(r.planes), dims, strides,
             box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -549,7 +555,7 @@ sq_status run_gemm(const GemmRequest &r, const GemmParams &p, cudaStream_t strea
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
       return SQ_ERR_CUDA;
   }
-  auto kernel = dualscale_gemm_kernel<BN, STAGES, OUT, SEGK, EPI_WARPS>;
+  auto kernel = dualscale_gemm_kernel<BN, STAGES, OUT, SEGK, EPI_WARPS, POL>;
   static bool attr_set[64] = {};  // per instantiation and device
   int dev = 0;
   cudaGetDevice(&dev);
@@ -563,6 +569,17 @@ sq_status run_gemm(const GemmRequest &r, const GemmParams &p, cudaStream_t strea
   const int grid = p.num_tiles < device_sm_count() ? p.num_tiles : device_sm_count();
   kernel<<<grid, threads_for(EPI_WARPS), L::BYTES, stream>>>(tmA, tmB, p);
   return cudaGetLastError() == cudaSuccess ? SQ_OK : SQ_ERR_CUDA;
+}
+
+// Tile configurations.  DualScale, one segment: 128 x 256 tiles, the + and -
+// accumulators fill TMEM (3 stages).  Single scale, one segment: 128 x 256
+// tiles with two TMEM buffers (4 stages).  Input-segmented: 128 x 128 tiles.
+template <int OUT, int POL>
+sq_status dispatch(const GemmRequest &r, const GemmParams &p, bool segk, int BN,
+                   cudaStream_t stream) {
+  if (segk) return run_gemm<128, 4, OUT, true, 16, POL>(r, p, stream);
+  if (BN == 256) return run_gemm<256, POL == 2 ? 3 : 4, OUT, false, 8, POL>(r, p, stream);
+  return run_gemm<128, 4, OUT, false, 8, POL>(r, p, stream);
 }
 
 }  // namespace
@@ -605,19 +622,18 @@ sq_status launch_gemm(const GemmRequest &r, cudaStream_t stream) {
   p.ldy = r.ldy;
   p.status = r.status;
 
-  if (r.out_kind == OUT_S32) {
-    if (segk) return run_gemm<128, 4, OUT_S32, true, 16>(r, p, stream);
-    return BN == 256 ? run_gemm<256, 3, OUT_S32, false, SQ_ONESEG_EPI_WARPS>(r, p, stream)
-                     : run_gemm<128, 4, OUT_S32, false, SQ_ONESEG_EPI_WARPS>(r, p, stream);
+  if (r.seg.P == 1) {
+    switch (r.out_kind) {
+      case OUT_S32: return dispatch<OUT_S32, 1>(r, p, segk, BN, stream);
+      case OUT_F32: return dispatch<OUT_F32, 1>(r, p, segk, BN, stream);
+      default: return dispatch<OUT_BF16, 1>(r, p, segk, BN, stream);
+    }
   }
-  if (r.out_kind == OUT_F32) {
-    if (segk) return run_gemm<128, 4, OUT_F32, true, 16>(r, p, stream);
-    return BN == 256 ? run_gemm<256, 3, OUT_F32, false, SQ_ONESEG_EPI_WARPS>(r, p, stream)
-                     : run_gemm<128, 4, OUT_F32, false, SQ_ONESEG_EPI_WARPS>(r, p, stream);
+  switch (r.out_kind) {
+    case OUT_S32: return dispatch<OUT_S32, 2>(r, p, segk, BN, stream);
+    case OUT_F32: return dispatch<OUT_F32, 2>(r, p, segk, BN, stream);
+    default: return dispatch<OUT_BF16, 2>(r, p, segk, BN, stream);
   }
-  if (segk) return run_gemm<128, 4, OUT_BF16, true, 16>(r, p, stream);
-  return BN == 256 ? run_gemm<256, 3, OUT_BF16, false, SQ_ONESEG_EPI_WARPS>(r, p, stream)
-                   : run_gemm<128, 4, OUT_BF16, false, SQ_ONESEG_EPI_WARPS>(r, p, stream);
 }
 
 }  // namespace sq

@@ -77,12 +77,20 @@ __global__ void __launch_bounds__(256) calib_reduce_kernel(const uint16_t *__res
   }
 }
 
-// Pass 2: s+ = max / 127, s- = |min| / 128; an empty side gets step 1.
-__global__ void calib_finalize_kernel(float *s_act, int n) {
+// Pass 2: s+ = max / 127, s- = |min| / 128; an empty side gets step 1.  In
+// single-scale mode both take max(max, |min|) / 127.
+__global__ void calib_finalize_kernel(float *s_act, int n, int single) {
   for (int t = threadIdx.x; t < n; t += blockDim.x) {
     const float hi = s_act[2 * t], nlo = s_act[2 * t + 1];
-    s_act[2 * t] = hi > 0.0f ? __fdiv_rn(hi, 127.0f) : 1.0f;
-    s_act[2 * t + 1] = nlo > 0.0f ? __fdiv_rn(nlo, 128.0f) : 1.0f;
+    if (single) {
+      const float amax = hi > nlo ? hi : nlo;
+      const float s = amax > 0.0f ? __fdiv_rn(amax, 127.0f) : 1.0f;
+      s_act[2 * t] = s;
+      s_act[2 * t + 1] = s;
+    } else {
+      s_act[2 * t] = hi > 0.0f ? __fdiv_rn(hi, 127.0f) : 1.0f;
+      s_act[2 * t + 1] = nlo > 0.0f ? __fdiv_rn(nlo, 128.0f) : 1.0f;
+    }
   }
 }
 
@@ -230,7 +238,7 @@ __global__ void __launch_bounds__(256, 3) quant_act_kernel(const __grid_constant
     const uint16_t *tile = reinterpret_cast<const uint16_t *>(qsmem + st * kQTileBytes);
     const int64_t r_base = static_cast<int64_t>(cur.rt) * kQRows;
     if (c0 < K) {
-      int8_t *plus = planes + (static_cast<int64_t>(cur.g) * 2) * plane_stride + c0;
+      int8_t *plus = planes + static_cast<int64_t>(cur.g) * seg.P * plane_stride + c0;
 #pragma unroll 2
       for (int rr = warp; rr < kQRows; rr += 8) {
         const int64_t r = r_base + rr;
@@ -240,8 +248,14 @@ __global__ void __launch_bounds__(256, 3) quant_act_kernel(const __grid_constant
         unpack8(v, xv);
         uint2 pk, nk;
         dualscale8(xv, p7, n7, pk, nk);
-        *reinterpret_cast<uint2 *>(plus + r * K) = pk;
-        *reinterpret_cast<uint2 *>(plus + plane_stride + r * K) = nk;
+        if (seg.P == 2) {
+          *reinterpret_cast<uint2 *>(plus + r * K) = pk;
+          *reinterpret_cast<uint2 *>(plus + plane_stride + r * K) = nk;
+        } else {
+          // single scale: one of the two codes of every element is 0, so the
+          // byte-wise OR is their sum
+          *reinterpret_cast<uint2 *>(plus + r * K) = make_uint2(pk.x | nk.x, pk.y | nk.y);
+        }
       }
     }
     __syncthreads();  // every warp is done with stage st
@@ -328,7 +342,7 @@ cudaError_t launch_calibrate_act(const uint16_t *x, int64_t M, int64_t K, int64_
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
-  calib_finalize_kernel<<<1, 256, 0, stream>>>(s_act, n);
+  calib_finalize_kernel<<<1, 256, 0, stream>>>(s_act, n, seg.P == 1 ? 1 : 0);
   return cudaGetLastError();
 }
 

@@ -15,6 +15,7 @@ struct SegParams {
   int32_t n_seg;  // segments
   int32_t G;      // activation groups
   int32_t S;      // K-segments (n_seg in input mode, else 1)
+  int32_t P;      // activation planes per group: 2 (DualScale) or 1 (single scale)
   int32_t off[SQ_MAX_SEGMENTS + 1];
 };
 

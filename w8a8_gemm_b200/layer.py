@@ -24,7 +24,8 @@ class DualScaleSegLinear:
     """
 
     def __init__(self, w: torch.Tensor, bias: Optional[torch.Tensor], d: Optional[torch.Tensor],
-                 seg: B.Segments, x_cal: torch.Tensor, out_dtype=torch.bfloat16):
+                 seg: B.Segments, x_cal: torch.Tensor, out_dtype=torch.bfloat16,
+                 adaptive: bool = False, asymmetry_threshold: float = 2.0):
         self.N, self.K = w.shape
         self.seg = seg
         self.G, self.S = seg.n_groups, seg.S
@@ -37,11 +38,24 @@ class DualScaleSegLinear:
         B.sq_quantize_weight_seg(w, d, seg, self.wq, self.s_w)
         self.s_act = torch.empty(self.G, self.S, 2, dtype=torch.float32, device=dev)
         B.sq_calibrate_act(x_cal, d, seg, self.s_act)
+        if adaptive and not seg.flags:
+            # Adaptive DualScale: keep the two steps only where the calibrated
+            # sides differ by at least `asymmetry_threshold` in some group and
+            # K-segment; otherwise switch the layer to one symmetric step.
+            hi = self.s_act[..., 0] * 127.0
+            lo = self.s_act[..., 1] * 128.0
+            ratio = torch.maximum(hi, lo) / torch.minimum(hi, lo).clamp_min(1e-30)
+            if float(ratio.max()) < asymmetry_threshold:
+                self.seg = B.Segments(seg.mode, seg.offsets, seg.n_groups,
+                                      B.SQ_FLAG_SINGLE_SCALE)
+                B.sq_calibrate_act(x_cal, d, self.seg, self.s_act)
+        self.single_scale = bool(self.seg.flags & B.SQ_FLAG_SINGLE_SCALE)
         self._planes = None
 
     def planes_for(self, M: int, device) -> torch.Tensor:
         if self._planes is None or self._planes.shape[2] != M:
-            self._planes = torch.empty(self.G, 2, M, self.K, dtype=torch.int8, device=device)
+            self._planes = torch.empty(self.G, self.seg.P, M, self.K, dtype=torch.int8,
+                                       device=device)
         return self._planes
 
     def quantize(self, x: torch.Tensor, planes: Optional[torch.Tensor] = None) -> torch.Tensor:
