@@ -26,6 +26,7 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <cstring>
 #include <mutex>
 
 #include "sm100.cuh"
@@ -65,7 +66,7 @@ struct GemmParams {
 
 // POL = activation planes per group: 2 for DualScale (X^+ and X^-), 1 for the
 // single-scale path (one merged plane).
-template <int BN, int STAGES, int EPI_WARPS, int POL>
+template <int BN, int STAGES, int EPI_WARPS, int POL, bool SEGK, bool TMA_STORE>
 struct Smem {
   static constexpr int A_BYTES = POL * BM * BK;  // X^+ tile, then X^- tile
   static constexpr int B_BYTES = BN * BK;
@@ -73,8 +74,13 @@ struct Smem {
   static constexpr int NBUF = 512 / (POL * BN);  // TMEM accumulator buffers
   static constexpr int EPI_OFFSET = STAGES * STAGE_BYTES;  // per-warp column constants
   static constexpr int COLS = BN / (EPI_WARPS / 4);  // columns per epilogue warp
-  static constexpr int EPI_BYTES = EPI_WARPS * 4 * COLS * 4;  // 2 buffers x 2 arrays
-  static constexpr int BAR_OFFSET = EPI_OFFSET + EPI_BYTES;
+  // two arrays of COLS floats per warp; multi-segment layers double-buffer them
+  static constexpr int CONST_FLOATS = (SEGK ? 2 : 1) * 2 * COLS;
+  static constexpr int EPI_BYTES = EPI_WARPS * CONST_FLOATS * 4;
+  // per-warp staging of one 32 x 32 bf16 output chunk for the tensor store
+  static constexpr int STG_OFFSET = EPI_OFFSET + EPI_BYTES;
+  static constexpr int STG_BYTES = TMA_STORE ? EPI_WARPS * 2048 : 0;
+  static constexpr int BAR_OFFSET = STG_OFFSET + STG_BYTES;
   static constexpr int NUM_BARS = 2 * STAGES + 2 * NBUF + 1;
   static constexpr int BYTES = BAR_OFFSET + NUM_BARS * 8 + 16 + 1024;  // + 1 KB alignment slack
 };
@@ -175,8 +181,11 @@ template <int BN, int STAGES, int OUT, bool SEGK, int EPI_WARPS, int POL>
 __global__ void __launch_bounds__(threads_for(EPI_WARPS), 1)
     dualscale_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                           const __grid_constant__ CUtensorMap tmB,
+                          const __grid_constant__ CUtensorMap tmY,
                           const __grid_constant__ GemmParams p) {
-  using L = Smem<BN, STAGES, EPI_WARPS, POL>;
+  // One-segment bf16 output leaves through shared memory and TMA stores.
+  constexpr bool TMA_STORE = (OUT == OUT_BF16) && !SEGK;
+  using L = Smem<BN, STAGES, EPI_WARPS, POL, SEGK, TMA_STORE>;
   constexpr int NBUF = L::NBUF;
   constexpr int ACC_COLS = POL * BN;  // TMEM columns of one accumulator buffer
   constexpr int HALF = L::COLS;      // columns per epilogue warp
@@ -321,8 +330,9 @@ __global__ void __launch_bounds__(threads_for(EPI_WARPS), 1)
     const int row = quarter * 32 + lane;
     const uint32_t lane_addr = static_cast<uint32_t>(quarter * 32) << 16;
     // Warp-private column constants in shared memory, read back as broadcast
-    // float4s: two buffers of [HALF] + [HALF] floats.
-    float *cst_base = reinterpret_cast<float *>(smem + L::EPI_OFFSET) + ew * 4 * HALF;
+    // float4s: [HALF] + [HALF] floats (two such buffers with several K-segments).
+    float *cst_base = reinterpret_cast<float *>(smem + L::EPI_OFFSET) + ew * L::CONST_FLOATS;
+    uint8_t *stg = smem + L::STG_OFFSET + ew * 2048;  // used when TMA_STORE
     uint32_t acc_iter = 0;
     for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x) {
       const int mt = tile / p.num_n_tiles, nt = tile % p.num_n_tiles;
@@ -406,7 +416,7 @@ __global__ void __launch_bounds__(threads_for(EPI_WARPS), 1)
             //   t = s+ f(A+) + s- f(A-);  y = s_w t + bias,
             // two columns per packed instruction (each lane rounds once per
             // operation, exactly as the scalar sequence does).
-            if (m < p.M) {
+            if (TMA_STORE || m < p.M) {
               const float4 *sw4 = reinterpret_cast<const float4 *>(cst + c * CW);
               const float4 *b4 = reinterpret_cast<const float4 *>(cst + HALF + c * CW);
               const uint64_t sp2 = f2pack(sp, sp), sm2 = f2pack(sm, sm);
@@ -436,7 +446,30 @@ __global__ void __launch_bounds__(threads_for(EPI_WARPS), 1)
                   f2unpack(y, v[j], v[j + 1]);
                 }
               }
-              store_row_chunk<OUT, CW>(p, m, n0, v);
+              if constexpr (TMA_STORE) {
+                // The warp's 32 rows x 32 columns go to its staging buffer (one
+                // 64-byte row per lane) and leave in one tensor store, which
+                // writes whole lines and drops rows >= M and columns >= N.
+                static_assert(CW == 32, "tensor-store chunk is 32 x 32");
+                if (lane == 0) bulk_wait_read_all();  // the previous chunk is out
+                __syncwarp();
+                uint4 *dst = reinterpret_cast<uint4 *>(stg + lane * 64);
+#pragma unroll
+                for (int q = 0; q < 4; ++q)
+                  dst[q] = make_uint4(pack_bf16x2(v[8 * q + 0], v[8 * q + 1]),
+                                      pack_bf16x2(v[8 * q + 2], v[8 * q + 3]),
+                                      pack_bf16x2(v[8 * q + 4], v[8 * q + 5]),
+                                      pack_bf16x2(v[8 * q + 6], v[8 * q + 7]));
+                fence_proxy_async_smem();
+                __syncwarp();
+                const int row0 = mt * BM + quarter * 32;
+                if (lane == 0 && row0 < p.M && n0 < p.N) {
+                  tma_store_2d(&tmY, stg, static_cast<int32_t>(n0), row0);
+                  bulk_commit_group();
+                }
+              } else {
+                store_row_chunk<OUT, CW>(p, m, n0, v);
+              }
             }
           }
         }
@@ -503,7 +536,11 @@ __global__ void __launch_bounds__(threads_for(EPI_WARPS), 1)
         __syncwarp();
       }
     }
-  epilogue_exit:;
+  epilogue_exit:
+    if constexpr (TMA_STORE) {
+      if (lane == 0) bulk_wait_all();  // every tensor store of this warp is complete
+      __syncwarp();
+    }
   }
 
   tc_fence_before();
@@ -525,7 +562,7 @@ int device_sm_count() {
 
 template <int BN, int STAGES, int OUT, bool SEGK, int EPI_WARPS, int POL>
 sq_status run_gemm(const GemmRequest &r, const GemmParams &p, cudaStream_t stream) {
-  using L = Smem<BN, STAGES, EPI_WARPS, POL>;
+  using L = Smem<BN, STAGES, EPI_WARPS, POL, SEGK, OUT == OUT_BF16 && !SEGK>;
   EncodeTiledFn enc = tensor_map_encoder();
   if (enc == nullptr) return SQ_ERR_CUDA;
   const int G = r.seg.G;
@@ -555,6 +592,20 @@ sq_status run_gemm(const GemmRequest &r, const GemmParams &p, cudaStream_t strea
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
       return SQ_ERR_CUDA;
   }
+  CUtensorMap tmY;
+  memset(&tmY, 0, sizeof tmY);
+  if (OUT == OUT_BF16 && !SEGK) {
+    // Y viewed as 2D bf16: x = N columns, y = M rows; 32 x 32 boxes.
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(r.N), static_cast<cuuint64_t>(r.M)};
+    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(r.ldy) * 2};
+    const cuuint32_t box[2] = {32, 32};
+    const cuuint32_t estr[2] = {1, 1};
+    if (enc(&tmY, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, r.y, dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+            CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return SQ_ERR_CUDA;
+  }
+  static_assert(L::BYTES <= 232448, "dynamic shared memory above the per-block limit");
   auto kernel = dualscale_gemm_kernel<BN, STAGES, OUT, SEGK, EPI_WARPS, POL>;
   static bool attr_set[64] = {};  // per instantiation and device
   int dev = 0;
@@ -567,7 +618,7 @@ sq_status run_gemm(const GemmRequest &r, const GemmParams &p, cudaStream_t strea
     attr_set[dev] = true;
   }
   const int grid = p.num_tiles < device_sm_count() ? p.num_tiles : device_sm_count();
-  kernel<<<grid, threads_for(EPI_WARPS), L::BYTES, stream>>>(tmA, tmB, p);
+  kernel<<<grid, threads_for(EPI_WARPS), L::BYTES, stream>>>(tmA, tmB, tmY, p);
   return cudaGetLastError() == cudaSuccess ? SQ_OK : SQ_ERR_CUDA;
 }
 
