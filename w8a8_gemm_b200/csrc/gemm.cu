@@ -81,6 +81,7 @@ struct Smem {
   static constexpr int STG_OFFSET = EPI_OFFSET + EPI_BYTES;
   static constexpr int STG_BYTES = TMA_STORE ? EPI_WARPS * 2048 : 0;
   static constexpr int BAR_OFFSET = STG_OFFSET + STG_BYTES;
+  static_assert(STG_OFFSET % 1024 == 0, "staging must be aligned to the swizzle pattern");
   static constexpr int NUM_BARS = 2 * STAGES + 2 * NBUF + 1;
   static constexpr int BYTES = BAR_OFFSET + NUM_BARS * 8 + 16 + 1024;  // + 1 KB alignment slack
 };
@@ -449,14 +450,18 @@ __global__ void __launch_bounds__(threads_for(EPI_WARPS), 1)
               if constexpr (TMA_STORE) {
                 // The warp's 32 rows x 32 columns go to its staging buffer (one
                 // 64-byte row per lane) and leave in one tensor store, which
-                // writes whole lines and drops rows >= M and columns >= N.
+                // writes whole lines and drops rows >= M and columns >= N.  The
+                // buffer uses the tensor map's 64-byte swizzle: 16-byte piece q
+                // of row r sits at piece q ^ ((r / 2) % 4), so each group of 8
+                // lanes stores to 8 distinct bank groups.
                 static_assert(CW == 32, "tensor-store chunk is 32 x 32");
                 if (lane == 0) bulk_wait_read_all();  // the previous chunk is out
                 __syncwarp();
                 uint4 *dst = reinterpret_cast<uint4 *>(stg + lane * 64);
+                const int swz = (lane >> 1) & 3;
 #pragma unroll
                 for (int q = 0; q < 4; ++q)
-                  dst[q] = make_uint4(pack_bf16x2(v[8 * q + 0], v[8 * q + 1]),
+                  dst[q ^ swz] = make_uint4(pack_bf16x2(v[8 * q + 0], v[8 * q + 1]),
                                       pack_bf16x2(v[8 * q + 2], v[8 * q + 3]),
                                       pack_bf16x2(v[8 * q + 4], v[8 * q + 5]),
                                       pack_bf16x2(v[8 * q + 6], v[8 * q + 7]));
@@ -601,7 +606,7 @@ sq_status run_gemm(const GemmRequest &r, const GemmParams &p, cudaStream_t strea
     const cuuint32_t box[2] = {32, 32};
     const cuuint32_t estr[2] = {1, 1};
     if (enc(&tmY, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, r.y, dims, strides, box, estr,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
             CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
       return SQ_ERR_CUDA;
   }
