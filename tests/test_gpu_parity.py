@@ -190,3 +190,48 @@ def test_full_size_configs_sampled_rows(cfg):
         assert rel_err_floor(gf["y"][torch.from_numpy(rows).cuda()].cpu().numpy(), r) <= FP32_TOL
         del g, gf
         torch.cuda.empty_cache()
+
+
+def _integer_layer(widths, seed, single):
+    """Input-segmented layer whose quantization is the identity: integer
+    activations in [-128, 127]; every segment's calibration slice spans
+    [-128, 127] (s+ = 127/127, s- = 128/128), or [-127, 127] for the single
+    step (s = 127/127); integer weights whose rows reach 127 in every segment
+    (s_w = 1).  Rows 0 and 1 are all 127 and all -128, weight rows 0 and 1 all
+    127 and all -127: their products are the largest accumulators a segment
+    of that width can hold.  Every fp32 sum stays below 2^24, so Y is the
+    exact integer product in any summation order."""
+    g = torch.Generator().manual_seed(seed)
+    K = sum(widths)
+    M, N = 130, 136
+    offsets = [0] + [int(v) for v in np.cumsum(widths)]
+    x = torch.randint(-128, 128, (M, K), generator=g).float()
+    x[0] = 127.0
+    x[1] = -128.0
+    x_cal = x[:2].clone()
+    if single:
+        x_cal[1] = -127.0
+    w = torch.randint(-127, 128, (N, K), generator=g).float()
+    w[:, offsets[:-1]] = 127.0
+    w[0] = 127.0
+    w[1] = -127.0
+    L = wl.Layer("int", x.to(torch.bfloat16), x_cal.to(torch.bfloat16), w.to(torch.bfloat16),
+                 None, None, wl.MODE_INPUT, offsets, 1)
+    exact = x.double().numpy() @ w.double().numpy().T
+    return L, exact
+
+
+@pytest.mark.parametrize("widths", [[256, 256], [256, 288], [32, 256, 96]])
+@pytest.mark.parametrize("single", [False, True])
+def test_input_segments_extreme_accumulators_exact(widths, single):
+    """The per-segment drains at the largest accumulators a segment allows
+    (|A| up to w * 128 * 127 for width w, beyond 2^22 for w = 288): with unit
+    scales every step is exact, so Y must equal the integer product."""
+    L, exact = _integer_layer(widths, sum(widths) + single, single)
+    prep = oracle_prep(L, single)
+    assert np.all(prep["s_act"] == 1.0) and np.all(prep["s_w"] == 1.0)
+    g = gpu_run(L, out_dtype=torch.float32, s32=True, single=single)
+    assert np.array_equal(g["acc"].cpu().numpy(), oracle_acc(L, prep))
+    y = g["y"].cpu().numpy()
+    assert np.array_equal(y.astype(np.float64), exact)
+    assert np.array_equal(oracle_y(L, prep).astype(np.float64), exact)

@@ -351,9 +351,11 @@ __global__ void __launch_bounds__(threads_for(EPI_WARPS), 1)
         __syncwarp();
       }
       // Multi-segment state: packed running sums (column pairs) and the next
-      // K-segment's weight scales, loaded one segment ahead.
+      // K-segment's weight and activation scales, loaded one segment ahead so
+      // that no global load latency sits between two drains.
       uint64_t run2[SEGK ? HALF / 2 : 1];
       float sw_next[SEGK ? HALF / 32 : 1];
+      float sp_next = 0.0f, sm_next = 0.0f;
       if constexpr (SEGK && OUT != OUT_S32) {
 #pragma unroll
         for (int j = 0; j < HALF / 2; ++j) run2[j] = 0ull;
@@ -362,11 +364,13 @@ __global__ void __launch_bounds__(threads_for(EPI_WARPS), 1)
           const int64_t n = nb + q * 32 + lane;
           sw_next[q] = n < p.N ? p.s_w[n] : 0.0f;
         }
+        sp_next = p.s_act[g * p.S * 2 + 0];
+        sm_next = p.s_act[g * p.S * 2 + 1];
       }
       const int units = SEGK ? p.S : 1;
       for (int u = 0; u < units; ++u) {
-        const float sp = p.s_act[(g * p.S + u) * 2 + 0];
-        const float sm = p.s_act[(g * p.S + u) * 2 + 1];
+        const float sp = (SEGK && OUT != OUT_S32) ? sp_next : p.s_act[(g * p.S + u) * 2 + 0];
+        const float sm = (SEGK && OUT != OUT_S32) ? sm_next : p.s_act[(g * p.S + u) * 2 + 1];
         float *cst = cst_base;
         if constexpr (SEGK && OUT != OUT_S32) {
           // Folded coefficients of K-segment u: c+- = s_w[u][n] * s+-[u], into
@@ -385,6 +389,8 @@ __global__ void __launch_bounds__(threads_for(EPI_WARPS), 1)
               const int64_t n = nb + q * 32 + lane;
               sw_next[q] = n < p.N ? swn[n] : 0.0f;
             }
+            sp_next = p.s_act[(g * p.S + u + 1) * 2 + 0];
+            sm_next = p.s_act[(g * p.S + u + 1) * 2 + 1];
           }
           __syncwarp();
         }
@@ -629,11 +635,16 @@ sq_status run_gemm(const GemmRequest &r, const GemmParams &p, cudaStream_t strea
 
 // Tile configurations.  DualScale, one segment: 128 x 256 tiles, the + and -
 // accumulators fill TMEM (3 stages).  Single scale, one segment: 128 x 256
-// tiles with two TMEM buffers (4 stages).  Input-segmented: 128 x 128 tiles.
+// tiles with two TMEM buffers (4 stages).  Input-segmented: 128 x 128 tiles
+// with two TMEM buffers and 16 epilogue warps for the per-segment drains, which
+// bound that path (int32 -> fp32 conversion and FMA per element and segment);
+// narrower tiles give more buffers but cost more than they save (measured).
+constexpr int kSegBN = 128;  // tile width of the input-segmented path
+
 template <int OUT, int POL>
 sq_status dispatch(const GemmRequest &r, const GemmParams &p, bool segk, int BN,
                    cudaStream_t stream) {
-  if (segk) return run_gemm<128, 4, OUT, true, 16, POL>(r, p, stream);
+  if (segk) return run_gemm<kSegBN, 4, OUT, true, 16, POL>(r, p, stream);
   if (BN == 256) return run_gemm<256, POL == 2 ? 3 : 4, OUT, false, 8, POL>(r, p, stream);
   return run_gemm<128, 4, OUT, false, 8, POL>(r, p, stream);
 }
@@ -643,7 +654,7 @@ sq_status dispatch(const GemmRequest &r, const GemmParams &p, bool segk, int BN,
 sq_status launch_gemm(const GemmRequest &r, cudaStream_t stream) {
   if (r.M == 0) return SQ_OK;
   const bool segk = r.seg.mode == SQ_SEG_INPUT && r.seg.S > 1;
-  int BN = segk ? 128 : SQ_GEMM_BN_ONE_SEG;
+  int BN = segk ? kSegBN : SQ_GEMM_BN_ONE_SEG;
   if (r.seg.G > 1) {
     for (int j = 0; j < r.seg.n_seg; ++j)
       if ((r.seg.off[j + 1] - r.seg.off[j]) % 256 != 0) BN = 128;
