@@ -35,11 +35,14 @@ def lib():
         L.orc_calibrate_act.argtypes = [p, i64, i64, i64, p, i32, i32, p, i32, i64, i32, p]
         L.orc_quantize_act.argtypes = [p, i64, i64, i64, p, p, i32, i32, p, i32, i64, i32, p]
         L.orc_quantize_weight.argtypes = [p, i64, i64, p, i32, i32, p, i32, p, p]
+        L.orc_quantize_weight_q.argtypes = [p, i64, i64, p, i32, i32, p, i32, i32, p, p]
+        L.orc_pack_w4.argtypes = [p, i64, i64, p]
         L.orc_gemm_s32.argtypes = [p, p, i64, i64, i64, i32, i32, p, i32, i32, p, i64, p, i32]
         L.orc_gemm.argtypes = [p, p, p, p, p, i64, i64, i64, i32, i32, p, i32, i32, p, i64, p,
                                i32]
         L.orc_num_threads.argtypes = []
         for f in (L.orc_calibrate_act, L.orc_quantize_act, L.orc_quantize_weight,
+                  L.orc_quantize_weight_q, L.orc_pack_w4,
                   L.orc_gemm_s32, L.orc_gemm, L.orc_num_threads):
             f.restype = ctypes.c_int
         _lib = L
@@ -102,18 +105,30 @@ def quantize_act(x_bits, s_act, d=None, mode=MODE_NONE, offsets=None, G=1, N=0,
     return planes
 
 
-def quantize_weight(w_bits, d=None, mode=MODE_NONE, offsets=None, G=1):
-    """Segment-wise AMax weight quantization: returns (wq int8 [N][K], s_w f32 [S][N])."""
+def quantize_weight(w_bits, d=None, mode=MODE_NONE, offsets=None, G=1, bits=8):
+    """Segment-wise AMax weight quantization: returns (wq int8 [N][K], s_w f32 [S][N]).
+    bits=8: codes in [-127, 127]; bits=4 (W4A8): codes in [-7, 7]."""
     w = _c(w_bits, np.uint16)
     N, K = w.shape
     off, n_seg, S = _seg(mode, offsets, G, N, K)
     d = _c(d, np.float32)
     wq = np.zeros((N, K), np.int8)
     s_w = np.zeros((S, N), np.float32)
-    _check(lib().orc_quantize_weight(_ptr(w), N, K, _ptr(d), mode, n_seg,
-                                     _ptr(off), G, _ptr(wq), _ptr(s_w)),
+    qmax = {8: 127, 4: 7}[bits]
+    _check(lib().orc_quantize_weight_q(_ptr(w), N, K, _ptr(d), mode, n_seg,
+                                       _ptr(off), G, qmax, _ptr(wq), _ptr(s_w)),
            "quantize_weight")
     return wq, s_w
+
+
+def pack_w4(wq):
+    """4-bit storage of codes in [-8, 7]: uint8 [N][K/2], channel 2j in the low
+    nibble and 2j + 1 in the high nibble (two's complement)."""
+    wq = _c(wq, np.int8)
+    N, K = wq.shape
+    out = np.zeros((N, K // 2), np.uint8)
+    _check(lib().orc_pack_w4(_ptr(wq), N, K, _ptr(out)), "pack_w4")
+    return out
 
 
 def _rows(rows, M):
@@ -162,7 +177,7 @@ def gemm(planes, wq, s_w, s_act, bias_bits=None, mode=MODE_NONE, offsets=None,
 
 
 def layer(x_bits, w_bits, x_cal_bits, d=None, bias_bits=None, mode=MODE_NONE,
-          offsets=None, G=1, rows=None, threads=1, single=False):
+          offsets=None, G=1, rows=None, threads=1, single=False, weight_bits=8):
     """Whole static pipeline on the CPU: calibrate, quantize both sides, GEMM.
 
     Returns a dict with s_act, planes, wq, s_w and y (fp32 rows)."""
@@ -170,11 +185,11 @@ def layer(x_bits, w_bits, x_cal_bits, d=None, bias_bits=None, mode=MODE_NONE,
     N = w.shape[0]
     s_act = calibrate_act(x_cal_bits, d, mode, offsets, G, N, single)
     planes = quantize_act(x_bits, s_act, d, mode, offsets, G, N, single)
-    wq, s_w = quantize_weight(w, d, mode, offsets, G)
+    wq, s_w = quantize_weight(w, d, mode, offsets, G, bits=weight_bits)
     y = gemm(planes, wq, s_w, s_act, bias_bits, mode, offsets, rows, threads)
     return dict(s_act=s_act, planes=planes, wq=wq, s_w=s_w, y=y)
 
 
 __all__ = ["MODE_NONE", "MODE_OUTPUT", "MODE_INPUT", "calibrate_act",
-           "quantize_act", "quantize_weight", "gemm_s32", "gemm", "layer",
+           "quantize_act", "quantize_weight", "pack_w4", "gemm_s32", "gemm", "layer",
            "num_threads", "lib"]

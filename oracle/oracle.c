@@ -38,6 +38,13 @@
  *    all-zero weight column segment gives s_w = 1.
  *  - Weights: symmetric AMax per output channel and per K-segment,
  *    s_w = amax / 127, q = rne(clamp(w' / s_w, -127, 127)).
+ *  - W4A8 (the papernotes page's and the author page's "SegQuant-4" / W4A8
+ *    rows in the results and deployment tables; the pages give no formula):
+ *    the same symmetric AMax rule with q_max = 7, s_w = amax / 7,
+ *    q = rne(clamp(w' / s_w, -7, 7)); activations stay DualScale int8 and the
+ *    integer product and epilogue are unchanged.  Storage: two codes per byte,
+ *    4-bit two's complement, channel 2j in the low nibble and 2j + 1 in the
+ *    high nibble (orc_pack_w4).
  *  - Output-segmented layers may carry their own activation parameters per
  *    output segment (a "group" g: its own d and s+/s-, hence its own planes).
  *    G = 1 is the pages' formula with one shared X^.
@@ -208,10 +215,12 @@ int orc_quantize_act(const uint16_t *x, int64_t M, int64_t K, int64_t ldx,
  * independently on every K-segment i; in output mode each output segment j
  * folds its own group's divisor d[j] when G > 1.
  * ------------------------------------------------------------------------- */
-int orc_quantize_weight(const uint16_t *w, int64_t N, int64_t K, const float *d,
-                        int mode, int n_seg, const int32_t *offsets, int G,
-                        int8_t *wq, float *s_w) {
+int orc_quantize_weight_q(const uint16_t *w, int64_t N, int64_t K, const float *d,
+                          int mode, int n_seg, const int32_t *offsets, int G,
+                          int qmax, int8_t *wq, float *s_w) {
   if (orc_check_seg(mode, n_seg, offsets, G, N, K)) return -1;
+  if (qmax != 127 && qmax != 7) return -1;
+  float fq = (float)qmax;
   int S = (mode == ORC_MODE_INPUT) ? n_seg : 1;
   for (int64_t n = 0; n < N; ++n) {
     int g = (mode == ORC_MODE_OUTPUT && G > 1)
@@ -226,17 +235,37 @@ int orc_quantize_weight(const uint16_t *w, int64_t N, int64_t K, const float *d,
         float a = fabsf(wv);
         if (a > amax) amax = a;
       }
-      float s = (amax > 0.0f) ? amax / 127.0f : 1.0f;
+      float s = (amax > 0.0f) ? amax / fq : 1.0f;
       s_w[(int64_t)i * N + n] = s;
       for (int64_t k = k0; k < k1; ++k) {
         float dv = d ? d[(int64_t)g * K + k] : 1.0f;
         float v = (orc_bf16(w[n * K + k]) * dv) / s;
-        if (v > 127.0f) v = 127.0f;
-        if (v < -127.0f) v = -127.0f;
+        if (v > fq) v = fq;
+        if (v < -fq) v = -fq;
         wq[n * K + k] = (int8_t)(int)rintf(v);
       }
     }
   }
+  return 0;
+}
+
+int orc_quantize_weight(const uint16_t *w, int64_t N, int64_t K, const float *d,
+                        int mode, int n_seg, const int32_t *offsets, int G,
+                        int8_t *wq, float *s_w) {
+  return orc_quantize_weight_q(w, N, K, d, mode, n_seg, offsets, G, 127, wq, s_w);
+}
+
+/* 4-bit storage of codes in [-8, 7]: byte [n][j] holds channel 2j in its low
+ * nibble and channel 2j + 1 in its high nibble, each as 4-bit two's complement.
+ * K must be even. */
+int orc_pack_w4(const int8_t *wq, int64_t N, int64_t K, uint8_t *packed) {
+  if (K % 2 != 0) return -1;
+  for (int64_t n = 0; n < N; ++n)
+    for (int64_t j = 0; j < K / 2; ++j) {
+      int lo = wq[n * K + 2 * j], hi = wq[n * K + 2 * j + 1];
+      if (lo < -8 || lo > 7 || hi < -8 || hi > 7) return -1;
+      packed[n * (K / 2) + j] = (uint8_t)((lo & 0xF) | ((hi & 0xF) << 4));
+    }
   return 0;
 }
 

@@ -97,6 +97,71 @@ def test_worked_weight_quant(golden_dir):
     assert wq.tolist() == qs
 
 
+def test_worked_weight_quant_w4(golden_dir):
+    fx = read_fixture(golden_dir, "weight_quant_w4_worked.txt")
+    rows, sws, qs, packed = [], [], [], []
+    for k, v in fx:
+        w, sw, q, pk = v.split("|")
+        rows.append(parse_floats(w))
+        sws.append(float(sw.split()[1]))
+        qs.append([int(t) for t in q.split()[1:]])
+        packed.append([int(t) for t in pk.split()[1:]])
+    wq, s_w = oracle.quantize_weight(bf16_bits(np.array(rows, np.float32)), bits=4)
+    assert s_w[0].tolist() == sws
+    assert wq.tolist() == qs
+    assert oracle.pack_w4(wq).tolist() == packed
+
+
+def test_w4_codes_bounds_and_half_step():
+    """W4 codes lie in [-7, 7], the largest |w| of each channel maps to +-7, and
+    every weight is within half a step of its reconstruction s_w q."""
+    rng = np.random.default_rng(7)
+    w = (rng.standard_normal((16, 96)) * rng.uniform(0.01, 1.0, (16, 1))).astype(np.float32)
+    wb = bf16_bits(w)
+    wf = (wb.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    wq, s_w = oracle.quantize_weight(wb, bits=4)
+    assert wq.min() >= -7 and wq.max() <= 7
+    arg = np.abs(wf).argmax(axis=1)
+    assert np.all(np.abs(wq[np.arange(16), arg]) == 7)
+    err = np.abs(wf - s_w[0][:, None].astype(np.float64) * wq)
+    assert np.all(err <= s_w[0][:, None] * (0.5 + 1e-6))
+
+
+def test_w4_input_segments_use_their_own_amax():
+    """With input segments every (channel, segment) pair has its own step."""
+    w = np.zeros((2, 64), np.float32)
+    w[:, :32] = 0.875      # segment 0: amax 7/8 -> s_w 1/8, codes 7
+    w[:, 32:] = -0.109375  # segment 1: amax 7/64 -> s_w 1/64, codes -7
+    wq, s_w = oracle.quantize_weight(bf16_bits(w), mode=oracle.MODE_INPUT, offsets=[0, 32, 64],
+                                     bits=4)
+    assert s_w.tolist() == [[0.125, 0.125], [0.015625, 0.015625]]
+    assert np.all(wq[:, :32] == 7) and np.all(wq[:, 32:] == -7)
+
+
+def test_w4_pack_nibble_order_and_range():
+    wq = np.array([[-8, 7, 1, -1, 0, -8]], np.int8)
+    assert oracle.pack_w4(wq).tolist() == [[0x78, 0xF1, 0x80]]
+    with pytest.raises(Exception):
+        oracle.pack_w4(np.array([[8, 0]], np.int8))
+
+
+def test_w4_layer_equals_brute_force_dequantized_product():
+    """W4A8 layer: the oracle's fp32 result against the dequantized operands
+    multiplied in float64 (the DualScale factorisation with 4-bit weights)."""
+    rng = np.random.default_rng(3)
+    M, K, N = 7, 96, 9
+    x = (rng.standard_normal((M, K)) * 2).astype(np.float32)
+    xc = (rng.standard_normal((32, K)) * 2).astype(np.float32)
+    w = (rng.standard_normal((N, K)) * 0.05).astype(np.float32)
+    r = oracle.layer(bf16_bits(x), bf16_bits(w), bf16_bits(xc), weight_bits=4)
+    s = r["s_act"][0, 0]
+    xt = s[0] * r["planes"][0, 0].astype(np.float64) + s[1] * r["planes"][0, 1]
+    wt = r["s_w"][0][:, None].astype(np.float64) * r["wq"]
+    assert r["wq"].min() >= -7 and r["wq"].max() <= 7
+    ref = xt @ wt.T
+    assert np.max(np.abs(r["y"] - ref)) <= 1e-5 * (np.abs(ref).max() + 1e-30)
+
+
 def _ints(s):
     return [int(v) for v in s.split()]
 
