@@ -174,7 +174,7 @@ def traffic_from_profile():
 
 # ------------------------------------------------------------- our path
 class GpuLayer:
-    def __init__(self, L, dev, adaptive=False):
+    def __init__(self, L, dev, adaptive=False, weight_bits=8, w_operand=None):
         from w8a8_gemm_b200 import binding as B
         from w8a8_gemm_b200.layer import DualScaleSegLinear
         self.L = L
@@ -183,7 +183,8 @@ class GpuLayer:
         d = None if L.d is None else L.d.to(dev)
         bias = None if L.bias is None else L.bias.to(dev)
         self.lin = DualScaleSegLinear(L.w.to(dev), bias, d, seg, L.x_cal.to(dev),
-                                      adaptive=adaptive)
+                                      adaptive=adaptive, weight_bits=weight_bits,
+                                      w_operand=w_operand)
         self.x = L.x.to(dev)
         self.planes = torch.empty(L.G, self.lin.seg.P, L.M, L.K, dtype=torch.int8, device=dev)
         self.y = torch.empty(L.M, L.N, dtype=torch.bfloat16, device=dev)
@@ -201,7 +202,12 @@ def run_ours(args, ws, rank, local):
     from w8a8_gemm_b200 import binding as B
     B.lib()  # fail loudly now if the library is missing
     layers_cpu = wl.config_layers(args.config, seed=0)
-    glayers = [GpuLayer(L, dev, adaptive=args.adaptive) for L in layers_cpu]
+    # W4A8: every layer keeps packed weights and expands them into one shared
+    # int8 operand buffer before its GEMM (inside the timed GEMM region).
+    w_operand = (torch.empty(max(L.N * L.K for L in layers_cpu), dtype=torch.int8, device=dev)
+                 if args.weight_bits == 4 else None)
+    glayers = [GpuLayer(L, dev, adaptive=args.adaptive, weight_bits=args.weight_bits,
+                        w_operand=w_operand) for L in layers_cpu]
     torch.cuda.synchronize()
     eff_ops = sum(layer_units(g.L, g.lin.seg.P)[0] for g in glayers)
     exe_ops = sum(layer_units(g.L, g.lin.seg.P)[1] for g in glayers)
@@ -267,7 +273,7 @@ def run_ours(args, ws, rank, local):
                                quant_us=1e3 * q_ms[i] / args.steps,
                                gemm_us=1e3 * g_ms[i] / args.steps)
                           for i, g in enumerate(glayers)],
-               launches=2 * nl * args.steps)
+               launches=(3 if args.weight_bits == 4 else 2) * nl * args.steps)
 
     # Each activation-quantize launch alone after an L2 flush: the kernel's own
     # HBM roofline, free of the write-back left in L2 by the previous kernel of
@@ -368,6 +374,9 @@ def main(argv=None):
     ap.add_argument("--e2e-steps", type=int, default=40)
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--weight-bits", type=int, default=8, choices=[8, 4],
+                    help="4: W4A8 weights (packed; expanded to the int8 operand before each "
+                         "GEMM, inside the timed GEMM region)")
     ap.add_argument("--adaptive", action="store_true",
                     help="single-scale path on layers whose calibrated sides differ by < 2x")
     args = ap.parse_args(argv)
@@ -436,6 +445,9 @@ def main(argv=None):
                               for p in res["per_layer"]],
                    "path": ("adaptive: single-scale where calibrated sides differ < 2x"
                             if args.adaptive else "DualScale on every layer"),
+                   "weights": ("W4A8: packed 4-bit codes, expanded to the int8 operand before "
+                               "each GEMM (counted in the GEMM time)"
+                               if args.weight_bits == 4 else "W8A8"),
                    "output": "bf16",
                    "l2": "flushed between steps, untimed: 512 MiB written, then 256 MiB read",
                    "parallelism": f"replicas x{n_gpus}"},

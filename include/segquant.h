@@ -90,6 +90,19 @@ typedef enum { SQ_OUT_BF16 = 0, SQ_OUT_F32 = 1 } sq_out_dtype;
 #define SQ_FLAG_SINGLE_SCALE 1
 
 /*
+ * SQ_FLAG_W4: the layer's weights are W4A8 codes ("SegQuant-4", the W4A8 rows
+ * of the results tables and the deployment-cost table of the papernotes.org
+ * and author pages; the pages give no formula, the reading is the W8 rule with
+ * q_max = 7).  They are stored packed (sq_quantize_weight_w4) and expanded by
+ * sq_unpack_weight_w4 into the int8 GEMM operand holding 16*q (the code in the
+ * high nibble of each byte).  With this flag sq_dualscale_seglinear_gemm
+ * multiplies s+ and s- by 2^-4 when it loads them, which is exact, so the
+ * result equals the W4A8 definition with codes q bit for bit.  The flag has no
+ * effect on the activation calls.
+ */
+#define SQ_FLAG_W4 2
+
+/*
  * Segment table (SegLinear).  `offsets` is a HOST array of n_seg + 1 strictly
  * increasing int32 values from 0 to the segmented extent (N for SQ_SEG_OUTPUT,
  * K for SQ_SEG_INPUT).  SQ_SEG_NONE takes n_seg = 1 and offsets may be NULL.
@@ -106,7 +119,7 @@ typedef struct {
   int32_t n_seg;           /* number of segments, 1..SQ_MAX_SEGMENTS */
   const int32_t *offsets;  /* host, n_seg + 1 entries            */
   int32_t n_groups;        /* G                                  */
-  int32_t flags;           /* 0 (DualScale) or SQ_FLAG_SINGLE_SCALE */
+  int32_t flags;           /* 0 or SQ_FLAG_SINGLE_SCALE, optionally | SQ_FLAG_W4 */
 } sq_segments;
 
 /*
@@ -166,6 +179,29 @@ SQ_API sq_status sq_quantize_weight_seg(const void *w, int64_t N, int64_t K,
                                  int8_t *wq, float *s_w, sq_stream_t stream);
 
 /*
+ * sq_quantize_weight_w4 -- W4A8 weight quantization (offline): the rule of
+ * sq_quantize_weight_seg with q_max = 7, s_w[i][n] = max_k |w'| / 7 (1 if 0),
+ * q = rne(clamp(w'/s_w, -7, 7)), stored two codes per byte: byte [n][j] holds
+ * channel 2j in its low nibble and 2j + 1 in its high nibble, 4-bit two's
+ * complement.
+ *   w    bf16 [N][K] (K % 16 == 0, 16-byte aligned);  d fp32 [G][K] or NULL
+ *   wq4  uint8 [N][K/2] output (16-byte aligned);  s_w fp32 [S][N] output
+ */
+SQ_API sq_status sq_quantize_weight_w4(const void *w, int64_t N, int64_t K,
+                                const float *d, const sq_segments *seg,
+                                uint8_t *wq4, float *s_w, sq_stream_t stream);
+
+/*
+ * sq_unpack_weight_w4 -- expands packed W4 codes into the int8 GEMM operand:
+ * wq[n][k] = 16 * q[n][k] (in [-112, 112]).  An HBM-bound pass over N*K/2 +
+ * N*K bytes, run before a GEMM with SQ_FLAG_W4; the caller owns both buffers,
+ * so one wq buffer can serve every W4 layer in turn.
+ *   wq4 uint8 [N][K/2], wq int8 [N][K], both 16-byte aligned, K % 16 == 0.
+ */
+SQ_API sq_status sq_unpack_weight_w4(const uint8_t *wq4, int64_t N, int64_t K, int8_t *wq,
+                              sq_stream_t stream);
+
+/*
  * sq_dualscale_seglinear_gemm -- the batched int8 GEMM with the fused DualScale
  * reconstruction.  Pages: papernotes.org section DualScale (one BatchedGEMM
  * launch over X^+ and X^-, results merged in a fused epilogue) and section
@@ -185,6 +221,8 @@ SQ_API sq_status sq_quantize_weight_seg(const void *w, int64_t N, int64_t K,
  *   y      bf16 or fp32 [M][ldy] output, ldy >= N, ldy*elem % 16 == 0,
  *          16-byte aligned
  *   K % 16 == 0, K >= 16; N >= 1; M == 0 is a valid no-op.
+ * With SQ_FLAG_W4, wq is the output of sq_unpack_weight_w4 (16 q) and the
+ * result is that of the codes q (see SQ_FLAG_W4).
  * Returns SQ_ERR_OVERFLOW when a K-segment is wider than 132104.
  */
 SQ_API sq_status sq_dualscale_seglinear_gemm(const int8_t *planes, const int8_t *wq,

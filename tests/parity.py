@@ -9,8 +9,8 @@ from w8a8_gemm_b200 import binding as B
 from w8a8_gemm_b200 import workloads as wl
 
 
-def segments(layer: wl.Layer, single=False) -> B.Segments:
-    flags = B.SQ_FLAG_SINGLE_SCALE if single else 0
+def segments(layer: wl.Layer, single=False, weight_bits=8) -> B.Segments:
+    flags = (B.SQ_FLAG_SINGLE_SCALE if single else 0) | (B.SQ_FLAG_W4 if weight_bits == 4 else 0)
     if layer.mode == wl.MODE_NONE:
         return B.Segments(B.SQ_SEG_NONE, None, 1, flags)
     return B.Segments(layer.mode, list(layer.offsets), layer.G, flags)
@@ -21,20 +21,30 @@ def oracle_offsets(layer: wl.Layer):
 
 
 def gpu_run(layer: wl.Layer, out_dtype=torch.float32, with_bias=True, s32=False,
-            single=False):
+            single=False, weight_bits=8):
     """CUDA path: weight quantization, calibration, activation quantization and
-    the fused GEMM, all through the library."""
+    the fused GEMM, all through the library.  weight_bits=4: W4A8 weights,
+    packed, then expanded into the GEMM operand (16 q); out["wq"] is then the
+    packed uint8 [N][K/2] and out["wq16"] the operand."""
     dev = torch.device("cuda")
-    seg = segments(layer, single)
+    seg = segments(layer, single, weight_bits)
     x = layer.x.to(dev)
     w = layer.w.to(dev)
     xc = layer.x_cal.to(dev)
     d = None if layer.d is None else layer.d.to(dev)
     bias = layer.bias.to(dev) if (with_bias and layer.bias is not None) else None
     M, K, N, G, S = layer.M, layer.K, layer.N, layer.G, layer.S
-    wq = torch.empty(N, K, dtype=torch.int8, device=dev)
     s_w = torch.empty(S, N, dtype=torch.float32, device=dev)
-    B.sq_quantize_weight_seg(w, d, seg, wq, s_w)
+    extra = {}
+    if weight_bits == 4:
+        wq4 = torch.empty(N, K // 2, dtype=torch.uint8, device=dev)
+        B.sq_quantize_weight_w4(w, d, seg, wq4, s_w)
+        wq = torch.empty(N, K, dtype=torch.int8, device=dev)
+        B.sq_unpack_weight_w4(wq4, wq)
+        extra = dict(wq=wq4, wq16=wq)
+    else:
+        wq = torch.empty(N, K, dtype=torch.int8, device=dev)
+        B.sq_quantize_weight_seg(w, d, seg, wq, s_w)
     s_act = torch.empty(G, S, 2, dtype=torch.float32, device=dev)
     B.sq_calibrate_act(xc, d, seg, s_act)
     planes = torch.empty(G, seg.P, M, K, dtype=torch.int8, device=dev)
@@ -43,6 +53,7 @@ def gpu_run(layer: wl.Layer, out_dtype=torch.float32, with_bias=True, s32=False,
     y = torch.empty(M, ldy, dtype=out_dtype, device=dev)[:, :N]
     B.sq_dualscale_seglinear_gemm(planes, wq, s_w, s_act, bias, y, seg)
     out = dict(wq=wq, s_w=s_w, s_act=s_act, planes=planes, y=y)
+    out.update(extra)
     if s32:
         acc = torch.empty(S, seg.P, M, N, dtype=torch.int32, device=dev)
         B.sq_debug_gemm_s32(planes, wq, seg, acc)
@@ -52,16 +63,21 @@ def gpu_run(layer: wl.Layer, out_dtype=torch.float32, with_bias=True, s32=False,
     return out
 
 
-def oracle_prep(layer: wl.Layer, single=False):
-    """Oracle calibration and quantization of both operands."""
+def oracle_prep(layer: wl.Layer, single=False, weight_bits=8):
+    """Oracle calibration and quantization of both operands (weight_bits=4:
+    W4A8 codes in [-7, 7] in "wq" and their packed storage in "wq4")."""
     off = oracle_offsets(layer)
     d = None if layer.d is None else layer.d.numpy()
     s_act = oracle.calibrate_act(wl.bits(layer.x_cal), d, layer.mode, off, layer.G, layer.N,
                                  single)
     planes = oracle.quantize_act(wl.bits(layer.x), s_act, d, layer.mode, off, layer.G, layer.N,
                                  single)
-    wq, s_w = oracle.quantize_weight(wl.bits(layer.w), d, layer.mode, off, layer.G)
-    return dict(s_act=s_act, planes=planes, wq=wq, s_w=s_w)
+    wq, s_w = oracle.quantize_weight(wl.bits(layer.w), d, layer.mode, off, layer.G,
+                                     bits=weight_bits)
+    out = dict(s_act=s_act, planes=planes, wq=wq, s_w=s_w)
+    if weight_bits == 4:
+        out["wq4"] = oracle.pack_w4(wq)
+    return out
 
 
 def oracle_y(layer, prep, rows=None, with_bias=True, threads=None):

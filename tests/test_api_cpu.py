@@ -109,7 +109,7 @@ def test_segment_table_validation(L):
 
 def test_unknown_flags_rejected(L):
     p = ctypes.c_void_p
-    s = B.Segments(B.SQ_SEG_NONE, None, 1, flags=2)
+    s = B.Segments(B.SQ_SEG_NONE, None, 1, flags=4)
     c, keep = s._c()
     assert L.sq_quantize_act(p(FAKE), 4, 32, 32, None, p(FAKE), ctypes.byref(c), p(FAKE),
                              None) == SQ_ERR_INVALID_ARG
@@ -152,3 +152,22 @@ def test_binding_without_library_fails_loudly(monkeypatch, tmp_path):
     monkeypatch.setattr(B, "_lib", None)
     with pytest.raises(RuntimeError, match="missing"):
         B.lib()
+
+
+def test_w4_calls_validate_on_host(L):
+    p = ctypes.c_void_p
+    c, keep = _seg(B.SQ_SEG_NONE, None)
+    # K not a multiple of 16
+    assert L.sq_quantize_weight_w4(p(FAKE), 8, 24, None, ctypes.byref(c), p(FAKE), p(FAKE),
+                                   None) == SQ_ERR_INVALID_ARG
+    # misaligned packed output
+    assert L.sq_quantize_weight_w4(p(FAKE), 8, 32, None, ctypes.byref(c), p(FAKE + 8), p(FAKE),
+                                   None) == SQ_ERR_ALIGNMENT
+    assert L.sq_unpack_weight_w4(p(FAKE), 0, 32, p(FAKE), None) == SQ_ERR_INVALID_ARG
+    assert L.sq_unpack_weight_w4(p(FAKE), 8, 40, p(FAKE), None) == SQ_ERR_INVALID_ARG
+    assert L.sq_unpack_weight_w4(p(FAKE + 4), 8, 32, p(FAKE), None) == SQ_ERR_ALIGNMENT
+    # the W4 flag is a valid segment-table flag, alone or with single scale
+    for flags in (B.SQ_FLAG_W4, B.SQ_FLAG_W4 | B.SQ_FLAG_SINGLE_SCALE):
+        cs, keep = B.Segments(B.SQ_SEG_NONE, None, 1, flags=flags)._c()
+        assert L.sq_dualscale_seglinear_gemm(None, None, None, None, None, None, 0,
+                                             0, 16, 64, 16, ctypes.byref(cs), None) == 0

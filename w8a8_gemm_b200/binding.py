@@ -23,8 +23,10 @@ SQ_SEG_NONE, SQ_SEG_OUTPUT, SQ_SEG_INPUT = 0, 1, 2
 SQ_OUT_BF16, SQ_OUT_F32 = 0, 1
 SQ_MAX_SEGMENTS = 64
 SQ_FLAG_SINGLE_SCALE = 1
+SQ_FLAG_W4 = 2
 
 EXPORTED = ("sq_calibrate_act", "sq_quantize_act", "sq_quantize_weight_seg",
+            "sq_quantize_weight_w4", "sq_unpack_weight_w4",
             "sq_dualscale_seglinear_gemm", "sq_debug_gemm_s32", "sq_get_device_status",
             "sq_status_string", "sq_version", "sq_debug_timeout_probe")
 
@@ -45,7 +47,8 @@ class _Segments(ctypes.Structure):
 class Segments:
     """SegLinear segment table: mode, boundaries (over N for output mode, over
     K for input mode), the number of activation groups G, and flags
-    (SQ_FLAG_SINGLE_SCALE for the single-scale path)."""
+    (SQ_FLAG_SINGLE_SCALE for the single-scale path, SQ_FLAG_W4 for a GEMM whose
+    weight operand comes from sq_unpack_weight_w4)."""
     mode: int = SQ_SEG_NONE
     offsets: Optional[Sequence[int]] = None
     n_groups: int = 1
@@ -92,6 +95,8 @@ def lib() -> ctypes.CDLL:
         L.sq_calibrate_act.argtypes = [p, i64, i64, i64, p, seg, p, p]
         L.sq_quantize_act.argtypes = [p, i64, i64, i64, p, p, seg, p, p]
         L.sq_quantize_weight_seg.argtypes = [p, i64, i64, p, seg, p, p, p]
+        L.sq_quantize_weight_w4.argtypes = [p, i64, i64, p, seg, p, p, p]
+        L.sq_unpack_weight_w4.argtypes = [p, i64, i64, p, p]
         L.sq_dualscale_seglinear_gemm.argtypes = [p, p, p, p, p, p, ctypes.c_int, i64, i64, i64,
                                                   i64, seg, p]
         L.sq_debug_gemm_s32.argtypes = [p, p, i64, i64, i64, seg, p, p]
@@ -101,6 +106,7 @@ def lib() -> ctypes.CDLL:
         L.sq_status_string.restype = ctypes.c_char_p
         L.sq_version.argtypes = []
         for f in (L.sq_calibrate_act, L.sq_quantize_act, L.sq_quantize_weight_seg,
+                  L.sq_quantize_weight_w4, L.sq_unpack_weight_w4,
                   L.sq_dualscale_seglinear_gemm, L.sq_debug_gemm_s32, L.sq_get_device_status,
                   L.sq_version, L.sq_debug_timeout_probe):
             f.restype = ctypes.c_int
@@ -186,6 +192,36 @@ def sq_quantize_weight_seg(w: torch.Tensor, d: Optional[torch.Tensor], seg: Segm
     _check(lib().sq_quantize_weight_seg(_ptr(w), N, K, _ptr(d), ctypes.byref(cs), _ptr(wq),
                                         _ptr(s_w), _stream()), "sq_quantize_weight_seg")
     return wq, s_w
+
+
+def sq_quantize_weight_w4(w: torch.Tensor, d: Optional[torch.Tensor], seg: Segments,
+                          wq4: torch.Tensor, s_w: torch.Tensor):
+    """W4A8 weight quantization: packed codes wq4 uint8 [N][K/2], s_w fp32 [S][N]."""
+    _need(w, torch.bfloat16, "w")
+    _need(d, torch.float32, "d", optional=True)
+    _need(wq4, torch.uint8, "wq4")
+    _need(s_w, torch.float32, "s_w")
+    N, K = w.shape
+    if not (w.is_contiguous() and wq4.is_contiguous() and s_w.is_contiguous()):
+        raise ValueError("w, wq4 and s_w must be contiguous")
+    if tuple(wq4.shape) != (N, K // 2):
+        raise ValueError(f"wq4 must be [{N}, {K // 2}]")
+    cs, keep = seg._c()
+    _check(lib().sq_quantize_weight_w4(_ptr(w), N, K, _ptr(d), ctypes.byref(cs), _ptr(wq4),
+                                       _ptr(s_w), _stream()), "sq_quantize_weight_w4")
+    return wq4, s_w
+
+
+def sq_unpack_weight_w4(wq4: torch.Tensor, wq: torch.Tensor) -> torch.Tensor:
+    """Packed W4 codes -> the int8 GEMM operand wq [N][K] = 16 q."""
+    _need(wq4, torch.uint8, "wq4")
+    _need(wq, torch.int8, "wq")
+    N, K = wq.shape
+    if tuple(wq4.shape) != (N, K // 2) or not (wq4.is_contiguous() and wq.is_contiguous()):
+        raise ValueError(f"wq4 must be contiguous [{N}, {K // 2}] and wq contiguous [{N}, {K}]")
+    _check(lib().sq_unpack_weight_w4(_ptr(wq4), N, K, _ptr(wq), _stream()),
+           "sq_unpack_weight_w4")
+    return wq
 
 
 def sq_dualscale_seglinear_gemm(planes: torch.Tensor, wq: torch.Tensor, s_w: torch.Tensor,

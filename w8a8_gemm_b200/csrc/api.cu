@@ -57,8 +57,9 @@ sq_status parse_segments(const sq_segments *seg, int64_t K, int64_t extent_n, Se
   if (seg->mode < SQ_SEG_NONE || seg->mode > SQ_SEG_INPUT) return SQ_ERR_INVALID_ARG;
   if (seg->n_seg < 1 || seg->n_seg > SQ_MAX_SEGMENTS || seg->n_groups < 1)
     return SQ_ERR_INVALID_ARG;
-  if (seg->flags != 0 && seg->flags != SQ_FLAG_SINGLE_SCALE) return SQ_ERR_INVALID_ARG;
+  if ((seg->flags & ~(SQ_FLAG_SINGLE_SCALE | SQ_FLAG_W4)) != 0) return SQ_ERR_INVALID_ARG;
   p.P = (seg->flags & SQ_FLAG_SINGLE_SCALE) ? 1 : 2;
+  p.w4 = (seg->flags & SQ_FLAG_W4) ? 1 : 0;
   p.mode = seg->mode;
   p.n_seg = seg->n_seg;
   p.G = seg->n_groups;
@@ -242,6 +243,31 @@ sq_status sq_quantize_weight_seg(const void *w, int64_t N, int64_t K, const floa
   SQ_TRY(check_device());
   return from_cuda(launch_quantize_weight(static_cast<const uint16_t *>(w), N, K, d, sp, wq, s_w,
                                           reinterpret_cast<cudaStream_t>(stream)));
+}
+
+sq_status sq_quantize_weight_w4(const void *w, int64_t N, int64_t K, const float *d,
+                                const sq_segments *seg, uint8_t *wq4, float *s_w,
+                                sq_stream_t stream) {
+  if (N < 1 || N > INT32_MAX) return SQ_ERR_INVALID_ARG;
+  SQ_TRY(check_k(K));
+  SegParams sp;
+  SQ_TRY(parse_segments(seg, K, N, &sp));
+  if (w == nullptr || wq4 == nullptr || s_w == nullptr) return SQ_ERR_INVALID_ARG;
+  if (!aligned(w, 16) || !aligned(wq4, 16) || !aligned(s_w, 4) || (d && !aligned(d, 4)))
+    return SQ_ERR_ALIGNMENT;
+  SQ_TRY(check_device());
+  return from_cuda(launch_quantize_weight_w4(static_cast<const uint16_t *>(w), N, K, d, sp, wq4,
+                                             s_w, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+sq_status sq_unpack_weight_w4(const uint8_t *wq4, int64_t N, int64_t K, int8_t *wq,
+                              sq_stream_t stream) {
+  if (N < 1 || N > INT32_MAX) return SQ_ERR_INVALID_ARG;
+  SQ_TRY(check_k(K));
+  if (wq4 == nullptr || wq == nullptr) return SQ_ERR_INVALID_ARG;
+  if (!aligned(wq4, 16) || !aligned(wq, 16)) return SQ_ERR_ALIGNMENT;
+  SQ_TRY(check_device());
+  return from_cuda(launch_unpack_w4(wq4, N, K, wq, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 sq_status sq_dualscale_seglinear_gemm(const int8_t *planes, const int8_t *wq, const float *s_w,

@@ -58,6 +58,9 @@ struct GemmParams {
   int32_t n_off[SQ_MAX_SEGMENTS + 1];
   const float *s_w;
   const float *s_act;
+  // Factor applied to s+ and s- as they are loaded: 1, or 2^-4 when the weight
+  // operand holds 16 q of W4A8 codes q (exact: a power of two).
+  float act_mul;
   const uint16_t *bias;
   void *y;
   int64_t ldy;
@@ -364,13 +367,17 @@ __global__ void __launch_bounds__(threads_for(EPI_WARPS), 1)
           const int64_t n = nb + q * 32 + lane;
           sw_next[q] = n < p.N ? p.s_w[n] : 0.0f;
         }
-        sp_next = p.s_act[g * p.S * 2 + 0];
-        sm_next = p.s_act[g * p.S * 2 + 1];
+        sp_next = __fmul_rn(p.s_act[g * p.S * 2 + 0], p.act_mul);
+        sm_next = __fmul_rn(p.s_act[g * p.S * 2 + 1], p.act_mul);
       }
       const int units = SEGK ? p.S : 1;
       for (int u = 0; u < units; ++u) {
-        const float sp = (SEGK && OUT != OUT_S32) ? sp_next : p.s_act[(g * p.S + u) * 2 + 0];
-        const float sm = (SEGK && OUT != OUT_S32) ? sm_next : p.s_act[(g * p.S + u) * 2 + 1];
+        const float sp = (SEGK && OUT != OUT_S32)
+                             ? sp_next
+                             : __fmul_rn(p.s_act[(g * p.S + u) * 2 + 0], p.act_mul);
+        const float sm = (SEGK && OUT != OUT_S32)
+                             ? sm_next
+                             : __fmul_rn(p.s_act[(g * p.S + u) * 2 + 1], p.act_mul);
         float *cst = cst_base;
         if constexpr (SEGK && OUT != OUT_S32) {
           // Folded coefficients of K-segment u: c+- = s_w[u][n] * s+-[u], into
@@ -389,8 +396,8 @@ __global__ void __launch_bounds__(threads_for(EPI_WARPS), 1)
               const int64_t n = nb + q * 32 + lane;
               sw_next[q] = n < p.N ? swn[n] : 0.0f;
             }
-            sp_next = p.s_act[(g * p.S + u + 1) * 2 + 0];
-            sm_next = p.s_act[(g * p.S + u + 1) * 2 + 1];
+            sp_next = __fmul_rn(p.s_act[(g * p.S + u + 1) * 2 + 0], p.act_mul);
+            sm_next = __fmul_rn(p.s_act[(g * p.S + u + 1) * 2 + 1], p.act_mul);
           }
           __syncwarp();
         }
@@ -684,6 +691,7 @@ sq_status launch_gemm(const GemmRequest &r, cudaStream_t stream) {
     for (int i = 0; i <= r.seg.n_seg; ++i) p.n_off[i] = r.seg.off[i];
   p.s_w = r.s_w;
   p.s_act = r.s_act;
+  p.act_mul = r.seg.w4 ? 0.0625f : 1.0f;
   p.bias = r.bias;
   p.y = r.y;
   p.ldy = r.ldy;

@@ -283,12 +283,22 @@ __device__ __forceinline__ float block_max(float v, float *red) {
   return r;
 }
 
+// QMAX = 127 (W8) or 7 (W4A8, "SegQuant-4"); with QMAX = 7 the codes are
+// stored two per byte (channel 2j in the low nibble, 2j + 1 in the high one,
+// 4-bit two's complement), each thread handling channel pairs.
+__device__ __forceinline__ int weight_code(float wv, float s, float qmax) {
+  const float v = fminf(fmaxf(__fdiv_rn(wv, s), -qmax), qmax);
+  return __float2int_rn(v);
+}
+
+template <int QMAX>
 __global__ void __launch_bounds__(256) quant_weight_kernel(const uint16_t *__restrict__ w,
                                                            int64_t N, int64_t K,
                                                            const float *__restrict__ d,
                                                            SegParams seg,
                                                            int8_t *__restrict__ wq,
                                                            float *__restrict__ s_w) {
+  constexpr float kQ = static_cast<float>(QMAX);
   __shared__ float red[32];
   const int64_t n = blockIdx.x;
   const int g = (seg.mode == SQ_SEG_OUTPUT && seg.G > 1) ? seg_index(seg.off, seg.n_seg, n) : 0;
@@ -303,13 +313,37 @@ __global__ void __launch_bounds__(256) quant_weight_kernel(const uint16_t *__res
       amax = fmaxf(amax, fabsf(wv));
     }
     amax = block_max(amax, red);
-    const float s = amax > 0.0f ? __fdiv_rn(amax, 127.0f) : 1.0f;
+    const float s = amax > 0.0f ? __fdiv_rn(amax, kQ) : 1.0f;
     if (threadIdx.x == 0) s_w[i * N + n] = s;
-    for (int64_t k = k0 + threadIdx.x; k < k1; k += blockDim.x) {
-      const float wv = dg ? __fmul_rn(bf16_bits_to_f32(row[k]), dg[k]) : bf16_bits_to_f32(row[k]);
-      const float v = fminf(fmaxf(__fdiv_rn(wv, s), -127.0f), 127.0f);
-      wq[n * K + k] = static_cast<int8_t>(__float2int_rn(v));
+    const auto wval = [&](int64_t k) {
+      return dg ? __fmul_rn(bf16_bits_to_f32(row[k]), dg[k]) : bf16_bits_to_f32(row[k]);
+    };
+    if constexpr (QMAX == 127) {
+      for (int64_t k = k0 + threadIdx.x; k < k1; k += blockDim.x)
+        wq[n * K + k] = static_cast<int8_t>(weight_code(wval(k), s, kQ));
+    } else {
+      // segment bounds are even (multiples of 32), so pairs never straddle one
+      uint8_t *packed = reinterpret_cast<uint8_t *>(wq) + n * (K / 2);
+      for (int64_t j = k0 / 2 + threadIdx.x; j < k1 / 2; j += blockDim.x) {
+        const int lo = weight_code(wval(2 * j), s, kQ), hi = weight_code(wval(2 * j + 1), s, kQ);
+        packed[j] = static_cast<uint8_t>((lo & 0xF) | ((hi & 0xF) << 4));
+      }
     }
+  }
+}
+
+// Packed W4 codes -> the int8 GEMM operand 16 q: each code moves into the high
+// nibble of its own byte (low nibble 0), so no sign extension is needed.  One
+// thread per 8 packed bytes (16 codes); a grid-stride loop over N*K/16 units.
+__global__ void __launch_bounds__(256) unpack_w4_kernel(const uint2 *__restrict__ src,
+                                                        uint4 *__restrict__ dst, int64_t units) {
+  for (int64_t u = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; u < units;
+       u += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const uint2 v = src[u];
+    const uint32_t e0 = (v.x & 0x0F0F0F0Fu) << 4, o0 = v.x & 0xF0F0F0F0u;  // channels 2j, 2j+1
+    const uint32_t e1 = (v.y & 0x0F0F0F0Fu) << 4, o1 = v.y & 0xF0F0F0F0u;
+    dst[u] = make_uint4(__byte_perm(e0, o0, 0x5140), __byte_perm(e0, o0, 0x7362),
+                        __byte_perm(e1, o1, 0x5140), __byte_perm(e1, o1, 0x7362));
   }
 }
 
@@ -380,7 +414,28 @@ cudaError_t launch_quantize_weight(const uint16_t *w, int64_t N, int64_t K, cons
                                    const SegParams &seg, int8_t *wq, float *s_w,
                                    cudaStream_t stream) {
   if (N == 0) return cudaSuccess;
-  quant_weight_kernel<<<static_cast<unsigned>(N), 256, 0, stream>>>(w, N, K, d, seg, wq, s_w);
+  quant_weight_kernel<127><<<static_cast<unsigned>(N), 256, 0, stream>>>(w, N, K, d, seg, wq, s_w);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_quantize_weight_w4(const uint16_t *w, int64_t N, int64_t K, const float *d,
+                                      const SegParams &seg, uint8_t *wq4, float *s_w,
+                                      cudaStream_t stream) {
+  if (N == 0) return cudaSuccess;
+  quant_weight_kernel<7><<<static_cast<unsigned>(N), 256, 0, stream>>>(
+      w, N, K, d, seg, reinterpret_cast<int8_t *>(wq4), s_w);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_unpack_w4(const uint8_t *wq4, int64_t N, int64_t K, int8_t *wq,
+                             cudaStream_t stream) {
+  const int64_t units = N * K / 16;  // K % 16 == 0
+  if (units == 0) return cudaSuccess;
+  int64_t blocks = (units + 255) / 256;
+  const int64_t cap = static_cast<int64_t>(num_sms()) * 8;
+  if (blocks > cap) blocks = cap;
+  unpack_w4_kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(
+      reinterpret_cast<const uint2 *>(wq4), reinterpret_cast<uint4 *>(wq), units);
   return cudaGetLastError();
 }
 

@@ -16,6 +16,7 @@ struct SegParams {
   int32_t G;      // activation groups
   int32_t S;      // K-segments (n_seg in input mode, else 1)
   int32_t P;      // activation planes per group: 2 (DualScale) or 1 (single scale)
+  int32_t w4;     // 1: the weight operand holds 16 q of W4A8 codes q (SQ_FLAG_W4)
   int32_t off[SQ_MAX_SEGMENTS + 1];
 };
 
@@ -36,6 +37,11 @@ sq_status launch_quantize_act(const uint16_t *x, int64_t M, int64_t K, int64_t l
 cudaError_t launch_quantize_weight(const uint16_t *w, int64_t N, int64_t K, const float *d,
                                    const SegParams &seg, int8_t *wq, float *s_w,
                                    cudaStream_t stream);
+cudaError_t launch_quantize_weight_w4(const uint16_t *w, int64_t N, int64_t K, const float *d,
+                                      const SegParams &seg, uint8_t *wq4, float *s_w,
+                                      cudaStream_t stream);
+cudaError_t launch_unpack_w4(const uint8_t *wq4, int64_t N, int64_t K, int8_t *wq,
+                             cudaStream_t stream);
 
 // ---- launcher (gemm.cu) ----------------------------------------------------
 enum OutKind { OUT_BF16 = 0, OUT_F32 = 1, OUT_S32 = 2 };

@@ -21,24 +21,43 @@ class DualScaleSegLinear:
     d      fp32 [G][K] SmoothQuant divisor or None
     seg    binding.Segments
     x_cal  bf16 [rows][K] calibration activations
+    weight_bits  8 (W8A8) or 4 (W4A8: weights kept packed, two codes per byte,
+           and expanded into the int8 GEMM operand before every GEMM; several
+           layers may share one operand buffer, `w_operand`, int8 [>= N*K])
     """
 
     def __init__(self, w: torch.Tensor, bias: Optional[torch.Tensor], d: Optional[torch.Tensor],
                  seg: B.Segments, x_cal: torch.Tensor, out_dtype=torch.bfloat16,
-                 adaptive: bool = False, asymmetry_threshold: float = 2.0):
+                 adaptive: bool = False, asymmetry_threshold: float = 2.0,
+                 weight_bits: int = 8, w_operand: Optional[torch.Tensor] = None):
+        if weight_bits not in (8, 4):
+            raise ValueError("weight_bits must be 8 or 4")
         self.N, self.K = w.shape
+        self.weight_bits = weight_bits
+        if weight_bits == 4:
+            seg = B.Segments(seg.mode, seg.offsets, seg.n_groups, seg.flags | B.SQ_FLAG_W4)
         self.seg = seg
         self.G, self.S = seg.n_groups, seg.S
         self.d = d
         self.bias = bias
         self.out_dtype = out_dtype
         dev = w.device
-        self.wq = torch.empty(self.N, self.K, dtype=torch.int8, device=dev)
         self.s_w = torch.empty(self.S, self.N, dtype=torch.float32, device=dev)
-        B.sq_quantize_weight_seg(w, d, seg, self.wq, self.s_w)
+        if weight_bits == 4:
+            self.wq4 = torch.empty(self.N, self.K // 2, dtype=torch.uint8, device=dev)
+            B.sq_quantize_weight_w4(w, d, seg, self.wq4, self.s_w)
+            if w_operand is None:
+                w_operand = torch.empty(self.N * self.K, dtype=torch.int8, device=dev)
+            if w_operand.numel() < self.N * self.K or w_operand.dtype != torch.int8:
+                raise ValueError("w_operand must be int8 with at least N*K elements")
+            self.wq = w_operand.view(-1)[: self.N * self.K].view(self.N, self.K)
+        else:
+            self.wq4 = None
+            self.wq = torch.empty(self.N, self.K, dtype=torch.int8, device=dev)
+            B.sq_quantize_weight_seg(w, d, seg, self.wq, self.s_w)
         self.s_act = torch.empty(self.G, self.S, 2, dtype=torch.float32, device=dev)
         B.sq_calibrate_act(x_cal, d, seg, self.s_act)
-        if adaptive and not seg.flags:
+        if adaptive and not seg.flags & B.SQ_FLAG_SINGLE_SCALE:
             # Adaptive DualScale: keep the two steps only where the calibrated
             # sides differ by at least `asymmetry_threshold` in some group and
             # K-segment; otherwise switch the layer to one symmetric step.
@@ -47,7 +66,7 @@ class DualScaleSegLinear:
             ratio = torch.maximum(hi, lo) / torch.minimum(hi, lo).clamp_min(1e-30)
             if float(ratio.max()) < asymmetry_threshold:
                 self.seg = B.Segments(seg.mode, seg.offsets, seg.n_groups,
-                                      B.SQ_FLAG_SINGLE_SCALE)
+                                      seg.flags | B.SQ_FLAG_SINGLE_SCALE)
                 B.sq_calibrate_act(x_cal, d, self.seg, self.s_act)
         self.single_scale = bool(self.seg.flags & B.SQ_FLAG_SINGLE_SCALE)
         self._planes = None
@@ -67,6 +86,8 @@ class DualScaleSegLinear:
         M = planes.shape[2]
         if y is None:
             y = torch.empty(M, self.N, dtype=self.out_dtype, device=planes.device)
+        if self.wq4 is not None:
+            B.sq_unpack_weight_w4(self.wq4, self.wq)
         return B.sq_dualscale_seglinear_gemm(planes, self.wq, self.s_w, self.s_act, self.bias,
                                              y, self.seg)
 
