@@ -22,7 +22,8 @@
  *
  * Conventions for every call:
  *  - Every pointer is a DEVICE pointer unless marked "host".  The caller owns
- *    all buffers; the library allocates no device memory in any call.
+ *    all buffers, workspaces included; the library allocates no device memory
+ *    in any call.
  *  - Calls are asynchronous on `stream` (0 = legacy default stream).  A return
  *    of SQ_OK means the arguments were valid and the kernels were launched;
  *    launch failures return SQ_ERR_CUDA.  Faults inside a kernel surface at
@@ -242,6 +243,55 @@ SQ_API sq_status sq_dualscale_seglinear_gemm(const int8_t *planes, const int8_t 
 SQ_API sq_status sq_debug_gemm_s32(const int8_t *planes, const int8_t *wq, int64_t M,
                             int64_t N, int64_t K, const sq_segments *seg,
                             int32_t *acc, sq_stream_t stream);
+
+/*
+ * Host-to-host execution of one layer with overlapped transfers.
+ *
+ * A pipeline owns three CUDA streams and a few events (host-side resources)
+ * and uses a caller-provided device workspace of two slots, each holding one
+ * chunk of `chunk_rows` activation rows (bf16), its planes and its output rows.
+ * sq_dualscale_seglinear_host copies the rows of x_host to the device chunk by
+ * chunk, runs sq_quantize_act and sq_dualscale_seglinear_gemm on each chunk and
+ * copies the output rows back, so that the host-to-device copy of chunk c + 1,
+ * the kernels of chunk c and the device-to-host copy of chunk c - 1 overlap.
+ * The result is that of the device calls on the whole layer, bit for bit: rows
+ * are independent in both kernels.  (The pages measure a single GPU's kernels;
+ * this is serving plumbing around them, not part of the method.)
+ *
+ * sq_host_pipeline_workspace_bytes -- workspace size for layers with K <= max_K,
+ * N <= max_N, G <= max_G and P <= max_P (P = 2 for DualScale, 1 single scale);
+ * 0 for invalid sizes.
+ *
+ * sq_host_pipeline_create -- chunk_rows >= 1; workspace: device memory of at
+ * least sq_host_pipeline_workspace_bytes(...) bytes, 256-byte aligned, owned by
+ * the caller and untouched by anything else while the pipeline is in use.
+ * Creates the streams and events on the current device.
+ *
+ * sq_host_pipeline_destroy -- waits for the pipeline's work, then releases its
+ * streams and events (not the workspace).  NULL is a no-op.
+ *
+ * sq_dualscale_seglinear_host -- arguments as in sq_quantize_act and
+ * sq_dualscale_seglinear_gemm, except that x_host (bf16 [M][ldx]) and y_host
+ * ([M][ldy], bf16 or fp32) are HOST pointers; page-locked memory is needed
+ * for the copies to overlap (pageable memory works, serialised).  The work is
+ * ordered after everything already enqueued on `stream`, and work enqueued on
+ * `stream` afterwards (e.g. cudaStreamSynchronize) waits for the whole layer.
+ * A pipeline serves one host thread at a time.
+ */
+typedef struct sq_host_pipeline sq_host_pipeline;
+
+SQ_API size_t sq_host_pipeline_workspace_bytes(int64_t chunk_rows, int64_t max_K, int64_t max_N,
+                                        int32_t max_G, int32_t max_P);
+SQ_API sq_status sq_host_pipeline_create(int64_t chunk_rows, int64_t max_K, int64_t max_N,
+                                  int32_t max_G, int32_t max_P, void *workspace,
+                                  size_t workspace_bytes, sq_host_pipeline **out);
+SQ_API sq_status sq_host_pipeline_destroy(sq_host_pipeline *pl);
+SQ_API sq_status sq_dualscale_seglinear_host(sq_host_pipeline *pl, const void *x_host,
+                                      int64_t M, int64_t K, int64_t ldx, const float *d,
+                                      const float *s_act, const int8_t *wq,
+                                      const float *s_w, const void *bias, void *y_host,
+                                      sq_out_dtype out_dtype, int64_t N, int64_t ldy,
+                                      const sq_segments *seg, sq_stream_t stream);
 
 /*
  * sq_debug_timeout_probe -- test only: launches one small kernel that waits on

@@ -43,7 +43,7 @@ def test_status_strings(L):
     assert B.status_string(0) == "SQ_OK"
     for code in range(-7, 0):
         assert B.status_string(code).startswith("SQ_ERR_")
-    assert B.lib().sq_version() == 101
+    assert B.lib().sq_version() == 102
 
 
 def _seg(mode, offsets, groups=1):
@@ -171,3 +171,25 @@ def test_w4_calls_validate_on_host(L):
         cs, keep = B.Segments(B.SQ_SEG_NONE, None, 1, flags=flags)._c()
         assert L.sq_dualscale_seglinear_gemm(None, None, None, None, None, None, 0,
                                              0, 16, 64, 16, ctypes.byref(cs), None) == 0
+
+
+def test_host_pipeline_validates_on_host(L):
+    p = ctypes.c_void_p
+    assert L.sq_host_pipeline_workspace_bytes(0, 64, 64, 1, 2) == 0
+    assert L.sq_host_pipeline_workspace_bytes(128, 24, 64, 1, 2) == 0      # K % 16 != 0
+    assert L.sq_host_pipeline_workspace_bytes(128, 64, 64, 1, 3) == 0      # P must be 1 or 2
+    need = L.sq_host_pipeline_workspace_bytes(128, 64, 64, 1, 2)
+    # two slots of x (128*64*2) + planes (2*128*64) + y (128*64*4), 256-byte rounded
+    assert need == 2 * (16384 + 16384 + 32768)
+    h = p()
+    assert L.sq_host_pipeline_create(128, 64, 64, 1, 2, None, need, ctypes.byref(h)) == \
+        SQ_ERR_INVALID_ARG
+    assert L.sq_host_pipeline_create(128, 64, 64, 1, 2, p(FAKE), need - 1, ctypes.byref(h)) == \
+        SQ_ERR_INVALID_ARG
+    assert L.sq_host_pipeline_create(128, 64, 64, 1, 2, p(FAKE + 16), need, ctypes.byref(h)) == \
+        SQ_ERR_ALIGNMENT
+    assert L.sq_host_pipeline_destroy(None) == 0
+    c, keep = _seg(B.SQ_SEG_NONE, None)
+    assert L.sq_dualscale_seglinear_host(None, p(FAKE), 8, 64, 64, None, p(FAKE), p(FAKE),
+                                         p(FAKE), None, p(FAKE), 0, 64, 64, ctypes.byref(c),
+                                         None) == SQ_ERR_INVALID_ARG

@@ -28,7 +28,9 @@ SQ_FLAG_W4 = 2
 EXPORTED = ("sq_calibrate_act", "sq_quantize_act", "sq_quantize_weight_seg",
             "sq_quantize_weight_w4", "sq_unpack_weight_w4",
             "sq_dualscale_seglinear_gemm", "sq_debug_gemm_s32", "sq_get_device_status",
-            "sq_status_string", "sq_version", "sq_debug_timeout_probe")
+            "sq_status_string", "sq_version", "sq_debug_timeout_probe",
+            "sq_host_pipeline_workspace_bytes", "sq_host_pipeline_create",
+            "sq_host_pipeline_destroy", "sq_dualscale_seglinear_host")
 
 
 class SegQuantError(RuntimeError):
@@ -102,11 +104,20 @@ def lib() -> ctypes.CDLL:
         L.sq_debug_gemm_s32.argtypes = [p, p, i64, i64, i64, seg, p, p]
         L.sq_get_device_status.argtypes = []
         L.sq_debug_timeout_probe.argtypes = [ctypes.c_uint32, p]
+        L.sq_host_pipeline_workspace_bytes.argtypes = [i64, i64, i64, ctypes.c_int32,
+                                                       ctypes.c_int32]
+        L.sq_host_pipeline_workspace_bytes.restype = ctypes.c_size_t
+        L.sq_host_pipeline_create.argtypes = [i64, i64, i64, ctypes.c_int32, ctypes.c_int32, p,
+                                              ctypes.c_size_t, ctypes.POINTER(p)]
+        L.sq_host_pipeline_destroy.argtypes = [p]
+        L.sq_dualscale_seglinear_host.argtypes = [p, p, i64, i64, i64, p, p, p, p, p, p,
+                                                  ctypes.c_int, i64, i64, seg, p]
         L.sq_status_string.argtypes = [ctypes.c_int]
         L.sq_status_string.restype = ctypes.c_char_p
         L.sq_version.argtypes = []
         for f in (L.sq_calibrate_act, L.sq_quantize_act, L.sq_quantize_weight_seg,
-                  L.sq_quantize_weight_w4, L.sq_unpack_weight_w4,
+                  L.sq_quantize_weight_w4, L.sq_unpack_weight_w4, L.sq_host_pipeline_create,
+                  L.sq_host_pipeline_destroy, L.sq_dualscale_seglinear_host,
                   L.sq_dualscale_seglinear_gemm, L.sq_debug_gemm_s32, L.sq_get_device_status,
                   L.sq_version, L.sq_debug_timeout_probe):
             f.restype = ctypes.c_int
@@ -262,6 +273,65 @@ def sq_debug_gemm_s32(planes: torch.Tensor, wq: torch.Tensor, seg: Segments,
     _check(lib().sq_debug_gemm_s32(_ptr(planes), _ptr(wq), M, N, K, ctypes.byref(cs), _ptr(acc),
                                    _stream()), "sq_debug_gemm_s32")
     return acc
+
+
+class HostPipeline:
+    """Streams, events and a device workspace (a torch tensor this object owns)
+    for sq_dualscale_seglinear_host: layers with K <= max_K, N <= max_N,
+    G <= max_G, P <= max_P, in chunks of chunk_rows rows."""
+
+    def __init__(self, chunk_rows: int, max_K: int, max_N: int, max_G: int = 1, max_P: int = 2,
+                 device=None):
+        L = lib()
+        nbytes = L.sq_host_pipeline_workspace_bytes(chunk_rows, max_K, max_N, max_G, max_P)
+        if nbytes == 0:
+            raise ValueError("invalid pipeline sizes")
+        self.workspace = torch.empty(nbytes, dtype=torch.uint8,
+                                     device=device or torch.device("cuda"))
+        self._h = ctypes.c_void_p()
+        _check(L.sq_host_pipeline_create(chunk_rows, max_K, max_N, max_G, max_P,
+                                         _ptr(self.workspace), nbytes, ctypes.byref(self._h)),
+               "sq_host_pipeline_create")
+
+    def close(self):
+        if self._h:
+            _check(lib().sq_host_pipeline_destroy(self._h), "sq_host_pipeline_destroy")
+            self._h = ctypes.c_void_p()
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+def sq_dualscale_seglinear_host(pl: HostPipeline, x_host: torch.Tensor, d: Optional[torch.Tensor],
+                                s_act: torch.Tensor, wq: torch.Tensor, s_w: torch.Tensor,
+                                bias: Optional[torch.Tensor], y_host: torch.Tensor,
+                                seg: Segments) -> torch.Tensor:
+    """One layer from host rows x_host (bf16 [M][K], CPU, pinned for overlap)
+    to host rows y_host (bf16 or fp32 [M][N], CPU) through the pipeline; the
+    weights and scales are CUDA tensors.  Ordered on torch's current stream."""
+    if x_host.is_cuda or y_host.is_cuda:
+        raise ValueError("x_host and y_host must be CPU tensors")
+    if x_host.dtype != torch.bfloat16 or y_host.dtype not in (torch.bfloat16, torch.float32):
+        raise ValueError("x_host must be bf16 and y_host bf16 or fp32")
+    _need(d, torch.float32, "d", optional=True)
+    _need(s_act, torch.float32, "s_act")
+    _need(wq, torch.int8, "wq")
+    _need(s_w, torch.float32, "s_w")
+    _need(bias, torch.bfloat16, "bias", optional=True)
+    M, K, ldx = _rows(x_host)
+    N = wq.shape[0]
+    if wq.shape[1] != K or y_host.shape[0] != M or y_host.shape[1] != N or y_host.stride(1) != 1:
+        raise ValueError("shape mismatch between x_host [M,K], wq [N,K] and y_host [M,N]")
+    out = SQ_OUT_BF16 if y_host.dtype == torch.bfloat16 else SQ_OUT_F32
+    cs, keep = seg._c()
+    _check(lib().sq_dualscale_seglinear_host(pl._h, _ptr(x_host), M, K, ldx, _ptr(d), _ptr(s_act),
+                                             _ptr(wq), _ptr(s_w), _ptr(bias), _ptr(y_host), out,
+                                             N, y_host.stride(0), ctypes.byref(cs), _stream()),
+           "sq_dualscale_seglinear_host")
+    return y_host
 
 
 def sq_get_device_status() -> int:

@@ -124,7 +124,7 @@ sq_status from_cuda(cudaError_t e) { return e == cudaSuccess ? SQ_OK : SQ_ERR_CU
 sq_status gemm_common(const int8_t *planes, const int8_t *wq, const float *s_w,
                       const float *s_act, const void *bias, void *y, int out_kind, int64_t M,
                       int64_t N, int64_t K, int64_t ldy, const sq_segments *seg,
-                      cudaStream_t stream) {
+                      cudaStream_t stream, bool launch = true) {
   if (M < 0 || M > INT32_MAX || N < 1 || N > INT32_MAX) return SQ_ERR_INVALID_ARG;
   SQ_TRY(check_k(K));
   SegParams sp;
@@ -143,6 +143,7 @@ sq_status gemm_common(const int8_t *planes, const int8_t *wq, const float *s_w,
     if ((ldy * elem) % 16 != 0) return SQ_ERR_ALIGNMENT;
   }
   SQ_TRY(check_device());
+  if (!launch) return SQ_OK;
   GemmRequest r;
   r.planes = planes;
   r.wq = wq;
@@ -161,7 +162,37 @@ sq_status gemm_common(const int8_t *planes, const int8_t *wq, const float *s_w,
   return launch_gemm(r, stream);
 }
 
+sq_status quantize_common(const void *x, int64_t M, int64_t K, int64_t ldx, const float *d,
+                          const float *s_act, const sq_segments *seg, int8_t *planes,
+                          cudaStream_t stream, bool launch = true) {
+  SQ_TRY(check_act(x, M, K, ldx));
+  SegParams sp;
+  SQ_TRY(parse_segments(seg, K, -1, &sp));
+  if (M == 0) return SQ_OK;
+  if (s_act == nullptr || planes == nullptr) return SQ_ERR_INVALID_ARG;
+  if (!aligned(s_act, 4) || (d && !aligned(d, 4)) || !aligned(planes, 16))
+    return SQ_ERR_ALIGNMENT;
+  SQ_TRY(check_device());
+  if (!launch) return SQ_OK;
+  int *status = device_status_word();
+  if (status == nullptr) return SQ_ERR_CUDA;
+  return launch_quantize_act(static_cast<const uint16_t *>(x), M, K, ldx, d, s_act, sp, planes,
+                             status, stream);
+}
+
 }  // namespace
+
+sq_status validate_quantize_act(const void *x, int64_t M, int64_t K, int64_t ldx, const float *d,
+                                const float *s_act, const sq_segments *seg, int8_t *planes) {
+  return quantize_common(x, M, K, ldx, d, s_act, seg, planes, nullptr, false);
+}
+
+sq_status validate_gemm(const int8_t *planes, const int8_t *wq, const float *s_w,
+                        const float *s_act, const void *bias, void *y, int out_kind, int64_t M,
+                        int64_t N, int64_t K, int64_t ldy, const sq_segments *seg) {
+  return gemm_common(planes, wq, s_w, s_act, bias, y, out_kind, M, N, K, ldy, seg, nullptr,
+                     false);
+}
 
 EncodeTiledFn tensor_map_encoder() {
   static EncodeTiledFn fn = nullptr;
@@ -216,18 +247,8 @@ sq_status sq_calibrate_act(const void *x, int64_t M, int64_t K, int64_t ldx, con
 sq_status sq_quantize_act(const void *x, int64_t M, int64_t K, int64_t ldx, const float *d,
                           const float *s_act, const sq_segments *seg, int8_t *planes,
                           sq_stream_t stream) {
-  SQ_TRY(check_act(x, M, K, ldx));
-  SegParams sp;
-  SQ_TRY(parse_segments(seg, K, -1, &sp));
-  if (M == 0) return SQ_OK;
-  if (s_act == nullptr || planes == nullptr) return SQ_ERR_INVALID_ARG;
-  if (!aligned(s_act, 4) || (d && !aligned(d, 4)) || !aligned(planes, 16))
-    return SQ_ERR_ALIGNMENT;
-  SQ_TRY(check_device());
-  int *status = device_status_word();
-  if (status == nullptr) return SQ_ERR_CUDA;
-  return launch_quantize_act(static_cast<const uint16_t *>(x), M, K, ldx, d, s_act, sp, planes,
-                             status, reinterpret_cast<cudaStream_t>(stream));
+  return quantize_common(x, M, K, ldx, d, s_act, seg, planes,
+                         reinterpret_cast<cudaStream_t>(stream));
 }
 
 sq_status sq_quantize_weight_seg(const void *w, int64_t N, int64_t K, const float *d,
@@ -322,6 +343,6 @@ const char *sq_status_string(sq_status s) {
   return "unknown sq_status";
 }
 
-int32_t sq_version(void) { return 101; }
+int32_t sq_version(void) { return 102; }
 
 }  // extern "C"

@@ -65,6 +65,14 @@ sq_status launch_gemm(const GemmRequest &req, cudaStream_t stream);
 // ---- test-only probe (probe.cu) --------------------------------------------
 cudaError_t launch_timeout_probe(uint32_t limit_us, int *status, cudaStream_t stream);
 
+// Host-side validation of a quantize / GEMM call without launching anything
+// (the checks of sq_quantize_act and sq_dualscale_seglinear_gemm).
+sq_status validate_quantize_act(const void *x, int64_t M, int64_t K, int64_t ldx, const float *d,
+                                const float *s_act, const sq_segments *seg, int8_t *planes);
+sq_status validate_gemm(const int8_t *planes, const int8_t *wq, const float *s_w,
+                        const float *s_act, const void *bias, void *y, int out_kind, int64_t M,
+                        int64_t N, int64_t K, int64_t ldy, const sq_segments *seg);
+
 // Device address of the library's error word on the current device.
 int *device_status_word();
 
