@@ -58,7 +58,7 @@ typedef struct CUstream_st *sq_stream_t;
 typedef enum {
   SQ_OK = 0,
   SQ_ERR_INVALID_ARG = -1,   /* null pointer, bad size, bad segment table     */
-  SQ_ERR_UNSUPPORTED = -2,   /* valid request this build does not implement  */
+  SQ_ERR_UNSUPPORTED = -2,   /* valid request the library does not implement  */
   SQ_ERR_ALIGNMENT = -3,     /* pointer / leading dimension misaligned       */
   SQ_ERR_OVERFLOW = -4,      /* a K-segment could overflow the int32 sum     */
   SQ_ERR_CUDA = -5,          /* a CUDA runtime call failed                    */
@@ -111,7 +111,7 @@ typedef enum { SQ_OUT_BF16 = 0, SQ_OUT_F32 = 1 } sq_out_dtype;
  * only, n_seg, so that every output segment has its own SmoothQuant divisor,
  * s+/s- and activation planes.  S, the number of K-segments, is n_seg for
  * SQ_SEG_INPUT and 1 otherwise.
- * Restrictions of this build: input-segment widths are multiples of 32 (the
+ * Restrictions of this library version: input-segment widths are multiples of 32 (the
  * int8 MMA K step) and at most 132104 (so 128*127*width < 2^31); with G > 1
  * output-segment widths are multiples of 128.
  */

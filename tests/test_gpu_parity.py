@@ -170,7 +170,7 @@ FULL = ["c1_tiny_dualscale", "c2_sd35_adanorm", "c3_sd35_attn_out", "c4_sd35_ffn
 
 @pytest.mark.parametrize("cfg", FULL)
 def test_full_size_configs_sampled_rows(cfg):
-    """BASELINE-sized layers: planes, weights and scales compared in full,
+    """Full-size workload layers: planes, weights and scales compared in full,
     outputs on every row of the first and last M tile plus a strided sample."""
     for L in wl.config_layers(cfg, seed=0):
         prep = oracle_prep(L)

@@ -333,7 +333,7 @@ const char *sq_status_string(sq_status s) {
   switch (s) {
     case SQ_OK: return "SQ_OK";
     case SQ_ERR_INVALID_ARG: return "SQ_ERR_INVALID_ARG: invalid argument";
-    case SQ_ERR_UNSUPPORTED: return "SQ_ERR_UNSUPPORTED: valid request this build does not implement";
+    case SQ_ERR_UNSUPPORTED: return "SQ_ERR_UNSUPPORTED: valid request the library does not implement";
     case SQ_ERR_ALIGNMENT: return "SQ_ERR_ALIGNMENT: pointer or leading dimension misaligned";
     case SQ_ERR_OVERFLOW: return "SQ_ERR_OVERFLOW: K-segment too wide for int32 accumulation";
     case SQ_ERR_CUDA: return "SQ_ERR_CUDA: a CUDA runtime call failed";
