@@ -41,9 +41,21 @@ def lib():
         L.orc_gemm.argtypes = [p, p, p, p, p, i64, i64, i64, i32, i32, p, i32, i32, p, i64, p,
                                i32]
         L.orc_num_threads.argtypes = []
+        L.orc_e4m3_encode.argtypes = [p, i64, p]
+        L.orc_e4m3_decode.argtypes = [p, i64, p]
+        L.orc_calibrate_act_fp8.argtypes = [p, i64, i64, i64, p, i32, i32, p, i32, i64, i32, p]
+        L.orc_quantize_act_fp8.argtypes = [p, i64, i64, i64, p, p, i32, i32, p, i32, i64, i32,
+                                           p]
+        L.orc_quantize_weight_fp8.argtypes = [p, i64, i64, p, i32, i32, p, i32, p, p]
+        L.orc_gemm_fp8_acc.argtypes = [p, p, i64, i64, i64, i32, i32, p, i32, i32, p, i64, p,
+                                       i32]
+        L.orc_gemm_fp8.argtypes = [p, p, p, p, p, i64, i64, i64, i32, i32, p, i32, i32, p, i64,
+                                   p, i32]
         for f in (L.orc_calibrate_act, L.orc_quantize_act, L.orc_quantize_weight,
                   L.orc_quantize_weight_q, L.orc_pack_w4,
-                  L.orc_gemm_s32, L.orc_gemm, L.orc_num_threads):
+                  L.orc_gemm_s32, L.orc_gemm, L.orc_num_threads, L.orc_e4m3_encode,
+                  L.orc_e4m3_decode, L.orc_calibrate_act_fp8, L.orc_quantize_act_fp8,
+                  L.orc_quantize_weight_fp8, L.orc_gemm_fp8_acc, L.orc_gemm_fp8):
             f.restype = ctypes.c_int
         _lib = L
     return _lib
@@ -190,6 +202,107 @@ def layer(x_bits, w_bits, x_cal_bits, d=None, bias_bits=None, mode=MODE_NONE,
     return dict(s_act=s_act, planes=planes, wq=wq, s_w=s_w, y=y)
 
 
+# ------------------------------------------------------------------ FP8 (E4M3)
+def e4m3_encode(v):
+    """fp32 -> E4M3 codes (uint8): round half to even, finite saturation to +-448,
+    NaN -> 0x7F."""
+    v = np.ascontiguousarray(np.asarray(v, dtype=np.float32))
+    out = np.zeros(v.shape, np.uint8)
+    _check(lib().orc_e4m3_encode(_ptr(v), v.size, _ptr(out)), "e4m3_encode")
+    return out
+
+
+def e4m3_decode(b):
+    """E4M3 codes (uint8) -> their fp32 values (NaN for 0x7F / 0xFF)."""
+    b = np.ascontiguousarray(np.asarray(b, dtype=np.uint8))
+    out = np.zeros(b.shape, np.float32)
+    _check(lib().orc_e4m3_decode(_ptr(b), b.size, _ptr(out)), "e4m3_decode")
+    return out
+
+
+def calibrate_act_fp8(x_bits, d=None, mode=MODE_NONE, offsets=None, G=1, N=0, single=False):
+    """AMax calibration of the FP8 path: s+ = max/448, s- = |min|/448."""
+    x = _c(x_bits, np.uint16)
+    M, K = x.shape
+    off, n_seg, S = _seg(mode, offsets, G, N, K)
+    d = _c(d, np.float32)
+    out = np.zeros((G, S, 2), np.float32)
+    _check(lib().orc_calibrate_act_fp8(_ptr(x), M, K, K, _ptr(d), mode, n_seg, _ptr(off), G, N,
+                                       int(single), _ptr(out)), "calibrate_act_fp8")
+    return out
+
+
+def quantize_act_fp8(x_bits, s_act, d=None, mode=MODE_NONE, offsets=None, G=1, N=0,
+                     single=False):
+    """DualScale planes of E4M3 codes: uint8 [G][2][M][K] ([G][1][M][K] single scale)."""
+    x = _c(x_bits, np.uint16)
+    M, K = x.shape
+    off, n_seg, S = _seg(mode, offsets, G, N, K)
+    s = _c(s_act, np.float32)
+    d = _c(d, np.float32)
+    planes = np.zeros((G, 1 if single else 2, M, K), np.uint8)
+    _check(lib().orc_quantize_act_fp8(_ptr(x), M, K, K, _ptr(d), _ptr(s), mode, n_seg, _ptr(off),
+                                      G, N, int(single), _ptr(planes)), "quantize_act_fp8")
+    return planes
+
+
+def quantize_weight_fp8(w_bits, d=None, mode=MODE_NONE, offsets=None, G=1):
+    """E4M3 weights: (wq uint8 [N][K], s_w f32 [S][N]) with s_w = amax/448."""
+    w = _c(w_bits, np.uint16)
+    N, K = w.shape
+    off, n_seg, S = _seg(mode, offsets, G, N, K)
+    d = _c(d, np.float32)
+    wq = np.zeros((N, K), np.uint8)
+    s_w = np.zeros((S, N), np.float32)
+    _check(lib().orc_quantize_weight_fp8(_ptr(w), N, K, _ptr(d), mode, n_seg, _ptr(off), G,
+                                         _ptr(wq), _ptr(s_w)), "quantize_weight_fp8")
+    return wq, s_w
+
+
+def gemm_fp8_acc(planes, wq, mode=MODE_NONE, offsets=None, rows=None, threads=1):
+    """Exact sums of E4M3 products rounded once to fp32: [S][P][rows][N]."""
+    planes = _c(planes, np.uint8)
+    wq = _c(wq, np.uint8)
+    G, P, M, K = planes.shape
+    N = wq.shape[0]
+    off, n_seg, S = _seg(mode, offsets, G, N, K)
+    r, n_rows = _rows(rows, M)
+    acc = np.zeros((S, P, n_rows, N), np.float32)
+    _check(lib().orc_gemm_fp8_acc(_ptr(planes), _ptr(wq), M, N, K, mode, n_seg, _ptr(off), G, P,
+                                  _ptr(r), n_rows, _ptr(acc), threads), "gemm_fp8_acc")
+    return acc
+
+
+def gemm_fp8(planes, wq, s_w, s_act, bias_bits=None, mode=MODE_NONE, offsets=None, rows=None,
+             threads=1):
+    """FP8 layer output fp32 [rows][N]: the W8A8 epilogue on the fp32 sums."""
+    planes = _c(planes, np.uint8)
+    wq = _c(wq, np.uint8)
+    G, P, M, K = planes.shape
+    N = wq.shape[0]
+    off, n_seg, S = _seg(mode, offsets, G, N, K)
+    r, n_rows = _rows(rows, M)
+    y = np.zeros((n_rows, N), np.float32)
+    _check(lib().orc_gemm_fp8(_ptr(planes), _ptr(wq), _ptr(_c(s_w, np.float32)),
+                              _ptr(_c(s_act, np.float32)), _ptr(_c(bias_bits, np.uint16)), M, N,
+                              K, mode, n_seg, _ptr(off), G, P, _ptr(r), n_rows, _ptr(y),
+                              threads), "gemm_fp8")
+    return y
+
+
+def layer_fp8(x_bits, w_bits, x_cal_bits, d=None, bias_bits=None, mode=MODE_NONE, offsets=None,
+              G=1, rows=None, threads=1, single=False):
+    """Whole FP8 pipeline on the CPU: calibrate, quantize both sides, GEMM."""
+    w = _c(w_bits, np.uint16)
+    N = w.shape[0]
+    s_act = calibrate_act_fp8(x_cal_bits, d, mode, offsets, G, N, single)
+    planes = quantize_act_fp8(x_bits, s_act, d, mode, offsets, G, N, single)
+    wq, s_w = quantize_weight_fp8(w, d, mode, offsets, G)
+    y = gemm_fp8(planes, wq, s_w, s_act, bias_bits, mode, offsets, rows, threads)
+    return dict(s_act=s_act, planes=planes, wq=wq, s_w=s_w, y=y)
+
+
 __all__ = ["MODE_NONE", "MODE_OUTPUT", "MODE_INPUT", "calibrate_act",
            "quantize_act", "quantize_weight", "pack_w4", "gemm_s32", "gemm", "layer",
-           "num_threads", "lib"]
+           "num_threads", "lib", "e4m3_encode", "e4m3_decode", "calibrate_act_fp8",
+           "quantize_act_fp8", "quantize_weight_fp8", "gemm_fp8_acc", "gemm_fp8", "layer_fp8"]

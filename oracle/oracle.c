@@ -363,3 +363,241 @@ int orc_gemm(const int8_t *planes, const int8_t *wq, const float *s_w,
   }
   return 0;
 }
+
+/* ===========================================================================
+ * FP8 variant (the pages' "W8A8(fp)" rows for SDXL in the results table,
+ * which they do not define).  Reading: both operands are FP8 E4M3 codes (the
+ * OCP "E4M3FN" format: 1 sign, 4 exponent bits with bias 7, 3 mantissa bits,
+ * no infinities, S.1111.111 is NaN, largest finite 448 = 1.75 * 2^8, smallest
+ * normal 2^-6, subnormals m * 2^-9).  DualScale steps become s+ = max/448 and
+ * s- = |min|/448 (single scale: the larger side / 448), weights
+ * s_w = amax/448; every code is e4m3(fl(v)) with round-half-to-even and
+ * finite saturation to +-448.  The products of two E4M3 values are exact; the
+ * oracle sums them exactly (in double, whose 53 bits hold every such sum for
+ * K < 2^15) and rounds the sum once to fp32; the epilogue is the W8A8 one.
+ * ========================================================================= */
+
+static float orc_e4m3_value(uint8_t b) {
+  int s = b >> 7, e = (b >> 3) & 0xF, m = b & 7;
+  float v;
+  if (e == 0xF && m == 7) return NAN;
+  if (e == 0)
+    v = ldexpf((float)m, -9); /* subnormal: m * 2^-9 */
+  else
+    v = ldexpf((float)(8 + m), e - 10); /* (1 + m/8) * 2^(e-7) */
+  return s ? -v : v;
+}
+
+/* fp32 -> E4M3 code, round half to even, |v| beyond 448 (infinities
+ * included) saturates to 448; NaN gives 0x7F. */
+static uint8_t orc_e4m3_code(float v) {
+  if (isnan(v)) return 0x7F;
+  uint8_t sign = signbit(v) ? 0x80 : 0x00;
+  float a = fabsf(v);
+  if (a >= 448.0f) return sign | 0x7E;
+  /* quantum of the binade of a: 2^(e-3) for normals (e >= -6), 2^-9 below */
+  int e;
+  frexpf(a, &e);         /* a = f * 2^e, f in [0.5, 1): binade exponent e - 1 */
+  int be = e - 1;
+  if (be < -6) be = -6;  /* subnormal range shares the quantum 2^-9 */
+  float q = ldexpf(1.0f, be - 3);
+  float n = rintf(a / q); /* exact division by a power of two, then RNE */
+  float r = n * q;        /* exact; may step into the next binade */
+  if (r > 448.0f) r = 448.0f;
+  /* encode r */
+  if (r == 0.0f) return sign;
+  int re;
+  frexpf(r, &re);
+  int rb = re - 1;
+  if (rb < -6) { /* subnormal: r = m * 2^-9 */
+    int m = (int)ldexpf(r, 9);
+    return sign | (uint8_t)m;
+  }
+  int m = (int)(ldexpf(r, -rb) * 8.0f) - 8;
+  return sign | (uint8_t)(((rb + 7) << 3) | m);
+}
+
+int orc_e4m3_encode(const float *v, int64_t n, uint8_t *out) {
+  for (int64_t i = 0; i < n; ++i) out[i] = orc_e4m3_code(v[i]);
+  return 0;
+}
+
+int orc_e4m3_decode(const uint8_t *b, int64_t n, float *out) {
+  for (int64_t i = 0; i < n; ++i) out[i] = orc_e4m3_value(b[i]);
+  return 0;
+}
+
+int orc_calibrate_act_fp8(const uint16_t *x, int64_t M, int64_t K, int64_t ldx,
+                          const float *d, int mode, int n_seg, const int32_t *offsets,
+                          int G, int64_t N, int single, float *s_act) {
+  if (orc_check_seg(mode, n_seg, offsets, G, N, K)) return -1;
+  int S = (mode == ORC_MODE_INPUT) ? n_seg : 1;
+  for (int g = 0; g < G; ++g) {
+    for (int i = 0; i < S; ++i) {
+      int64_t c0 = (S == 1) ? 0 : offsets[i];
+      int64_t c1 = (S == 1) ? K : offsets[i + 1];
+      float hi = 0.0f, lo = 0.0f;
+      for (int64_t m = 0; m < M; ++m)
+        for (int64_t c = c0; c < c1; ++c) {
+          float dv = d ? d[(int64_t)g * K + c] : 1.0f;
+          float u = orc_bf16(x[m * ldx + c]) / dv;
+          if (u > hi) hi = u;
+          if (u < lo) lo = u;
+        }
+      float sp = (hi > 0.0f) ? hi / 448.0f : 1.0f;
+      float sm = (lo < 0.0f) ? (-lo) / 448.0f : 1.0f;
+      if (single) {
+        float amax = (hi > -lo) ? hi : -lo;
+        sp = (amax > 0.0f) ? amax / 448.0f : 1.0f;
+        sm = sp;
+      }
+      s_act[((int64_t)g * S + i) * 2 + 0] = sp;
+      s_act[((int64_t)g * S + i) * 2 + 1] = sm;
+    }
+  }
+  return 0;
+}
+
+/* Planes of E4M3 codes [G][P][M][K].  x >= 0 (-0.0 included): the + plane
+ * holds e4m3(fl(x * m+)) and the - plane 0x00; x < 0: the - plane holds
+ * e4m3(fl(x * m-)) and the + plane 0x00; NaN: both 0x00.  Single scale: one
+ * plane holding the code of whichever branch applies. */
+int orc_quantize_act_fp8(const uint16_t *x, int64_t M, int64_t K, int64_t ldx,
+                         const float *d, const float *s_act, int mode, int n_seg,
+                         const int32_t *offsets, int G, int64_t N, int single,
+                         uint8_t *planes) {
+  if (orc_check_seg(mode, n_seg, offsets, G, N, K)) return -1;
+  int S = (mode == ORC_MODE_INPUT) ? n_seg : 1;
+  int P = single ? 1 : 2;
+  for (int g = 0; g < G; ++g) {
+    uint8_t *plus = planes + ((int64_t)g * P + 0) * M * K;
+    uint8_t *minus = planes + ((int64_t)g * P + (P - 1)) * M * K;
+    for (int64_t m = 0; m < M; ++m)
+      for (int64_t c = 0; c < K; ++c) {
+        int i = (S == 1) ? 0 : orc_seg_index(offsets, n_seg, c);
+        float sp = s_act[((int64_t)g * S + i) * 2 + 0];
+        float sm = s_act[((int64_t)g * S + i) * 2 + 1];
+        float dv = d ? d[(int64_t)g * K + c] : 1.0f;
+        float mp = 1.0f / (dv * sp);
+        float mm = 1.0f / (dv * sm);
+        float xv = orc_bf16(x[m * ldx + c]);
+        uint8_t qp = 0, qm = 0;
+        if (xv < 0.0f)
+          qm = orc_e4m3_code(xv * mm);
+        else if (xv >= 0.0f)
+          qp = orc_e4m3_code(xv * mp);
+        if (single) {
+          plus[m * K + c] = (xv < 0.0f) ? qm : qp;
+        } else {
+          plus[m * K + c] = qp;
+          minus[m * K + c] = qm;
+        }
+      }
+  }
+  return 0;
+}
+
+int orc_quantize_weight_fp8(const uint16_t *w, int64_t N, int64_t K, const float *d,
+                            int mode, int n_seg, const int32_t *offsets, int G,
+                            uint8_t *wq, float *s_w) {
+  if (orc_check_seg(mode, n_seg, offsets, G, N, K)) return -1;
+  int S = (mode == ORC_MODE_INPUT) ? n_seg : 1;
+  for (int64_t n = 0; n < N; ++n) {
+    int g = (mode == ORC_MODE_OUTPUT && G > 1) ? orc_seg_index(offsets, n_seg, n) : 0;
+    for (int i = 0; i < S; ++i) {
+      int64_t k0 = (S == 1) ? 0 : offsets[i];
+      int64_t k1 = (S == 1) ? K : offsets[i + 1];
+      float amax = 0.0f;
+      for (int64_t k = k0; k < k1; ++k) {
+        float dv = d ? d[(int64_t)g * K + k] : 1.0f;
+        float a = fabsf(orc_bf16(w[n * K + k]) * dv);
+        if (a > amax) amax = a;
+      }
+      float s = (amax > 0.0f) ? amax / 448.0f : 1.0f;
+      s_w[(int64_t)i * N + n] = s;
+      for (int64_t k = k0; k < k1; ++k) {
+        float dv = d ? d[(int64_t)g * K + k] : 1.0f;
+        wq[n * K + k] = orc_e4m3_code((orc_bf16(w[n * K + k]) * dv) / s);
+      }
+    }
+  }
+  return 0;
+}
+
+/* Exact per-segment products of E4M3 codes, rounded once to fp32:
+ * acc layout [S][P][n_rows][N] (fp32). */
+int orc_gemm_fp8_acc(const uint8_t *planes, const uint8_t *wq, int64_t M, int64_t N,
+                     int64_t K, int mode, int n_seg, const int32_t *offsets, int G,
+                     int P, const int64_t *rows, int64_t n_rows, float *acc,
+                     int n_threads) {
+  if (orc_check_seg(mode, n_seg, offsets, G, N, K)) return -1;
+  if (P != 1 && P != 2) return -1;
+  int S = (mode == ORC_MODE_INPUT) ? n_seg : 1;
+  if (rows == NULL) n_rows = M;
+#ifdef _OPENMP
+  if (n_threads < 1) n_threads = 1;
+#pragma omp parallel for schedule(dynamic, 1) num_threads(n_threads)
+#endif
+  for (int64_t r = 0; r < n_rows; ++r) {
+    int64_t m = rows ? rows[r] : r;
+    for (int64_t n = 0; n < N; ++n) {
+      int g = (mode == ORC_MODE_OUTPUT && G > 1) ? orc_seg_index(offsets, n_seg, n) : 0;
+      const uint8_t *wn = wq + n * K;
+      for (int i = 0; i < S; ++i) {
+        int64_t k0 = (S == 1) ? 0 : offsets[i];
+        int64_t k1 = (S == 1) ? K : offsets[i + 1];
+        for (int pl = 0; pl < P; ++pl) {
+          const uint8_t *xq = planes + (((int64_t)g * P + pl) * M + m) * K;
+          double a = 0.0;
+          for (int64_t k = k0; k < k1; ++k)
+            a += (double)orc_e4m3_value(xq[k]) * (double)orc_e4m3_value(wn[k]);
+          acc[(((int64_t)i * P + pl) * n_rows + r) * N + n] = (float)a;
+        }
+      }
+    }
+  }
+  return 0;
+}
+
+/* Full FP8 layer: the W8A8 epilogue with f(A) replaced by the fp32 sums. */
+int orc_gemm_fp8(const uint8_t *planes, const uint8_t *wq, const float *s_w,
+                 const float *s_act, const uint16_t *bias, int64_t M, int64_t N,
+                 int64_t K, int mode, int n_seg, const int32_t *offsets, int G, int P,
+                 const int64_t *rows, int64_t n_rows, float *y, int n_threads) {
+  if (orc_check_seg(mode, n_seg, offsets, G, N, K)) return -1;
+  if (P != 1 && P != 2) return -1;
+  int S = (mode == ORC_MODE_INPUT) ? n_seg : 1;
+  if (rows == NULL) n_rows = M;
+  float *acc = (float *)malloc(sizeof(float) * (size_t)S * P * n_rows * N);
+  if (!acc) return -2;
+  int rc = orc_gemm_fp8_acc(planes, wq, M, N, K, mode, n_seg, offsets, G, P, rows, n_rows,
+                            acc, n_threads);
+  if (rc) {
+    free(acc);
+    return rc;
+  }
+  for (int64_t r = 0; r < n_rows; ++r)
+    for (int64_t n = 0; n < N; ++n) {
+      int g = (mode == ORC_MODE_OUTPUT && G > 1) ? orc_seg_index(offsets, n_seg, n) : 0;
+      float yv = 0.0f;
+      for (int i = 0; i < S; ++i) {
+        float sp = s_act[((int64_t)g * S + i) * 2 + 0];
+        float sm = s_act[((int64_t)g * S + i) * 2 + 1];
+        float ap = acc[(((int64_t)i * P + 0) * n_rows + r) * N + n];
+        float t;
+        if (P == 2) {
+          float am = acc[(((int64_t)i * P + 1) * n_rows + r) * N + n];
+          float tp = sp * ap;
+          float tm = sm * am;
+          t = tp + tm;
+        } else {
+          t = sp * ap;
+        }
+        yv = yv + s_w[(int64_t)i * N + n] * t;
+      }
+      if (bias) yv = yv + orc_bf16(bias[n]);
+      y[r * N + n] = yv;
+    }
+  free(acc);
+  return 0;
+}
