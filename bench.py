@@ -175,7 +175,7 @@ def traffic_from_profile():
 
 # ------------------------------------------------------------- our path
 class GpuLayer:
-    def __init__(self, L, dev, adaptive=False, weight_bits=8, w_operand=None):
+    def __init__(self, L, dev, adaptive=False, weight_bits=8, w_operand=None, fp8=False):
         from w8a8_gemm_b200 import binding as B
         from w8a8_gemm_b200.layer import DualScaleSegLinear
         self.L = L
@@ -185,7 +185,7 @@ class GpuLayer:
         bias = None if L.bias is None else L.bias.to(dev)
         self.lin = DualScaleSegLinear(L.w.to(dev), bias, d, seg, L.x_cal.to(dev),
                                       adaptive=adaptive, weight_bits=weight_bits,
-                                      w_operand=w_operand)
+                                      w_operand=w_operand, fp8=fp8)
         self.x = L.x.to(dev)
         self.planes = torch.empty(L.G, self.lin.seg.P, L.M, L.K, dtype=torch.int8, device=dev)
         self.y = torch.empty(L.M, L.N, dtype=torch.bfloat16, device=dev)
@@ -218,7 +218,7 @@ def run_ours(args, ws, rank, local):
     w_operand = (torch.empty(max(L.N * L.K for L in layers_cpu), dtype=torch.int8, device=dev)
                  if args.weight_bits == 4 else None)
     glayers = [GpuLayer(L, dev, adaptive=args.adaptive, weight_bits=args.weight_bits,
-                        w_operand=w_operand) for L in layers_cpu]
+                        w_operand=w_operand, fp8=args.fp8) for L in layers_cpu]
     torch.cuda.synchronize()
     eff_ops = sum(layer_units(g.L, g.lin.seg.P)[0] for g in glayers)
     exe_ops = sum(layer_units(g.L, g.lin.seg.P)[1] for g in glayers)
@@ -388,6 +388,8 @@ def main(argv=None):
     ap.add_argument("--weight-bits", type=int, default=8, choices=[8, 4],
                     help="4: W4A8 weights (packed; expanded to the int8 operand before each "
                          "GEMM, inside the timed GEMM region)")
+    ap.add_argument("--fp8", action="store_true",
+                    help="FP8 E4M3 codes for activations and weights (tcgen05 kind::f8f6f4)")
     ap.add_argument("--adaptive", action="store_true",
                     help="single-scale path on layers whose calibrated sides differ by < 2x")
     args = ap.parse_args(argv)
@@ -448,7 +450,7 @@ def main(argv=None):
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": "s8",
+        "dtype": "e4m3" if args.fp8 else "s8",
         "data": "synthetic (seeded SD3.5/FLUX-shaped activations and weights)",
         "config": {"workload": f"{args.config}: {wl.CONFIGS[args.config]}",
                    "layers": [{k: v for k, v in p.items()
@@ -458,7 +460,8 @@ def main(argv=None):
                             if args.adaptive else "DualScale on every layer"),
                    "weights": ("W4A8: packed 4-bit codes, expanded to the int8 operand before "
                                "each GEMM (counted in the GEMM time)"
-                               if args.weight_bits == 4 else "W8A8"),
+                               if args.weight_bits == 4 else
+                               "FP8 E4M3 activations and weights" if args.fp8 else "W8A8"),
                    "output": "bf16",
                    "l2": "flushed between steps, untimed: 512 MiB written, then 256 MiB read",
                    "parallelism": f"replicas x{n_gpus}"},
@@ -473,7 +476,8 @@ def main(argv=None):
                      "peak": round(int8_peak_burst, 1), "unit": "TOPS",
                      "frac": round(gemm_tops / int8_peak_burst, 4),
                      "traffic": traffic,
-                     "kernel": "dualscale_gemm_kernel (tcgen05 kind::i8)",
+                     "kernel": ("dualscale_gemm_kernel (tcgen05 kind::f8f6f4)" if args.fp8
+                                else "dualscale_gemm_kernel (tcgen05 kind::i8)"),
                      "peak_source": f"{peak_src}: bf16 burst {peaks['bf16_tflops']} TF/s x 2 "
                                     f"(nominal INT8/bf16 ratio); sustained-based INT8 peak "
                                     f"{round(int8_peak_sust, 1)}",

@@ -104,6 +104,21 @@ typedef enum { SQ_OUT_BF16 = 0, SQ_OUT_F32 = 1 } sq_out_dtype;
 #define SQ_FLAG_W4 2
 
 /*
+ * SQ_FLAG_FP8: the FP8 variant (the "W8A8(fp)" rows of the results table for
+ * SDXL, which the pages do not define).  Reading: every code is FP8 E4M3 (1
+ * sign, 4 exponent bits with bias 7, 3 mantissa bits, largest finite 448, no
+ * infinities, 0x7F/0xFF NaN), stored as its bit pattern in the int8 buffers.
+ * Calibration: s+ = max/448 and s- = |min|/448 (single scale: the larger side
+ * / 448).  Quantization: x >= 0 -> X^+ = e4m3(fl(x*m+)), X^- = 0x00; x < 0 ->
+ * X^- = e4m3(fl(x*m-)), X^+ = 0x00; NaN -> both 0x00; e4m3() rounds half to
+ * even and saturates finite values to +-448.  Weights: s_w = amax/448,
+ * W^ = e4m3(fl(w'/s_w)).  GEMM: tcgen05 kind::f8f6f4 with fp32 accumulation
+ * (exact products; sums in the tensor core's fp32, order unspecified), the
+ * W8A8 epilogue on the fp32 sums.  Not combinable with SQ_FLAG_W4.
+ */
+#define SQ_FLAG_FP8 4
+
+/*
  * Segment table (SegLinear).  `offsets` is a HOST array of n_seg + 1 strictly
  * increasing int32 values from 0 to the segmented extent (N for SQ_SEG_OUTPUT,
  * K for SQ_SEG_INPUT).  SQ_SEG_NONE takes n_seg = 1 and offsets may be NULL.
@@ -120,7 +135,7 @@ typedef struct {
   int32_t n_seg;           /* number of segments, 1..SQ_MAX_SEGMENTS */
   const int32_t *offsets;  /* host, n_seg + 1 entries            */
   int32_t n_groups;        /* G                                  */
-  int32_t flags;           /* 0 or SQ_FLAG_SINGLE_SCALE, optionally | SQ_FLAG_W4 */
+  int32_t flags;           /* 0 or SQ_FLAG_SINGLE_SCALE, | SQ_FLAG_W4 or SQ_FLAG_FP8 */
 } sq_segments;
 
 /*

@@ -9,8 +9,9 @@ from w8a8_gemm_b200 import binding as B
 from w8a8_gemm_b200 import workloads as wl
 
 
-def segments(layer: wl.Layer, single=False, weight_bits=8) -> B.Segments:
-    flags = (B.SQ_FLAG_SINGLE_SCALE if single else 0) | (B.SQ_FLAG_W4 if weight_bits == 4 else 0)
+def segments(layer: wl.Layer, single=False, weight_bits=8, fp8=False) -> B.Segments:
+    flags = ((B.SQ_FLAG_SINGLE_SCALE if single else 0) | (B.SQ_FLAG_W4 if weight_bits == 4 else 0)
+             | (B.SQ_FLAG_FP8 if fp8 else 0))
     if layer.mode == wl.MODE_NONE:
         return B.Segments(B.SQ_SEG_NONE, None, 1, flags)
     return B.Segments(layer.mode, list(layer.offsets), layer.G, flags)
@@ -21,13 +22,14 @@ def oracle_offsets(layer: wl.Layer):
 
 
 def gpu_run(layer: wl.Layer, out_dtype=torch.float32, with_bias=True, s32=False,
-            single=False, weight_bits=8):
+            single=False, weight_bits=8, fp8=False):
     """CUDA path: weight quantization, calibration, activation quantization and
     the fused GEMM, all through the library.  weight_bits=4: W4A8 weights,
     packed, then expanded into the GEMM operand (16 q); out["wq"] is then the
-    packed uint8 [N][K/2] and out["wq16"] the operand."""
+    packed uint8 [N][K/2] and out["wq16"] the operand.  fp8=True: E4M3 codes
+    in the int8 buffers, and out["acc"] holds the fp32 sums' bit patterns."""
     dev = torch.device("cuda")
-    seg = segments(layer, single, weight_bits)
+    seg = segments(layer, single, weight_bits, fp8)
     x = layer.x.to(dev)
     w = layer.w.to(dev)
     xc = layer.x_cal.to(dev)
@@ -63,11 +65,19 @@ def gpu_run(layer: wl.Layer, out_dtype=torch.float32, with_bias=True, s32=False,
     return out
 
 
-def oracle_prep(layer: wl.Layer, single=False, weight_bits=8):
+def oracle_prep(layer: wl.Layer, single=False, weight_bits=8, fp8=False):
     """Oracle calibration and quantization of both operands (weight_bits=4:
-    W4A8 codes in [-7, 7] in "wq" and their packed storage in "wq4")."""
+    W4A8 codes in [-7, 7] in "wq" and their packed storage in "wq4"; fp8:
+    E4M3 codes as uint8)."""
     off = oracle_offsets(layer)
     d = None if layer.d is None else layer.d.numpy()
+    if fp8:
+        s_act = oracle.calibrate_act_fp8(wl.bits(layer.x_cal), d, layer.mode, off, layer.G,
+                                         layer.N, single)
+        planes = oracle.quantize_act_fp8(wl.bits(layer.x), s_act, d, layer.mode, off, layer.G,
+                                         layer.N, single)
+        wq, s_w = oracle.quantize_weight_fp8(wl.bits(layer.w), d, layer.mode, off, layer.G)
+        return dict(s_act=s_act, planes=planes, wq=wq, s_w=s_w, fp8=True)
     s_act = oracle.calibrate_act(wl.bits(layer.x_cal), d, layer.mode, off, layer.G, layer.N,
                                  single)
     planes = oracle.quantize_act(wl.bits(layer.x), s_act, d, layer.mode, off, layer.G, layer.N,
@@ -82,6 +92,10 @@ def oracle_prep(layer: wl.Layer, single=False, weight_bits=8):
 
 def oracle_y(layer, prep, rows=None, with_bias=True, threads=None):
     bias = wl.bits(layer.bias) if (with_bias and layer.bias is not None) else None
+    if prep.get("fp8"):
+        return oracle.gemm_fp8(prep["planes"], prep["wq"], prep["s_w"], prep["s_act"], bias,
+                               layer.mode, oracle_offsets(layer), rows=rows,
+                               threads=threads or oracle.num_threads())
     return oracle.gemm(prep["planes"], prep["wq"], prep["s_w"], prep["s_act"], bias, layer.mode,
                        oracle_offsets(layer), rows=rows,
                        threads=threads or oracle.num_threads())
@@ -128,3 +142,14 @@ def sample_rows(M: int, bm: int = 128, stride: int = 97):
     rows |= set(range(max(0, M - bm), M))
     rows |= set(range(0, M, stride))
     return np.array(sorted(rows), dtype=np.int64)
+
+
+def oracle_acc_fp8(layer, prep, rows=None, threads=None, absolute=False):
+    """FP8: the exact sums of E4M3 products rounded once to fp32; with
+    absolute=True the sums of |products| (sign bits cleared), which bound the
+    rounding error of any fp32 summation order."""
+    planes, wq = prep["planes"], prep["wq"]
+    if absolute:
+        planes, wq = planes & 0x7F, wq & 0x7F
+    return oracle.gemm_fp8_acc(planes, wq, layer.mode, oracle_offsets(layer), rows=rows,
+                               threads=threads or oracle.num_threads())

@@ -109,7 +109,12 @@ def test_segment_table_validation(L):
 
 def test_unknown_flags_rejected(L):
     p = ctypes.c_void_p
-    s = B.Segments(B.SQ_SEG_NONE, None, 1, flags=4)
+    s = B.Segments(B.SQ_SEG_NONE, None, 1, flags=8)
+    c, keep = s._c()
+    assert L.sq_quantize_act(p(FAKE), 4, 32, 32, None, p(FAKE), ctypes.byref(c), p(FAKE),
+                             None) == SQ_ERR_INVALID_ARG
+    # W4 weights and FP8 codes do not combine
+    s = B.Segments(B.SQ_SEG_NONE, None, 1, flags=B.SQ_FLAG_W4 | B.SQ_FLAG_FP8)
     c, keep = s._c()
     assert L.sq_quantize_act(p(FAKE), 4, 32, 32, None, p(FAKE), ctypes.byref(c), p(FAKE),
                              None) == SQ_ERR_INVALID_ARG

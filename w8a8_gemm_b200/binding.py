@@ -24,6 +24,7 @@ SQ_OUT_BF16, SQ_OUT_F32 = 0, 1
 SQ_MAX_SEGMENTS = 64
 SQ_FLAG_SINGLE_SCALE = 1
 SQ_FLAG_W4 = 2
+SQ_FLAG_FP8 = 4
 
 EXPORTED = ("sq_calibrate_act", "sq_quantize_act", "sq_quantize_weight_seg",
             "sq_quantize_weight_w4", "sq_unpack_weight_w4",
@@ -50,7 +51,8 @@ class Segments:
     """SegLinear segment table: mode, boundaries (over N for output mode, over
     K for input mode), the number of activation groups G, and flags
     (SQ_FLAG_SINGLE_SCALE for the single-scale path, SQ_FLAG_W4 for a GEMM whose
-    weight operand comes from sq_unpack_weight_w4)."""
+    weight operand comes from sq_unpack_weight_w4, SQ_FLAG_FP8 for E4M3 codes in
+    the int8 buffers)."""
     mode: int = SQ_SEG_NONE
     offsets: Optional[Sequence[int]] = None
     n_groups: int = 1

@@ -57,9 +57,12 @@ sq_status parse_segments(const sq_segments *seg, int64_t K, int64_t extent_n, Se
   if (seg->mode < SQ_SEG_NONE || seg->mode > SQ_SEG_INPUT) return SQ_ERR_INVALID_ARG;
   if (seg->n_seg < 1 || seg->n_seg > SQ_MAX_SEGMENTS || seg->n_groups < 1)
     return SQ_ERR_INVALID_ARG;
-  if ((seg->flags & ~(SQ_FLAG_SINGLE_SCALE | SQ_FLAG_W4)) != 0) return SQ_ERR_INVALID_ARG;
+  if ((seg->flags & ~(SQ_FLAG_SINGLE_SCALE | SQ_FLAG_W4 | SQ_FLAG_FP8)) != 0)
+    return SQ_ERR_INVALID_ARG;
+  if ((seg->flags & SQ_FLAG_W4) && (seg->flags & SQ_FLAG_FP8)) return SQ_ERR_INVALID_ARG;
   p.P = (seg->flags & SQ_FLAG_SINGLE_SCALE) ? 1 : 2;
   p.w4 = (seg->flags & SQ_FLAG_W4) ? 1 : 0;
+  p.fp8 = (seg->flags & SQ_FLAG_FP8) ? 1 : 0;
   p.mode = seg->mode;
   p.n_seg = seg->n_seg;
   p.G = seg->n_groups;
@@ -273,7 +276,7 @@ sq_status sq_quantize_weight_w4(const void *w, int64_t N, int64_t K, const float
   SQ_TRY(check_k(K));
   SegParams sp;
   SQ_TRY(parse_segments(seg, K, N, &sp));
-  if (w == nullptr || wq4 == nullptr || s_w == nullptr) return SQ_ERR_INVALID_ARG;
+  if (w == nullptr || wq4 == nullptr || s_w == nullptr || sp.fp8) return SQ_ERR_INVALID_ARG;
   if (!aligned(w, 16) || !aligned(wq4, 16) || !aligned(s_w, 4) || (d && !aligned(d, 4)))
     return SQ_ERR_ALIGNMENT;
   SQ_TRY(check_device());

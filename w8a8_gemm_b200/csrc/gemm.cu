@@ -181,7 +181,18 @@ __device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, uint32_t (&r)[CW]) 
 // One CTA per SM (shared memory allows no more).  Its warps spread over the four
 // 16K-register sub-partitions (10 warps: 3/3/2/2, a thread at most 168
 // registers; 18 warps: 5/5/4/4, at most 96).
-template <int BN, int STAGES, int OUT, bool SEGK, int EPI_WARPS, int POL>
+// accumulator word -> fp32: int32 (kind::i8, RN conversion) or the fp32 bits
+// themselves (kind::f8f6f4).
+template <bool F8>
+__device__ __forceinline__ float acc_f32(uint32_t v) {
+  if constexpr (F8)
+    return __uint_as_float(v);
+  else
+    return __int2float_rn(static_cast<int32_t>(v));
+}
+
+// F8: E4M3 planes and weights (kind::f8f6f4, fp32 accumulators) instead of int8.
+template <int BN, int STAGES, int OUT, bool SEGK, int EPI_WARPS, int POL, bool F8>
 __global__ void __launch_bounds__(threads_for(EPI_WARPS), 1)
     dualscale_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                           const __grid_constant__ CUtensorMap tmB,
@@ -269,7 +280,7 @@ __global__ void __launch_bounds__(threads_for(EPI_WARPS), 1)
   } else if (warp == 1) {
     // ---------------------------------------------------------- MMA issuer
     if (lane == 0) {
-      constexpr uint32_t idesc = idesc_i8(BM, BN);
+      constexpr uint32_t idesc = F8 ? idesc_e4m3(BM, BN) : idesc_i8(BM, BN);
       int stage = 0;
       uint32_t phase = 0;
       uint32_t acc_iter = 0;
@@ -306,10 +317,17 @@ __global__ void __launch_bounds__(threads_for(EPI_WARPS), 1)
               seg_end = p.k_off[seg + 1];
             }
             const uint64_t b_desc = sdesc_kmajor_sw128(sb + kk * MMA_K);
-            mma_i8(d_plus, sdesc_kmajor_sw128(sa + kk * MMA_K), b_desc, idesc, accumulate);
-            if (POL == 2)
-              mma_i8(d_plus + BN, sdesc_kmajor_sw128(sa + BM * BK + kk * MMA_K), b_desc, idesc,
-                     accumulate);
+            if constexpr (F8) {
+              mma_e4m3(d_plus, sdesc_kmajor_sw128(sa + kk * MMA_K), b_desc, idesc, accumulate);
+              if (POL == 2)
+                mma_e4m3(d_plus + BN, sdesc_kmajor_sw128(sa + BM * BK + kk * MMA_K), b_desc,
+                         idesc, accumulate);
+            } else {
+              mma_i8(d_plus, sdesc_kmajor_sw128(sa + kk * MMA_K), b_desc, idesc, accumulate);
+              if (POL == 2)
+                mma_i8(d_plus + BN, sdesc_kmajor_sw128(sa + BM * BK + kk * MMA_K), b_desc,
+                       idesc, accumulate);
+            }
             accumulate = 1;
           }
           mma_commit(&empty[stage]);  // frees the stage once these MMAs finish
@@ -442,15 +460,13 @@ __global__ void __launch_bounds__(threads_for(EPI_WARPS), 1)
 #pragma unroll
                 for (int h = 0; h < 2; ++h) {
                   const int j = 4 * q + 2 * h;
-                  const uint64_t fp = f2pack(__int2float_rn(static_cast<int32_t>(ap[j])),
-                                             __int2float_rn(static_cast<int32_t>(ap[j + 1])));
+                  const uint64_t fp = f2pack(acc_f32<F8>(ap[j]), acc_f32<F8>(ap[j + 1]));
                   // Each step is one packed FMA with a zero addend or a unit
                   // factor, i.e. exactly one rounding of the scalar product
                   // or sum, and nothing the compiler could contract further.
                   uint64_t t;
                   if constexpr (POL == 2) {
-                    const uint64_t fm = f2pack(__int2float_rn(static_cast<int32_t>(am[j])),
-                                               __int2float_rn(static_cast<int32_t>(am[j + 1])));
+                    const uint64_t fm = f2pack(acc_f32<F8>(am[j]), acc_f32<F8>(am[j + 1]));
                     t = ffma2(one2, ffma2(sp2, fp, zero2), ffma2(sm2, fm, zero2));
                   } else {
                     t = ffma2(sp2, fp, zero2);  // single scale: t = s f(A)
@@ -508,8 +524,7 @@ __global__ void __launch_bounds__(threads_for(EPI_WARPS), 1)
               const int j = 4 * q;
               uint64_t &r0 = run2[c * 8 + 2 * q], &r1 = run2[c * 8 + 2 * q + 1];
               const auto cvt2 = [](uint32_t x, uint32_t y) {
-                return f2pack(__int2float_rn(static_cast<int32_t>(x)),
-                              __int2float_rn(static_cast<int32_t>(y)));
+                return f2pack(acc_f32<F8>(x), acc_f32<F8>(y));
               };
               r0 = ffma2(f2pack(a.x, a.y), cvt2(ap[j], ap[j + 1]), r0);
               r1 = ffma2(f2pack(a.z, a.w), cvt2(ap[j + 2], ap[j + 3]), r1);
@@ -578,7 +593,7 @@ int device_sm_count() {
   return sms > 0 ? sms : 148;
 }
 
-template <int BN, int STAGES, int OUT, bool SEGK, int EPI_WARPS, int POL>
+template <int BN, int STAGES, int OUT, bool SEGK, int EPI_WARPS, int POL, bool F8>
 sq_status run_gemm(const GemmRequest &r, const GemmParams &p, cudaStream_t stream) {
   using L = Smem<BN, STAGES, EPI_WARPS, POL, SEGK, OUT == OUT_BF16 && !SEGK>;
   EncodeTiledFn enc = tensor_map_encoder();
@@ -624,7 +639,7 @@ sq_status run_gemm(const GemmRequest &r, const GemmParams &p, cudaStream_t strea
       return SQ_ERR_CUDA;
   }
   static_assert(L::BYTES <= 232448, "dynamic shared memory above the per-block limit");
-  auto kernel = dualscale_gemm_kernel<BN, STAGES, OUT, SEGK, EPI_WARPS, POL>;
+  auto kernel = dualscale_gemm_kernel<BN, STAGES, OUT, SEGK, EPI_WARPS, POL, F8>;
   static bool attr_set[64] = {};  // per instantiation and device
   int dev = 0;
   cudaGetDevice(&dev);
@@ -648,12 +663,19 @@ sq_status run_gemm(const GemmRequest &r, const GemmParams &p, cudaStream_t strea
 // narrower tiles give more buffers but cost more than they save (measured).
 constexpr int kSegBN = 128;  // tile width of the input-segmented path
 
-template <int OUT, int POL>
+template <int OUT, int POL, bool F8>
 sq_status dispatch(const GemmRequest &r, const GemmParams &p, bool segk, int BN,
                    cudaStream_t stream) {
-  if (segk) return run_gemm<kSegBN, 4, OUT, true, 16, POL>(r, p, stream);
-  if (BN == 256) return run_gemm<256, POL == 2 ? 3 : 4, OUT, false, 8, POL>(r, p, stream);
-  return run_gemm<128, 4, OUT, false, 8, POL>(r, p, stream);
+  if (segk) return run_gemm<kSegBN, 4, OUT, true, 16, POL, F8>(r, p, stream);
+  if (BN == 256) return run_gemm<256, POL == 2 ? 3 : 4, OUT, false, 8, POL, F8>(r, p, stream);
+  return run_gemm<128, 4, OUT, false, 8, POL, F8>(r, p, stream);
+}
+
+template <int OUT, int POL>
+sq_status dispatch_kind(const GemmRequest &r, const GemmParams &p, bool segk, int BN,
+                        cudaStream_t stream) {
+  return r.seg.fp8 ? dispatch<OUT, POL, true>(r, p, segk, BN, stream)
+                   : dispatch<OUT, POL, false>(r, p, segk, BN, stream);
 }
 
 }  // namespace
@@ -699,15 +721,15 @@ sq_status launch_gemm(const GemmRequest &r, cudaStream_t stream) {
 
   if (r.seg.P == 1) {
     switch (r.out_kind) {
-      case OUT_S32: return dispatch<OUT_S32, 1>(r, p, segk, BN, stream);
-      case OUT_F32: return dispatch<OUT_F32, 1>(r, p, segk, BN, stream);
-      default: return dispatch<OUT_BF16, 1>(r, p, segk, BN, stream);
+      case OUT_S32: return dispatch_kind<OUT_S32, 1>(r, p, segk, BN, stream);
+      case OUT_F32: return dispatch_kind<OUT_F32, 1>(r, p, segk, BN, stream);
+      default: return dispatch_kind<OUT_BF16, 1>(r, p, segk, BN, stream);
     }
   }
   switch (r.out_kind) {
-    case OUT_S32: return dispatch<OUT_S32, 2>(r, p, segk, BN, stream);
-    case OUT_F32: return dispatch<OUT_F32, 2>(r, p, segk, BN, stream);
-    default: return dispatch<OUT_BF16, 2>(r, p, segk, BN, stream);
+    case OUT_S32: return dispatch_kind<OUT_S32, 2>(r, p, segk, BN, stream);
+    case OUT_F32: return dispatch_kind<OUT_F32, 2>(r, p, segk, BN, stream);
+    default: return dispatch_kind<OUT_BF16, 2>(r, p, segk, BN, stream);
   }
 }
 

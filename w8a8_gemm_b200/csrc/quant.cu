@@ -7,6 +7,7 @@
 // Every fp32 operation that decides an integer code is written with an explicit
 // round-to-nearest intrinsic so that no contraction or approximation changes it.
 #include <cuda_bf16.h>
+#include <cuda_fp8.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -78,18 +79,20 @@ __global__ void __launch_bounds__(256) calib_reduce_kernel(const uint16_t *__res
 }
 
 // Pass 2: s+ = max / 127, s- = |min| / 128; an empty side gets step 1.  In
-// single-scale mode both take max(max, |min|) / 127.
-__global__ void calib_finalize_kernel(float *s_act, int n, int single) {
+// single-scale mode both take max(max, |min|) / 127.  FP8 (E4M3): both
+// divisors are 448.
+__global__ void calib_finalize_kernel(float *s_act, int n, int single, int fp8) {
+  const float qp = fp8 ? 448.0f : 127.0f, qm = fp8 ? 448.0f : 128.0f;
   for (int t = threadIdx.x; t < n; t += blockDim.x) {
     const float hi = s_act[2 * t], nlo = s_act[2 * t + 1];
     if (single) {
       const float amax = hi > nlo ? hi : nlo;
-      const float s = amax > 0.0f ? __fdiv_rn(amax, 127.0f) : 1.0f;
+      const float s = amax > 0.0f ? __fdiv_rn(amax, qp) : 1.0f;
       s_act[2 * t] = s;
       s_act[2 * t + 1] = s;
     } else {
-      s_act[2 * t] = hi > 0.0f ? __fdiv_rn(hi, 127.0f) : 1.0f;
-      s_act[2 * t + 1] = nlo > 0.0f ? __fdiv_rn(nlo, 128.0f) : 1.0f;
+      s_act[2 * t] = hi > 0.0f ? __fdiv_rn(hi, qp) : 1.0f;
+      s_act[2 * t + 1] = nlo > 0.0f ? __fdiv_rn(nlo, qm) : 1.0f;
     }
   }
 }
@@ -141,6 +144,41 @@ __device__ __forceinline__ void dualscale8(const float (&x)[8], const float (&p7
   minus = make_uint2(pack4_lo(qm[0], qm[1], qm[2], qm[3]), pack4_lo(qm[4], qm[5], qm[6], qm[7]));
 }
 
+// FP8 (E4M3) codes of eight channels, with the multipliers m+ and m- as they
+// are (no 2^-7 pre-scaling): v = fl(x * m), code = e4m3(v), round half to even
+// with saturation to +-448 (the CUDA conversion intrinsics).  x >= 0 (-0.0
+// included) fills the + plane, x < 0 the - plane, NaN neither.
+__device__ __forceinline__ uint32_t e4m3x4(float a, float b, float c, float d) {
+  const uint32_t lo = __nv_cvt_float2_to_fp8x2(make_float2(a, b), __NV_SATFINITE, __NV_E4M3);
+  const uint32_t hi = __nv_cvt_float2_to_fp8x2(make_float2(c, d), __NV_SATFINITE, __NV_E4M3);
+  return lo | (hi << 16);
+}
+
+__device__ __forceinline__ void dualscale8_fp8(const float (&x)[8], const float (&mp)[8],
+                                               const float (&mm)[8], uint2 &plus, uint2 &minus) {
+  float vp[8], vm[8];
+  uint32_t pos = 0, neg = 0;  // byte masks of the two branches
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    vp[j] = __fmul_rn(x[j], mp[j]);
+    vm[j] = __fmul_rn(x[j], mm[j]);
+    const int sh = 8 * (j & 3);
+    if (j == 4) {
+      plus.x = pos;
+      minus.x = neg;
+      pos = neg = 0;
+    }
+    if (x[j] >= 0.0f) pos |= 0xFFu << sh;
+    if (x[j] < 0.0f) neg |= 0xFFu << sh;
+  }
+  plus.y = pos;
+  minus.y = neg;
+  plus.x &= e4m3x4(vp[0], vp[1], vp[2], vp[3]);
+  plus.y &= e4m3x4(vp[4], vp[5], vp[6], vp[7]);
+  minus.x &= e4m3x4(vm[0], vm[1], vm[2], vm[3]);
+  minus.y &= e4m3x4(vm[4], vm[5], vm[6], vm[7]);
+}
+
 // Work unit = one activation group g and one tile of 32 rows x 256 channels.
 // Units are numbered group-major, then column block, then row tile, and every
 // block takes one contiguous range of them: the grid is balanced to within one
@@ -152,6 +190,8 @@ __device__ __forceinline__ void dualscale8(const float (&x)[8], const float (&p7
 // memory; every warp then takes whole rows of the staged tile (lane = 8
 // channels, one conflict-free 16-byte shared load) and writes 8 bytes per plane
 // per row, 256 contiguous bytes per warp.
+// FP8 keeps m+ and m- unscaled in p7 and n7.
+template <bool FP8>
 __device__ __forceinline__ void load_multipliers(int g, int64_t c0, int64_t K, const float *d,
                                                  const float *s_act, const SegParams &seg,
                                                  float (&p7)[8], float (&n7)[8]) {
@@ -161,8 +201,9 @@ __device__ __forceinline__ void load_multipliers(int g, int64_t c0, int64_t K, c
 #pragma unroll
   for (int j = 0; j < 8; ++j) {
     const float dv = d ? d[g * K + c0 + j] : 1.0f;
-    p7[j] = __fdiv_rn(1.0f, __fmul_rn(dv, sp)) * 0.0078125f;
-    n7[j] = __fdiv_rn(1.0f, __fmul_rn(dv, sm)) * -0.0078125f;
+    const float mp = __fdiv_rn(1.0f, __fmul_rn(dv, sp)), mm = __fdiv_rn(1.0f, __fmul_rn(dv, sm));
+    p7[j] = FP8 ? mp : mp * 0.0078125f;
+    n7[j] = FP8 ? mm : mm * -0.0078125f;
   }
 }
 
@@ -187,6 +228,7 @@ struct UnitCursor {
   }
 };
 
+template <bool FP8>
 __global__ void __launch_bounds__(256, 3) quant_act_kernel(const __grid_constant__ CUtensorMap tmX,
                                                            int64_t M, int64_t K,
                                                            const float *__restrict__ d,
@@ -228,7 +270,7 @@ __global__ void __launch_bounds__(256, 3) quant_act_kernel(const __grid_constant
     if (cur.g != key_g || cur.cb != key_cb) {
       key_g = cur.g;
       key_cb = cur.cb;
-      load_multipliers(cur.g, c0, K, d, s_act, seg, p7, n7);
+      load_multipliers<FP8>(cur.g, c0, K, d, s_act, seg, p7, n7);
     }
     const int st = it % kQStages;
     if (!mbar_wait(&full[st], (it / kQStages) & 1, kQuantWaitNs)) {
@@ -247,13 +289,16 @@ __global__ void __launch_bounds__(256, 3) quant_act_kernel(const __grid_constant
         float xv[8];
         unpack8(v, xv);
         uint2 pk, nk;
-        dualscale8(xv, p7, n7, pk, nk);
+        if constexpr (FP8)
+          dualscale8_fp8(xv, p7, n7, pk, nk);
+        else
+          dualscale8(xv, p7, n7, pk, nk);
         if (seg.P == 2) {
           *reinterpret_cast<uint2 *>(plus + r * K) = pk;
           *reinterpret_cast<uint2 *>(plus + plane_stride + r * K) = nk;
         } else {
-          // single scale: one of the two codes of every element is 0, so the
-          // byte-wise OR is their sum
+          // single scale: at most one of the two codes of an element is
+          // non-zero (int8: the OR is their sum; FP8: the branch's code)
           *reinterpret_cast<uint2 *>(plus + r * K) = make_uint2(pk.x | nk.x, pk.y | nk.y);
         }
       }
@@ -285,7 +330,8 @@ __device__ __forceinline__ float block_max(float v, float *red) {
 
 // QMAX = 127 (W8) or 7 (W4A8, "SegQuant-4"); with QMAX = 7 the codes are
 // stored two per byte (channel 2j in the low nibble, 2j + 1 in the high one,
-// 4-bit two's complement), each thread handling channel pairs.
+// 4-bit two's complement), each thread handling channel pairs.  QMAX = 448:
+// FP8 E4M3 codes e4m3(fl(w'/s_w)) (round half to even, saturating).
 __device__ __forceinline__ int weight_code(float wv, float s, float qmax) {
   const float v = fminf(fmaxf(__fdiv_rn(wv, s), -qmax), qmax);
   return __float2int_rn(v);
@@ -321,6 +367,10 @@ __global__ void __launch_bounds__(256) quant_weight_kernel(const uint16_t *__res
     if constexpr (QMAX == 127) {
       for (int64_t k = k0 + threadIdx.x; k < k1; k += blockDim.x)
         wq[n * K + k] = static_cast<int8_t>(weight_code(wval(k), s, kQ));
+    } else if constexpr (QMAX == 448) {
+      for (int64_t k = k0 + threadIdx.x; k < k1; k += blockDim.x)
+        wq[n * K + k] = static_cast<int8_t>(
+            __nv_cvt_float_to_fp8(__fdiv_rn(wval(k), s), __NV_SATFINITE, __NV_E4M3));
     } else {
       // segment bounds are even (multiples of 32), so pairs never straddle one
       uint8_t *packed = reinterpret_cast<uint8_t *>(wq) + n * (K / 2);
@@ -376,7 +426,7 @@ cudaError_t launch_calibrate_act(const uint16_t *x, int64_t M, int64_t K, int64_
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
-  calib_finalize_kernel<<<1, 256, 0, stream>>>(s_act, n, seg.P == 1 ? 1 : 0);
+  calib_finalize_kernel<<<1, 256, 0, stream>>>(s_act, n, seg.P == 1 ? 1 : 0, seg.fp8);
   return cudaGetLastError();
 }
 
@@ -402,11 +452,12 @@ sq_status launch_quantize_act(const uint16_t *x, int64_t M, int64_t K, int64_t l
   int64_t nblk = static_cast<int64_t>(num_sms()) * 3;
   if (nblk > n_units) nblk = n_units;
   const size_t smem = kQStages * kQTileBytes + kQStages * sizeof(uint64_t);
-  if (cudaFuncSetAttribute(quant_act_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  auto kernel = seg.fp8 ? quant_act_kernel<true> : quant_act_kernel<false>;
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(smem)) != cudaSuccess)
     return SQ_ERR_CUDA;
-  quant_act_kernel<<<static_cast<unsigned>(nblk), 256, smem, stream>>>(tmX, M, K, d, s_act, seg,
-                                                                       planes, status);
+  kernel<<<static_cast<unsigned>(nblk), 256, smem, stream>>>(tmX, M, K, d, s_act, seg, planes,
+                                                             status);
   return cudaGetLastError() == cudaSuccess ? SQ_OK : SQ_ERR_CUDA;
 }
 
@@ -414,7 +465,12 @@ cudaError_t launch_quantize_weight(const uint16_t *w, int64_t N, int64_t K, cons
                                    const SegParams &seg, int8_t *wq, float *s_w,
                                    cudaStream_t stream) {
   if (N == 0) return cudaSuccess;
-  quant_weight_kernel<127><<<static_cast<unsigned>(N), 256, 0, stream>>>(w, N, K, d, seg, wq, s_w);
+  if (seg.fp8)
+    quant_weight_kernel<448><<<static_cast<unsigned>(N), 256, 0, stream>>>(w, N, K, d, seg, wq,
+                                                                          s_w);
+  else
+    quant_weight_kernel<127><<<static_cast<unsigned>(N), 256, 0, stream>>>(w, N, K, d, seg, wq,
+                                                                          s_w);
   return cudaGetLastError();
 }
 

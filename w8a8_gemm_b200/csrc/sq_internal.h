@@ -17,6 +17,7 @@ struct SegParams {
   int32_t S;      // K-segments (n_seg in input mode, else 1)
   int32_t P;      // activation planes per group: 2 (DualScale) or 1 (single scale)
   int32_t w4;     // 1: the weight operand holds 16 q of W4A8 codes q (SQ_FLAG_W4)
+  int32_t fp8;    // 1: codes are FP8 E4M3 bit patterns (SQ_FLAG_FP8)
   int32_t off[SQ_MAX_SEGMENTS + 1];
 };
 

@@ -24,18 +24,25 @@ class DualScaleSegLinear:
     weight_bits  8 (W8A8) or 4 (W4A8: weights kept packed, two codes per byte,
            and expanded into the int8 GEMM operand before every GEMM; several
            layers may share one operand buffer, `w_operand`, int8 [>= N*K])
+    fp8    FP8 E4M3 codes for activations and weights (SQ_FLAG_FP8) instead of int8
     """
 
     def __init__(self, w: torch.Tensor, bias: Optional[torch.Tensor], d: Optional[torch.Tensor],
                  seg: B.Segments, x_cal: torch.Tensor, out_dtype=torch.bfloat16,
                  adaptive: bool = False, asymmetry_threshold: float = 2.0,
-                 weight_bits: int = 8, w_operand: Optional[torch.Tensor] = None):
+                 weight_bits: int = 8, w_operand: Optional[torch.Tensor] = None,
+                 fp8: bool = False):
         if weight_bits not in (8, 4):
             raise ValueError("weight_bits must be 8 or 4")
+        if fp8 and weight_bits == 4:
+            raise ValueError("FP8 codes and W4 weights do not combine")
         self.N, self.K = w.shape
         self.weight_bits = weight_bits
+        self.fp8 = fp8
         if weight_bits == 4:
             seg = B.Segments(seg.mode, seg.offsets, seg.n_groups, seg.flags | B.SQ_FLAG_W4)
+        if fp8:
+            seg = B.Segments(seg.mode, seg.offsets, seg.n_groups, seg.flags | B.SQ_FLAG_FP8)
         self.seg = seg
         self.G, self.S = seg.n_groups, seg.S
         self.d = d
@@ -61,8 +68,8 @@ class DualScaleSegLinear:
             # Adaptive DualScale: keep the two steps only where the calibrated
             # sides differ by at least `asymmetry_threshold` in some group and
             # K-segment; otherwise switch the layer to one symmetric step.
-            hi = self.s_act[..., 0] * 127.0
-            lo = self.s_act[..., 1] * 128.0
+            hi = self.s_act[..., 0] * (448.0 if fp8 else 127.0)
+            lo = self.s_act[..., 1] * (448.0 if fp8 else 128.0)
             ratio = torch.maximum(hi, lo) / torch.minimum(hi, lo).clamp_min(1e-30)
             if float(ratio.max()) < asymmetry_threshold:
                 self.seg = B.Segments(seg.mode, seg.offsets, seg.n_groups,
