@@ -156,27 +156,15 @@ __device__ __forceinline__ uint32_t e4m3x4(float a, float b, float c, float d) {
 
 __device__ __forceinline__ void dualscale8_fp8(const float (&x)[8], const float (&mp)[8],
                                                const float (&mm)[8], uint2 &plus, uint2 &minus) {
+  // The branch that does not apply converts +0.0, whose code is 0x00.
   float vp[8], vm[8];
-  uint32_t pos = 0, neg = 0;  // byte masks of the two branches
 #pragma unroll
   for (int j = 0; j < 8; ++j) {
-    vp[j] = __fmul_rn(x[j], mp[j]);
-    vm[j] = __fmul_rn(x[j], mm[j]);
-    const int sh = 8 * (j & 3);
-    if (j == 4) {
-      plus.x = pos;
-      minus.x = neg;
-      pos = neg = 0;
-    }
-    if (x[j] >= 0.0f) pos |= 0xFFu << sh;
-    if (x[j] < 0.0f) neg |= 0xFFu << sh;
+    vp[j] = x[j] >= 0.0f ? __fmul_rn(x[j], mp[j]) : 0.0f;
+    vm[j] = x[j] < 0.0f ? __fmul_rn(x[j], mm[j]) : 0.0f;
   }
-  plus.y = pos;
-  minus.y = neg;
-  plus.x &= e4m3x4(vp[0], vp[1], vp[2], vp[3]);
-  plus.y &= e4m3x4(vp[4], vp[5], vp[6], vp[7]);
-  minus.x &= e4m3x4(vm[0], vm[1], vm[2], vm[3]);
-  minus.y &= e4m3x4(vm[4], vm[5], vm[6], vm[7]);
+  plus = make_uint2(e4m3x4(vp[0], vp[1], vp[2], vp[3]), e4m3x4(vp[4], vp[5], vp[6], vp[7]));
+  minus = make_uint2(e4m3x4(vm[0], vm[1], vm[2], vm[3]), e4m3x4(vm[4], vm[5], vm[6], vm[7]));
 }
 
 // Work unit = one activation group g and one tile of 32 rows x 256 channels.
