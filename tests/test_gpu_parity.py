@@ -37,6 +37,9 @@ SMALL = {
     "input_heads": lambda: wl.outproj_layer("heads", 300, 448, 264, 64, seed=5),
     "input_mixed": _input_layer_mixed,
     "input_wide": lambda: wl.outproj_layer("wide", 130, 1024, 136, 512, seed=6),
+    # the most segments a table may hold (SQ_MAX_SEGMENTS = 64)
+    "input_max_segments": lambda: wl.outproj_layer("maxin", 130, 2048, 136, 32, seed=12),
+    "output_max_segments": lambda: wl.adanorm_layer("maxout", 130, 256, 64 * 9, 64, seed=13, G=1),
     "output_g1": lambda: wl.adanorm_layer("o1", 200, 256, 768, 3, seed=7, G=1),
     "output_g3": lambda: wl.adanorm_layer("o3", 200, 256, 768, 3, seed=8, G=3),
     "output_g2_bn128": lambda: wl.adanorm_layer("o2", 130, 128, 256, 2, seed=9, G=2),

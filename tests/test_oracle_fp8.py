@@ -114,3 +114,12 @@ def test_fp8_weights_hit_448_and_stay_within_half_a_quantum():
     u = wf / s_w[0][:, None]
     quantum = np.exp2(np.floor(np.log2(np.maximum(np.abs(u), 2.0 ** -6))) - 3)
     assert np.all(np.abs(vals - u) <= quantum / 2 * (1 + 1e-6))
+
+
+def test_fp8_weight_step_is_amax_over_448():
+    """s_w = amax / 448 exactly: amax = 7/8 gives s_w = 2^-9, and the codes of
+    w = 7/8, 7/16, -7/32, 1/64 are then e4m3 of 448, 224, -112, 8 (all exact)."""
+    w = np.array([[0.875, 0.4375, -0.21875, 0.015625] + [0.0] * 12], np.float32)
+    wq, s_w = oracle.quantize_weight_fp8(bf16_bits(w))
+    assert s_w.tolist() == [[2.0 ** -9]]
+    assert oracle.e4m3_decode(wq[0, :4]).tolist() == [448.0, 224.0, -112.0, 8.0]
