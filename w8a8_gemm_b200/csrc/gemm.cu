@@ -248,6 +248,7 @@ __global__ void __launch_bounds__(threads_for(EPI_WARPS), 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  grid_dependency_wait();  // the prologue above touches no global memory
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -651,7 +652,19 @@ sq_status run_gemm(const GemmRequest &r, const GemmParams &p, cudaStream_t strea
     attr_set[dev] = true;
   }
   const int grid = p.num_tiles < device_sm_count() ? p.num_tiles : device_sm_count();
-  kernel<<<grid, threads_for(EPI_WARPS), L::BYTES, stream>>>(tmA, tmB, tmY, p);
+  // Programmatic dependent launch: CTAs may run their prologue (barriers,
+  // TMEM allocation) while the preceding kernel finishes.
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(threads_for(EPI_WARPS));
+  cfg.dynamicSmemBytes = L::BYTES;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, kernel, tmA, tmB, tmY, p) != cudaSuccess) return SQ_ERR_CUDA;
   return cudaGetLastError() == cudaSuccess ? SQ_OK : SQ_ERR_CUDA;
 }
 

@@ -239,6 +239,9 @@ __global__ void __launch_bounds__(256, 3) quant_act_kernel(const __grid_constant
     for (int st = 0; st < kQStages; ++st) mbar_init(&full[st], 1);
     fence_mbar_init();
     prefetch_tmap(&tmX);
+  }
+  grid_dependency_wait();  // nothing above touches global memory
+  if (tid == 0) {
     fetch.set(u_begin, n_cb, n_rt);
     for (int st = 0; st < kQStages && st < n_mine; ++st) {
       mbar_arrive_expect_tx(&full[st], kQTileBytes);
@@ -444,8 +447,20 @@ sq_status launch_quantize_act(const uint16_t *x, int64_t M, int64_t K, int64_t l
   if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(smem)) != cudaSuccess)
     return SQ_ERR_CUDA;
-  kernel<<<static_cast<unsigned>(nblk), 256, smem, stream>>>(tmX, M, K, d, s_act, seg, planes,
-                                                             status);
+  // Programmatic dependent launch: the blocks may start their prologue while
+  // the preceding kernel finishes; they wait for it before touching memory.
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(nblk));
+  cfg.blockDim = dim3(256);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, kernel, tmX, M, K, d, s_act, seg, planes, status) != cudaSuccess)
+    return SQ_ERR_CUDA;
   return cudaGetLastError() == cudaSuccess ? SQ_OK : SQ_ERR_CUDA;
 }
 

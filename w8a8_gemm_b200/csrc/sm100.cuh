@@ -133,6 +133,15 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
+// Programmatic dependent launch: wait until the preceding kernel in the
+// stream has completed and its memory is visible (a no-op without one).  A
+// kernel launched with programmatic stream serialization may start its
+// prologue while that kernel's last CTAs still run; it must not touch global
+// memory before this wait.
+__device__ __forceinline__ void grid_dependency_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
 __device__ __forceinline__ void prefetch_tmap(const CUtensorMap *map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(map) : "memory");
 }
