@@ -401,16 +401,66 @@ def test_output_segments_equal_concatenation():
         assert np.array_equal(full["y"][:, n0:n1], part["y"])
 
 
+def rn_f32(v: Fraction) -> float:
+    """Round an exact rational to the nearest fp32 value, ties to even
+    (normal and subnormal range), written from the IEEE definition."""
+    if v == 0:
+        return 0.0
+    sign = -1 if v < 0 else 1
+    a = abs(v)
+    m, e = math.frexp(float(a))          # float(a) is within one ulp: adjust
+    e -= 1                               # a in [2^e, 2^(e+1)) after the fix-up
+    while Fraction(2) ** e > a:
+        e -= 1
+    while Fraction(2) ** (e + 1) <= a:
+        e += 1
+    q = Fraction(2) ** (max(e, -126) - 23)
+    return sign * float(round(a / q) * q)   # Fraction.__round__: half to even
+
+
+def fma_f32(a: float, b: float, c: float) -> float:
+    return rn_f32(Fraction(a) * Fraction(b) + Fraction(c))
+
+
+def test_rn_f32_matches_numpy_rounding():
+    rng = np.random.default_rng(0)
+    for v in rng.standard_normal(2000) * np.exp2(rng.integers(-140, 100, 2000)):
+        assert rn_f32(Fraction(float(v))) == float(np.float32(v))
+
+
+@pytest.mark.parametrize("single", [False, True])
+def test_one_segment_epilogue_order(single):
+    """One K-segment: y = fma(c-, f(A-), fma(c+, f(A+), bias)) with
+    c+- = fl(s_w s+-) (single scale: y = fma(c, f(A), bias)), recomputed in
+    exact rational arithmetic from the oracle's own accumulators and scales."""
+    L = _c1_like(M=6, K=96, N=7, seed=12)
+    xb, wb = wl.bits(L.x), wl.bits(L.w)
+    bias = (np.random.default_rng(4).standard_normal(7) * 0.1).astype(np.float32)
+    bb = bf16_bits(bias)
+    r = oracle.layer(xb, wb, wl.bits(L.x_cal), None, bb, single=single)
+    acc = oracle.gemm_s32(r["planes"], r["wq"])
+    b32 = bits_to_f32(bb)
+    for m in range(6):
+        for n in range(7):
+            cp = float(np.float32(r["s_w"][0, n]) * np.float32(r["s_act"][0, 0, 0]))
+            y = fma_f32(cp, float(np.float32(acc[0, 0, m, n])), float(b32[n]))
+            if not single:
+                cm = float(np.float32(r["s_w"][0, n]) * np.float32(r["s_act"][0, 0, 1]))
+                y = fma_f32(cm, float(np.float32(acc[0, 1, m, n])), y)
+            assert r["y"][m, n] == np.float32(y)
+
+
 def test_input_segments_equal_sum():
     """Input-segmented Y = sum_i X^_i W^_i: the int32 partials equal those of
-    standalone per-segment products, and Y equals the ascending fp32 sum of the
-    per-segment outputs with the bias added once."""
-    L = wl.outproj_layer("t", 37, 128, 45, 32, seed=8)
+    standalone per-segment products, and Y is the sum of the per-segment terms
+    c+_i f(A+_i) + c-_i f(A-_i), c+-_i = fl(s_w[i] s+-_i), accumulated from the
+    bias with one exactly rounded fused multiply-add per term, segments in
+    ascending order (recomputed here in exact rational arithmetic)."""
+    L = wl.outproj_layer("t", 9, 128, 11, 32, seed=8)
     d = L.d.numpy()
     xb, wb, bb = wl.bits(L.x), wl.bits(L.w), wl.bits(L.bias)
     full = oracle.layer(xb, wb, wl.bits(L.x_cal), d, bb, MODE_INPUT, L.offsets)
     acc = oracle.gemm_s32(full["planes"], full["wq"], MODE_INPUT, L.offsets)
-    ysum = np.zeros_like(full["y"])
     for i in range(4):
         k0, k1 = L.offsets[i], L.offsets[i + 1]
         part = oracle.layer(np.ascontiguousarray(xb[:, k0:k1]),
@@ -421,9 +471,17 @@ def test_input_segments_equal_sum():
         assert np.array_equal(part["s_w"][0], full["s_w"][i])
         pacc = oracle.gemm_s32(part["planes"], part["wq"])
         assert np.array_equal(pacc[0], acc[i])
-        ysum = (ysum + part["y"]).astype(np.float32)
-    ysum = (ysum + bits_to_f32(bb)[None]).astype(np.float32)
-    assert np.array_equal(ysum, full["y"])
+    bias = bits_to_f32(bb)
+    s_act, s_w = full["s_act"], full["s_w"]
+    for m in range(L.M):
+        for n in range(L.N):
+            y = float(bias[n])
+            for i in range(4):
+                cp = float(np.float32(s_w[i, n]) * np.float32(s_act[0, i, 0]))
+                cm = float(np.float32(s_w[i, n]) * np.float32(s_act[0, i, 1]))
+                y = fma_f32(cp, float(np.float32(acc[i, 0, m, n])), y)
+                y = fma_f32(cm, float(np.float32(acc[i, 1, m, n])), y)
+            assert full["y"][m, n] == np.float32(y)
 
 
 # ------------------------------------------- brute-force float64 reconstruction
