@@ -53,12 +53,13 @@
  *    s = max(max u, -min u) / 127 for both signs, i.e. the DualScale quantizer
  *    with s+ = s-, whose two planes are then one: q = q+ + q- in [-128, 127],
  *    and one integer product A = sum q w.  Planes [G][1][M][K].
- *  - Epilogue in fp32, fixed order (the pages fix none): y starts at the bias
- *    (0 without one); for each K-segment i in ascending order, with the
- *    folded coefficients c+_i = fl(s_w[i][n] * s+_i), c-_i = fl(s_w[i][n] *
- *    s-_i) of the products s+ s_w and s- s_w the reconstruction formula shows,
- *    y = fma(c+_i, f(A+_i), y), then y = fma(c-_i, f(A-_i), y); single scale:
- *    y = fma(c_i, f(A_i), y).  f is int32 -> fp32 round-to-nearest; fma rounds
+ *  - Epilogue in fp32, fixed order (the pages fix none), read left to right
+ *    as the reconstruction formula is written: y starts at 0; for each
+ *    K-segment i in ascending order, with the folded coefficients
+ *    c+_i = fl(s_w[i][n] * s+_i), c-_i = fl(s_w[i][n] * s-_i) of the products
+ *    s+ s_w and s- s_w the formula shows, y = fma(c+_i, f(A+_i), y), then
+ *    y = fma(c-_i, f(A-_i), y) (single scale: y = fma(c_i, f(A_i), y)); the
+ *    bias is added last.  f is int32 -> fp32 round-to-nearest; fma rounds
  *    once.
  *
  * Layouts (row-major, innermost last):
@@ -314,9 +315,9 @@ int orc_gemm_s32(const int8_t *planes, const int8_t *wq, int64_t M, int64_t N,
 
 /* ---------------------------------------------------------------------------
  * Full layer: integer products, then the DualScale reconstruction in fp32
- *   y[m][n] = bias[n] + sum_i (s_w[i][n] s+_i) f(A+_i) + (s_w[i][n] s-_i) f(A-_i)
- * accumulated from the bias with one fused multiply-add per term, segments in
- * ascending order, + before -.  bias: bf16 bits [N] or NULL.  y [n_rows][N].
+ *   y[m][n] = sum_i (s_w[i][n] s+_i) f(A+_i) + (s_w[i][n] s-_i) f(A-_i) + bias[n]
+ * with one fused multiply-add per term, segments in ascending order, + before
+ * -, and the bias added last.  bias: bf16 bits [N] or NULL.  y [n_rows][N].
  * ------------------------------------------------------------------------- */
 int orc_gemm(const int8_t *planes, const int8_t *wq, const float *s_w,
              const float *s_act, const uint16_t *bias, int64_t M, int64_t N,
@@ -339,7 +340,7 @@ int orc_gemm(const int8_t *planes, const int8_t *wq, const float *s_w,
       const int8_t *xp = planes + (((int64_t)g * P + 0) * M + m) * K;
       const int8_t *xm = planes + (((int64_t)g * P + (P - 1)) * M + m) * K;
       const int8_t *wn = wq + n * K;
-      float yv = bias ? orc_bf16(bias[n]) : 0.0f;
+      float yv = 0.0f;
       for (int i = 0; i < S; ++i) {
         int64_t k0 = (S == 1) ? 0 : offsets[i];
         int64_t k1 = (S == 1) ? K : offsets[i + 1];
@@ -360,6 +361,7 @@ int orc_gemm(const int8_t *planes, const int8_t *wq, const float *s_w,
           yv = fmaf(cp, (float)a, yv);
         }
       }
+      if (bias) yv = yv + orc_bf16(bias[n]);
       y[r * N + n] = yv;
     }
   }
@@ -581,7 +583,7 @@ int orc_gemm_fp8(const uint8_t *planes, const uint8_t *wq, const float *s_w,
   for (int64_t r = 0; r < n_rows; ++r)
     for (int64_t n = 0; n < N; ++n) {
       int g = (mode == ORC_MODE_OUTPUT && G > 1) ? orc_seg_index(offsets, n_seg, n) : 0;
-      float yv = bias ? orc_bf16(bias[n]) : 0.0f;
+      float yv = 0.0f;
       for (int i = 0; i < S; ++i) {
         float sw = s_w[(int64_t)i * N + n];
         float cp = sw * s_act[((int64_t)g * S + i) * 2 + 0];
@@ -589,6 +591,7 @@ int orc_gemm_fp8(const uint8_t *planes, const uint8_t *wq, const float *s_w,
         yv = fmaf(cp, acc[(((int64_t)i * P + 0) * n_rows + r) * N + n], yv);
         if (P == 2) yv = fmaf(cm, acc[(((int64_t)i * P + 1) * n_rows + r) * N + n], yv);
       }
+      if (bias) yv = yv + orc_bf16(bias[n]);
       y[r * N + n] = yv;
     }
   free(acc);

@@ -2,11 +2,10 @@
 
 Bar (as fixed for this method): int8 planes, int8 weights, the scales that
 come out of calibration and the int32 accumulators are bit-exact; fp32 output
-within max |y - r| / (|r| + 1e-3 rms(r)) <= 1e-3.  With one K-segment the
-epilogue runs the oracle's fp32 operations in the oracle's order, so fp32 is
-bit-exact and bf16 equals RNE_bf16(oracle fp32).  With several K-segments the
-terms are accumulated with fused multiply-adds, so bf16 is held to the fp32
-criterion widened by one bf16 ulp.
+within max |y - r| / (|r| + 1e-3 rms(r)) <= 1e-3.  The epilogue runs the
+oracle's fp32 operations in the oracle's order (a fused multiply-add per term,
+from the bias) for one and for several K-segments, so the fp32 output is
+bit-exact and the bf16 output equals RNE_bf16(oracle fp32) as well.
 """
 import numpy as np
 import pytest
@@ -16,8 +15,7 @@ import oracle
 from w8a8_gemm_b200 import binding as B
 from w8a8_gemm_b200 import workloads as wl
 
-from parity import (bf16_close, bf16_ulp_diff, gpu_run, oracle_acc, oracle_prep, oracle_y, rel_err_floor,
-                    sample_rows, segments)
+from parity import (bf16_ulp_diff, gpu_run, oracle_acc, oracle_prep, oracle_y, rel_err_floor, sample_rows, segments)
 
 pytestmark = pytest.mark.gpu
 FP32_TOL = 1e-3
@@ -59,13 +57,9 @@ def _check_layer(L, full_rows=True):
     r = oracle_y(L, prep)
     y = g["y"].cpu().numpy()
     assert rel_err_floor(y, r) <= FP32_TOL
-    if L.S == 1:
-        assert np.array_equal(y, r)          # same fp32 operations, same order
+    assert np.array_equal(y, r)              # same fp32 operations, same order
     gb = gpu_run(L, out_dtype=torch.bfloat16)
-    if L.S == 1:
-        assert bf16_ulp_diff(gb["y"], r) == 0
-    else:
-        assert bf16_close(gb["y"], r)
+    assert bf16_ulp_diff(gb["y"], r) == 0    # RNE of the same fp32 value
 
 
 @pytest.mark.parametrize("name", sorted(SMALL))
@@ -185,12 +179,9 @@ def test_full_size_configs_sampled_rows(cfg):
         rows = sample_rows(L.M)
         r = oracle_y(L, prep, rows=rows)
         yb = g["y"][torch.from_numpy(rows).cuda()]
-        if L.S == 1:
-            assert bf16_ulp_diff(yb, r) == 0
-        else:
-            assert bf16_close(yb, r)
+        assert bf16_ulp_diff(yb, r) == 0
         gf = gpu_run(L, out_dtype=torch.float32)
-        assert rel_err_floor(gf["y"][torch.from_numpy(rows).cuda()].cpu().numpy(), r) <= FP32_TOL
+        assert np.array_equal(gf["y"][torch.from_numpy(rows).cuda()].cpu().numpy(), r)
         del g, gf
         torch.cuda.empty_cache()
 

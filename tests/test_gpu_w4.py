@@ -9,8 +9,7 @@ import torch
 
 from w8a8_gemm_b200 import workloads as wl
 
-from parity import (bf16_close, bf16_ulp_diff, gpu_run, oracle_acc, oracle_prep, oracle_y,
-                    rel_err_floor, sample_rows)
+from parity import (bf16_ulp_diff, gpu_run, oracle_acc, oracle_prep, oracle_y, rel_err_floor, sample_rows)
 
 pytestmark = pytest.mark.gpu
 
@@ -36,15 +35,10 @@ def test_w4_layers_against_oracle(name, single):
     assert np.array_equal(g["acc"].cpu().numpy(), 16 * oracle_acc(L, prep))
     r = oracle_y(L, prep)
     y = g["y"].cpu().numpy()
-    if L.S == 1:
-        assert np.array_equal(y, r)
-    else:
-        assert rel_err_floor(y, r) <= 1e-3
+    assert rel_err_floor(y, r) <= 1e-3
+    assert np.array_equal(y, r)
     gb = gpu_run(L, out_dtype=torch.bfloat16, single=single, weight_bits=4)
-    if L.S == 1:
-        assert bf16_ulp_diff(gb["y"], r) == 0
-    else:
-        assert bf16_close(gb["y"], r)
+    assert bf16_ulp_diff(gb["y"], r) == 0
 
 
 def test_w4_full_size_ffn_sampled_rows():

@@ -430,9 +430,9 @@ def test_rn_f32_matches_numpy_rounding():
 
 @pytest.mark.parametrize("single", [False, True])
 def test_one_segment_epilogue_order(single):
-    """One K-segment: y = fma(c-, f(A-), fma(c+, f(A+), bias)) with
-    c+- = fl(s_w s+-) (single scale: y = fma(c, f(A), bias)), recomputed in
-    exact rational arithmetic from the oracle's own accumulators and scales."""
+    """One K-segment: y = fma(c-, f(A-), fl(c+ f(A+))) + bias with
+    c+- = fl(s_w s+-) (single scale: y = fl(c f(A)) + bias), recomputed in exact
+    rational arithmetic from the oracle's own accumulators and scales."""
     L = _c1_like(M=6, K=96, N=7, seed=12)
     xb, wb = wl.bits(L.x), wl.bits(L.w)
     bias = (np.random.default_rng(4).standard_normal(7) * 0.1).astype(np.float32)
@@ -443,19 +443,20 @@ def test_one_segment_epilogue_order(single):
     for m in range(6):
         for n in range(7):
             cp = float(np.float32(r["s_w"][0, n]) * np.float32(r["s_act"][0, 0, 0]))
-            y = fma_f32(cp, float(np.float32(acc[0, 0, m, n])), float(b32[n]))
+            y = fma_f32(cp, float(np.float32(acc[0, 0, m, n])), 0.0)
             if not single:
                 cm = float(np.float32(r["s_w"][0, n]) * np.float32(r["s_act"][0, 0, 1]))
                 y = fma_f32(cm, float(np.float32(acc[0, 1, m, n])), y)
+            y = rn_f32(Fraction(y) + Fraction(float(b32[n])))
             assert r["y"][m, n] == np.float32(y)
 
 
 def test_input_segments_equal_sum():
     """Input-segmented Y = sum_i X^_i W^_i: the int32 partials equal those of
     standalone per-segment products, and Y is the sum of the per-segment terms
-    c+_i f(A+_i) + c-_i f(A-_i), c+-_i = fl(s_w[i] s+-_i), accumulated from the
-    bias with one exactly rounded fused multiply-add per term, segments in
-    ascending order (recomputed here in exact rational arithmetic)."""
+    c+_i f(A+_i) + c-_i f(A-_i), c+-_i = fl(s_w[i] s+-_i), accumulated with one
+    exactly rounded fused multiply-add per term, segments in ascending order,
+    and the bias added last (recomputed here in exact rational arithmetic)."""
     L = wl.outproj_layer("t", 9, 128, 11, 32, seed=8)
     d = L.d.numpy()
     xb, wb, bb = wl.bits(L.x), wl.bits(L.w), wl.bits(L.bias)
@@ -475,12 +476,13 @@ def test_input_segments_equal_sum():
     s_act, s_w = full["s_act"], full["s_w"]
     for m in range(L.M):
         for n in range(L.N):
-            y = float(bias[n])
+            y = 0.0
             for i in range(4):
                 cp = float(np.float32(s_w[i, n]) * np.float32(s_act[0, i, 0]))
                 cm = float(np.float32(s_w[i, n]) * np.float32(s_act[0, i, 1]))
                 y = fma_f32(cp, float(np.float32(acc[i, 0, m, n])), y)
                 y = fma_f32(cm, float(np.float32(acc[i, 1, m, n])), y)
+            y = rn_f32(Fraction(y) + Fraction(float(bias[n])))
             assert full["y"][m, n] == np.float32(y)
 
 

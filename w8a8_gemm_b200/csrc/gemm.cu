@@ -77,8 +77,10 @@ struct Smem {
   static constexpr int NBUF = 512 / (POL * BN);  // TMEM accumulator buffers
   static constexpr int EPI_OFFSET = STAGES * STAGE_BYTES;  // per-warp column constants
   static constexpr int COLS = BN / (EPI_WARPS / 4);  // columns per epilogue warp
-  // two arrays of COLS floats per warp; multi-segment layers double-buffer them
-  static constexpr int CONST_FLOATS = (SEGK ? 2 : 1) * 2 * COLS;
+  // per warp: one K-segment: s_w and bias (COLS floats each); several
+  // K-segments: c+ and c- double-buffered (the bias goes, at the end of a
+  // tile, into the buffer the last K-segment did not use)
+  static constexpr int CONST_FLOATS = (SEGK ? 4 : 2) * COLS;
   static constexpr int EPI_BYTES = EPI_WARPS * CONST_FLOATS * 4;
   // per-warp staging of one 32 x 32 bf16 output chunk for the tensor store
   static constexpr int STG_OFFSET = EPI_OFFSET + EPI_BYTES;
@@ -353,7 +355,8 @@ __global__ void __launch_bounds__(threads_for(EPI_WARPS), 1)
     const int row = quarter * 32 + lane;
     const uint32_t lane_addr = static_cast<uint32_t>(quarter * 32) << 16;
     // Warp-private column constants in shared memory, read back as broadcast
-    // float4s: [HALF] + [HALF] floats (two such buffers with several K-segments).
+    // float4s: s_w and bias, [HALF] floats each (with several K-segments two
+    // buffers of c+ = fl(s_w s+) and c- = fl(s_w s-)).
     float *cst_base = reinterpret_cast<float *>(smem + L::EPI_OFFSET) + ew * L::CONST_FLOATS;
     uint8_t *stg = smem + L::STG_OFFSET + ew * 2048;  // used when TMA_STORE
     uint32_t acc_iter = 0;
@@ -445,10 +448,11 @@ __global__ void __launch_bounds__(threads_for(EPI_WARPS), 1)
                 }
             }
           } else if constexpr (!SEGK) {
-            // One K-segment: the fp32 operations in the reference order
-            //   t = s+ f(A+) + s- f(A-);  y = s_w t + bias,
-            // two columns per packed instruction (each lane rounds once per
-            // operation, exactly as the scalar sequence does).
+            // One K-segment, in the reference order: y = fma(c-, f(A-),
+            // fl(c+ f(A+))) + bias with c+- = fl(s_w s+-), or
+            // y = fl(c f(A)) + bias for a single scale; two columns per packed
+            // instruction (each lane rounds once per product, fused
+            // multiply-add and sum, as the scalar sequence does).
             if (TMA_STORE || m < p.M) {
               const float4 *sw4 = reinterpret_cast<const float4 *>(cst + c * CW);
               const float4 *b4 = reinterpret_cast<const float4 *>(cst + HALF + c * CW);
@@ -461,19 +465,14 @@ __global__ void __launch_bounds__(threads_for(EPI_WARPS), 1)
 #pragma unroll
                 for (int h = 0; h < 2; ++h) {
                   const int j = 4 * q + 2 * h;
+                  const uint64_t w2 = h ? f2pack(w.z, w.w) : f2pack(w.x, w.y);
                   const uint64_t fp = f2pack(acc_f32<F8>(ap[j]), acc_f32<F8>(ap[j + 1]));
-                  // Each step is one packed FMA with a zero addend or a unit
-                  // factor, i.e. exactly one rounding of the scalar product
-                  // or sum, and nothing the compiler could contract further.
-                  uint64_t t;
+                  uint64_t y = ffma2(ffma2(w2, sp2, zero2), fp, zero2);
                   if constexpr (POL == 2) {
                     const uint64_t fm = f2pack(acc_f32<F8>(am[j]), acc_f32<F8>(am[j + 1]));
-                    t = ffma2(one2, ffma2(sp2, fp, zero2), ffma2(sm2, fm, zero2));
-                  } else {
-                    t = ffma2(sp2, fp, zero2);  // single scale: t = s f(A)
+                    y = ffma2(ffma2(w2, sm2, zero2), fm, y);
                   }
-                  const uint64_t u = ffma2(h ? f2pack(w.z, w.w) : f2pack(w.x, w.y), t, zero2);
-                  const uint64_t y = ffma2(one2, u, h ? f2pack(b.z, b.w) : f2pack(b.x, b.y));
+                  y = ffma2(one2, y, h ? f2pack(b.z, b.w) : f2pack(b.x, b.y));
                   f2unpack(y, v[j], v[j + 1]);
                 }
               }
@@ -509,8 +508,9 @@ __global__ void __launch_bounds__(threads_for(EPI_WARPS), 1)
           }
         }
         if constexpr (SEGK && OUT != OUT_S32) {
-          // Several K-segments: y += c+ f(A+) + c- f(A-), two columns per packed
-          // instruction, 16 columns per TMEM load to keep register pressure low.
+          // Several K-segments: y = fma(c-, f(A-), fma(c+, f(A+), y)) from
+          // y = 0, two columns per packed instruction, 16 columns per TMEM
+          // load to keep register pressure low; the bias is added at the end.
 #pragma unroll
           for (int c = 0; c < HALF / 16; ++c) {
             uint32_t ap[16], am[16];
