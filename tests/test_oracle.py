@@ -451,7 +451,8 @@ def test_one_segment_epilogue_order(single):
             assert r["y"][m, n] == np.float32(y)
 
 
-def test_input_segments_equal_sum():
+@pytest.mark.parametrize("single", [False, True])
+def test_input_segments_equal_sum(single):
     """Input-segmented Y = sum_i X^_i W^_i: the int32 partials equal those of
     standalone per-segment products, and Y is the sum of the per-segment terms
     c+_i f(A+_i) + c-_i f(A-_i), c+-_i = fl(s_w[i] s+-_i), accumulated with one
@@ -460,14 +461,14 @@ def test_input_segments_equal_sum():
     L = wl.outproj_layer("t", 9, 128, 11, 32, seed=8)
     d = L.d.numpy()
     xb, wb, bb = wl.bits(L.x), wl.bits(L.w), wl.bits(L.bias)
-    full = oracle.layer(xb, wb, wl.bits(L.x_cal), d, bb, MODE_INPUT, L.offsets)
+    full = oracle.layer(xb, wb, wl.bits(L.x_cal), d, bb, MODE_INPUT, L.offsets, single=single)
     acc = oracle.gemm_s32(full["planes"], full["wq"], MODE_INPUT, L.offsets)
     for i in range(4):
         k0, k1 = L.offsets[i], L.offsets[i + 1]
         part = oracle.layer(np.ascontiguousarray(xb[:, k0:k1]),
                             np.ascontiguousarray(wb[:, k0:k1]),
                             np.ascontiguousarray(wl.bits(L.x_cal)[:, k0:k1]),
-                            d[:, k0:k1])
+                            d[:, k0:k1], single=single)
         assert np.array_equal(part["planes"][0], full["planes"][0][:, :, k0:k1])
         assert np.array_equal(part["s_w"][0], full["s_w"][i])
         pacc = oracle.gemm_s32(part["planes"], part["wq"])
@@ -481,7 +482,8 @@ def test_input_segments_equal_sum():
                 cp = float(np.float32(s_w[i, n]) * np.float32(s_act[0, i, 0]))
                 cm = float(np.float32(s_w[i, n]) * np.float32(s_act[0, i, 1]))
                 y = fma_f32(cp, float(np.float32(acc[i, 0, m, n])), y)
-                y = fma_f32(cm, float(np.float32(acc[i, 1, m, n])), y)
+                if not single:
+                    y = fma_f32(cm, float(np.float32(acc[i, 1, m, n])), y)
             y = rn_f32(Fraction(y) + Fraction(float(bias[n])))
             assert full["y"][m, n] == np.float32(y)
 
