@@ -226,10 +226,12 @@ SQ_API sq_status sq_unpack_weight_w4(const uint8_t *wq4, int64_t N, int64_t K, i
  *   A+_i[m][n] = sum_{k in segment i} X^+[g(n)][m][k] * W^[n][k]   (same for -)
  * Epilogue in fp32, never leaving the chip:
  *   y[m][n] = sum_i s_w[i][n] * (s+[g][i]*f(A+_i) + s-[g][i]*f(A-_i)) + bias[n]
- * with f = int32 -> fp32 round-to-nearest.  With S == 1 the operations run in
- * exactly this order; with S > 1 each segment's term is accumulated as
- * (s_w s+) f(A+) + (s_w s-) f(A-) with fused multiply-adds (same value up to
- * fp32 rounding).  Output rounds to bf16 (RN) or stays fp32.
+ * with f = int32 -> fp32 round-to-nearest, evaluated in one fixed fp32 order
+ * for every segment mode: c+- = fl(s_w[i][n] * s+-[g][i]); y = 0; for each
+ * segment i ascending y = fma(c+, f(A+_i), y), then y = fma(c-, f(A-_i), y);
+ * finally y = y + bias[n].  The result is therefore a deterministic function
+ * of the inputs, independent of tiling.  Output rounds to bf16 (RN) or stays
+ * fp32.
  *   planes int8 [G][P][M][K] from sq_quantize_act (P = 1 with
  *          SQ_FLAG_SINGLE_SCALE: one product, y = sum_i s_w[i][n] s[g][i] f(A_i)
  *          + bias, s = s_act[g][i][0]); wq int8 [N][K]

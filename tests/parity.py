@@ -126,9 +126,9 @@ def bf16_ulp_diff(y_bf16: torch.Tensor, r_f32: np.ndarray) -> int:
 
 
 def bf16_close(y_bf16: torch.Tensor, r_f32: np.ndarray, tol: float = 1e-3) -> bool:
-    """bf16 output check for the multi-segment epilogue, whose fp32 value may
-    differ from the oracle's by fp32 reordering: |y - r| <= ulp_bf16(r) +
-    tol * (|r| + 1e-3 rms(r)), the fp32 criterion widened by one bf16 ulp."""
+    """bf16 output check where the fp32 accumulation order is the tensor
+    core's (FP8 products summed in fp32 inside the MMA): |y - r| <= ulp_bf16(r)
+    + tol * (|r| + 1e-3 rms(r)), the fp32 criterion widened by one bf16 ulp."""
     r = r_f32.astype(np.float64)
     y = y_bf16.float().cpu().numpy().astype(np.float64)
     rms = float(np.sqrt(np.mean(r * r))) if r.size else 0.0

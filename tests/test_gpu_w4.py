@@ -1,8 +1,8 @@
 """W4A8 ("SegQuant-4") through the CUDA path against the oracle: packed 4-bit
 weight codes and their scales bit-exact, the expanded GEMM operand equal to
 16 x the codes, raw accumulators equal to 16 x the oracle's, and outputs held
-to the same bar as W8A8 (one K-segment: fp32 bit-exact, bf16 = RNE of the
-oracle; several: the fp32 criterion widened by one bf16 ulp)."""
+to the same bar as W8A8 (fp32 bit-exact and bf16 = RNE of the oracle, for
+every segment mode)."""
 import numpy as np
 import pytest
 import torch
