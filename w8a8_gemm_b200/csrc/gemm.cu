@@ -376,8 +376,9 @@ __global__ void __launch_bounds__(threads_for(EPI_WARPS), 1)
         __syncwarp();
       }
       // Multi-segment state: packed running sums (column pairs) and the next
-      // K-segment's weight and activation scales, loaded one segment ahead so
-      // that no global load latency sits between two drains.
+      // K-segment's weight and activation scales, loaded one segment ahead and
+      // not used (not even scaled by act_mul) until that segment starts, so
+      // that no instruction waits for a global load between two drains.
       uint64_t run2[SEGK ? HALF / 2 : 1];
       float sw_next[SEGK ? HALF / 32 : 1];
       float sp_next = 0.0f, sm_next = 0.0f;
@@ -389,17 +390,17 @@ __global__ void __launch_bounds__(threads_for(EPI_WARPS), 1)
           const int64_t n = nb + q * 32 + lane;
           sw_next[q] = n < p.N ? p.s_w[n] : 0.0f;
         }
-        sp_next = __fmul_rn(p.s_act[g * p.S * 2 + 0], p.act_mul);
-        sm_next = __fmul_rn(p.s_act[g * p.S * 2 + 1], p.act_mul);
+        sp_next = p.s_act[g * p.S * 2 + 0];
+        sm_next = p.s_act[g * p.S * 2 + 1];
       }
       const int units = SEGK ? p.S : 1;
       for (int u = 0; u < units; ++u) {
-        const float sp = (SEGK && OUT != OUT_S32)
-                             ? sp_next
-                             : __fmul_rn(p.s_act[(g * p.S + u) * 2 + 0], p.act_mul);
-        const float sm = (SEGK && OUT != OUT_S32)
-                             ? sm_next
-                             : __fmul_rn(p.s_act[(g * p.S + u) * 2 + 1], p.act_mul);
+        const float sp = __fmul_rn((SEGK && OUT != OUT_S32) ? sp_next
+                                                            : p.s_act[(g * p.S + u) * 2 + 0],
+                                   p.act_mul);
+        const float sm = __fmul_rn((SEGK && OUT != OUT_S32) ? sm_next
+                                                            : p.s_act[(g * p.S + u) * 2 + 1],
+                                   p.act_mul);
         float *cst = cst_base;
         if constexpr (SEGK && OUT != OUT_S32) {
           // Folded coefficients of K-segment u: c+- = s_w[u][n] * s+-[u], into
@@ -418,8 +419,8 @@ __global__ void __launch_bounds__(threads_for(EPI_WARPS), 1)
               const int64_t n = nb + q * 32 + lane;
               sw_next[q] = n < p.N ? swn[n] : 0.0f;
             }
-            sp_next = __fmul_rn(p.s_act[(g * p.S + u + 1) * 2 + 0], p.act_mul);
-            sm_next = __fmul_rn(p.s_act[(g * p.S + u + 1) * 2 + 1], p.act_mul);
+            sp_next = p.s_act[(g * p.S + u + 1) * 2 + 0];
+            sm_next = p.s_act[(g * p.S + u + 1) * 2 + 1];
           }
           __syncwarp();
         }
@@ -509,36 +510,43 @@ __global__ void __launch_bounds__(threads_for(EPI_WARPS), 1)
         }
         if constexpr (SEGK && OUT != OUT_S32) {
           // Several K-segments: y = fma(c-, f(A-), fma(c+, f(A+), y)) from
-          // y = 0, two columns per packed instruction, 16 columns per TMEM
-          // load to keep register pressure low; the bias is added at the end.
+          // y = 0, two columns per packed instruction; the bias is added at
+          // the end.  The warp folds in its 32 columns of A+, then copies
+          // those of A- into registers and hands the TMEM buffer back before
+          // folding them in, so that the MMAs of the segment after next
+          // overlap the rest of this segment's arithmetic.
+          static_assert(HALF == 32, "one 32-column TMEM load per polarity");
+          const auto cvt2 = [](uint32_t x, uint32_t y) {
+            return f2pack(acc_f32<F8>(x), acc_f32<F8>(y));
+          };
+          const auto fold = [&](const uint32_t(&acc)[32], const float *c) {
+            const float4 *c4 = reinterpret_cast<const float4 *>(c);
 #pragma unroll
-          for (int c = 0; c < HALF / 16; ++c) {
-            uint32_t ap[16], am[16];
-            tmem_ld_32x32b_x16(t_plus + c * 16, ap);
-            if constexpr (POL == 2) tmem_ld_32x32b_x16(t_plus + BN + c * 16, am);
-            tmem_ld_wait();
-            const float4 *cp4 = reinterpret_cast<const float4 *>(cst + c * 16);
-            const float4 *cm4 = reinterpret_cast<const float4 *>(cst + HALF + c * 16);
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              const float4 a = cp4[q], b = cm4[q];
+            for (int q = 0; q < 8; ++q) {
+              const float4 w = c4[q];
               const int j = 4 * q;
-              uint64_t &r0 = run2[c * 8 + 2 * q], &r1 = run2[c * 8 + 2 * q + 1];
-              const auto cvt2 = [](uint32_t x, uint32_t y) {
-                return f2pack(acc_f32<F8>(x), acc_f32<F8>(y));
-              };
-              r0 = ffma2(f2pack(a.x, a.y), cvt2(ap[j], ap[j + 1]), r0);
-              r1 = ffma2(f2pack(a.z, a.w), cvt2(ap[j + 2], ap[j + 3]), r1);
-              if constexpr (POL == 2) {
-                r0 = ffma2(f2pack(b.x, b.y), cvt2(am[j], am[j + 1]), r0);
-                r1 = ffma2(f2pack(b.z, b.w), cvt2(am[j + 2], am[j + 3]), r1);
-              }
+              run2[2 * q] = ffma2(f2pack(w.x, w.y), cvt2(acc[j], acc[j + 1]), run2[2 * q]);
+              run2[2 * q + 1] =
+                  ffma2(f2pack(w.z, w.w), cvt2(acc[j + 2], acc[j + 3]), run2[2 * q + 1]);
             }
+          };
+          uint32_t acc[32];
+          tmem_ld_32x32b_x32(t_plus, acc);
+          tmem_ld_wait();
+          if constexpr (POL == 2) {
+            fold(acc, cst);
+            tmem_ld_32x32b_x32(t_plus + BN, acc);
+            tmem_ld_wait();
           }
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&acc_empty[buf]);
+          fold(acc, POL == 2 ? cst + HALF : cst);
+        } else {
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&acc_empty[buf]);
         }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&acc_empty[buf]);
         ++acc_iter;
       }
       if constexpr (SEGK && OUT != OUT_S32) {
