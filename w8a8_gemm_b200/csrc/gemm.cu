@@ -171,6 +171,28 @@ __device__ __forceinline__ void store_row_chunk(const GemmParams &p, int64_t m, 
   }
 }
 
+// Two adjacent output columns n, n + 1 of row m (n even; n + 1 may be >= N).
+template <int OUT>
+__device__ __forceinline__ void store_pair(const GemmParams &p, int64_t m, int64_t n, float y0,
+                                           float y1) {
+  if (n >= p.N) return;
+  if (OUT == OUT_BF16) {
+    uint16_t *row = reinterpret_cast<uint16_t *>(p.y) + m * p.ldy;
+    if (n + 1 < p.N) {
+      *reinterpret_cast<uint32_t *>(row + n) = pack_bf16x2(y0, y1);
+    } else {
+      const __nv_bfloat16 b = __float2bfloat16_rn(y0);
+      row[n] = *reinterpret_cast<const uint16_t *>(&b);
+    }
+  } else {
+    float *row = reinterpret_cast<float *>(p.y) + m * p.ldy;
+    if (n + 1 < p.N)
+      *reinterpret_cast<float2 *>(row + n) = make_float2(y0, y1);
+    else
+      row[n] = y0;
+  }
+}
+
 // TMEM columns of one chunk: 16 or 32 per lane.
 template <int CW>
 __device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, uint32_t (&r)[CW]) {
@@ -206,7 +228,6 @@ __global__ void __launch_bounds__(threads_for(EPI_WARPS), 1)
   constexpr int NBUF = L::NBUF;
   constexpr int ACC_COLS = POL * BN;  // TMEM columns of one accumulator buffer
   constexpr int HALF = L::COLS;      // columns per epilogue warp
-  constexpr int CHUNKS = HALF / 32;  // 32-column groups (final multi-segment stores)
   // TMEM chunk of the one-segment epilogue: 32 columns with 8 warps, 16 with
   // more warps (their register budget is smaller).
   constexpr int CW = EPI_WARPS >= 16 ? 16 : 32;
@@ -511,37 +532,48 @@ __global__ void __launch_bounds__(threads_for(EPI_WARPS), 1)
         if constexpr (SEGK && OUT != OUT_S32) {
           // Several K-segments: y = fma(c-, f(A-), fma(c+, f(A+), y)) from
           // y = 0, two columns per packed instruction; the bias is added at
-          // the end.  The warp folds in its 32 columns of A+, then copies
-          // those of A- into registers and hands the TMEM buffer back before
-          // folding them in, so that the MMAs of the segment after next
-          // overlap the rest of this segment's arithmetic.
-          static_assert(HALF == 32, "one 32-column TMEM load per polarity");
+          // the end.  The accumulators are read in the 16x256b pattern: a
+          // thread holds rows t/4 + {0, 8, 16, 24} of the warp's 32 and
+          // columns 8j + 2 (t % 4) + {0, 1}, j < 4, so it needs 8 of the 32
+          // column coefficients per polarity (4 float2 reads instead of 8
+          // float4), which keeps the shared-memory pipe off the critical path.
+          // run2[8k + 2j + h] holds row 16k + 8h + t/4, column pair j.  The
+          // warp folds in A+, copies A- into registers and hands the TMEM
+          // buffer back before folding A- in, so that the MMAs of the segment
+          // after next overlap the rest of this segment's arithmetic.
+          static_assert(HALF == 32, "one 32-column TMEM block per polarity and warp");
+          const int q2 = 2 * (lane & 3);
           const auto cvt2 = [](uint32_t x, uint32_t y) {
             return f2pack(acc_f32<F8>(x), acc_f32<F8>(y));
           };
-          const auto fold = [&](const uint32_t(&acc)[32], const float *c) {
-            const float4 *c4 = reinterpret_cast<const float4 *>(c);
+          const auto fold = [&](const uint32_t(&lo)[16], const uint32_t(&hi)[16],
+                                const float *c) {
 #pragma unroll
-            for (int q = 0; q < 8; ++q) {
-              const float4 w = c4[q];
-              const int j = 4 * q;
-              run2[2 * q] = ffma2(f2pack(w.x, w.y), cvt2(acc[j], acc[j + 1]), run2[2 * q]);
-              run2[2 * q + 1] =
-                  ffma2(f2pack(w.z, w.w), cvt2(acc[j + 2], acc[j + 3]), run2[2 * q + 1]);
+            for (int j = 0; j < 4; ++j) {
+              const uint64_t cj = *reinterpret_cast<const uint64_t *>(c + 8 * j + q2);
+#pragma unroll
+              for (int h = 0; h < 2; ++h) {
+                const int r = 4 * j + 2 * h;
+                run2[2 * j + h] = ffma2(cj, cvt2(lo[r], lo[r + 1]), run2[2 * j + h]);
+                run2[8 + 2 * j + h] = ffma2(cj, cvt2(hi[r], hi[r + 1]), run2[8 + 2 * j + h]);
+              }
             }
           };
-          uint32_t acc[32];
-          tmem_ld_32x32b_x32(t_plus, acc);
+          constexpr uint32_t kLanes16 = 16u << 16;
+          uint32_t lo[16], hi[16];
+          tmem_ld_16x256b_x4(t_plus, lo);
+          tmem_ld_16x256b_x4(t_plus + kLanes16, hi);
           tmem_ld_wait();
           if constexpr (POL == 2) {
-            fold(acc, cst);
-            tmem_ld_32x32b_x32(t_plus + BN, acc);
+            fold(lo, hi, cst);
+            tmem_ld_16x256b_x4(t_plus + BN, lo);
+            tmem_ld_16x256b_x4(t_plus + BN + kLanes16, hi);
             tmem_ld_wait();
           }
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(&acc_empty[buf]);
-          fold(acc, POL == 2 ? cst + HALF : cst);
+          fold(lo, hi, POL == 2 ? cst + HALF : cst);
         } else {
           tc_fence_before();
           __syncwarp();
@@ -556,25 +588,23 @@ __global__ void __launch_bounds__(threads_for(EPI_WARPS), 1)
           bst[j] = (p.bias != nullptr && n < p.N) ? bf16_to_f32(p.bias[n]) : 0.0f;
         }
         __syncwarp();
-        if (m < p.M) {
+        // Rows and columns in the 16x256b pattern of the drains.
+        const int q2 = 2 * (lane & 3);
 #pragma unroll
-          for (int c = 0; c < CHUNKS; ++c) {
-            const float4 *b4 = reinterpret_cast<const float4 *>(bst + c * 32);
-            float v[32];
+        for (int k = 0; k < 2; ++k)
 #pragma unroll
-            for (int q = 0; q < 8; ++q) {
-              const float4 b = b4[q];
-              float r0, r1, r2, r3;
-              f2unpack(run2[c * 16 + 2 * q], r0, r1);
-              f2unpack(run2[c * 16 + 2 * q + 1], r2, r3);
-              v[4 * q + 0] = __fadd_rn(r0, b.x);
-              v[4 * q + 1] = __fadd_rn(r1, b.y);
-              v[4 * q + 2] = __fadd_rn(r2, b.z);
-              v[4 * q + 3] = __fadd_rn(r3, b.w);
+          for (int h = 0; h < 2; ++h) {
+            const int64_t mr = static_cast<int64_t>(mt) * BM + quarter * 32 + 16 * k + 8 * h + (lane >> 2);
+            if (mr < p.M) {
+#pragma unroll
+              for (int j = 0; j < 4; ++j) {
+                const float2 b = *reinterpret_cast<const float2 *>(bst + 8 * j + q2);
+                float r0, r1;
+                f2unpack(run2[8 * k + 2 * j + h], r0, r1);
+                store_pair<OUT>(p, mr, nb + 8 * j + q2, __fadd_rn(r0, b.x), __fadd_rn(r1, b.y));
+              }
             }
-            store_row_chunk<OUT>(p, m, nb + c * 32, v);
           }
-        }
         __syncwarp();
       }
     }
