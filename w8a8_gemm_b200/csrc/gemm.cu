@@ -588,21 +588,56 @@ __global__ void __launch_bounds__(threads_for(EPI_WARPS), 1)
           bst[j] = (p.bias != nullptr && n < p.N) ? bf16_to_f32(p.bias[n]) : 0.0f;
         }
         __syncwarp();
-        // Rows and columns in the 16x256b pattern of the drains.
-        const int q2 = 2 * (lane & 3);
+        // Rows and columns in the 16x256b pattern of the drains: thread t
+        // holds, for each of its 4 rows, column pairs 8j + 2q (q = t % 4).
+        const int q = lane & 3;
 #pragma unroll
         for (int k = 0; k < 2; ++k)
 #pragma unroll
           for (int h = 0; h < 2; ++h) {
             const int64_t mr = static_cast<int64_t>(mt) * BM + quarter * 32 + 16 * k + 8 * h + (lane >> 2);
-            if (mr < p.M) {
+            float y[8];  // pairs j = 0..3
 #pragma unroll
-              for (int j = 0; j < 4; ++j) {
-                const float2 b = *reinterpret_cast<const float2 *>(bst + 8 * j + q2);
-                float r0, r1;
-                f2unpack(run2[8 * k + 2 * j + h], r0, r1);
-                store_pair<OUT>(p, mr, nb + 8 * j + q2, __fadd_rn(r0, b.x), __fadd_rn(r1, b.y));
+            for (int j = 0; j < 4; ++j) {
+              const float2 b = *reinterpret_cast<const float2 *>(bst + 8 * j + 2 * q);
+              f2unpack(run2[8 * k + 2 * j + h], y[2 * j], y[2 * j + 1]);
+              y[2 * j] = __fadd_rn(y[2 * j], b.x);
+              y[2 * j + 1] = __fadd_rn(y[2 * j + 1], b.y);
+            }
+            if constexpr (OUT == OUT_BF16) {
+              // The 4 lanes of a row exchange bf16 pairs (a 4 x 4 transpose in
+              // two xor rounds) so that lane q ends with columns 8q .. 8q + 7
+              // and writes them with one 16-byte store.
+              uint32_t w[4];
+#pragma unroll
+              for (int j = 0; j < 4; ++j) w[j] = pack_bf16x2(y[2 * j], y[2 * j + 1]);
+              {
+                const bool up = q & 2;  // swap the off-diagonal 2 x 2 blocks
+                const uint32_t s0 = __shfl_xor_sync(0xffffffffu, up ? w[0] : w[2], 2);
+                const uint32_t s1 = __shfl_xor_sync(0xffffffffu, up ? w[1] : w[3], 2);
+                if (up) { w[0] = s0; w[1] = s1; } else { w[2] = s0; w[3] = s1; }
               }
+              {
+                const bool odd = q & 1;  // transpose each 2 x 2 block
+                const uint32_t s0 = __shfl_xor_sync(0xffffffffu, odd ? w[0] : w[1], 1);
+                const uint32_t s1 = __shfl_xor_sync(0xffffffffu, odd ? w[2] : w[3], 1);
+                if (odd) { w[0] = s0; w[2] = s1; } else { w[1] = s0; w[3] = s1; }
+              }
+              const int64_t n0 = nb + 8 * q;
+              if (mr < p.M && n0 < p.N) {
+                uint16_t *row = reinterpret_cast<uint16_t *>(p.y) + mr * p.ldy;
+                if (n0 + 8 <= p.N) {
+                  *reinterpret_cast<uint4 *>(row + n0) = make_uint4(w[0], w[1], w[2], w[3]);
+                } else {
+#pragma unroll
+                  for (int e = 0; e < 8; ++e)
+                    if (n0 + e < p.N) row[n0 + e] = static_cast<uint16_t>(w[e >> 1] >> (16 * (e & 1)));
+                }
+              }
+            } else if (mr < p.M) {
+#pragma unroll
+              for (int j = 0; j < 4; ++j)
+                store_pair<OUT>(p, mr, nb + 8 * j + 2 * q, y[2 * j], y[2 * j + 1]);
             }
           }
         __syncwarp();
