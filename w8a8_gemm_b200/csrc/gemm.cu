@@ -77,10 +77,11 @@ struct Smem {
   static constexpr int NBUF = 512 / (POL * BN);  // TMEM accumulator buffers
   static constexpr int EPI_OFFSET = STAGES * STAGE_BYTES;  // per-warp column constants
   static constexpr int COLS = BN / (EPI_WARPS / 4);  // columns per epilogue warp
-  // per warp: one K-segment: s_w and bias (COLS floats each); several
+  // per warp: one K-segment: the folded c+ = fl(s_w s+), c- = fl(s_w s-)
+  // and the bias (COLS floats each; c- unused with one plane); several
   // K-segments: c+ and c- double-buffered (the bias goes, at the end of a
   // tile, into the buffer the last K-segment did not use)
-  static constexpr int CONST_FLOATS = (SEGK ? 4 : 2) * COLS;
+  static constexpr int CONST_FLOATS = (SEGK ? 4 : 3) * COLS;
   static constexpr int EPI_BYTES = EPI_WARPS * CONST_FLOATS * 4;
   // per-warp staging of one 32 x 32 bf16 output chunk for the tensor store
   static constexpr int STG_OFFSET = EPI_OFFSET + EPI_BYTES;
@@ -133,42 +134,6 @@ __device__ __forceinline__ float bf16_to_f32(uint16_t h) {
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<const uint32_t *>(&v);
-}
-
-template <int OUT, int W = 32>
-__device__ __forceinline__ void store_row_chunk(const GemmParams &p, int64_t m, int64_t n0,
-                                                const float (&v)[W]) {
-  if (OUT == OUT_BF16) {
-    uint16_t *row = reinterpret_cast<uint16_t *>(p.y) + m * p.ldy;
-    if (n0 + W <= p.N) {
-      uint4 *dst = reinterpret_cast<uint4 *>(row + n0);
-#pragma unroll
-      for (int q = 0; q < W / 8; ++q)
-        dst[q] = make_uint4(pack_bf16x2(v[8 * q + 0], v[8 * q + 1]),
-                            pack_bf16x2(v[8 * q + 2], v[8 * q + 3]),
-                            pack_bf16x2(v[8 * q + 4], v[8 * q + 5]),
-                            pack_bf16x2(v[8 * q + 6], v[8 * q + 7]));
-    } else {
-#pragma unroll
-      for (int j = 0; j < W; ++j)
-        if (n0 + j < p.N) {
-          const __nv_bfloat16 b = __float2bfloat16_rn(v[j]);
-          row[n0 + j] = *reinterpret_cast<const uint16_t *>(&b);
-        }
-    }
-  } else {
-    float *row = reinterpret_cast<float *>(p.y) + m * p.ldy;
-    if (n0 + W <= p.N) {
-      float4 *dst = reinterpret_cast<float4 *>(row + n0);
-#pragma unroll
-      for (int q = 0; q < W / 4; ++q)
-        dst[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
-    } else {
-#pragma unroll
-      for (int j = 0; j < W; ++j)
-        if (n0 + j < p.N) row[n0 + j] = v[j];
-    }
-  }
 }
 
 // Two adjacent output columns n, n + 1 of row m (n even; n + 1 may be >= N).
@@ -387,12 +352,18 @@ __global__ void __launch_bounds__(threads_for(EPI_WARPS), 1)
       const int64_t m = static_cast<int64_t>(mt) * BM + row;
       const int64_t nb = static_cast<int64_t>(nt) * BN + half * HALF;
       if constexpr (!SEGK && OUT != OUT_S32) {
-        // s_w and bias of this warp's columns, staged while the MMAs run.
+        // The folded c+- = fl(s_w s+-) and the bias of this warp's columns,
+        // staged while the MMAs run (one K-segment: s_act[g][0]).
+        const float sp0 = __fmul_rn(p.s_act[g * 2 + 0], p.act_mul);
+        const float sm0 = __fmul_rn(p.s_act[g * 2 + 1], p.act_mul);
         __syncwarp();
         for (int j = lane; j < HALF; j += 32) {
           const int64_t n = nb + j;
-          cst_base[j] = n < p.N ? p.s_w[n] : 0.0f;
-          cst_base[HALF + j] = (p.bias != nullptr && n < p.N) ? bf16_to_f32(p.bias[n]) : 0.0f;
+          const float w = n < p.N ? p.s_w[n] : 0.0f;
+          cst_base[j] = __fmaf_rn(w, sp0, 0.0f);
+          if constexpr (POL == 2) cst_base[HALF + j] = __fmaf_rn(w, sm0, 0.0f);
+          cst_base[POL * HALF + j] =
+              (p.bias != nullptr && n < p.N) ? bf16_to_f32(p.bias[n]) : 0.0f;
         }
         __syncwarp();
       }
@@ -452,12 +423,12 @@ __global__ void __launch_bounds__(threads_for(EPI_WARPS), 1)
         const uint32_t t_plus = tmem_base + lane_addr + buf * ACC_COLS + half * HALF;
 #pragma unroll
         for (int c = 0; c < ((SEGK && OUT != OUT_S32) ? 0 : HALF / CW); ++c) {
-          uint32_t ap[CW], am[CW];
-          tmem_ld_cols<CW>(t_plus + c * CW, ap);
-          if constexpr (POL == 2) tmem_ld_cols<CW>(t_plus + BN + c * CW, am);
-          tmem_ld_wait();
           const int64_t n0 = nb + c * CW;
           if constexpr (OUT == OUT_S32) {
+            uint32_t ap[CW], am[CW];
+            tmem_ld_cols<CW>(t_plus + c * CW, ap);
+            if constexpr (POL == 2) tmem_ld_cols<CW>(t_plus + BN + c * CW, am);
+            tmem_ld_wait();
             if (m < p.M) {
               int32_t *accp = reinterpret_cast<int32_t *>(p.y) +
                               ((static_cast<int64_t>(u) * POL) * p.M + m) * p.N;
@@ -471,60 +442,74 @@ __global__ void __launch_bounds__(threads_for(EPI_WARPS), 1)
             }
           } else if constexpr (!SEGK) {
             // One K-segment, in the reference order: y = fma(c-, f(A-),
-            // fl(c+ f(A+))) + bias with c+- = fl(s_w s+-), or
-            // y = fl(c f(A)) + bias for a single scale; two columns per packed
-            // instruction (each lane rounds once per product, fused
-            // multiply-add and sum, as the scalar sequence does).
-            if (TMA_STORE || m < p.M) {
-              const float4 *sw4 = reinterpret_cast<const float4 *>(cst + c * CW);
-              const float4 *b4 = reinterpret_cast<const float4 *>(cst + HALF + c * CW);
-              const uint64_t sp2 = f2pack(sp, sp), sm2 = f2pack(sm, sm);
-              const uint64_t zero2 = f2pack(0.0f, 0.0f), one2 = f2pack(1.0f, 1.0f);
-              float v[CW];
+            // fl(c+ f(A+))) + bias with the folded c+- = fl(s_w s+-) staged per
+            // column, or y = fl(c f(A)) + bias for a single scale; each step one
+            // rounding, two columns per packed instruction.  The 32-column
+            // chunk is read in the 16x256b pattern: thread t holds rows
+            // 16k + 8h + t/4 (k, h < 2) and the column pairs 8j + 2 (t % 4)
+            // (j < 4), so it reads 4 float2 of each constant, not 8 float4.
+            static_assert(CW == 32, "32-column chunks");
+            constexpr uint32_t kLanes16 = 16u << 16;
+            uint32_t pl[16], ph[16], ml[POL == 2 ? 16 : 1], mh[POL == 2 ? 16 : 1];
+            tmem_ld_16x256b_x4(t_plus + c * 32, pl);
+            tmem_ld_16x256b_x4(t_plus + c * 32 + kLanes16, ph);
+            if constexpr (POL == 2) {
+              tmem_ld_16x256b_x4(t_plus + BN + c * 32, ml);
+              tmem_ld_16x256b_x4(t_plus + BN + c * 32 + kLanes16, mh);
+            }
+            tmem_ld_wait();
+            const int q = lane & 3;
+            const float *cpc = cst + c * 32 + 2 * q;
+            const float *cmc = cst + HALF + c * 32 + 2 * q;
+            const float *bc = cst + POL * HALF + c * 32 + 2 * q;
+            const uint64_t zero2 = f2pack(0.0f, 0.0f), one2 = f2pack(1.0f, 1.0f);
+            if constexpr (TMA_STORE) {
+              if (lane == 0) bulk_wait_read_all();  // the previous chunk is out
+              __syncwarp();
+            }
 #pragma unroll
-              for (int q = 0; q < CW / 4; ++q) {
-                const float4 w = sw4[q], b = b4[q];
+            for (int j = 0; j < 4; ++j) {
+              const uint64_t cp = *reinterpret_cast<const uint64_t *>(cpc + 8 * j);
+              const uint64_t b = *reinterpret_cast<const uint64_t *>(bc + 8 * j);
+              uint64_t cm = 0;
+              if constexpr (POL == 2) cm = *reinterpret_cast<const uint64_t *>(cmc + 8 * j);
+#pragma unroll
+              for (int k = 0; k < 2; ++k)
 #pragma unroll
                 for (int h = 0; h < 2; ++h) {
-                  const int j = 4 * q + 2 * h;
-                  const uint64_t w2 = h ? f2pack(w.z, w.w) : f2pack(w.x, w.y);
-                  const uint64_t fp = f2pack(acc_f32<F8>(ap[j]), acc_f32<F8>(ap[j + 1]));
-                  uint64_t y = ffma2(ffma2(w2, sp2, zero2), fp, zero2);
+                  const int r = 4 * j + 2 * h;
+                  const uint32_t a0 = k ? ph[r] : pl[r], a1 = k ? ph[r + 1] : pl[r + 1];
+                  uint64_t y = ffma2(cp, f2pack(acc_f32<F8>(a0), acc_f32<F8>(a1)), zero2);
                   if constexpr (POL == 2) {
-                    const uint64_t fm = f2pack(acc_f32<F8>(am[j]), acc_f32<F8>(am[j + 1]));
-                    y = ffma2(ffma2(w2, sm2, zero2), fm, y);
+                    const uint32_t b0 = k ? mh[r] : ml[r], b1 = k ? mh[r + 1] : ml[r + 1];
+                    y = ffma2(cm, f2pack(acc_f32<F8>(b0), acc_f32<F8>(b1)), y);
                   }
-                  y = ffma2(one2, y, h ? f2pack(b.z, b.w) : f2pack(b.x, b.y));
-                  f2unpack(y, v[j], v[j + 1]);
+                  y = ffma2(one2, y, b);
+                  float y0, y1;
+                  f2unpack(y, y0, y1);
+                  const int rr = 16 * k + 8 * h + (lane >> 2);  // row within the warp's 32
+                  if constexpr (TMA_STORE) {
+                    // Staging buffer in the tensor map's 64-byte swizzle:
+                    // 16-byte piece j of row rr sits at piece j ^ ((rr / 2) % 4),
+                    // so the 8 rows x 16 bytes of one store instruction fall
+                    // into 8 distinct bank groups.
+                    *reinterpret_cast<uint32_t *>(stg + rr * 64 + ((j ^ ((rr >> 1) & 3)) << 4) +
+                                                  4 * q) = pack_bf16x2(y0, y1);
+                  } else {
+                    const int64_t mr = static_cast<int64_t>(mt) * BM + quarter * 32 + rr;
+                    if (mr < p.M) store_pair<OUT>(p, mr, n0 + 8 * j + 2 * q, y0, y1);
+                  }
                 }
-              }
-              if constexpr (TMA_STORE) {
-                // The warp's 32 rows x 32 columns go to its staging buffer (one
-                // 64-byte row per lane) and leave in one tensor store, which
-                // writes whole lines and drops rows >= M and columns >= N.  The
-                // buffer uses the tensor map's 64-byte swizzle: 16-byte piece q
-                // of row r sits at piece q ^ ((r / 2) % 4), so each group of 8
-                // lanes stores to 8 distinct bank groups.
-                static_assert(CW == 32, "tensor-store chunk is 32 x 32");
-                if (lane == 0) bulk_wait_read_all();  // the previous chunk is out
-                __syncwarp();
-                uint4 *dst = reinterpret_cast<uint4 *>(stg + lane * 64);
-                const int swz = (lane >> 1) & 3;
-#pragma unroll
-                for (int q = 0; q < 4; ++q)
-                  dst[q ^ swz] = make_uint4(pack_bf16x2(v[8 * q + 0], v[8 * q + 1]),
-                                      pack_bf16x2(v[8 * q + 2], v[8 * q + 3]),
-                                      pack_bf16x2(v[8 * q + 4], v[8 * q + 5]),
-                                      pack_bf16x2(v[8 * q + 6], v[8 * q + 7]));
-                fence_proxy_async_smem();
-                __syncwarp();
-                const int row0 = mt * BM + quarter * 32;
-                if (lane == 0 && row0 < p.M && n0 < p.N) {
-                  tma_store_2d(&tmY, stg, static_cast<int32_t>(n0), row0);
-                  bulk_commit_group();
-                }
-              } else {
-                store_row_chunk<OUT, CW>(p, m, n0, v);
+            }
+            if constexpr (TMA_STORE) {
+              // The warp's 32 rows x 32 columns leave in one tensor store,
+              // which writes whole lines and drops rows >= M and columns >= N.
+              fence_proxy_async_smem();
+              __syncwarp();
+              const int row0 = mt * BM + quarter * 32;
+              if (lane == 0 && row0 < p.M && n0 < p.N) {
+                tma_store_2d(&tmY, stg, static_cast<int32_t>(n0), row0);
+                bulk_commit_group();
               }
             }
           }
