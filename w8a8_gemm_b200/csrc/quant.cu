@@ -178,18 +178,29 @@ __device__ __forceinline__ void dualscale8_fp8(const float (&x)[8], const float 
 // memory; every warp then takes whole rows of the staged tile (lane = 8
 // channels, one conflict-free 16-byte shared load) and writes 8 bytes per plane
 // per row, 256 contiguous bytes per warp.
-// FP8 keeps m+ and m- unscaled in p7 and n7.
-template <bool FP8>
-__device__ __forceinline__ void load_multipliers(int g, int64_t c0, int64_t K, const float *d,
-                                                 const float *s_act, const SegParams &seg,
-                                                 float (&p7)[8], float (&n7)[8]) {
+// FP8 keeps m+ and m- unscaled in p7 and n7.  fetch_scales reads the inputs
+// of one (group, column block) into registers (s+, s- in sc[0..1], the eight
+// divisors in p7) and fold_multipliers turns them into the multipliers, so
+// that the reads can be issued ahead of the first tile copies.
+__device__ __forceinline__ void fetch_scales(int g, int64_t c0, int64_t K, const float *d,
+                                             const float *s_act, const SegParams &seg,
+                                             float (&sc)[2], float (&p7)[8]) {
   if (c0 >= K) return;
   const int i = (seg.mode == SQ_SEG_INPUT) ? seg_index(seg.off, seg.n_seg, c0) : 0;
-  const float sp = s_act[(g * seg.S + i) * 2 + 0], sm = s_act[(g * seg.S + i) * 2 + 1];
+  sc[0] = s_act[(g * seg.S + i) * 2 + 0];
+  sc[1] = s_act[(g * seg.S + i) * 2 + 1];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) p7[j] = d ? d[g * K + c0 + j] : 1.0f;
+}
+template <bool FP8>
+__device__ __forceinline__ void fold_multipliers(int64_t c0, int64_t K, const float (&sc)[2],
+                                                 float (&p7)[8], float (&n7)[8]) {
+  if (c0 >= K) return;
 #pragma unroll
   for (int j = 0; j < 8; ++j) {
-    const float dv = d ? d[g * K + c0 + j] : 1.0f;
-    const float mp = __fdiv_rn(1.0f, __fmul_rn(dv, sp)), mm = __fdiv_rn(1.0f, __fmul_rn(dv, sm));
+    const float dv = p7[j];
+    const float mp = __fdiv_rn(1.0f, __fmul_rn(dv, sc[0]));
+    const float mm = __fdiv_rn(1.0f, __fmul_rn(dv, sc[1]));
     p7[j] = FP8 ? mp : mp * 0.0078125f;
     n7[j] = FP8 ? mm : mm * -0.0078125f;
   }
@@ -241,6 +252,14 @@ __global__ void __launch_bounds__(256, 3) quant_act_kernel(const __grid_constant
     prefetch_tmap(&tmX);
   }
   grid_dependency_wait();  // nothing above touches global memory
+  // The first unit's scales are requested before the tile copies, so that
+  // these small reads do not queue behind the whole grid's tile traffic.
+  UnitCursor cur;
+  cur.set(u_begin, n_cb, n_rt);
+  float sc[2], p7[8], n7[8];
+  if (n_mine > 0)
+    fetch_scales(cur.g, static_cast<int64_t>(cur.cb) * kWarpCols + lane * kColsPerThread, K, d,
+                 s_act, seg, sc, p7);
   if (tid == 0) {
     fetch.set(u_begin, n_cb, n_rt);
     for (int st = 0; st < kQStages && st < n_mine; ++st) {
@@ -251,17 +270,18 @@ __global__ void __launch_bounds__(256, 3) quant_act_kernel(const __grid_constant
     }
   }
   __syncthreads();  // barriers initialised
-  UnitCursor cur;
-  cur.set(u_begin, n_cb, n_rt);
-  float p7[8], n7[8];
-  int key_g = -1, key_cb = -1;  // (group, column block) of the multipliers held
+  if (n_mine > 0)
+    fold_multipliers<FP8>(static_cast<int64_t>(cur.cb) * kWarpCols + lane * kColsPerThread, K, sc,
+                          p7, n7);
+  int key_g = cur.g, key_cb = cur.cb;  // (group, column block) of the multipliers held
   const int64_t plane_stride = M * K;
   for (int it = 0; it < n_mine; ++it, cur.next(n_cb, n_rt)) {
     const int64_t c0 = static_cast<int64_t>(cur.cb) * kWarpCols + lane * kColsPerThread;
     if (cur.g != key_g || cur.cb != key_cb) {
       key_g = cur.g;
       key_cb = cur.cb;
-      load_multipliers<FP8>(cur.g, c0, K, d, s_act, seg, p7, n7);
+      fetch_scales(cur.g, c0, K, d, s_act, seg, sc, p7);
+      fold_multipliers<FP8>(c0, K, sc, p7, n7);
     }
     const int st = it % kQStages;
     if (!mbar_wait(&full[st], (it / kQStages) & 1, kQuantWaitNs)) {
