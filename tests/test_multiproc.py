@@ -56,3 +56,18 @@ def test_two_rank_max_over_ranks():
 def test_single_process_aggregate_is_identity():
     import bench
     assert bench.aggregate_over_ranks(3.5) == 3.5
+
+
+def test_reference_arm_other_ranks_exit_without_work(capsys, monkeypatch):
+    """Under torchrun the reference arm (the CPU oracle) runs on rank 0 only:
+    every other rank returns 0 at once and prints nothing, without loading the
+    oracle."""
+    import argparse
+    import sys
+
+    import bench
+    monkeypatch.delitem(sys.modules, "oracle", raising=False)
+    args = argparse.Namespace(config="c1_tiny_dualscale", steps=1, warmup=0, gpus=2)
+    assert bench.main_reference(args, 2, 1) == 0
+    assert capsys.readouterr().out == ""
+    assert "oracle" not in sys.modules
