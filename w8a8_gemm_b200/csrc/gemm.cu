@@ -9,16 +9,19 @@
 // share every weight tile staged in shared memory and accumulate side by side
 // in tensor memory, so the X^- product never reaches HBM.
 //
-// Structure (one persistent CTA per SM, 320 threads):
+// Structure (one persistent CTA per SM; 320 threads, 576 for input-segmented
+// layers):
 //   warp 0      TMA producer: per 128-byte k-block, one 3D box {128 B, 128
 //               rows, 2 planes} of [X^+; X^-] and one box {128 B, BN rows} of
 //               W^, into a STAGES-deep ring guarded by mbarriers;
 //   warp 1      TMEM owner and MMA issuer (one thread): tcgen05.mma kind::i8,
 //               M = 128, N = BN, K = 32, two per k-step (X^+ and X^-);
-//   warps 2-9   epilogue: tcgen05.ld of both accumulators, fp32 reconstruction,
-//               bias, bf16/fp32 stores.  Input-segmented layers drain one
-//               accumulator pair per K-segment into fp32 running sums held in
-//               registers while the MMA warp fills the other TMEM buffer.
+//   warps 2-    epilogue (8 warps, 16 for input-segmented layers): tcgen05.ld
+//               of both accumulators in the 16x256b pattern, fp32
+//               reconstruction, bias, bf16/fp32 stores.  Input-segmented
+//               layers drain one accumulator pair per K-segment into fp32
+//               running sums held in registers while the MMA warp fills the
+//               other TMEM buffer.
 // TMEM holds 512 columns: BN = 256 gives one buffer (+ and - of 256 columns);
 // BN = 128 gives two, so drains overlap the next segment's MMAs.
 #include <cuda.h>
@@ -193,8 +196,8 @@ __global__ void __launch_bounds__(threads_for(EPI_WARPS), 1)
   constexpr int NBUF = L::NBUF;
   constexpr int ACC_COLS = POL * BN;  // TMEM columns of one accumulator buffer
   constexpr int HALF = L::COLS;      // columns per epilogue warp
-  // TMEM chunk of the one-segment epilogue: 32 columns with 8 warps, 16 with
-  // more warps (their register budget is smaller).
+  // Column chunk of the one-segment epilogue (32) and of the raw-accumulator
+  // output: 32 columns with 8 warps, 16 with 16 (a smaller register budget).
   constexpr int CW = EPI_WARPS >= 16 ? 16 : 32;
   static_assert(EPI_WARPS % 4 == 0 && HALF % 32 == 0, "epilogue split");
   static_assert(NBUF >= 1, "BN too large for TMEM");
@@ -340,9 +343,10 @@ __global__ void __launch_bounds__(threads_for(EPI_WARPS), 1)
     const int half = ew >> 2;           // which column part of the tile
     const int row = quarter * 32 + lane;
     const uint32_t lane_addr = static_cast<uint32_t>(quarter * 32) << 16;
-    // Warp-private column constants in shared memory, read back as broadcast
-    // float4s: s_w and bias, [HALF] floats each (with several K-segments two
-    // buffers of c+ = fl(s_w s+) and c- = fl(s_w s-)).
+    // Warp-private column constants in shared memory, read back as float2
+    // pairs: with one K-segment c+ = fl(s_w s+), c- = fl(s_w s-) and the bias,
+    // [HALF] floats each; with several, two buffers of c+ and c- (the bias
+    // goes, at the end of a tile, into the buffer the last segment did not use).
     float *cst_base = reinterpret_cast<float *>(smem + L::EPI_OFFSET) + ew * L::CONST_FLOATS;
     uint8_t *stg = smem + L::STG_OFFSET + ew * 2048;  // used when TMA_STORE
     uint32_t acc_iter = 0;
@@ -387,17 +391,13 @@ __global__ void __launch_bounds__(threads_for(EPI_WARPS), 1)
       }
       const int units = SEGK ? p.S : 1;
       for (int u = 0; u < units; ++u) {
-        const float sp = __fmul_rn((SEGK && OUT != OUT_S32) ? sp_next
-                                                            : p.s_act[(g * p.S + u) * 2 + 0],
-                                   p.act_mul);
-        const float sm = __fmul_rn((SEGK && OUT != OUT_S32) ? sm_next
-                                                            : p.s_act[(g * p.S + u) * 2 + 1],
-                                   p.act_mul);
         float *cst = cst_base;
         if constexpr (SEGK && OUT != OUT_S32) {
           // Folded coefficients of K-segment u: c+- = s_w[u][n] * s+-[u], into
           // buffer u & 1 (the other buffer may still be read by segment u - 1
           // only in program order of this warp, so no wait is needed).
+          const float sp = __fmul_rn(sp_next, p.act_mul);
+          const float sm = __fmul_rn(sm_next, p.act_mul);
           cst = cst_base + (u & 1) * 2 * HALF;
 #pragma unroll
           for (int q = 0; q < HALF / 32; ++q) {
