@@ -580,7 +580,8 @@ __global__ void __launch_bounds__(threads_for(EPI_WARPS), 1)
         for (int k = 0; k < 2; ++k)
 #pragma unroll
           for (int h = 0; h < 2; ++h) {
-            const int64_t mr = static_cast<int64_t>(mt) * BM + quarter * 32 + 16 * k + 8 * h + (lane >> 2);
+            const int64_t mr =
+                static_cast<int64_t>(mt) * BM + quarter * 32 + 16 * k + 8 * h + (lane >> 2);
             float y[8];  // pairs j = 0..3
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
@@ -616,7 +617,8 @@ __global__ void __launch_bounds__(threads_for(EPI_WARPS), 1)
                 } else {
 #pragma unroll
                   for (int e = 0; e < 8; ++e)
-                    if (n0 + e < p.N) row[n0 + e] = static_cast<uint16_t>(w[e >> 1] >> (16 * (e & 1)));
+                    if (n0 + e < p.N)
+                      row[n0 + e] = static_cast<uint16_t>(w[e >> 1] >> (16 * (e & 1)));
                 }
               }
             } else if (mr < p.M) {
