@@ -18,6 +18,7 @@ LAYERS = {
     "none_tails": lambda: wl.gelu_layer("none", 300, 416, 520, seed=41, bias=True),
     "none_ragged": lambda: wl.gelu_layer("rag", 5, 48, 13, seed=42, bias=True),
     "input_heads": lambda: wl.outproj_layer("heads", 300, 448, 264, 64, seed=43),
+    "input_odd_n": lambda: wl.outproj_layer("oddn", 150, 256, 261, 64, seed=45),
     "output_groups": lambda: wl.adanorm_layer("og", 130, 256, 768, 3, seed=44, G=3),
 }
 

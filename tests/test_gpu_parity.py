@@ -35,6 +35,8 @@ SMALL = {
     "input_heads": lambda: wl.outproj_layer("heads", 300, 448, 264, 64, seed=5),
     "input_mixed": _input_layer_mixed,
     "input_wide": lambda: wl.outproj_layer("wide", 130, 1024, 136, 512, seed=6),
+    # N = 261: the last 8-column store of a row crosses N (element-wise tail)
+    "input_odd_n": lambda: wl.outproj_layer("oddn", 150, 256, 261, 64, seed=14),
     # the most segments a table may hold (SQ_MAX_SEGMENTS = 64)
     "input_max_segments": lambda: wl.outproj_layer("maxin", 130, 2048, 136, 32, seed=12),
     "output_max_segments": lambda: wl.adanorm_layer("maxout", 130, 256, 64 * 9, 64, seed=13, G=1),

@@ -16,6 +16,7 @@ LAYERS = {
     "none_tails": lambda: wl.gelu_layer("none", 300, 416, 520, seed=1, bias=True),
     "none_ragged": lambda: wl.gelu_layer("rag", 5, 48, 13, seed=3, bias=True),
     "input_heads": lambda: wl.outproj_layer("heads", 300, 448, 264, 64, seed=5),
+    "input_odd_n": lambda: wl.outproj_layer("oddn", 150, 256, 261, 64, seed=15),
     "output_g3": lambda: wl.adanorm_layer("o3", 200, 256, 768, 3, seed=8, G=3),
     "output_g2_bn128": lambda: wl.adanorm_layer("o2", 130, 128, 256, 2, seed=9, G=2),
 }

@@ -17,6 +17,7 @@ LAYERS = {
     "none_tails": lambda: wl.gelu_layer("none", 300, 416, 520, seed=21, bias=True),
     "none_ragged": lambda: wl.gelu_layer("rag", 5, 48, 13, seed=22, bias=True),
     "input_heads": lambda: wl.outproj_layer("heads", 300, 448, 264, 64, seed=23),
+    "input_odd_n": lambda: wl.outproj_layer("oddn", 150, 256, 261, 64, seed=26),
     "output_g1": lambda: wl.adanorm_layer("o1", 200, 256, 768, 3, seed=24, G=1),
     "output_groups": lambda: wl.adanorm_layer("og", 130, 256, 768, 3, seed=25, G=3),
 }
