@@ -277,7 +277,8 @@ SQ_API sq_status sq_debug_gemm_s32(const int8_t *planes, const int8_t *wq, int64
  *
  * sq_host_pipeline_workspace_bytes -- workspace size for layers with K <= max_K,
  * N <= max_N, G <= max_G and P <= max_P (P = 2 for DualScale, 1 single scale);
- * 0 for invalid sizes.
+ * 0 for invalid sizes, including chunk_rows * max_K or chunk_rows * max_N above
+ * 2^44 elements.
  *
  * sq_host_pipeline_create -- chunk_rows >= 1; workspace: device memory of at
  * least sq_host_pipeline_workspace_bytes(...) bytes, 256-byte aligned, owned by
@@ -286,6 +287,9 @@ SQ_API sq_status sq_debug_gemm_s32(const int8_t *planes, const int8_t *wq, int64
  *
  * sq_host_pipeline_destroy -- waits for the pipeline's work, then releases its
  * streams and events (not the workspace).  NULL is a no-op.
+ *
+ * If sq_dualscale_seglinear_host fails after it has enqueued work, it waits for
+ * the pipeline's streams before returning the error.
  *
  * sq_dualscale_seglinear_host -- arguments as in sq_quantize_act and
  * sq_dualscale_seglinear_gemm, except that x_host (bf16 [M][ldx]) and y_host

@@ -183,6 +183,9 @@ def test_host_pipeline_validates_on_host(L):
     assert L.sq_host_pipeline_workspace_bytes(0, 64, 64, 1, 2) == 0
     assert L.sq_host_pipeline_workspace_bytes(128, 24, 64, 1, 2) == 0      # K % 16 != 0
     assert L.sq_host_pipeline_workspace_bytes(128, 64, 64, 1, 3) == 0      # P must be 1 or 2
+    # sizes whose byte counts would not fit 64 bits are rejected, not wrapped
+    assert L.sq_host_pipeline_workspace_bytes(2**31 - 1, 2**31 - 16, 2**31 - 1, 64, 2) == 0
+    assert L.sq_host_pipeline_workspace_bytes(2**31 - 1, 2**20, 64, 1, 2) == 0
     need = L.sq_host_pipeline_workspace_bytes(128, 64, 64, 1, 2)
     # two slots of x (128*64*2) + planes (2*128*64) + y (128*64*4), 256-byte rounded
     assert need == 2 * (16384 + 16384 + 32768)

@@ -34,6 +34,9 @@ bool slot_layout(int64_t chunk, int64_t K, int64_t N, int32_t G, int32_t P, size
       N > INT32_MAX || G < 1 || G > SQ_MAX_SEGMENTS || P < 1 || P > 2)
     return false;
   const int64_t n_pad = (N + 7) / 8 * 8;  // output rows 16-byte aligned for bf16 and fp32
+  // Every product below then stays far inside 64 bits.
+  constexpr int64_t kMaxElems = int64_t(1) << 44;
+  if (chunk > kMaxElems / K || chunk > kMaxElems / n_pad) return false;
   const size_t x_bytes = static_cast<size_t>(chunk) * K * 2;
   const size_t planes_bytes = static_cast<size_t>(G) * P * chunk * K;
   const size_t y_bytes = static_cast<size_t>(chunk) * n_pad * 4;
@@ -157,7 +160,17 @@ sq_status sq_dualscale_seglinear_host(sq_host_pipeline *pl, const void *x_host, 
   }
   cudaStream_t user = reinterpret_cast<cudaStream_t>(stream);
   auto cu = [](cudaError_t e) { return e == cudaSuccess; };
-  if (!cu(cudaEventRecord(pl->ev_start, user)) || !cu(cudaStreamWaitEvent(pl->s_in, pl->ev_start, 0)) ||
+  // After a failure past the first enqueue, wait for the pipeline's streams
+  // before returning, so that no copy or kernel of this call is still in
+  // flight when the caller sees the error.
+  auto fail = [pl](sq_status st) {
+    cudaStreamSynchronize(pl->s_in);
+    cudaStreamSynchronize(pl->s_comp);
+    cudaStreamSynchronize(pl->s_out);
+    return st;
+  };
+  if (!cu(cudaEventRecord(pl->ev_start, user)) ||
+      !cu(cudaStreamWaitEvent(pl->s_in, pl->ev_start, 0)) ||
       !cu(cudaStreamWaitEvent(pl->s_comp, pl->ev_start, 0)) ||
       !cu(cudaStreamWaitEvent(pl->s_out, pl->ev_start, 0)))
     return SQ_ERR_CUDA;
@@ -172,28 +185,29 @@ sq_status sq_dualscale_seglinear_host(sq_host_pipeline *pl, const void *x_host, 
     uint8_t *y_dev = pl->slot[s] + pl->y_off;
     // The slot's previous chunk (c - 2) must have been quantized before its
     // rows are overwritten, and copied out before its planes and output are.
-    if (c >= 2 && !cu(cudaStreamWaitEvent(pl->s_in, pl->ev_comp[s], 0))) return SQ_ERR_CUDA;
+    if (c >= 2 && !cu(cudaStreamWaitEvent(pl->s_in, pl->ev_comp[s], 0))) return fail(SQ_ERR_CUDA);
     if (!cu(cudaMemcpy2DAsync(x_dev, K * 2, static_cast<const uint8_t *>(x_host) + r0 * ldx * 2,
                               ldx * 2, K * 2, rows, cudaMemcpyHostToDevice, pl->s_in)) ||
         !cu(cudaEventRecord(pl->ev_in[s], pl->s_in)) ||
         !cu(cudaStreamWaitEvent(pl->s_comp, pl->ev_in[s], 0)))
-      return SQ_ERR_CUDA;
-    if (c >= 2 && !cu(cudaStreamWaitEvent(pl->s_comp, pl->ev_out[s], 0))) return SQ_ERR_CUDA;
+      return fail(SQ_ERR_CUDA);
+    if (c >= 2 && !cu(cudaStreamWaitEvent(pl->s_comp, pl->ev_out[s], 0))) return fail(SQ_ERR_CUDA);
     sq_stream_t comp = reinterpret_cast<sq_stream_t>(pl->s_comp);
     sq_status st = sq_quantize_act(x_dev, rows, K, K, d, s_act, seg, planes_dev, comp);
-    if (st != SQ_OK) return st;
+    if (st != SQ_OK) return fail(st);
     st = sq_dualscale_seglinear_gemm(planes_dev, wq, s_w, s_act, bias, y_dev, out_dtype, rows, N,
                                      K, n_pad, seg, comp);
-    if (st != SQ_OK) return st;
+    if (st != SQ_OK) return fail(st);
     if (!cu(cudaEventRecord(pl->ev_comp[s], pl->s_comp)) ||
         !cu(cudaStreamWaitEvent(pl->s_out, pl->ev_comp[s], 0)) ||
         !cu(cudaMemcpy2DAsync(static_cast<uint8_t *>(y_host) + r0 * ldy * elem, ldy * elem, y_dev,
                               n_pad * elem, N * elem, rows, cudaMemcpyDeviceToHost, pl->s_out)) ||
         !cu(cudaEventRecord(pl->ev_out[s], pl->s_out)))
-      return SQ_ERR_CUDA;
+      return fail(SQ_ERR_CUDA);
   }
-  if (!cu(cudaEventRecord(pl->ev_done, pl->s_out)) || !cu(cudaStreamWaitEvent(user, pl->ev_done, 0)))
-    return SQ_ERR_CUDA;
+  if (!cu(cudaEventRecord(pl->ev_done, pl->s_out)) ||
+      !cu(cudaStreamWaitEvent(user, pl->ev_done, 0)))
+    return fail(SQ_ERR_CUDA);
   return SQ_OK;
 }
 
