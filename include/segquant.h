@@ -238,7 +238,7 @@ SQ_API sq_status sq_unpack_weight_w4(const uint8_t *wq4, int64_t N, int64_t K, i
  *   s_w fp32 [S][N]; s_act fp32 [G][S][2]; bias bf16 [N] or NULL
  *   y      bf16 or fp32 [M][ldy] output, ldy >= N, ldy*elem % 16 == 0,
  *          16-byte aligned
- *   K % 16 == 0, K >= 16; N >= 1; M == 0 is a valid no-op.
+ *   K % 16 == 0, K >= 16; N >= 1; M * N <= 2^44; M == 0 is a valid no-op.
  * With SQ_FLAG_W4, wq is the output of sq_unpack_weight_w4 (16 q) and the
  * result is that of the codes q (see SQ_FLAG_W4).
  * Returns SQ_ERR_OVERFLOW when a K-segment is wider than 132104.

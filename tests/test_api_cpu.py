@@ -135,6 +135,11 @@ def test_gemm_overflow_and_layout_checks(L):
     # ldy < N
     assert L.sq_dualscale_seglinear_gemm(p(FAKE), p(FAKE), p(FAKE), p(FAKE), None, p(FAKE), 0,
                                          8, 16, 64, 8, ctypes.byref(c), None) == SQ_ERR_INVALID_ARG
+    # an output of more than 2^44 elements (M, N each within int32)
+    big = 2**31 - 1
+    assert L.sq_dualscale_seglinear_gemm(p(FAKE), p(FAKE), p(FAKE), p(FAKE), None, p(FAKE), 0,
+                                         big, big, 64, big + 1, ctypes.byref(c),
+                                         None) == SQ_ERR_INVALID_ARG
     # bf16 output rows must start 16-byte aligned (ldy multiple of 8)
     assert L.sq_dualscale_seglinear_gemm(p(FAKE), p(FAKE), p(FAKE), p(FAKE), None, p(FAKE), 0,
                                          8, 20, 64, 20, ctypes.byref(c), None) == SQ_ERR_ALIGNMENT

@@ -129,6 +129,9 @@ sq_status gemm_common(const int8_t *planes, const int8_t *wq, const float *s_w,
                       int64_t N, int64_t K, int64_t ldy, const sq_segments *seg,
                       cudaStream_t stream, bool launch = true) {
   if (M < 0 || M > INT32_MAX || N < 1 || N > INT32_MAX) return SQ_ERR_INVALID_ARG;
+  // An output of more than 2^44 elements fits no device; the bound keeps the
+  // kernel's tile count (at most 2^30 tiles of 128 x 128) inside int32.
+  if (M * N > (int64_t(1) << 44)) return SQ_ERR_INVALID_ARG;
   SQ_TRY(check_k(K));
   SegParams sp;
   SQ_TRY(parse_segments(seg, K, N, &sp));
