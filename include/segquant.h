@@ -147,7 +147,7 @@ typedef struct {
  * lo = min(0, min u); s+ = hi/127 (1 if hi == 0), s- = -lo/128 (1 if lo == 0).
  * NaN inputs are ignored.
  *   x      bf16 [M][ldx]; M >= 1, K >= 16, K % 16 == 0, ldx >= K, ldx % 8 == 0,
- *          x 16-byte aligned
+ *          M * ldx <= 2^44, x 16-byte aligned
  *   d      fp32 [G][K] divisor (> 0, finite) or NULL for d = 1
  *   s_act  fp32 [G][S][2] output, {s+, s-} per group and K-segment
  * With SQ_FLAG_SINGLE_SCALE: s+ = s- = max(hi, -lo)/127 (1 if both are 0).

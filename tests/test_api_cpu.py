@@ -70,6 +70,11 @@ def test_quantize_act_rejects_bad_shapes(L):
     # ldx not a multiple of 8 elements
     assert L.sq_quantize_act(p(FAKE), 4, 32, 36, None, p(FAKE), ctypes.byref(c), p(FAKE),
                              None) == SQ_ERR_ALIGNMENT
+    # an input of more than 2^44 elements (including a huge row stride)
+    assert L.sq_quantize_act(p(FAKE), 2**31 - 1, 2**20, 2**20, None, p(FAKE), ctypes.byref(c),
+                             p(FAKE), None) == SQ_ERR_INVALID_ARG
+    assert L.sq_quantize_act(p(FAKE), 2**20, 32, 2**62, None, p(FAKE), ctypes.byref(c), p(FAKE),
+                             None) == SQ_ERR_INVALID_ARG
 
 
 def test_segment_table_validation(L):

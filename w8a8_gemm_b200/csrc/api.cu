@@ -111,6 +111,9 @@ sq_status check_act(const void *x, int64_t M, int64_t K, int64_t ldx) {
   sq_status st = check_k(K);
   if (st != SQ_OK) return st;
   if (ldx < K) return SQ_ERR_INVALID_ARG;
+  // More than 2^44 input elements fit no device; the bound keeps the
+  // quantizer's work-unit arithmetic far inside int64.
+  if (M > 0 && ldx > (int64_t(1) << 44) / M) return SQ_ERR_INVALID_ARG;
   if (M > 0 && x == nullptr) return SQ_ERR_INVALID_ARG;
   if (ldx % 8 != 0 || !aligned(x, 16)) return SQ_ERR_ALIGNMENT;
   return SQ_OK;
