@@ -49,6 +49,7 @@ METRIC = "DualScale-SegLinear W8A8 GEMM effective TOPS & % of B200 INT8 peak; qu
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 INT8_OVER_BF16 = 4.5 / 2.25   # dense INT8 / dense bf16, nominal B200 ratio
 E2E_CHUNK_ROWS = 2048          # rows per chunk of the host entry point (e2e leg)
+REF_BUDGET_S = 120.0           # CPU seconds of the whole reference-arm run (oracle)
 FLUSH_BYTES = 512 << 20       # written between steps (4x the 126 MB L2) ...
 SWEEP_BYTES = 256 << 20       # ... then a second buffer is read, so the L2 holds clean lines
 SMI_FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
@@ -536,10 +537,9 @@ def main_reference(args, ws, rank):
     layers = wl.config_layers(args.config, seed=0)
     thr = oracle.num_threads()
     prepared = prepare_oracle(layers)
-    total_budget_s = 120.0
     probe = oracle_sample(layers, 1.0, thr, prepared)
     per_row_s = probe["seconds"] / probe["rows"]
-    rows = max(1, int(total_budget_s / (args.steps + args.warmup) / per_row_s))
+    rows = max(1, int(REF_BUDGET_S / (args.steps + args.warmup) / per_row_s))
     rows = min(rows, min(L.M for L in layers))
 
     def step():
