@@ -49,6 +49,8 @@ def lib():
         L.orc_quantize_weight_fp8.argtypes = [p, i64, i64, p, i32, i32, p, i32, p, p]
         L.orc_gemm_fp8_acc.argtypes = [p, p, i64, i64, i64, i32, i32, p, i32, i32, p, i64, p,
                                        i32]
+        L.orc_gelu_bf16.argtypes = [p, i64, p]
+        L.orc_gelu_parts.argtypes = [p, i64, p, p, p, p]
         L.orc_gemm_fp8.argtypes = [p, p, p, p, p, i64, i64, i64, i32, i32, p, i32, i32, p, i64,
                                    p, i32]
         for f in (L.orc_calibrate_act, L.orc_quantize_act, L.orc_quantize_weight,
@@ -302,7 +304,29 @@ def layer_fp8(x_bits, w_bits, x_cal_bits, d=None, bias_bits=None, mode=MODE_NONE
     return dict(s_act=s_act, planes=planes, wq=wq, s_w=s_w, y=y)
 
 
+def gelu_bf16(y):
+    """bf16(gelu(bf16(y))) of fp32 values, as bf16 bit patterns (uint16): the
+    FFN activation between fc1 and fc2, tanh approximation, for the fused
+    producer."""
+    y = _c(y, np.float32)
+    out = np.empty(y.shape, np.uint16)
+    _check(lib().orc_gelu_bf16(_ptr(y), y.size, _ptr(out)), "gelu_bf16")
+    return out
+
+
+def gelu_parts(x):
+    """The pieces of gelu_bf16 on fp32 inputs: e^x (for 0 <= x <= 18), tanh,
+    gelu, and bf16 rounding (bit patterns)."""
+    x = _c(x, np.float32)
+    e, t, g = (np.empty(x.shape, np.float32) for _ in range(3))
+    b = np.empty(x.shape, np.uint16)
+    _check(lib().orc_gelu_parts(_ptr(x), x.size, _ptr(e), _ptr(t), _ptr(g), _ptr(b)),
+           "gelu_parts")
+    return dict(exp=e, tanh=t, gelu=g, bf16=b)
+
+
 __all__ = ["MODE_NONE", "MODE_OUTPUT", "MODE_INPUT", "calibrate_act",
            "quantize_act", "quantize_weight", "pack_w4", "gemm_s32", "gemm", "layer",
            "num_threads", "lib", "e4m3_encode", "e4m3_decode", "calibrate_act_fp8",
-           "quantize_act_fp8", "quantize_weight_fp8", "gemm_fp8_acc", "gemm_fp8", "layer_fp8"]
+           "quantize_act_fp8", "quantize_weight_fp8", "gemm_fp8_acc", "gemm_fp8", "layer_fp8",
+           "gelu_bf16", "gelu_parts"]

@@ -597,3 +597,86 @@ int orc_gemm_fp8(const uint8_t *planes, const uint8_t *wq, const float *s_w,
   free(acc);
   return 0;
 }
+
+
+/* ------------------------------------------------------------------------
+ * FFN activation between the two linears (the input of fc2 is GELU of fc1's
+ * output; "SegQuant" papernotes.org, section DualScale, polarity table row
+ * "FFN (DiT)"), for the fused producer.  The pages name the activation but
+ * give no formula; the models' FFNs use the tanh approximation
+ *   gelu(x) = x/2 * (1 + tanh(sqrt(2/pi) * (x + 0.044715 x^3))).
+ * It is written out here as a fixed sequence of fp32 operations, each rounded
+ * once (this file is built with -ffp-contract=off), so that a GPU running the
+ * same sequence gets the same bits:
+ *   tanh(u) = 1 - 2 / (e^(2|u|) + 1), sign of u; 1 for |u| >= 9 (the fp32
+ *             value of tanh there is 1);
+ *   e^z     (0 <= z <= 18): z = n ln2 + f with n = rint(z / ln2), |f| <= ln2/2
+ *             (Cody and Waite's reduction, ln2 split into a head exact in
+ *             n * head and a tail), e^f by its Taylor series to degree 7
+ *             (remainder below 2^-27), times 2^n (exact).
+ * The values are rounded to bf16 before and after (the models' activation
+ * type), round half to even.
+ * ------------------------------------------------------------------------ */
+static uint16_t orc_bf16_rne(float v) {
+  uint32_t u;
+  memcpy(&u, &v, sizeof u);
+  if ((u & 0x7fffffffu) > 0x7f800000u) return (uint16_t)((u >> 16) | 0x40u);  /* NaN stays NaN */
+  u += 0x7fffu + ((u >> 16) & 1u);
+  return (uint16_t)(u >> 16);
+}
+
+static float orc_exp_0_18(float z) {
+  const float inv_ln2 = 0x1.715476p+0f;   /* fp32(1/ln 2) */
+  const float ln2_hi = 0x1.62e4p-1f;      /* 17 significant bits: n * ln2_hi is exact */
+  const float ln2_lo = 0x1.7f7d1cp-20f;   /* fp32(ln 2 - ln2_hi) */
+  const float n = rintf(z * inv_ln2);
+  float f = fmaf(-n, ln2_hi, z);
+  f = fmaf(-n, ln2_lo, f);
+  float p = 0x1.a01a02p-13f;              /* 1/7! */
+  p = fmaf(p, f, 0x1.6c16c2p-10f);        /* 1/6! */
+  p = fmaf(p, f, 0x1.111112p-7f);         /* 1/5! */
+  p = fmaf(p, f, 0x1.555556p-5f);         /* 1/4! */
+  p = fmaf(p, f, 0x1.555556p-3f);         /* 1/3! */
+  p = fmaf(p, f, 0.5f);
+  p = fmaf(p, f, 1.0f);
+  p = fmaf(p, f, 1.0f);
+  return p * ldexpf(1.0f, (int)n);
+}
+
+static float orc_tanh(float u) {
+  const float a = fabsf(u);
+  float t = 1.0f;
+  if (a < 9.0f) {
+    const float e = orc_exp_0_18(2.0f * a);
+    t = 1.0f - 2.0f / (e + 1.0f);
+  }
+  return u < 0.0f ? -t : t;
+}
+
+static float orc_gelu_tanh(float x) {
+  const float k0 = 0x1.988454p-1f;   /* fp32(sqrt(2/pi)) */
+  const float k1 = 0x1.6e4e26p-5f;   /* fp32(0.044715) */
+  const float x3 = (x * x) * x;
+  const float u = k0 * fmaf(k1, x3, x);
+  const float t = orc_tanh(u);
+  return (0.5f * x) * (1.0f + t);
+}
+
+/* bf16(gelu(bf16(y))) for n fp32 values, as bf16 bit patterns. */
+int orc_gelu_bf16(const float *y, int64_t n, uint16_t *out) {
+  if (n < 0 || (n > 0 && (y == NULL || out == NULL))) return -1;
+  for (int64_t i = 0; i < n; ++i) out[i] = orc_bf16_rne(orc_gelu_tanh(orc_bf16(orc_bf16_rne(y[i]))));
+  return 0;
+}
+
+/* The pieces, for the pins: bf16 rounding, e^z on [0, 18], tanh and gelu. */
+int orc_gelu_parts(const float *x, int64_t n, float *exp_out, float *tanh_out, float *gelu_out,
+                   uint16_t *bf16_out) {
+  for (int64_t i = 0; i < n; ++i) {
+    if (exp_out) exp_out[i] = orc_exp_0_18(x[i]);
+    if (tanh_out) tanh_out[i] = orc_tanh(x[i]);
+    if (gelu_out) gelu_out[i] = orc_gelu_tanh(x[i]);
+    if (bf16_out) bf16_out[i] = orc_bf16_rne(x[i]);
+  }
+  return 0;
+}
