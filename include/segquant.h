@@ -252,6 +252,39 @@ SQ_API sq_status sq_dualscale_seglinear_gemm(const int8_t *planes, const int8_t 
                                       sq_stream_t stream);
 
 /*
+ * sq_dualscale_seglinear_gemm_gelu_quant -- the fused producer of an FFN's
+ * second linear: the same GEMM and epilogue as sq_dualscale_seglinear_gemm,
+ * but instead of y it writes the next layer's DualScale activation planes of
+ *   x2 = bf16(gelu(bf16(y)))
+ * (pages: papernotes.org section DualScale, whose polarity table measures the
+ * FFN's GELU output, the next layer's input; the pages give no GELU formula,
+ * the models use the tanh approximation
+ *   gelu(x) = x/2 (1 + tanh(sqrt(2/pi) (x + 0.044715 x^3))),
+ * evaluated here as one fixed sequence of fp32 operations: tanh from e^(2|u|)
+ * by Cody and Waite's reduction and a degree-7 Taylor series, 1 for |u| >= 9).
+ * The next layer's codes follow sq_quantize_act with d = 1 and its steps
+ * s_act_next = {s+, s-}: m+- = fl(1/s+-), x2 >= 0: q+ = rne(min(x2 m+, 127)),
+ * x2 < 0: q- = rne(max(x2 m-, -128)).  Its planes never round-trip through a
+ * bf16 activation in HBM.
+ *   planes, wq, s_w, s_act, bias, M, N, K, seg: as in
+ *          sq_dualscale_seglinear_gemm; seg must be SQ_SEG_NONE (one K-segment,
+ *          one group) and not SQ_FLAG_FP8 (SQ_ERR_UNSUPPORTED otherwise)
+ *   s_act_next fp32 [2] device {s+, s-} of the next layer (one group, one
+ *          K-segment, no SmoothQuant divisor), positive and finite
+ *   flags_next 0 (DualScale: planes_next int8 [2][M][N]) or
+ *          SQ_FLAG_SINGLE_SCALE (one merged plane [1][M][N])
+ *   planes_next int8 output, 16-byte aligned; N % 16 == 0 (it is the next
+ *          layer's K)
+ */
+SQ_API sq_status sq_dualscale_seglinear_gemm_gelu_quant(const int8_t *planes, const int8_t *wq,
+                                                       const float *s_w, const float *s_act,
+                                                       const void *bias, int64_t M, int64_t N,
+                                                       int64_t K, const sq_segments *seg,
+                                                       const float *s_act_next,
+                                                       int32_t flags_next, int8_t *planes_next,
+                                                       sq_stream_t stream);
+
+/*
  * sq_debug_gemm_s32 -- the same tensor-core kernel, storing the raw int32
  * accumulators instead of the epilogue, for bit-exact checks.
  *   acc int32 [S][P][M][N] output (16-byte aligned), polarity 0 = A+, 1 = A-;

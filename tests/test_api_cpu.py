@@ -43,7 +43,7 @@ def test_status_strings(L):
     assert B.status_string(0) == "SQ_OK"
     for code in range(-7, 0):
         assert B.status_string(code).startswith("SQ_ERR_")
-    assert B.lib().sq_version() == 102
+    assert B.lib().sq_version() == 103
 
 
 def _seg(mode, offsets, groups=1):
@@ -211,3 +211,24 @@ def test_host_pipeline_validates_on_host(L):
     assert L.sq_dualscale_seglinear_host(None, p(FAKE), 8, 64, 64, None, p(FAKE), p(FAKE),
                                          p(FAKE), None, p(FAKE), 0, 64, 64, ctypes.byref(c),
                                          None) == SQ_ERR_INVALID_ARG
+
+
+def test_gelu_quant_validation(L):
+    """The fused producer's host checks, before any launch."""
+    p = ctypes.c_void_p
+    none, keep0 = _seg(B.SQ_SEG_NONE, None)
+    inp, keep1 = _seg(B.SQ_SEG_INPUT, [0, 32, 64])
+    f = L.sq_dualscale_seglinear_gemm_gelu_quant
+    args = lambda seg, N=64, s_next=FAKE, flags=0: (p(FAKE), p(FAKE), p(FAKE), p(FAKE), None,
+                                                    8, N, 64, ctypes.byref(seg), p(s_next),
+                                                    flags, p(FAKE), None)
+    assert f(*args(inp)) == SQ_ERR_UNSUPPORTED            # this layer: one K-segment only
+    assert f(*args(none, flags=B.SQ_FLAG_W4)) == SQ_ERR_INVALID_ARG   # next: 0 or single scale
+    assert f(*args(none, N=40)) == SQ_ERR_ALIGNMENT       # N is the next layer's K: % 16
+    assert f(*args(none, s_next=0)) == SQ_ERR_INVALID_ARG  # the next layer's steps
+    fp8, keep2 = B.Segments(B.SQ_SEG_NONE, None, 1, B.SQ_FLAG_FP8)._c()
+    assert f(*args(fp8)) == SQ_ERR_UNSUPPORTED
+    # M == 0 is a valid no-op that never touches CUDA
+    assert f(p(FAKE), p(FAKE), p(FAKE), p(FAKE), None, 0, 64, 64, ctypes.byref(none), p(FAKE), 0,
+             p(FAKE), None) == 0
+

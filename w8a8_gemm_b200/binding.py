@@ -28,7 +28,8 @@ SQ_FLAG_FP8 = 4
 
 EXPORTED = ("sq_calibrate_act", "sq_quantize_act", "sq_quantize_weight_seg",
             "sq_quantize_weight_w4", "sq_unpack_weight_w4",
-            "sq_dualscale_seglinear_gemm", "sq_debug_gemm_s32", "sq_get_device_status",
+            "sq_dualscale_seglinear_gemm", "sq_dualscale_seglinear_gemm_gelu_quant",
+            "sq_debug_gemm_s32", "sq_get_device_status",
             "sq_status_string", "sq_version", "sq_debug_timeout_probe",
             "sq_host_pipeline_workspace_bytes", "sq_host_pipeline_create",
             "sq_host_pipeline_destroy", "sq_dualscale_seglinear_host")
@@ -103,6 +104,8 @@ def lib() -> ctypes.CDLL:
         L.sq_unpack_weight_w4.argtypes = [p, i64, i64, p, p]
         L.sq_dualscale_seglinear_gemm.argtypes = [p, p, p, p, p, p, ctypes.c_int, i64, i64, i64,
                                                   i64, seg, p]
+        L.sq_dualscale_seglinear_gemm_gelu_quant.argtypes = [p, p, p, p, p, i64, i64, i64, seg,
+                                                             p, ctypes.c_int32, p, p]
         L.sq_debug_gemm_s32.argtypes = [p, p, i64, i64, i64, seg, p, p]
         L.sq_get_device_status.argtypes = []
         L.sq_debug_timeout_probe.argtypes = [ctypes.c_uint32, p]
@@ -120,7 +123,8 @@ def lib() -> ctypes.CDLL:
         for f in (L.sq_calibrate_act, L.sq_quantize_act, L.sq_quantize_weight_seg,
                   L.sq_quantize_weight_w4, L.sq_unpack_weight_w4, L.sq_host_pipeline_create,
                   L.sq_host_pipeline_destroy, L.sq_dualscale_seglinear_host,
-                  L.sq_dualscale_seglinear_gemm, L.sq_debug_gemm_s32, L.sq_get_device_status,
+                  L.sq_dualscale_seglinear_gemm, L.sq_dualscale_seglinear_gemm_gelu_quant,
+                  L.sq_debug_gemm_s32, L.sq_get_device_status,
                   L.sq_version, L.sq_debug_timeout_probe):
             f.restype = ctypes.c_int
         _lib = L
@@ -259,6 +263,36 @@ def sq_dualscale_seglinear_gemm(planes: torch.Tensor, wq: torch.Tensor, s_w: tor
                                              ctypes.byref(cs), _stream()),
            "sq_dualscale_seglinear_gemm")
     return y
+
+
+def sq_dualscale_seglinear_gemm_gelu_quant(planes: torch.Tensor, wq: torch.Tensor,
+                                           s_w: torch.Tensor, s_act: torch.Tensor,
+                                           bias: Optional[torch.Tensor], seg: Segments,
+                                           s_act_next: torch.Tensor, planes_next: torch.Tensor,
+                                           single_next: bool = False) -> torch.Tensor:
+    """The fused producer: the next layer's planes of bf16(gelu(bf16(y))) into
+    planes_next (int8 [1][P'][M][N], P' = 2, or 1 with single_next), with its
+    steps s_act_next (fp32 [2] = {s+, s-}).  This layer: one K-segment."""
+    _need(planes, torch.int8, "planes")
+    _need(wq, torch.int8, "wq")
+    _need(s_w, torch.float32, "s_w")
+    _need(s_act, torch.float32, "s_act")
+    _need(bias, torch.bfloat16, "bias", optional=True)
+    _need(s_act_next, torch.float32, "s_act_next")
+    _need(planes_next, torch.int8, "planes_next")
+    G, P, M, K = planes.shape
+    N = wq.shape[0]
+    pn = 1 if single_next else 2
+    if (P != seg.P or wq.shape[1] != K or s_act_next.numel() != 2
+            or tuple(planes_next.shape) != (1, pn, M, N) or not planes_next.is_contiguous()):
+        raise ValueError("shape mismatch between planes [G,P,M,K], wq [N,K] and "
+                         "planes_next [1,P',M,N]")
+    cs, keep = seg._c()
+    _check(lib().sq_dualscale_seglinear_gemm_gelu_quant(
+        _ptr(planes), _ptr(wq), _ptr(s_w), _ptr(s_act), _ptr(bias), M, N, K, ctypes.byref(cs),
+        _ptr(s_act_next), SQ_FLAG_SINGLE_SCALE if single_next else 0, _ptr(planes_next),
+        _stream()), "sq_dualscale_seglinear_gemm_gelu_quant")
+    return planes_next
 
 
 def sq_debug_gemm_s32(planes: torch.Tensor, wq: torch.Tensor, seg: Segments,

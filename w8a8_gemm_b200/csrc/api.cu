@@ -130,7 +130,8 @@ sq_status from_cuda(cudaError_t e) { return e == cudaSuccess ? SQ_OK : SQ_ERR_CU
 sq_status gemm_common(const int8_t *planes, const int8_t *wq, const float *s_w,
                       const float *s_act, const void *bias, void *y, int out_kind, int64_t M,
                       int64_t N, int64_t K, int64_t ldy, const sq_segments *seg,
-                      cudaStream_t stream, bool launch = true) {
+                      cudaStream_t stream, bool launch = true, const float *s_next = nullptr,
+                      int p_next = 0) {
   if (M < 0 || M > INT32_MAX || N < 1 || N > INT32_MAX) return SQ_ERR_INVALID_ARG;
   // An output of more than 2^44 elements fits no device; the bound keeps the
   // kernel's tile count (at most 2^30 tiles of 128 x 128) inside int32.
@@ -146,7 +147,14 @@ sq_status gemm_common(const int8_t *planes, const int8_t *wq, const float *s_w,
   if (s_w && !aligned(s_w, 4)) return SQ_ERR_ALIGNMENT;
   if (s_act && !aligned(s_act, 4)) return SQ_ERR_ALIGNMENT;
   if (bias && !aligned(bias, 2)) return SQ_ERR_ALIGNMENT;
-  if (out_kind != OUT_S32) {
+  if (out_kind == OUT_PLANES) {
+    // the fused producer: this layer one K-segment and one group, int8 codes;
+    // the next layer's planes [p_next][M][N] (N is its K)
+    if (sp.mode != SQ_SEG_NONE || sp.fp8) return SQ_ERR_UNSUPPORTED;
+    if (s_next == nullptr || (p_next != 1 && p_next != 2) || ldy != N)
+      return SQ_ERR_INVALID_ARG;
+    if (!aligned(s_next, 4) || N % 16 != 0) return SQ_ERR_ALIGNMENT;
+  } else if (out_kind != OUT_S32) {
     const int64_t elem = (out_kind == OUT_BF16) ? 2 : 4;
     if (ldy < N) return SQ_ERR_INVALID_ARG;
     if ((ldy * elem) % 16 != 0) return SQ_ERR_ALIGNMENT;
@@ -166,6 +174,8 @@ sq_status gemm_common(const int8_t *planes, const int8_t *wq, const float *s_w,
   r.N = N;
   r.K = K;
   r.seg = sp;
+  r.s_next = s_next;
+  r.p_next = p_next;
   r.status = device_status_word();
   if (r.status == nullptr) return SQ_ERR_CUDA;
   return launch_gemm(r, stream);
@@ -310,6 +320,18 @@ sq_status sq_dualscale_seglinear_gemm(const int8_t *planes, const int8_t *wq, co
                      reinterpret_cast<cudaStream_t>(stream));
 }
 
+sq_status sq_dualscale_seglinear_gemm_gelu_quant(const int8_t *planes, const int8_t *wq,
+                                                const float *s_w, const float *s_act,
+                                                const void *bias, int64_t M, int64_t N, int64_t K,
+                                                const sq_segments *seg, const float *s_act_next,
+                                                int32_t flags_next, int8_t *planes_next,
+                                                sq_stream_t stream) {
+  if (flags_next != 0 && flags_next != SQ_FLAG_SINGLE_SCALE) return SQ_ERR_INVALID_ARG;
+  const int p_next = (flags_next & SQ_FLAG_SINGLE_SCALE) ? 1 : 2;
+  return gemm_common(planes, wq, s_w, s_act, bias, planes_next, OUT_PLANES, M, N, K, N, seg,
+                     reinterpret_cast<cudaStream_t>(stream), true, s_act_next, p_next);
+}
+
 sq_status sq_debug_gemm_s32(const int8_t *planes, const int8_t *wq, int64_t M, int64_t N,
                             int64_t K, const sq_segments *seg, int32_t *acc,
                             sq_stream_t stream) {
@@ -352,6 +374,6 @@ const char *sq_status_string(sq_status s) {
   return "unknown sq_status";
 }
 
-int32_t sq_version(void) { return 102; }
+int32_t sq_version(void) { return 103; }
 
 }  // extern "C"

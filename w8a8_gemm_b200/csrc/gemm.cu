@@ -68,6 +68,8 @@ struct GemmParams {
   void *y;
   int64_t ldy;
   int *status;
+  const float *s_next;  // OUT_PLANES: the next layer's {s+, s-}
+  int32_t p_next;       // OUT_PLANES: its planes (2, or 1 single scale)
 };
 
 // POL = activation planes per group: 2 for DualScale (X^+ and X^-), 1 for the
@@ -134,6 +136,56 @@ __device__ __forceinline__ float bf16_to_f32(uint16_t h) {
   return __uint_as_float(static_cast<uint32_t>(h) << 16);
 }
 
+// ---- the FFN activation of the fused producer (OUT_PLANES) ----------------
+// gelu(x) = x/2 (1 + tanh(sqrt(2/pi) (x + 0.044715 x^3))), the tanh
+// approximation the models' FFNs use between the two linears, as one fixed
+// sequence of fp32 operations, each rounded once:
+//   tanh(u) = 1 - 2 / (e^(2|u|) + 1) with the sign of u; 1 for |u| >= 9;
+//   e^z (0 <= z <= 18): z = n ln2 + f, n = rint(z / ln2) (Cody and Waite's
+//   reduction with ln2 split into a head exact in n * head and a tail), e^f by
+//   its Taylor series to degree 7, times 2^n.
+__device__ __forceinline__ float exp_0_18(float z) {
+  const float n = rintf(__fmul_rn(z, 0x1.715476p+0f));  // z / ln2
+  float f = __fmaf_rn(-n, 0x1.62e4p-1f, z);             // ln2 head (17 bits)
+  f = __fmaf_rn(-n, 0x1.7f7d1cp-20f, f);                // ln2 tail
+  float q = 0x1.a01a02p-13f;                            // 1/7!
+  q = __fmaf_rn(q, f, 0x1.6c16c2p-10f);                 // 1/6!
+  q = __fmaf_rn(q, f, 0x1.111112p-7f);                  // 1/5!
+  q = __fmaf_rn(q, f, 0x1.555556p-5f);                  // 1/4!
+  q = __fmaf_rn(q, f, 0x1.555556p-3f);                  // 1/3!
+  q = __fmaf_rn(q, f, 0.5f);
+  q = __fmaf_rn(q, f, 1.0f);
+  q = __fmaf_rn(q, f, 1.0f);
+  return __fmul_rn(q, __int_as_float((static_cast<int>(n) + 127) << 23));  // 2^n, 0 <= n <= 26
+}
+
+__device__ __forceinline__ float gelu_tanh(float x) {
+  const float x3 = __fmul_rn(__fmul_rn(x, x), x);
+  const float u = __fmul_rn(0x1.988454p-1f, __fmaf_rn(0x1.6e4e26p-5f, x3, x));
+  const float a = fabsf(u);
+  float t = 1.0f;
+  if (a < 9.0f) {
+    const float e = exp_0_18(__fmul_rn(2.0f, a));
+    t = __fsub_rn(1.0f, __fdiv_rn(2.0f, __fadd_rn(e, 1.0f)));
+  }
+  if (u < 0.0f) t = -t;
+  return __fmul_rn(__fmul_rn(0.5f, x), __fadd_rn(1.0f, t));
+}
+
+// DualScale codes of the next layer's input x2 = bf16(gelu(bf16(y))), with its
+// folded multipliers m+- = 1/s+-: x2 >= 0 gives q+ = rne(min(x2 m+, 127)),
+// x2 < 0 gives q- = rne(max(x2 m-, -128)); the other code is 0.
+__device__ __forceinline__ void gelu_codes(float y, float mp, float mm, int &qp, int &qm) {
+  const float xb = __bfloat162float(__float2bfloat16_rn(y));
+  const float x2 = __bfloat162float(__float2bfloat16_rn(gelu_tanh(xb)));
+  qp = 0;
+  qm = 0;
+  if (x2 < 0.0f)
+    qm = __float2int_rn(fmaxf(__fmul_rn(x2, mm), -128.0f));
+  else
+    qp = __float2int_rn(fminf(__fmul_rn(x2, mp), 127.0f));
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<const uint32_t *>(&v);
@@ -190,8 +242,10 @@ __global__ void __launch_bounds__(threads_for(EPI_WARPS), 1)
                           const __grid_constant__ CUtensorMap tmB,
                           const __grid_constant__ CUtensorMap tmY,
                           const __grid_constant__ GemmParams p) {
-  // One-segment bf16 output leaves through shared memory and TMA stores.
-  constexpr bool TMA_STORE = (OUT == OUT_BF16) && !SEGK;
+  // One-segment bf16 output (and the next layer's planes) leave through
+  // shared memory and TMA stores.
+  constexpr bool TMA_STORE = (OUT == OUT_BF16 || OUT == OUT_PLANES) && !SEGK;
+  static_assert(OUT != OUT_PLANES || (!SEGK && !F8), "planes output: one K-segment, int8");
   using L = Smem<BN, STAGES, EPI_WARPS, POL, SEGK, TMA_STORE>;
   constexpr int NBUF = L::NBUF;
   constexpr int ACC_COLS = POL * BN;  // TMEM columns of one accumulator buffer
@@ -350,6 +404,12 @@ __global__ void __launch_bounds__(threads_for(EPI_WARPS), 1)
     float *cst_base = reinterpret_cast<float *>(smem + L::EPI_OFFSET) + ew * L::CONST_FLOATS;
     uint8_t *stg = smem + L::STG_OFFSET + ew * 2048;  // used when TMA_STORE
     uint32_t acc_iter = 0;
+    // OUT_PLANES: the next layer's folded multipliers m+- = fl(1/s+-).
+    float mp_next = 0.0f, mm_next = 0.0f;
+    if constexpr (OUT == OUT_PLANES) {
+      mp_next = __fdiv_rn(1.0f, p.s_next[0]);
+      mm_next = __fdiv_rn(1.0f, p.s_next[1]);
+    }
     for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x) {
       const int mt = tile / p.num_n_tiles, nt = tile % p.num_n_tiles;
       const int g = group_of_tile(p, nt, BN);
@@ -488,7 +548,21 @@ __global__ void __launch_bounds__(threads_for(EPI_WARPS), 1)
                   float y0, y1;
                   f2unpack(y, y0, y1);
                   const int rr = 16 * k + 8 * h + (lane >> 2);  // row within the warp's 32
-                  if constexpr (TMA_STORE) {
+                  if constexpr (OUT == OUT_PLANES) {
+                    // Two 32 x 32-byte staging blocks (X^+ then X^-), row-major:
+                    // columns 8j + 2q and 8j + 2q + 1 as one 16-bit store each.
+                    int qp0, qm0, qp1, qm1;
+                    gelu_codes(y0, mp_next, mm_next, qp0, qm0);
+                    gelu_codes(y1, mp_next, mm_next, qp1, qm1);
+                    uint16_t *dst = reinterpret_cast<uint16_t *>(stg + rr * 32 + 8 * j + 2 * q);
+                    if (p.p_next == 2) {
+                      dst[0] = static_cast<uint16_t>((qp0 & 0xFF) | ((qp1 & 0xFF) << 8));
+                      dst[512] = static_cast<uint16_t>((qm0 & 0xFF) | ((qm1 & 0xFF) << 8));
+                    } else {  // single scale: one merged plane (one code is 0)
+                      dst[0] = static_cast<uint16_t>(((qp0 + qm0) & 0xFF) |
+                                                     (((qp1 + qm1) & 0xFF) << 8));
+                    }
+                  } else if constexpr (TMA_STORE) {
                     // Staging buffer in the tensor map's 64-byte swizzle:
                     // 16-byte piece j of row rr sits at piece j ^ ((rr / 2) % 4),
                     // so the 8 rows x 16 bytes of one store instruction fall
@@ -502,13 +576,19 @@ __global__ void __launch_bounds__(threads_for(EPI_WARPS), 1)
                 }
             }
             if constexpr (TMA_STORE) {
-              // The warp's 32 rows x 32 columns leave in one tensor store,
-              // which writes whole lines and drops rows >= M and columns >= N.
+              // The warp's 32 rows x 32 columns leave in one tensor store per
+              // plane, which writes whole lines and drops rows >= M and
+              // columns >= N.
               fence_proxy_async_smem();
               __syncwarp();
               const int row0 = mt * BM + quarter * 32;
               if (lane == 0 && row0 < p.M && n0 < p.N) {
-                tma_store_2d(&tmY, stg, static_cast<int32_t>(n0), row0);
+                if constexpr (OUT == OUT_PLANES) {
+                  for (int pl = 0; pl < p.p_next; ++pl)
+                    tma_store_3d(&tmY, stg + pl * 1024, static_cast<int32_t>(n0), row0, pl);
+                } else {
+                  tma_store_2d(&tmY, stg, static_cast<int32_t>(n0), row0);
+                }
                 bulk_commit_group();
               }
             }
@@ -656,7 +736,7 @@ int device_sm_count() {
 
 template <int BN, int STAGES, int OUT, bool SEGK, int EPI_WARPS, int POL, bool F8>
 sq_status run_gemm(const GemmRequest &r, const GemmParams &p, cudaStream_t stream) {
-  using L = Smem<BN, STAGES, EPI_WARPS, POL, SEGK, OUT == OUT_BF16 && !SEGK>;
+  using L = Smem<BN, STAGES, EPI_WARPS, POL, SEGK, (OUT == OUT_BF16 || OUT == OUT_PLANES) && !SEGK>;
   EncodeTiledFn enc = tensor_map_encoder();
   if (enc == nullptr) return SQ_ERR_CUDA;
   const int G = r.seg.G;
@@ -688,6 +768,20 @@ sq_status run_gemm(const GemmRequest &r, const GemmParams &p, cudaStream_t strea
   }
   CUtensorMap tmY;
   memset(&tmY, 0, sizeof tmY);
+  if (OUT == OUT_PLANES) {
+    // The next layer's planes as 3D int8: x = N columns, y = M rows, z = plane;
+    // 32 x 32 boxes, one plane each.
+    const cuuint64_t dims[3] = {static_cast<cuuint64_t>(r.N), static_cast<cuuint64_t>(r.M),
+                                static_cast<cuuint64_t>(r.p_next)};
+    const cuuint64_t strides[2] = {static_cast<cuuint64_t>(r.N),
+                                   static_cast<cuuint64_t>(r.N) * static_cast<cuuint64_t>(r.M)};
+    const cuuint32_t box[3] = {32, 32, 1};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    if (enc(&tmY, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, r.y, dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+            CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return SQ_ERR_CUDA;
+  }
   if (OUT == OUT_BF16 && !SEGK) {
     // Y viewed as 2D bf16: x = N columns, y = M rows; 32 x 32 boxes.
     const cuuint64_t dims[2] = {static_cast<cuuint64_t>(r.N), static_cast<cuuint64_t>(r.M)};
@@ -739,14 +833,20 @@ constexpr int kSegBN = 128;  // tile width of the input-segmented path
 template <int OUT, int POL, bool F8>
 sq_status dispatch(const GemmRequest &r, const GemmParams &p, bool segk, int BN,
                    cudaStream_t stream) {
+  if constexpr (OUT == OUT_PLANES) {
+    // one K-segment, one group (checked by the caller)
+    return run_gemm<256, POL == 2 ? 3 : 4, OUT, false, 8, POL, false>(r, p, stream);
+  } else {
   if (segk) return run_gemm<kSegBN, 4, OUT, true, 16, POL, F8>(r, p, stream);
   if (BN == 256) return run_gemm<256, POL == 2 ? 3 : 4, OUT, false, 8, POL, F8>(r, p, stream);
   return run_gemm<128, 4, OUT, false, 8, POL, F8>(r, p, stream);
+  }
 }
 
 template <int OUT, int POL>
 sq_status dispatch_kind(const GemmRequest &r, const GemmParams &p, bool segk, int BN,
                         cudaStream_t stream) {
+  if constexpr (OUT == OUT_PLANES) return dispatch<OUT, POL, false>(r, p, segk, BN, stream);
   return r.seg.fp8 ? dispatch<OUT, POL, true>(r, p, segk, BN, stream)
                    : dispatch<OUT, POL, false>(r, p, segk, BN, stream);
 }
@@ -791,17 +891,21 @@ sq_status launch_gemm(const GemmRequest &r, cudaStream_t stream) {
   p.y = r.y;
   p.ldy = r.ldy;
   p.status = r.status;
+  p.s_next = r.s_next;
+  p.p_next = r.p_next;
 
   if (r.seg.P == 1) {
     switch (r.out_kind) {
       case OUT_S32: return dispatch_kind<OUT_S32, 1>(r, p, segk, BN, stream);
       case OUT_F32: return dispatch_kind<OUT_F32, 1>(r, p, segk, BN, stream);
+      case OUT_PLANES: return dispatch_kind<OUT_PLANES, 1>(r, p, segk, BN, stream);
       default: return dispatch_kind<OUT_BF16, 1>(r, p, segk, BN, stream);
     }
   }
   switch (r.out_kind) {
     case OUT_S32: return dispatch_kind<OUT_S32, 2>(r, p, segk, BN, stream);
     case OUT_F32: return dispatch_kind<OUT_F32, 2>(r, p, segk, BN, stream);
+    case OUT_PLANES: return dispatch_kind<OUT_PLANES, 2>(r, p, segk, BN, stream);
     default: return dispatch_kind<OUT_BF16, 2>(r, p, segk, BN, stream);
   }
 }

@@ -45,7 +45,9 @@ cudaError_t launch_unpack_w4(const uint8_t *wq4, int64_t N, int64_t K, int8_t *w
                              cudaStream_t stream);
 
 // ---- launcher (gemm.cu) ----------------------------------------------------
-enum OutKind { OUT_BF16 = 0, OUT_F32 = 1, OUT_S32 = 2 };
+// OUT_PLANES: the next layer's int8 activation planes, from bf16(gelu(bf16(y)))
+// (the fused producer of an FFN's second linear).
+enum OutKind { OUT_BF16 = 0, OUT_F32 = 1, OUT_S32 = 2, OUT_PLANES = 3 };
 
 struct GemmRequest {
   const int8_t *planes;
@@ -59,6 +61,10 @@ struct GemmRequest {
   int64_t M, N, K;
   SegParams seg;
   int *status;  // device error word
+  // OUT_PLANES: the next layer's steps {s+, s-} (fp32 [2], device) and its
+  // planes per group (2 DualScale, 1 single scale); y is int8 [p_next][M][N].
+  const float *s_next = nullptr;
+  int p_next = 0;
 };
 
 sq_status launch_gemm(const GemmRequest &req, cudaStream_t stream);
