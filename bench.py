@@ -75,6 +75,18 @@ def layer_units(L, P=2):
     return eff, P * eff, quant_bytes
 
 
+def ffn_pairs(layers):
+    """(i, i + 1) for every FFN pair fc1 -> fc2 of a configuration: both one
+    segment, fc2's input the width of fc1's output, fc2 without a divisor."""
+    out = []
+    for i in range(len(layers) - 1):
+        a, b = layers[i], layers[i + 1]
+        if (a.name.endswith("fc1") and b.name.endswith("fc2") and a.mode == wl.MODE_NONE
+                and b.mode == wl.MODE_NONE and b.d is None and a.N == b.K and a.M == b.M):
+            out.append((i, i + 1))
+    return out
+
+
 def dist_env():
     ws = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -190,12 +202,22 @@ class GpuLayer:
         self.x = L.x.to(dev)
         self.planes = torch.empty(L.G, self.lin.seg.P, L.M, L.K, dtype=torch.int8, device=dev)
         self.y = torch.empty(L.M, L.N, dtype=torch.bfloat16, device=dev)
+        self.fused_next = None  # fused producer: the layer whose planes this GEMM writes
+        self.produced = False   # this layer's planes come from the previous GEMM
 
     def quantize(self):
-        self.lin.quantize(self.x, self.planes)
+        if not self.produced:
+            self.lin.quantize(self.x, self.planes)
 
     def gemm(self):
-        self.lin.gemm(self.planes, self.y)
+        if self.fused_next is None:
+            self.lin.gemm(self.planes, self.y)
+            return
+        self.lin.gemm_gelu_quant(self.planes, self.fused_next.lin, self.fused_next.planes)
+
+    def kernels(self):
+        """This library's kernel launches per step."""
+        return ((0 if self.produced else 1) + 1 + (1 if self.lin.wq4 is not None else 0))
 
     def host_call(self, pl, x_host, y_host):
         """The layer from host rows to host rows through the library's host
@@ -220,10 +242,16 @@ def run_ours(args, ws, rank, local):
                  if args.weight_bits == 4 else None)
     glayers = [GpuLayer(L, dev, adaptive=args.adaptive, weight_bits=args.weight_bits,
                         w_operand=w_operand, fp8=args.fp8) for L in layers_cpu]
+    if args.fused_gelu:
+        # FFN pairs: fc1's GEMM writes fc2's planes of bf16(gelu(bf16(y1)))
+        for a, b in ffn_pairs(layers_cpu):
+            glayers[a].fused_next = glayers[b]
+            glayers[b].produced = True
     torch.cuda.synchronize()
     eff_ops = sum(layer_units(g.L, g.lin.seg.P)[0] for g in glayers)
     exe_ops = sum(layer_units(g.L, g.lin.seg.P)[1] for g in glayers)
-    qbytes = sum(layer_units(g.L, g.lin.seg.P)[2] for g in glayers)
+    # bytes of the activation-quantize kernels that run (a produced layer has none)
+    qbytes = sum(layer_units(g.L, g.lin.seg.P)[2] for g in glayers if not g.produced)
     flush = torch.empty(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
     sweep = torch.ones(SWEEP_BYTES // 4, dtype=torch.float32, device=dev)
     sink = torch.empty((), dtype=torch.float32, device=dev)
@@ -306,7 +334,7 @@ def run_ours(args, ws, rank, local):
                                gemm_us=1e3 * g_ms[i])
                           for i, g in enumerate(glayers)],
                breakdown_steps=n_bd,
-               launches=(3 if args.weight_bits == 4 else 2) * nl * args.steps)
+               launches=sum(g.kernels() for g in glayers) * args.steps)
 
     # Each activation-quantize launch alone after an L2 flush: the kernel's own
     # HBM roofline, free of the write-back left in L2 by the previous kernel of
@@ -314,6 +342,8 @@ def run_ours(args, ws, rank, local):
     iso_steps = max(3, min(args.steps, 200))
     iso_ms = [0.0] * nl
     for i, g in enumerate(glayers):
+        if g.produced:
+            continue
         ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
               for _ in range(iso_steps)]
         for k in range(iso_steps):
@@ -328,29 +358,47 @@ def run_ours(args, ws, rank, local):
     # End to end through the library's host entry point: every layer's input
     # rows come from pinned host memory and its output rows go back to it, in
     # chunks whose copies overlap the kernels (sq_dualscale_seglinear_host).
+    # A fused FFN pair runs as one block: X1 from the host, fc2's planes stay on
+    # the device, Y2 back to the host.
     from w8a8_gemm_b200 import binding as B
-    hx = [g.x.cpu().pin_memory() for g in glayers]
-    hy = [torch.empty(g.L.M, g.L.N, dtype=torch.bfloat16).pin_memory() for g in glayers]
+    hx = [None if g.produced else g.x.cpu().pin_memory() for g in glayers]
+    hy = [None if g.fused_next is not None else
+          torch.empty(g.L.M, g.L.N, dtype=torch.bfloat16).pin_memory() for g in glayers]
+
+    def e2e_layer(i, g):
+        if g.produced:
+            return
+        if g.fused_next is None:
+            g.host_call(pl, hx[i], hy[i])
+            return
+        nxt = g.fused_next
+        j = glayers.index(nxt)
+        g.x.copy_(hx[i], non_blocking=True)
+        g.quantize()
+        g.gemm()
+        nxt.gemm()
+        hy[j].copy_(nxt.y, non_blocking=True)
+
     pl = B.HostPipeline(E2E_CHUNK_ROWS, max(g.L.K for g in glayers), max(g.L.N for g in glayers),
                         max(g.L.G for g in glayers), max(g.lin.seg.P for g in glayers),
                         device=dev)
     e2e_steps = max(3, min(args.steps, args.e2e_steps))
     for _ in range(2):
         for i, g in enumerate(glayers):
-            g.host_call(pl, hx[i], hy[i])
+            e2e_layer(i, g)
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
     for _ in range(e2e_steps):
         for i, g in enumerate(glayers):
-            g.host_call(pl, hx[i], hy[i])
+            e2e_layer(i, g)
     e1.record(stream)
     torch.cuda.synchronize()
     pl.close()
     e2e_ms = aggregate_over_ranks(e0.elapsed_time(e1), "max", device=dev) / e2e_steps
     res["e2e_ms"] = e2e_ms
-    res["h2d"] = sum(t.numel() * t.element_size() for t in hx)
-    res["d2h"] = sum(t.numel() * t.element_size() for t in hy)
+    res["h2d"] = sum(t.numel() * t.element_size() for t in hx if t is not None)
+    res["d2h"] = sum(t.numel() * t.element_size() for t in hy if t is not None)
     return res, layers_cpu
 
 
@@ -369,28 +417,32 @@ def prepare_oracle(layers):
     return prepared
 
 
-def oracle_rows(prepared, rows: int, threads: int):
+def oracle_rows(prepared, rows: int, threads: int, pairs=()):
     """One pass of the oracle's per-batch work (activation quantization and the
     DualScale GEMM) over the first `rows` rows of every layer; returns
-    (seconds, effective ops)."""
+    (seconds, effective ops).  For each (a, b) in pairs, layer b's input is
+    bf16(gelu(bf16(y_a))) instead of its own X (the fused producer's step)."""
     import oracle
+    produced = {b: a for a, b in pairs}
     t0 = time.perf_counter()
     ops = 0.0
-    for L, off, d, s_act, wq, s_w, bias in prepared:
-        planes = oracle.quantize_act(wl.bits(L.x[:rows]), s_act, d, L.mode, off, L.G, L.N)
-        oracle.gemm(planes, wq, s_w, s_act, bias, L.mode, off, threads=threads)
+    y_prev = None
+    for i, (L, off, d, s_act, wq, s_w, bias) in enumerate(prepared):
+        x = oracle.gelu_bf16(y_prev) if i in produced else wl.bits(L.x[:rows])
+        planes = oracle.quantize_act(x, s_act, d, L.mode, off, L.G, L.N)
+        y_prev = oracle.gemm(planes, wq, s_w, s_act, bias, L.mode, off, threads=threads)
         ops += 2.0 * rows * L.N * L.K
     return time.perf_counter() - t0, ops
 
 
-def oracle_sample(layers, target_s: float, threads: int, prepared=None):
+def oracle_sample(layers, target_s: float, threads: int, prepared=None, pairs=()):
     """Times the CPU oracle on a row sample of every layer, sized so that the
     timed work takes about target_s seconds."""
     prepared = prepared or prepare_oracle(layers)
     max_rows = min(L.M for L in layers)
     rows = 4
     while True:
-        dt, ops = oracle_rows(prepared, rows, threads)
+        dt, ops = oracle_rows(prepared, rows, threads, pairs)
         if dt >= 0.5 * target_s or rows >= max_rows:
             return dict(rows=rows, seconds=dt, eff_ops=ops, tops=ops / dt / 1e12)
         rows = min(max_rows, max(rows * 2, int(rows * target_s / max(dt, 1e-3))))
@@ -414,9 +466,16 @@ def main(argv=None):
                     help="FP8 E4M3 codes for activations and weights (tcgen05 kind::f8f6f4)")
     ap.add_argument("--adaptive", action="store_true",
                     help="single-scale path on layers whose calibrated sides differ by < 2x")
+    ap.add_argument("--fused-gelu", action="store_true",
+                    help="FFN pairs: fc1's GEMM applies the GELU and writes fc2's activation "
+                         "planes (the fused producer); fc2 runs no quantize kernel")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+    if args.fused_gelu and args.fp8:
+        ap.error("--fused-gelu takes int8 codes, not --fp8")
+    if args.fused_gelu and not ffn_pairs(wl.config_layers(args.config, seed=0)):
+        ap.error(f"--fused-gelu: no FFN pair in {args.config}")
     ws, rank, local = dist_env()
     n_gpus = max(args.gpus, ws)
 
@@ -451,14 +510,18 @@ def main(argv=None):
     quant_gbs = res["qbytes"] / (res["quant_ms"] * 1e-3) / 1e9
     quant_iso_gbs = res["qbytes"] / (sum(res["quant_isolated_ms"]) * 1e-3) / 1e9
     traffic, traffic_note = traffic_from_profile()
+    if args.fused_gelu:
+        traffic, traffic_note = None, "the profile's counters are for the GEMM without the fused producer"
     cpu = None
     if n_gpus == 1 and not args.no_cpu_baseline:
         import oracle
         thr = oracle.num_threads()
-        s = oracle_sample(layers, args.cpu_seconds, thr)
+        pairs = ffn_pairs(layers) if args.fused_gelu else []
+        s = oracle_sample(layers, args.cpu_seconds, thr, pairs=pairs)
         cpu = {"value": s["tops"], "unit": "TOPS", "cores": thr, "kind": "oracle",
                "sample": f"first {s['rows']} rows of every layer of {args.config} "
-                         f"(quantize + GEMM, calibration and weights prepared untimed), "
+                         f"(quantize + GEMM, calibration and weights prepared untimed"
+                         f"{'; fc2 input = bf16(gelu(bf16(fc1 output)))' if pairs else ''}), "
                          f"{s['seconds']:.1f} s"}
     e2e_tops = n_gpus * res["eff_ops"] / (res["e2e_ms"] * 1e-3) / 1e12
     out = {
@@ -485,6 +548,9 @@ def main(argv=None):
                                if args.weight_bits == 4 else
                                "FP8 E4M3 activations and weights" if args.fp8 else "W8A8"),
                    "output": "bf16",
+                   "producer": ("fused: fc1's epilogue writes fc2's planes of "
+                                "bf16(gelu(bf16(y1))), no fc2 quantize kernel"
+                                if args.fused_gelu else "separate activation-quantize kernels"),
                    "l2": "flushed between steps, untimed: 512 MiB written, then 256 MiB read",
                    "parallelism": f"replicas x{n_gpus}"},
         "executed_tops": round(n_gpus * exe_tops_step, 2),
@@ -518,8 +584,11 @@ def main(argv=None):
         "e2e": {"value": round(e2e_tops, 3), "unit": "TOPS",
                 "h2d_bytes_per_step": res["h2d"], "d2h_bytes_per_step": res["d2h"],
                 "ms_per_step": round(res["e2e_ms"], 4),
-                "via": (f"sq_dualscale_seglinear_host, {E2E_CHUNK_ROWS}-row chunks, pinned host "
-                        "rows in and out of every layer")},
+                "via": ((f"FFN pairs as one fused block (X1 from pinned host memory, Y2 back); "
+                         f"other layers through sq_dualscale_seglinear_host, "
+                         f"{E2E_CHUNK_ROWS}-row chunks") if args.fused_gelu else
+                        (f"sq_dualscale_seglinear_host, {E2E_CHUNK_ROWS}-row chunks, pinned "
+                         "host rows in and out of every layer"))},
         "gpu_launches": res["launches"],
         "clocks": res["clocks"],
         "wall_s_timed_region": round(res["wall_s"], 3),
@@ -537,13 +606,14 @@ def main_reference(args, ws, rank):
     layers = wl.config_layers(args.config, seed=0)
     thr = oracle.num_threads()
     prepared = prepare_oracle(layers)
-    probe = oracle_sample(layers, 1.0, thr, prepared)
+    pairs = ffn_pairs(layers) if args.fused_gelu else []
+    probe = oracle_sample(layers, 1.0, thr, prepared, pairs=pairs)
     per_row_s = probe["seconds"] / probe["rows"]
     rows = max(1, int(REF_BUDGET_S / (args.steps + args.warmup) / per_row_s))
     rows = min(rows, min(L.M for L in layers))
 
     def step():
-        oracle_rows(prepared, rows, thr)
+        oracle_rows(prepared, rows, thr, pairs)
 
     for _ in range(args.warmup):
         step()
@@ -559,7 +629,9 @@ def main_reference(args, ws, rank):
            "scaling": "weak", "vs_baseline": None, "dtype": "s8",
            "data": "synthetic (seeded SD3.5/FLUX-shaped activations and weights)",
            "config": {"workload": f"{args.config}: {wl.CONFIGS[args.config]}",
-                      "sample_rows_per_layer": rows},
+                      "sample_rows_per_layer": rows,
+                      "producer": ("fused: fc2's input = bf16(gelu(bf16(fc1 output)))"
+                                   if args.fused_gelu else "separate activation quantize")},
            "cpu_baseline": {"value": round(tops, 6), "unit": "TOPS", "cores": thr,
                             "kind": "oracle",
                             "sample": f"first {rows} rows of every layer per step"},

@@ -98,5 +98,24 @@ class DualScaleSegLinear:
         return B.sq_dualscale_seglinear_gemm(planes, self.wq, self.s_w, self.s_act, self.bias,
                                              y, self.seg)
 
+    def gemm_gelu_quant(self, planes: torch.Tensor, nxt: "DualScaleSegLinear",
+                        planes_next: Optional[torch.Tensor] = None) -> torch.Tensor:
+        """This layer's GEMM fused with the next layer's input: returns nxt's
+        activation planes of bf16(gelu(bf16(y))) (an FFN's fc1 feeding fc2),
+        computed in this GEMM's epilogue with nxt's calibrated steps.  This
+        layer: one K-segment; nxt: one group and K-segment, no divisor."""
+        if nxt.d is not None or nxt.seg.mode != B.SQ_SEG_NONE:
+            raise ValueError("the next layer must have one segment and no SmoothQuant divisor")
+        M = planes.shape[2]
+        if planes_next is None:
+            planes_next = torch.empty(1, nxt.seg.P, M, nxt.K, dtype=torch.int8,
+                                      device=planes.device)
+        if self.wq4 is not None:
+            B.sq_unpack_weight_w4(self.wq4, self.wq)
+        return B.sq_dualscale_seglinear_gemm_gelu_quant(planes, self.wq, self.s_w, self.s_act,
+                                                        self.bias, self.seg,
+                                                        nxt.s_act.reshape(2), planes_next,
+                                                        single_next=nxt.seg.P == 1)
+
     def __call__(self, x: torch.Tensor, y: Optional[torch.Tensor] = None) -> torch.Tensor:
         return self.gemm(self.quantize(x), y)
