@@ -156,18 +156,20 @@ __device__ __forceinline__ float exp_0_18(float z) {
   q = __fmaf_rn(q, f, 0.5f);
   q = __fmaf_rn(q, f, 1.0f);
   q = __fmaf_rn(q, f, 1.0f);
-  return __fmul_rn(q, __int_as_float((static_cast<int>(n) + 127) << 23));  // 2^n, 0 <= n <= 26
+  // 2^n, 0 <= n <= 26: n as an integer from the bits of 1.5 * 2^23 + n (exact)
+  const int ni = __float_as_int(__fadd_rn(n, 12582912.0f)) - 0x4B400000;
+  return __fmul_rn(q, __int_as_float((ni + 127) << 23));
 }
 
 __device__ __forceinline__ float gelu_tanh(float x) {
   const float x3 = __fmul_rn(__fmul_rn(x, x), x);
   const float u = __fmul_rn(0x1.988454p-1f, __fmaf_rn(0x1.6e4e26p-5f, x3, x));
+  // Branch-free: e^(2|u|) with |u| capped at 9, and 1 selected from 9 on.
+  // 2 / d = 2 RN(1/d) exactly (d = e + 1 in [2, e^18 + 1]: no underflow).
   const float a = fabsf(u);
-  float t = 1.0f;
-  if (a < 9.0f) {
-    const float e = exp_0_18(__fmul_rn(2.0f, a));
-    t = __fsub_rn(1.0f, __fdiv_rn(2.0f, __fadd_rn(e, 1.0f)));
-  }
+  const float e = exp_0_18(__fmul_rn(2.0f, fminf(a, 9.0f)));
+  float t = __fsub_rn(1.0f, __fmul_rn(2.0f, __frcp_rn(__fadd_rn(e, 1.0f))));
+  t = a < 9.0f ? t : 1.0f;
   if (u < 0.0f) t = -t;
   return __fmul_rn(__fmul_rn(0.5f, x), __fadd_rn(1.0f, t));
 }
@@ -178,12 +180,13 @@ __device__ __forceinline__ float gelu_tanh(float x) {
 __device__ __forceinline__ void gelu_codes(float y, float mp, float mm, int &qp, int &qm) {
   const float xb = __bfloat162float(__float2bfloat16_rn(y));
   const float x2 = __bfloat162float(__float2bfloat16_rn(gelu_tanh(xb)));
-  qp = 0;
-  qm = 0;
-  if (x2 < 0.0f)
-    qm = __float2int_rn(fmaxf(__fmul_rn(x2, mm), -128.0f));
-  else
-    qp = __float2int_rn(fminf(__fmul_rn(x2, mp), 127.0f));
+  // rne of a value in [-128, 127]: the integer part of the bits of
+  // 1.5 * 2^23 + v, where the add rounds to the nearest integer, ties to even.
+  const bool neg = x2 < 0.0f;
+  const float v = neg ? fmaxf(__fmul_rn(x2, mm), -128.0f) : fminf(__fmul_rn(x2, mp), 127.0f);
+  const int q = __float_as_int(__fadd_rn(v, 12582912.0f)) - 0x4B400000;
+  qp = neg ? 0 : q;
+  qm = neg ? q : 0;
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
