@@ -275,6 +275,8 @@ SQ_API sq_status sq_dualscale_seglinear_gemm(const int8_t *planes, const int8_t 
  *          SQ_FLAG_SINGLE_SCALE (one merged plane [1][M][N])
  *   planes_next int8 output, 16-byte aligned; N % 16 == 0 (it is the next
  *          layer's K)
+ * y is finite whenever the scales and the bias are; the codes of a
+ * non-finite y are unspecified.
  */
 SQ_API sq_status sq_dualscale_seglinear_gemm_gelu_quant(const int8_t *planes, const int8_t *wq,
                                                        const float *s_w, const float *s_act,
