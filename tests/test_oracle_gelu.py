@@ -84,3 +84,30 @@ def test_gelu_bf16_close_to_torch():
     ulp = np.exp2(np.floor(np.log2(np.maximum(np.abs(b), 2.0 ** -126))) - 7)
     assert np.all(np.abs(a - b) <= np.maximum(ulp, 2.0 ** -21))
     assert np.mean(ours == theirs) >= 0.99
+
+
+def test_identities_of_the_branch_free_form():
+    """The arithmetic facts the GPU's form of the same operations rests on,
+    checked in IEEE fp32 (numpy): 2/d == 2 RN(1/d) for the divisors e + 1 in
+    [2, e^18 + 1] (whole binades exhaustively, the rest sampled), and the
+    integer read from the bits of 1.5 * 2^23 + v is rne(v) on [-128, 127]."""
+    two, one = np.float32(2.0), np.float32(1.0)
+    for lo in (2.0, 4.0, float(2 ** 25)):
+        d = np.arange(np.float32(lo).view(np.int32), np.float32(2 * lo).view(np.int32),
+                      dtype=np.int32).view(np.float32)
+        assert np.array_equal(two / d, two * (one / d))
+    rng = np.random.default_rng(7)
+    d = np.exp(rng.uniform(np.log(2.0), np.log(math.exp(18) + 1), 2_000_000)).astype(np.float32)
+    assert np.array_equal(two / d, two * (one / d))
+    # rne on [-128, 127] by the bits of 1.5 * 2^23 + v: every half and a dense grid
+    v = np.concatenate([np.arange(-256, 255, dtype=np.float32) / np.float32(2),
+                        _grid(-128.0, 127.0, 1_000_001)])
+    q = (v + np.float32(12582912.0)).view(np.int32) - 0x4B400000
+    assert np.array_equal(q, np.rint(v).astype(np.int32))
+    # the capped exponent and selected 1 give the same tanh as the branch
+    u = _grid(-30.0, 30.0, 600001)
+    a = np.abs(u)
+    e = oracle.gelu_parts(np.float32(2.0) * np.minimum(a, np.float32(9.0)))["exp"]
+    t = np.where(a < 9.0, one - two * (one / (e + one)), one).astype(np.float32)
+    t = np.where(u < 0.0, -t, t)
+    assert np.array_equal(t, oracle.gelu_parts(u)["tanh"])
