@@ -73,3 +73,29 @@ def test_host_path_empty_batch_is_noop():
     B.sq_dualscale_seglinear_host(pl, x, None, g["s_act"], g["wq"], g["s_w"], None, y, seg)
     torch.cuda.synchronize()
     pl.close()
+
+
+def test_host_calls_on_two_streams_do_not_race_on_the_workspace():
+    """Two calls on one pipeline, each on its own stream, with no ordering
+    between the streams: the second call's first chunks reuse the workspace
+    slots the first call's last chunks used, and must wait for them.  Both
+    outputs must still equal the device path's bit for bit."""
+    La = wl.gelu_layer("race_a", 700, 416, 520, seed=41, bias=True)
+    Lb = wl.gelu_layer("race_b", 700, 416, 520, seed=42, bias=True)
+    ga, gb = gpu_run(La), gpu_run(Lb)
+    seg = segments(La)
+    pl = B.HostPipeline(64, La.K, La.N)
+    outs = []
+    streams = [torch.cuda.Stream(), torch.cuda.Stream()]
+    for L, g, st in ((La, ga, streams[0]), (Lb, gb, streams[1])):
+        x_host = L.x.contiguous().pin_memory()
+        y_host = torch.full((L.M, L.N), float("nan"), dtype=torch.float32).pin_memory()
+        with torch.cuda.stream(st):
+            B.sq_dualscale_seglinear_host(pl, x_host, None, g["s_act"], g["wq"], g["s_w"],
+                                          L.bias.cuda(), y_host, seg)
+        outs.append((x_host, y_host))
+    torch.cuda.synchronize()
+    assert B.sq_get_device_status() == 0
+    pl.close()
+    assert torch.equal(outs[0][1], ga["y"].cpu())
+    assert torch.equal(outs[1][1], gb["y"].cpu())

@@ -183,15 +183,18 @@ sq_status sq_dualscale_seglinear_host(sq_host_pipeline *pl, const void *x_host, 
     uint8_t *x_dev = pl->slot[s] + pl->x_off;
     int8_t *planes_dev = reinterpret_cast<int8_t *>(pl->slot[s] + pl->planes_off);
     uint8_t *y_dev = pl->slot[s] + pl->y_off;
-    // The slot's previous chunk (c - 2) must have been quantized before its
-    // rows are overwritten, and copied out before its planes and output are.
-    if (c >= 2 && !cu(cudaStreamWaitEvent(pl->s_in, pl->ev_comp[s], 0))) return fail(SQ_ERR_CUDA);
+    // The slot's previous chunk -- chunk c - 2 of this call, or the last chunk
+    // an earlier call ran in this slot, whichever stream that call was given --
+    // must have been quantized before its rows are overwritten, and copied out
+    // before its planes and output are.  Waiting on an event that was never
+    // recorded (a fresh pipeline) returns at once.
+    if (!cu(cudaStreamWaitEvent(pl->s_in, pl->ev_comp[s], 0))) return fail(SQ_ERR_CUDA);
     if (!cu(cudaMemcpy2DAsync(x_dev, K * 2, static_cast<const uint8_t *>(x_host) + r0 * ldx * 2,
                               ldx * 2, K * 2, rows, cudaMemcpyHostToDevice, pl->s_in)) ||
         !cu(cudaEventRecord(pl->ev_in[s], pl->s_in)) ||
         !cu(cudaStreamWaitEvent(pl->s_comp, pl->ev_in[s], 0)))
       return fail(SQ_ERR_CUDA);
-    if (c >= 2 && !cu(cudaStreamWaitEvent(pl->s_comp, pl->ev_out[s], 0))) return fail(SQ_ERR_CUDA);
+    if (!cu(cudaStreamWaitEvent(pl->s_comp, pl->ev_out[s], 0))) return fail(SQ_ERR_CUDA);
     sq_stream_t comp = reinterpret_cast<sq_stream_t>(pl->s_comp);
     sq_status st = sq_quantize_act(x_dev, rows, K, K, d, s_act, seg, planes_dev, comp);
     if (st != SQ_OK) return fail(st);
