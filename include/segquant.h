@@ -23,7 +23,9 @@
  * Conventions for every call:
  *  - Every pointer is a DEVICE pointer unless marked "host".  The caller owns
  *    all buffers, workspaces included; the library allocates no device memory
- *    in any call.
+ *    in any call.  (The one exception to caller-owned memory is the fixed
+ *    scratch array of sq_dualscale_seglinear_host_noalloc, which is part of
+ *    the library's device image.)
  *  - Calls are asynchronous on `stream` (0 = legacy default stream).  A return
  *    of SQ_OK means the arguments were valid and the kernels were launched;
  *    launch failures return SQ_ERR_CUDA.  Faults inside a kernel surface at
@@ -63,7 +65,8 @@ typedef enum {
   SQ_ERR_OVERFLOW = -4,      /* a K-segment could overflow the int32 sum     */
   SQ_ERR_CUDA = -5,          /* a CUDA runtime call failed                    */
   SQ_ERR_DEVICE_TIMEOUT = -6,/* a kernel gave up waiting (see status call)    */
-  SQ_ERR_NO_DEVICE = -7      /* no sm_100 device is current                   */
+  SQ_ERR_NO_DEVICE = -7,     /* no sm_100 device is current                   */
+  SQ_ERR_TOO_LARGE = -8      /* one row does not fit a fixed-size scratch     */
 } sq_status;
 
 typedef enum {
@@ -348,6 +351,68 @@ SQ_API sq_status sq_dualscale_seglinear_host(sq_host_pipeline *pl, const void *x
                                       const float *s_w, const void *bias, void *y_host,
                                       sq_out_dtype out_dtype, int64_t N, int64_t ldy,
                                       const sq_segments *seg, sq_stream_t stream);
+
+/*
+ * sq_dualscale_seglinear_host_noalloc -- the host-to-host layer of
+ * sq_dualscale_seglinear_host for callers that cannot allocate device memory.
+ * (The pages have no counterpart: this is deployment plumbing, not part of the
+ * method.)
+ *
+ * Who needs it: a library that is loaded into a host application which owns
+ * the device-memory budget (a plug-in of an inference server, an embedded
+ * runtime) is often not allowed to call cudaMalloc at all; a latency-critical
+ * loop cannot afford cudaMalloc and cudaFree, which may synchronise the whole
+ * device and stall every other stream; and a process already at the edge of
+ * the device's memory cannot count on an allocation succeeding in the middle
+ * of its work.  Such callers cannot provide the workspace that
+ * sq_host_pipeline_create needs.
+ *
+ * This call needs none.  Its device scratch is one fixed array of
+ * SQ_NOALLOC_SCRATCH_BYTES (32 MiB) inside the library's device image: every
+ * GPU on which the library is loaded holds it until the process exits.  The
+ * call itself calls no cudaMalloc, cudaFree or other allocating routine, and
+ * it creates no streams or events.
+ *
+ * Arguments and results are those of sq_dualscale_seglinear_host without the
+ * pipeline: x_host (bf16 [M][ldx]) and y_host ([M][ldy], bf16 or fp32) are
+ * HOST pointers (page-locked or pageable), the other pointers are device
+ * buffers the caller owns, and the output equals the device calls
+ * sq_quantize_act + sq_dualscale_seglinear_gemm on the whole layer bit for
+ * bit.  Rows are processed in chunks as large as the scratch allows (a
+ * multiple of 128 rows when at least 128 fit), all on `stream`, one after the
+ * other: copy in, quantize, GEMM, copy out.  Nothing overlaps, so it is slower
+ * than a pipeline, and work enqueued on `stream` afterwards waits for the
+ * whole layer.
+ *
+ * Limit: one row's x (2K bytes), planes (G*P*K bytes) and output (4 bytes per
+ * column, N rounded up to a multiple of 8), each region rounded up to 256
+ * bytes, must fit in SQ_NOALLOC_SCRATCH_BYTES; otherwise the call returns
+ * SQ_ERR_TOO_LARGE and enqueues nothing.  Other errors as in
+ * sq_dualscale_seglinear_host; after a failure past the first enqueue the call
+ * waits for `stream` before it returns.
+ *
+ * Sharing: every call on a device uses the same scratch, and the scratch keeps
+ * whatever the last call left in it.  Nothing in it has to start at zero:
+ * each chunk's rows, planes and output are written in full before they are
+ * read.  Calls that can overlap on the GPU -- calls on different streams, or
+ * from several host threads, without an ordering between them -- race on the
+ * scratch and corrupt each other's results; order them on one stream (or with
+ * events).
+ *
+ * First call: the first call on each device looks up the scratch's device
+ * address (cudaGetSymbolAddress), which may load the library's device code on
+ * that device.  Make that first call before any stream capture begins.
+ */
+#define SQ_NOALLOC_SCRATCH_BYTES (32u * 1024u * 1024u)
+
+SQ_API sq_status sq_dualscale_seglinear_host_noalloc(const void *x_host, int64_t M, int64_t K,
+                                                     int64_t ldx, const float *d,
+                                                     const float *s_act, const int8_t *wq,
+                                                     const float *s_w, const void *bias,
+                                                     void *y_host, sq_out_dtype out_dtype,
+                                                     int64_t N, int64_t ldy,
+                                                     const sq_segments *seg,
+                                                     sq_stream_t stream);
 
 /*
  * sq_debug_timeout_probe -- test only: launches one small kernel that waits on

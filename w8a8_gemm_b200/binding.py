@@ -32,7 +32,9 @@ EXPORTED = ("sq_calibrate_act", "sq_quantize_act", "sq_quantize_weight_seg",
             "sq_debug_gemm_s32", "sq_get_device_status",
             "sq_status_string", "sq_version", "sq_debug_timeout_probe",
             "sq_host_pipeline_workspace_bytes", "sq_host_pipeline_create",
-            "sq_host_pipeline_destroy", "sq_dualscale_seglinear_host")
+            "sq_host_pipeline_destroy", "sq_dualscale_seglinear_host",
+            "sq_dualscale_seglinear_host_noalloc")
+SQ_NOALLOC_SCRATCH_BYTES = 32 * 1024 * 1024
 
 
 class SegQuantError(RuntimeError):
@@ -117,12 +119,15 @@ def lib() -> ctypes.CDLL:
         L.sq_host_pipeline_destroy.argtypes = [p]
         L.sq_dualscale_seglinear_host.argtypes = [p, p, i64, i64, i64, p, p, p, p, p, p,
                                                   ctypes.c_int, i64, i64, seg, p]
+        L.sq_dualscale_seglinear_host_noalloc.argtypes = [p, i64, i64, i64, p, p, p, p, p, p,
+                                                          ctypes.c_int, i64, i64, seg, p]
         L.sq_status_string.argtypes = [ctypes.c_int]
         L.sq_status_string.restype = ctypes.c_char_p
         L.sq_version.argtypes = []
         for f in (L.sq_calibrate_act, L.sq_quantize_act, L.sq_quantize_weight_seg,
                   L.sq_quantize_weight_w4, L.sq_unpack_weight_w4, L.sq_host_pipeline_create,
                   L.sq_host_pipeline_destroy, L.sq_dualscale_seglinear_host,
+                  L.sq_dualscale_seglinear_host_noalloc,
                   L.sq_dualscale_seglinear_gemm, L.sq_dualscale_seglinear_gemm_gelu_quant,
                   L.sq_debug_gemm_s32, L.sq_get_device_status,
                   L.sq_version, L.sq_debug_timeout_probe):
@@ -367,6 +372,38 @@ def sq_dualscale_seglinear_host(pl: HostPipeline, x_host: torch.Tensor, d: Optio
                                              _ptr(wq), _ptr(s_w), _ptr(bias), _ptr(y_host), out,
                                              N, y_host.stride(0), ctypes.byref(cs), _stream()),
            "sq_dualscale_seglinear_host")
+    return y_host
+
+
+def sq_dualscale_seglinear_host_noalloc(x_host: torch.Tensor, d: Optional[torch.Tensor],
+                                        s_act: torch.Tensor, wq: torch.Tensor,
+                                        s_w: torch.Tensor, bias: Optional[torch.Tensor],
+                                        y_host: torch.Tensor, seg: Segments) -> torch.Tensor:
+    """The layer of sq_dualscale_seglinear_host without a pipeline or a
+    workspace: for callers that may not allocate device memory.  The library's
+    fixed device scratch (SQ_NOALLOC_SCRATCH_BYTES) holds the chunks; every
+    call on a device shares it, so calls must not overlap on the GPU.  Ordered
+    on torch's current stream."""
+    if x_host.is_cuda or y_host.is_cuda:
+        raise ValueError("x_host and y_host must be CPU tensors")
+    if x_host.dtype != torch.bfloat16 or y_host.dtype not in (torch.bfloat16, torch.float32):
+        raise ValueError("x_host must be bf16 and y_host bf16 or fp32")
+    _need(d, torch.float32, "d", optional=True)
+    _need(s_act, torch.float32, "s_act")
+    _need(wq, torch.int8, "wq")
+    _need(s_w, torch.float32, "s_w")
+    _need(bias, torch.bfloat16, "bias", optional=True)
+    M, K, ldx = _rows(x_host)
+    N = wq.shape[0]
+    if wq.shape[1] != K or y_host.shape[0] != M or y_host.shape[1] != N or y_host.stride(1) != 1:
+        raise ValueError("shape mismatch between x_host [M,K], wq [N,K] and y_host [M,N]")
+    out = SQ_OUT_BF16 if y_host.dtype == torch.bfloat16 else SQ_OUT_F32
+    cs, keep = seg._c()
+    _check(lib().sq_dualscale_seglinear_host_noalloc(_ptr(x_host), M, K, ldx, _ptr(d),
+                                                     _ptr(s_act), _ptr(wq), _ptr(s_w), _ptr(bias),
+                                                     _ptr(y_host), out, N, y_host.stride(0),
+                                                     ctypes.byref(cs), _stream()),
+           "sq_dualscale_seglinear_host_noalloc")
     return y_host
 
 

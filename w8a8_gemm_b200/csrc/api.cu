@@ -370,6 +370,7 @@ const char *sq_status_string(sq_status s) {
     case SQ_ERR_CUDA: return "SQ_ERR_CUDA: a CUDA runtime call failed";
     case SQ_ERR_DEVICE_TIMEOUT: return "SQ_ERR_DEVICE_TIMEOUT: a kernel gave up waiting on a barrier";
     case SQ_ERR_NO_DEVICE: return "SQ_ERR_NO_DEVICE: no sm_100 device is current";
+    case SQ_ERR_TOO_LARGE: return "SQ_ERR_TOO_LARGE: one row does not fit the fixed scratch";
   }
   return "unknown sq_status";
 }

@@ -6,6 +6,7 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <mutex>
 #include <new>
 
 #include "sq_internal.h"
@@ -56,6 +57,53 @@ void release(sq_host_pipeline *pl) {
   for (cudaStream_t *st : ss)
     if (*st) cudaStreamDestroy(*st);
   delete pl;
+}
+
+// ---- fixed scratch of sq_dualscale_seglinear_host_noalloc -----------------
+// One statically sized buffer in the library's device image: every device that
+// loads the library holds it until the process exits, and every call of the
+// no-allocation entry point on that device shares it.  Host code must not use
+// the symbol itself as a pointer (on the host it names a stand-in, not device
+// memory); its device address is looked up once per device.
+__device__ __align__(256) uint8_t g_noalloc_scratch[SQ_NOALLOC_SCRATCH_BYTES];
+
+constexpr int kMaxDevices = 64;
+
+// Device address of g_noalloc_scratch on the current device, or nullptr.
+uint8_t *noalloc_scratch() {
+  static uint8_t *addr[kMaxDevices] = {};
+  static std::mutex mu;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+    cudaGetLastError();
+    return nullptr;
+  }
+  std::lock_guard<std::mutex> lock(mu);
+  if (addr[dev] == nullptr) {
+    void *p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) {
+      cudaGetLastError();
+      return nullptr;
+    }
+    addr[dev] = static_cast<uint8_t *>(p);
+  }
+  return addr[dev];
+}
+
+// Most rows per chunk whose x rows, planes and output rows fit the scratch
+// together (the slot layout of the pipelines), at most M; 0 if not one row fits.
+int64_t noalloc_chunk_rows(int64_t M, int64_t K, int64_t N, int32_t G, int32_t P) {
+  size_t x_off, planes_off, y_off, slot_bytes;
+  const int64_t n_pad = (N + 7) / 8 * 8;
+  const int64_t per_row = 2 * K + static_cast<int64_t>(G) * P * K + 4 * n_pad;
+  int64_t rows = static_cast<int64_t>(SQ_NOALLOC_SCRATCH_BYTES) / per_row;
+  if (rows >= 128) rows = rows / 128 * 128;  // whole GEMM row tiles
+  if (rows > M) rows = M;
+  // each region is rounded up to 256 bytes: step down until the slot fits
+  while (rows > 0 && (!slot_layout(rows, K, N, G, P, &x_off, &planes_off, &y_off, &slot_bytes) ||
+                      slot_bytes > SQ_NOALLOC_SCRATCH_BYTES))
+    --rows;
+  return rows;
 }
 
 }  // namespace
@@ -211,6 +259,69 @@ sq_status sq_dualscale_seglinear_host(sq_host_pipeline *pl, const void *x_host, 
   if (!cu(cudaEventRecord(pl->ev_done, pl->s_out)) ||
       !cu(cudaStreamWaitEvent(user, pl->ev_done, 0)))
     return fail(SQ_ERR_CUDA);
+  return SQ_OK;
+}
+
+sq_status sq_dualscale_seglinear_host_noalloc(const void *x_host, int64_t M, int64_t K,
+                                              int64_t ldx, const float *d, const float *s_act,
+                                              const int8_t *wq, const float *s_w,
+                                              const void *bias, void *y_host,
+                                              sq_out_dtype out_dtype, int64_t N, int64_t ldy,
+                                              const sq_segments *seg, sq_stream_t stream) {
+  if (out_dtype != SQ_OUT_BF16 && out_dtype != SQ_OUT_F32) return SQ_ERR_INVALID_ARG;
+  if (M < 0 || M > INT32_MAX || K < 16 || K % 16 != 0 || K > INT32_MAX || N < 1 ||
+      N > INT32_MAX || ldx < K || ldy < N)
+    return SQ_ERR_INVALID_ARG;
+  const int32_t G = seg ? seg->n_groups : 1;
+  const int32_t P = (seg && (seg->flags & SQ_FLAG_SINGLE_SCALE)) ? 1 : 2;
+  if (G < 1 || G > SQ_MAX_SEGMENTS) return SQ_ERR_INVALID_ARG;
+  // One row of x, its planes and its output must fit the fixed scratch.
+  const int64_t chunk = noalloc_chunk_rows(M > 0 ? M : 1, K, N, G, P);
+  if (chunk < 1) return SQ_ERR_TOO_LARGE;
+  if (M == 0) return SQ_OK;
+  if (x_host == nullptr || y_host == nullptr) return SQ_ERR_INVALID_ARG;
+  uint8_t *scratch = noalloc_scratch();
+  if (scratch == nullptr) return SQ_ERR_CUDA;
+  size_t x_off, planes_off, y_off, slot_bytes;
+  if (!slot_layout(chunk, K, N, G, P, &x_off, &planes_off, &y_off, &slot_bytes))
+    return SQ_ERR_INVALID_ARG;
+  uint8_t *x_dev = scratch + x_off;
+  int8_t *planes_dev = reinterpret_cast<int8_t *>(scratch + planes_off);
+  uint8_t *y_dev = scratch + y_off;
+  const size_t elem = out_dtype == SQ_OUT_BF16 ? 2 : 4;
+  const int64_t n_pad = (N + 7) / 8 * 8;
+  // Every check of the device calls, before anything is enqueued: chunks
+  // differ only in their row count.
+  sq_status st = validate_quantize_act(x_dev, chunk, K, K, d, s_act, seg, planes_dev);
+  if (st != SQ_OK) return st;
+  st = validate_gemm(planes_dev, wq, s_w, s_act, bias, y_dev,
+                     out_dtype == SQ_OUT_BF16 ? OUT_BF16 : OUT_F32, chunk, N, K, n_pad, seg);
+  if (st != SQ_OK) return st;
+  cudaStream_t user = reinterpret_cast<cudaStream_t>(stream);
+  // After a failure past the first enqueue, wait for the caller's stream, so
+  // that no copy or kernel of this call is still in flight on return.
+  auto fail = [user](sq_status code) {
+    cudaStreamSynchronize(user);
+    return code;
+  };
+  // Everything runs on the caller's stream, chunk after chunk through the one
+  // scratch region: a chunk's rows are copied in only after the previous
+  // chunk's output has been copied out.
+  for (int64_t r0 = 0; r0 < M; r0 += chunk) {
+    const int64_t rows = (M - r0) < chunk ? (M - r0) : chunk;
+    if (cudaMemcpy2DAsync(x_dev, K * 2, static_cast<const uint8_t *>(x_host) + r0 * ldx * 2,
+                          ldx * 2, K * 2, rows, cudaMemcpyHostToDevice, user) != cudaSuccess)
+      return fail(SQ_ERR_CUDA);
+    st = sq_quantize_act(x_dev, rows, K, K, d, s_act, seg, planes_dev, stream);
+    if (st != SQ_OK) return fail(st);
+    st = sq_dualscale_seglinear_gemm(planes_dev, wq, s_w, s_act, bias, y_dev, out_dtype, rows, N,
+                                     K, n_pad, seg, stream);
+    if (st != SQ_OK) return fail(st);
+    if (cudaMemcpy2DAsync(static_cast<uint8_t *>(y_host) + r0 * ldy * elem, ldy * elem, y_dev,
+                          n_pad * elem, N * elem, rows, cudaMemcpyDeviceToHost,
+                          user) != cudaSuccess)
+      return fail(SQ_ERR_CUDA);
+  }
   return SQ_OK;
 }
 
