@@ -29,9 +29,12 @@
  *    s+ = max/127.  X^- lies in [-128, 0], X^+ in [0, 127].
  *  - "round" is round-half-to-even, in fp32.
  *  - The SmoothQuant divisor d (per group, per input channel, > 0) is an input.
- *    Activations are quantized as x / d, weights as w * d.  The quantizer
- *    multiplies by a folded reciprocal: t = fl(d * s), m = fl(1 / t),
- *    v = fl(x * m), q = rne(clamp(v)).  Both sides take this decision in fp32.
+ *    Activations are quantized as x / d, weights as w * d.  The quantizer is
+ *    the pages' round(u / s) evaluated in fp32 with IEEE divisions: the
+ *    smoothed activation u = fl(x / d) (u = x when there is no divisor), the
+ *    quotient v = fl(u / s+-), then q = rne(clamp(v)).  Where v itself lands
+ *    on a half-integer, the tie goes to the even code, even if the exact
+ *    quotient u / s lay on one side of it.
  *  - Out-of-range values saturate: q+ <= 127, q- >= -128.  NaN goes to 0 in
  *    both planes (neither x < 0 nor x >= 0 holds); -0.0 goes to the + plane.
  *  - Degenerate calibration: max <= 0 gives s+ = 1, min >= 0 gives s- = 1; an
@@ -171,7 +174,10 @@ int orc_calibrate_act(const uint16_t *x, int64_t M, int64_t K, int64_t ldx,
 }
 
 /* ---------------------------------------------------------------------------
- * DualScale activation quantization (Q_dual) with SmoothQuant divisor.
+ * DualScale activation quantization (Q_dual) with SmoothQuant divisor:
+ * author page section 3, Q_dual(x) = round(x/s-) for x < 0 and round(x/s+)
+ * for x >= 0, applied to the smoothed activation u = x / d.  Both quotients
+ * are fp32 IEEE divisions; the clamps are the int8 code range.
  * ------------------------------------------------------------------------- */
 int orc_quantize_act(const uint16_t *x, int64_t M, int64_t K, int64_t ldx,
                      const float *d, const float *s_act, int mode, int n_seg,
@@ -188,17 +194,15 @@ int orc_quantize_act(const uint16_t *x, int64_t M, int64_t K, int64_t ldx,
         int i = (S == 1) ? 0 : orc_seg_index(offsets, n_seg, c);
         float sp = s_act[((int64_t)g * S + i) * 2 + 0];
         float sm = s_act[((int64_t)g * S + i) * 2 + 1];
-        float dv = d ? d[(int64_t)g * K + c] : 1.0f;
-        float mp = 1.0f / (dv * sp); /* folded reciprocal, two fp32 ops */
-        float mm = 1.0f / (dv * sm);
         float xv = orc_bf16(x[m * ldx + c]);
+        float u = d ? xv / d[(int64_t)g * K + c] : xv; /* smoothed activation */
         int qp = 0, qm = 0;
-        if (xv < 0.0f) { /* X- branch: round(x / s-) */
-          float v = xv * mm;
+        if (xv < 0.0f) { /* X- branch: round(u / s-) */
+          float v = u / sm;
           if (v < -128.0f) v = -128.0f;
           qm = (int)rintf(v);
-        } else if (xv >= 0.0f) { /* X+ branch: round(x / s+) */
-          float v = xv * mp;
+        } else if (xv >= 0.0f) { /* X+ branch: round(u / s+) */
+          float v = u / sp;
           if (v > 127.0f) v = 127.0f;
           qp = (int)rintf(v);
         }
@@ -462,9 +466,10 @@ int orc_calibrate_act_fp8(const uint16_t *x, int64_t M, int64_t K, int64_t ldx,
   return 0;
 }
 
-/* Planes of E4M3 codes [G][P][M][K].  x >= 0 (-0.0 included): the + plane
- * holds e4m3(fl(x * m+)) and the - plane 0x00; x < 0: the - plane holds
- * e4m3(fl(x * m-)) and the + plane 0x00; NaN: both 0x00.  Single scale: one
+/* Planes of E4M3 codes [G][P][M][K], with u = fl(x / d) and fp32 IEEE
+ * divisions as in orc_quantize_act.  x >= 0 (-0.0 included): the + plane
+ * holds e4m3(fl(u / s+)) and the - plane 0x00; x < 0: the - plane holds
+ * e4m3(fl(u / s-)) and the + plane 0x00; NaN: both 0x00.  Single scale: one
  * plane holding the code of whichever branch applies. */
 int orc_quantize_act_fp8(const uint16_t *x, int64_t M, int64_t K, int64_t ldx,
                          const float *d, const float *s_act, int mode, int n_seg,
@@ -481,15 +486,13 @@ int orc_quantize_act_fp8(const uint16_t *x, int64_t M, int64_t K, int64_t ldx,
         int i = (S == 1) ? 0 : orc_seg_index(offsets, n_seg, c);
         float sp = s_act[((int64_t)g * S + i) * 2 + 0];
         float sm = s_act[((int64_t)g * S + i) * 2 + 1];
-        float dv = d ? d[(int64_t)g * K + c] : 1.0f;
-        float mp = 1.0f / (dv * sp);
-        float mm = 1.0f / (dv * sm);
         float xv = orc_bf16(x[m * ldx + c]);
+        float u = d ? xv / d[(int64_t)g * K + c] : xv;
         uint8_t qp = 0, qm = 0;
         if (xv < 0.0f)
-          qm = orc_e4m3_code(xv * mm);
+          qm = orc_e4m3_code(u / sm);
         else if (xv >= 0.0f)
-          qp = orc_e4m3_code(xv * mp);
+          qp = orc_e4m3_code(u / sp);
         if (single) {
           plus[m * K + c] = (xv < 0.0f) ? qm : qp;
         } else {
