@@ -235,7 +235,7 @@ def run_ours(args, ws, rank, local):
     torch.cuda.set_device(dev)
     from w8a8_gemm_b200 import binding as B
     B.lib()  # fail loudly now if the library is missing
-    layers_cpu = wl.config_layers(args.config, seed=0)
+    layers_cpu = wl.config_layers(args.config, seed=0, G_output=args.g_output)
     # W4A8: every layer keeps packed weights and expands them into one shared
     # int8 operand buffer before its GEMM (inside the timed GEMM region).
     w_operand = (torch.empty(max(L.N * L.K for L in layers_cpu), dtype=torch.int8, device=dev)
@@ -466,6 +466,9 @@ def main(argv=None):
                     help="FP8 E4M3 codes for activations and weights (tcgen05 kind::f8f6f4)")
     ap.add_argument("--adaptive", action="store_true",
                     help="single-scale path on layers whose calibrated sides differ by < 2x")
+    ap.add_argument("--g-output", type=int, default=None, choices=[1],
+                    help="1: output-segmented layers share one activation group (one X^, the "
+                         "pages' output-segmented formula) instead of one group per segment")
     ap.add_argument("--fused-gelu", action="store_true",
                     help="FFN pairs: fc1's GEMM applies the GELU and writes fc2's activation "
                          "planes (the fused producer); fc2 runs no quantize kernel")
@@ -474,7 +477,8 @@ def main(argv=None):
         ap.error("--warmup must be >= 3")
     if args.fused_gelu and args.fp8:
         ap.error("--fused-gelu takes int8 codes, not --fp8")
-    if args.fused_gelu and not ffn_pairs(wl.config_layers(args.config, seed=0)):
+    if args.fused_gelu and not ffn_pairs(wl.config_layers(args.config, seed=0,
+                                                          G_output=args.g_output)):
         ap.error(f"--fused-gelu: no FFN pair in {args.config}")
     ws, rank, local = dist_env()
     n_gpus = max(args.gpus, ws)
@@ -547,6 +551,10 @@ def main(argv=None):
                                "each GEMM (counted in the GEMM time)"
                                if args.weight_bits == 4 else
                                "FP8 E4M3 activations and weights" if args.fp8 else "W8A8"),
+                   "activation_groups": ("G = 1 on output-segmented layers (one shared X^)"
+                                         if args.g_output == 1 else
+                                         "one group per output segment (G = n_seg) where "
+                                         "the workload has output segments"),
                    "output": "bf16",
                    "producer": ("fused: fc1's epilogue writes fc2's planes of "
                                 "bf16(gelu(bf16(y1))), no fc2 quantize kernel"
@@ -603,7 +611,7 @@ def main_reference(args, ws, rank):
     if rank != 0:
         return 0
     import oracle
-    layers = wl.config_layers(args.config, seed=0)
+    layers = wl.config_layers(args.config, seed=0, G_output=args.g_output)
     thr = oracle.num_threads()
     prepared = prepare_oracle(layers)
     pairs = ffn_pairs(layers) if args.fused_gelu else []

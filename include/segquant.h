@@ -112,9 +112,10 @@ typedef enum { SQ_OUT_BF16 = 0, SQ_OUT_F32 = 1 } sq_out_dtype;
  * sign, 4 exponent bits with bias 7, 3 mantissa bits, largest finite 448, no
  * infinities, 0x7F/0xFF NaN), stored as its bit pattern in the int8 buffers.
  * Calibration: s+ = max/448 and s- = |min|/448 (single scale: the larger side
- * / 448).  Quantization: x >= 0 -> X^+ = e4m3(fl(x*m+)), X^- = 0x00; x < 0 ->
- * X^- = e4m3(fl(x*m-)), X^+ = 0x00; NaN -> both 0x00; e4m3() rounds half to
- * even and saturates finite values to +-448.  Weights: s_w = amax/448,
+ * / 448).  Quantization, with u = fl(x / d) as for int8: x >= 0 -> X^+ =
+ * e4m3(fl(u / s+)), X^- = 0x00; x < 0 -> X^- = e4m3(fl(u / s-)), X^+ = 0x00;
+ * NaN -> both 0x00; e4m3() rounds half to even and saturates finite values to
+ * +-448.  Weights: s_w = amax/448,
  * W^ = e4m3(fl(w'/s_w)).  GEMM: tcgen05 kind::f8f6f4 with fp32 accumulation
  * (exact products; sums in the tensor core's fp32, order unspecified), the
  * W8A8 epilogue on the fp32 sums.  Not combinable with SQ_FLAG_W4.
@@ -164,14 +165,17 @@ SQ_API sq_status sq_calibrate_act(const void *x, int64_t M, int64_t K, int64_t l
  * sq_quantize_act -- DualScale activation quantization (the HBM-bound step).
  * Pages: author page section 3 (Q_dual), papernotes.org section DualScale.
  * For every element x (bf16, exact in fp32) of channel c in K-segment i and
- * every group g:
- *   m+ = 1/(d[g][c]*s+[g][i]), m- = 1/(d[g][c]*s-[g][i])   (fp32, each op RN)
- *   x >= 0: X^+ = rne(min(x*m+, 127)),  X^- = 0
- *   x <  0: X^- = rne(max(x*m-, -128)), X^+ = 0
- *   NaN   : both 0.   (-0.0 counts as x >= 0; rne = round half to even.)
+ * every group g, with the smoothed activation u = fl(x / d[g][c]) (u = x when
+ * d is NULL) and the quotients rounded to fp32 (IEEE division):
+ *   x >= 0: X^+ = rne(min(fl(u / s+[g][i]), 127)),  X^- = 0
+ *   x <  0: X^- = rne(max(fl(u / s-[g][i]), -128)), X^+ = 0
+ *   NaN   : both 0.   (-0.0 counts as x >= 0; rne = round half to even, so a
+ *   quotient that is itself a half-integer goes to the even code.)
+ * The kernel forms each quotient from the rounded reciprocal with one FMA
+ * correction, which gives the IEEE quotient exactly under these bounds:
  *   x      bf16 [M][ldx], constraints as in sq_calibrate_act
- *   d      fp32 [G][K] or NULL;  s_act fp32 [G][S][2] (positive, finite, with
- *          d*s a normal float)
+ *   d      fp32 [G][K] or NULL;  s_act fp32 [G][S][2]; every d and s finite
+ *          and within [2^-40, 2^40] (codes are unspecified otherwise)
  *   planes int8 [G][2][M][K] output, 16-byte aligned
  * With SQ_FLAG_SINGLE_SCALE the two codes of an element are written as their
  * sum, one plane per group: planes int8 [G][1][M][K].
@@ -266,14 +270,14 @@ SQ_API sq_status sq_dualscale_seglinear_gemm(const int8_t *planes, const int8_t 
  * evaluated here as one fixed sequence of fp32 operations: tanh from e^(2|u|)
  * by Cody and Waite's reduction and a degree-7 Taylor series, 1 for |u| >= 9).
  * The next layer's codes follow sq_quantize_act with d = 1 and its steps
- * s_act_next = {s+, s-}: m+- = fl(1/s+-), x2 >= 0: q+ = rne(min(x2 m+, 127)),
- * x2 < 0: q- = rne(max(x2 m-, -128)).  Its planes never round-trip through a
- * bf16 activation in HBM.
+ * s_act_next = {s+, s-}: x2 >= 0: q+ = rne(min(fl(x2 / s+), 127)),
+ * x2 < 0: q- = rne(max(fl(x2 / s-), -128)).  Its planes never round-trip
+ * through a bf16 activation in HBM.
  *   planes, wq, s_w, s_act, bias, M, N, K, seg: as in
  *          sq_dualscale_seglinear_gemm; seg must be SQ_SEG_NONE (one K-segment,
  *          one group) and not SQ_FLAG_FP8 (SQ_ERR_UNSUPPORTED otherwise)
  *   s_act_next fp32 [2] device {s+, s-} of the next layer (one group, one
- *          K-segment, no SmoothQuant divisor), positive and finite
+ *          K-segment, no SmoothQuant divisor), within [2^-40, 2^40]
  *   flags_next 0 (DualScale: planes_next int8 [2][M][N]) or
  *          SQ_FLAG_SINGLE_SCALE (one merged plane [1][M][N])
  *   planes_next int8 output, 16-byte aligned; N % 16 == 0 (it is the next

@@ -79,6 +79,42 @@ def test_every_bf16_value_quantizes_like_oracle():
     assert np.array_equal(planes.cpu().numpy(), ref)
 
 
+_NP2_STEPS = [(float.fromhex("0x1.fd0eb8p-8"), float.fromhex("0x1.0adc5p-7")),
+              (float.fromhex("0x1.945622p-6"), float.fromhex("0x1.0624dcp-8")),
+              (float.fromhex("0x1.1cf06ap-8"), float.fromhex("0x1.fffffep-6")),
+              (0.0123457, 0.000731), (0.2718, 0.0031416), (0.00057, 0.0419)]
+
+
+@pytest.mark.parametrize("fp8", [False, True])
+@pytest.mark.parametrize("single", [False, True])
+@pytest.mark.parametrize("with_d", [False, True])
+def test_every_bf16_value_at_non_power_of_two_steps(with_d, single, fp8):
+    """Every bf16 pattern at steps that are not powers of two, where the form of
+    the quotient decides the code: the kernel's corrected reciprocal must give
+    the oracle's rne(fl(fl(x/d)/s)) (FP8: e4m3(fl(fl(x/d)/s))) bit for bit.
+    With a divisor, every one of the 256 channels has its own d."""
+    allbits = np.arange(65536, dtype=np.uint32).astype(np.uint16).reshape(256, 256)
+    x = torch.from_numpy(allbits.view(np.int16)).view(torch.bfloat16).cuda()
+    d = None
+    if with_d:
+        d = np.exp(np.random.default_rng(5).uniform(-4, 4, (1, 256))).astype(np.float32)
+        d[0, :4] = [3.0, 2.5, 0.7071068, 1.0]
+    P = 1 if single else 2
+    flags = (B.SQ_FLAG_SINGLE_SCALE if single else 0) | (B.SQ_FLAG_FP8 if fp8 else 0)
+    for sp, sm in _NP2_STEPS:
+        if single:
+            sm = sp
+        s_act = np.array([[[sp, sm]]], np.float32)
+        if fp8:
+            ref = oracle.quantize_act_fp8(allbits, s_act, d=d, single=single).view(np.int8)
+        else:
+            ref = oracle.quantize_act(allbits, s_act, d=d, single=single)
+        planes = torch.empty(1, P, 256, 256, dtype=torch.int8, device="cuda")
+        B.sq_quantize_act(x, None if d is None else torch.from_numpy(d).cuda(),
+                          torch.from_numpy(s_act).cuda(), B.Segments(flags=flags), planes)
+        assert np.array_equal(planes.cpu().numpy(), ref), (sp, sm)
+
+
 @pytest.mark.parametrize("kind", ["positive", "negative", "zero", "nan_and_inf", "mixed"])
 def test_calibration_degenerate_slices_on_gpu(kind):
     """AMax calibration on the GPU equals the oracle's, bit for bit, including
@@ -164,7 +200,7 @@ def test_input_segments_sum_on_gpu():
 
 
 FULL = ["c1_tiny_dualscale", "c2_sd35_adanorm", "c3_sd35_attn_out", "c4_sd35_ffn",
-        "c5_flux_block"]
+        "c5_flux_block", "c5_flux_adanorm_m2"]
 
 
 @pytest.mark.parametrize("cfg", FULL)
@@ -185,6 +221,49 @@ def test_full_size_configs_sampled_rows(cfg):
         gf = gpu_run(L, out_dtype=torch.float32)
         assert np.array_equal(gf["y"][torch.from_numpy(rows).cuda()].cpu().numpy(), r)
         del g, gf
+        torch.cuda.empty_cache()
+
+
+@pytest.mark.parametrize("cfg", ["c2_sd35_adanorm", "c5_flux_block", "c5_flux_adanorm_m2"])
+def test_full_size_shared_activation_group(cfg):
+    """The output-segmented layers with one shared activation group (G = 1,
+    one X^ for every output segment, the pages' output-segmented formula) at
+    full size: planes in full, int32 accumulators and outputs on the sampled
+    rows."""
+    for L in wl.config_layers(cfg, seed=0, G_output=1):
+        if L.mode != wl.MODE_OUTPUT:
+            continue
+        assert L.G == 1
+        prep = oracle_prep(L)
+        g = gpu_run(L, out_dtype=torch.float32, s32=True)
+        assert np.array_equal(g["s_act"].cpu().numpy(), prep["s_act"])
+        assert np.array_equal(g["wq"].cpu().numpy(), prep["wq"])
+        assert np.array_equal(g["planes"].cpu().numpy(), prep["planes"])
+        rows = sample_rows(L.M)
+        idx = torch.from_numpy(rows).cuda()
+        assert np.array_equal(g["acc"][:, :, idx].cpu().numpy(), oracle_acc(L, prep, rows=rows))
+        assert np.array_equal(g["y"][idx].cpu().numpy(), oracle_y(L, prep, rows=rows))
+        del g
+        torch.cuda.empty_cache()
+
+
+@pytest.mark.parametrize("cfg", FULL)
+def test_full_size_int32_accumulators_sampled_rows(cfg):
+    """The raw int32 accumulators of every full-size workload layer, per
+    K-segment and polarity, against the oracle's int32 products on the sampled
+    rows: above 2^24 the fp32 output rounds the accumulator, so an off-by-one
+    there could hide behind an output that still matches (K = 6144 allows
+    |A| up to 128 * 127 * 6144, about 10^8)."""
+    for L in wl.config_layers(cfg, seed=0):
+        prep = oracle_prep(L)
+        g = gpu_run(L, out_dtype=torch.float32, s32=True)
+        assert np.array_equal(g["planes"].cpu().numpy(), prep["planes"])
+        rows = sample_rows(L.M)
+        ref = oracle_acc(L, prep, rows=rows)
+        got = g["acc"][:, :, torch.from_numpy(rows).cuda()].cpu().numpy()
+        assert got.shape == ref.shape
+        assert np.array_equal(got, ref), L.name
+        del g
         torch.cuda.empty_cache()
 
 

@@ -174,16 +174,24 @@ __device__ __forceinline__ float gelu_tanh(float x) {
   return __fmul_rn(__fmul_rn(0.5f, x), __fadd_rn(1.0f, t));
 }
 
-// DualScale codes of the next layer's input x2 = bf16(gelu(bf16(y))), with its
-// folded multipliers m+- = 1/s+-: x2 >= 0 gives q+ = rne(min(x2 m+, 127)),
-// x2 < 0 gives q- = rne(max(x2 m-, -128)); the other code is 0.
-__device__ __forceinline__ void gelu_codes(float y, float mp, float mm, int &qp, int &qm) {
+// DualScale codes of the next layer's input x2 = bf16(gelu(bf16(y))), the
+// activation quantizer's rule with d = 1: x2 >= 0 gives q+ = rne(min(fl(x2/s+),
+// 127)), x2 < 0 gives q- = rne(max(fl(x2/s-), -128)); the other code is 0.  The
+// quotient is the correctly rounded one, formed from r = fl(1/s) by
+// Markstein's correction: q0 = fl(x2 r), then fl(q0 + (x2 - q0 s) r).  Where
+// x2 r overflows, the correction yields NaN, and fminf / fmaxf return the
+// clamp bound: the saturated code.
+__device__ __forceinline__ void gelu_codes(float y, float sp, float rp, float sm, float rm,
+                                           int &qp, int &qm) {
   const float xb = __bfloat162float(__float2bfloat16_rn(y));
   const float x2 = __bfloat162float(__float2bfloat16_rn(gelu_tanh(xb)));
   // rne of a value in [-128, 127]: the integer part of the bits of
   // 1.5 * 2^23 + v, where the add rounds to the nearest integer, ties to even.
   const bool neg = x2 < 0.0f;
-  const float v = neg ? fmaxf(__fmul_rn(x2, mm), -128.0f) : fminf(__fmul_rn(x2, mp), 127.0f);
+  const float s = neg ? sm : sp, r = neg ? rm : rp;
+  const float q0 = __fmul_rn(x2, r);
+  const float quot = __fmaf_rn(__fmaf_rn(-q0, s, x2), r, q0);
+  const float v = neg ? fmaxf(quot, -128.0f) : fminf(quot, 127.0f);
   const int q = __float_as_int(__fadd_rn(v, 12582912.0f)) - 0x4B400000;
   qp = neg ? 0 : q;
   qm = neg ? q : 0;
@@ -407,11 +415,13 @@ __global__ void __launch_bounds__(threads_for(EPI_WARPS), 1)
     float *cst_base = reinterpret_cast<float *>(smem + L::EPI_OFFSET) + ew * L::CONST_FLOATS;
     uint8_t *stg = smem + L::STG_OFFSET + ew * 2048;  // used when TMA_STORE
     uint32_t acc_iter = 0;
-    // OUT_PLANES: the next layer's folded multipliers m+- = fl(1/s+-).
-    float mp_next = 0.0f, mm_next = 0.0f;
+    // OUT_PLANES: the next layer's steps s+- and their reciprocals fl(1/s+-).
+    float sp_nx = 1.0f, rp_nx = 1.0f, sm_nx = 1.0f, rm_nx = 1.0f;
     if constexpr (OUT == OUT_PLANES) {
-      mp_next = __fdiv_rn(1.0f, p.s_next[0]);
-      mm_next = __fdiv_rn(1.0f, p.s_next[1]);
+      sp_nx = p.s_next[0];
+      sm_nx = p.s_next[1];
+      rp_nx = __frcp_rn(sp_nx);
+      rm_nx = __frcp_rn(sm_nx);
     }
     for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x) {
       const int mt = tile / p.num_n_tiles, nt = tile % p.num_n_tiles;
@@ -555,8 +565,8 @@ __global__ void __launch_bounds__(threads_for(EPI_WARPS), 1)
                     // Two 32 x 32-byte staging blocks (X^+ then X^-), row-major:
                     // columns 8j + 2q and 8j + 2q + 1 as one 16-bit store each.
                     int qp0, qm0, qp1, qm1;
-                    gelu_codes(y0, mp_next, mm_next, qp0, qm0);
-                    gelu_codes(y1, mp_next, mm_next, qp1, qm1);
+                    gelu_codes(y0, sp_nx, rp_nx, sm_nx, rm_nx, qp0, qm0);
+                    gelu_codes(y1, sp_nx, rp_nx, sm_nx, rm_nx, qp1, qm1);
                     uint16_t *dst = reinterpret_cast<uint16_t *>(stg + rr * 32 + 8 * j + 2 * q);
                     if (p.p_next == 2) {
                       dst[0] = static_cast<uint16_t>((qp0 & 0xFF) | ((qp1 & 0xFF) << 8));

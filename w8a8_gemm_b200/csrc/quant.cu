@@ -98,10 +98,56 @@ __global__ void calib_finalize_kernel(float *s_act, int n, int single, int fp8) 
 }
 
 // ---------------------------------------------------- activation quantize
+// The codes are round(u / s) with u = fl(x / d) and the quotients rounded to
+// fp32 first (IEEE division), then to an integer (half to even).  A quotient
+// a / b is formed without a divide: with r = fl(1/b), q0 = fl(a r) is within
+// an ulp of a / b, the residual a - q0 b is exact in one FMA, and
+// fl(q0 + (a - q0 b) r) is the correctly rounded quotient (Markstein's
+// correction, "Computation of elementary functions on the IBM RISC System/6000
+// processor", IBM J. Res. Dev. 34(1), 1990).  The identity holds for every
+// bf16 dividend and every fp32 divisor significand (checked exhaustively on
+// the CPU) and for fp32 dividends (sampled); it needs dividend, divisor and
+// residual away from the ends of the fp32 range, hence the bounds on d and s
+// in the library's header.
+
 // sat(a * b) clamped to [0, 1]; NaN gives +0.
 __device__ __forceinline__ float mul_sat(float a, float b) {
   float r;
   asm("fma.rn.sat.f32 %0, %1, %2, 0f00000000;" : "=f"(r) : "f"(a), "f"(b));
+  return r;
+}
+__device__ __forceinline__ float fma_sat(float a, float b, float c) {
+  float r;
+  asm("fma.rn.sat.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+__device__ __forceinline__ uint64_t pack2(float a, float b) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+  return r;
+}
+__device__ __forceinline__ void unpack2(uint64_t v, float &a, float &b) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(v));
+}
+__device__ __forceinline__ uint64_t ffma2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t fmul2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+// min / max that keep a NaN operand (the plain forms return the other one)
+__device__ __forceinline__ float min_nan(float a, float b) {
+  float r;
+  asm("min.NaN.f32 %0, %1, %2;" : "=f"(r) : "f"(a), "f"(b));
+  return r;
+}
+__device__ __forceinline__ float max_nan(float a, float b) {
+  float r;
+  asm("max.NaN.f32 %0, %1, %2;" : "=f"(r) : "f"(a), "f"(b));
   return r;
 }
 
@@ -113,55 +159,102 @@ __device__ __forceinline__ uint32_t pack4_lo(uint32_t a, uint32_t b, uint32_t c,
 // Bit patterns of fl(1.5 * 2^23 + k * u0) and fl(1.5 * 2^23 + k * u1), one packed
 // FMA (f32x2) for both; the low byte of each is rne(k * u) for |k u| <= 128.
 __device__ __forceinline__ void round2(float u0, float u1, float k, uint32_t &r0, uint32_t &r1) {
-  uint64_t a, b, c, d;
-  asm("mov.b64 %0, {%1, %2};" : "=l"(a) : "f"(u0), "f"(u1));
-  asm("mov.b64 %0, {%1, %1};" : "=l"(b) : "f"(k));
-  asm("mov.b64 %0, {%1, %1};" : "=l"(c) : "f"(12582912.0f));
-  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  const uint64_t d = ffma2(pack2(u0, u1), pack2(k, k), pack2(12582912.0f, 12582912.0f));
   asm("mov.b64 {%0, %1}, %2;" : "=r"(r0), "=r"(r1) : "l"(d));
 }
 
-// Eight channels x of one row -> X^+ and X^- codes, 8 bytes each, with the
-// multipliers pre-scaled by 2^-7: p7 = m+ / 128, n7 = -m- / 128.
-//   u+ = sat(x * p7) = clamp(fl(x * m+), 0, 128) / 128   (power-of-two scaling
-//        commutes with rounding, so this is exact; x < 0 and NaN give 0)
-//   q+ = rne(128 u+): the FP add of 1.5 * 2^23 rounds to nearest even and the
-//        code is the low byte of the sum's bits; 128 is then lowered to 127.
-//   u- = sat(x * n7) = clamp(-fl(x * m-), 0, 128) / 128, q- = -rne(128 u-).
-// This is the case-wise Q_dual with the reference's clamps: x >= 0 (including
-// -0.0) gives a code in [0, 127] and none in X^-, x < 0 the reverse, NaN 0.
-__device__ __forceinline__ void dualscale8(const float (&x)[8], const float (&p7)[8],
-                                           const float (&n7)[8], uint2 &plus, uint2 &minus) {
+// Per-thread constants of the current (group, column block): the thread's
+// eight channels share one K-segment (segment widths are multiples of 32), so
+// one step pair serves them all; the divisors are per channel.
+//   int8: r7p = fl(1/s+)/128, m128p = -128 s+; r7m = -fl(1/s-)/128, m128m = 128 s-
+//   FP8:  r7p = fl(1/s+), m128p = -s+, lim_p = 1024 s+; the same with s-.
+//   nd = -d, rd = fl(1/d), ld = the overflow clamp min(FLT_MAX/2 * d, FLT_MAX)
+//   (HAS_D only).
+struct StepConsts {
+  float r7p, m128p, r7m, m128m, lim_p, lim_m;
+  float nd[8], rd[8], ld[8];
+};
+
+// u = fl(x / d) for eight channels (HAS_D), Markstein's correction in packed
+// FMAs.  x is first clamped to +-min(FLT_MAX/2 * d, FLT_MAX) so that no step
+// overflows (the clamp keeps NaN; a clamped value's code saturates, like the
+// value's own).
+__device__ __forceinline__ void smooth8(float (&x)[8], const StepConsts &k) {
+#pragma unroll
+  for (int j = 0; j < 8; j += 2) {
+    const float x0 = max_nan(min_nan(x[j], k.ld[j]), -k.ld[j]);
+    const float x1 = max_nan(min_nan(x[j + 1], k.ld[j + 1]), -k.ld[j + 1]);
+    const uint64_t xx = pack2(x0, x1), rd = pack2(k.rd[j], k.rd[j + 1]);
+    const uint64_t q0 = fmul2(xx, rd);
+    const uint64_t e = ffma2(q0, pack2(k.nd[j], k.nd[j + 1]), xx);  // x - q0 d, exact
+    unpack2(ffma2(e, rd, q0), x[j], x[j + 1]);
+  }
+}
+
+// sat(fl(u / s) / 128) for two channels of one polarity, everything scaled by
+// 2^-7 (exact) so that .sat clamps to the code range: q0 = sat(u fl(1/s)/128)
+// (x on the other side of zero, NaN and overflow all clamp), the residual
+// u - q0 * 128 s in one packed FMA, then v = sat(q0 + e fl(1/s)/128).  For the
+// - plane r7 and the residual's factor carry the other sign, so that v is
+// sat(fl(-u / s-) / 128) for u < 0 and 0 otherwise.
+__device__ __forceinline__ void quot2_sat(float u0, float u1, float r7, float m128, float &v0,
+                                          float &v1) {
+  const float a0 = mul_sat(u0, r7), a1 = mul_sat(u1, r7);
+  float e0, e1;
+  unpack2(ffma2(pack2(a0, a1), pack2(m128, m128), pack2(u0, u1)), e0, e1);
+  v0 = fma_sat(e0, r7, a0);
+  v1 = fma_sat(e1, r7, a1);
+}
+
+// Eight channels u of one row -> X^+ and X^- codes, 8 bytes each:
+//   q+ = rne(128 v+), v+ = sat(fl(u / s+) / 128): the FP add of 1.5 * 2^23
+//        rounds to nearest even and the code is the low byte of the sum's
+//        bits; 128 is then lowered to 127 with a byte-wise unsigned min;
+//   q- = -rne(128 v-), v- = sat(fl(-u / s-) / 128), codes in [-128, 0].
+// This is the case-wise Q_dual with the reference's clamps: u >= 0 (including
+// -0.0) gives a code in [0, 127] and none in X^-, u < 0 the reverse, NaN 0.
+__device__ __forceinline__ void dualscale8(const float (&u)[8], const StepConsts &k,
+                                           uint2 &plus, uint2 &minus) {
   uint32_t qp[8], qm[8];
 #pragma unroll
   for (int j = 0; j < 8; j += 2) {
-    // rne(128 u) + 1.5 * 2^23 for two channels per packed FMA
-    round2(mul_sat(x[j], p7[j]), mul_sat(x[j + 1], p7[j + 1]), 128.0f, qp[j], qp[j + 1]);
-    round2(mul_sat(x[j], n7[j]), mul_sat(x[j + 1], n7[j + 1]), -128.0f, qm[j], qm[j + 1]);
+    float vp0, vp1, vm0, vm1;
+    quot2_sat(u[j], u[j + 1], k.r7p, k.m128p, vp0, vp1);
+    quot2_sat(u[j], u[j + 1], k.r7m, k.m128m, vm0, vm1);
+    round2(vp0, vp1, 128.0f, qp[j], qp[j + 1]);
+    round2(vm0, vm1, -128.0f, qm[j], qm[j + 1]);
   }
   plus = make_uint2(__vminu4(pack4_lo(qp[0], qp[1], qp[2], qp[3]), 0x7F7F7F7Fu),
                     __vminu4(pack4_lo(qp[4], qp[5], qp[6], qp[7]), 0x7F7F7F7Fu));
   minus = make_uint2(pack4_lo(qm[0], qm[1], qm[2], qm[3]), pack4_lo(qm[4], qm[5], qm[6], qm[7]));
 }
 
-// FP8 (E4M3) codes of eight channels, with the multipliers m+ and m- as they
-// are (no 2^-7 pre-scaling): v = fl(x * m), code = e4m3(v), round half to even
-// with saturation to +-448 (the CUDA conversion intrinsics).  x >= 0 (-0.0
-// included) fills the + plane, x < 0 the - plane, NaN neither.
+// FP8 (E4M3) codes of eight channels: v = fl(u / s) by the same correction
+// (unscaled), code = e4m3(v), round half to even with saturation to +-448 (the
+// CUDA conversion intrinsics).  u is clamped to 1024 s on its own side first
+// (beyond that the code saturates anyway), which keeps every step finite.
+// x >= 0 (-0.0 included) fills the + plane, x < 0 the - plane, NaN neither;
+// the branch that does not apply converts +0.0, whose code is 0x00.  The
+// quotient takes the sign of x, which the correction loses for x = -0.0.
 __device__ __forceinline__ uint32_t e4m3x4(float a, float b, float c, float d) {
   const uint32_t lo = __nv_cvt_float2_to_fp8x2(make_float2(a, b), __NV_SATFINITE, __NV_E4M3);
   const uint32_t hi = __nv_cvt_float2_to_fp8x2(make_float2(c, d), __NV_SATFINITE, __NV_E4M3);
   return lo | (hi << 16);
 }
 
-__device__ __forceinline__ void dualscale8_fp8(const float (&x)[8], const float (&mp)[8],
-                                               const float (&mm)[8], uint2 &plus, uint2 &minus) {
-  // The branch that does not apply converts +0.0, whose code is 0x00.
+__device__ __forceinline__ float quot_fp8(float u, float x, float r, float ms) {
+  const float q0 = __fmul_rn(u, r);
+  const float v = __fmaf_rn(__fmaf_rn(q0, ms, u), r, q0);
+  return __int_as_float(__float_as_int(v) | (__float_as_int(x) & 0x80000000));
+}
+
+__device__ __forceinline__ void dualscale8_fp8(const float (&x)[8], const float (&u)[8],
+                                               const StepConsts &k, uint2 &plus, uint2 &minus) {
   float vp[8], vm[8];
 #pragma unroll
   for (int j = 0; j < 8; ++j) {
-    vp[j] = x[j] >= 0.0f ? __fmul_rn(x[j], mp[j]) : 0.0f;
-    vm[j] = x[j] < 0.0f ? __fmul_rn(x[j], mm[j]) : 0.0f;
+    vp[j] = x[j] >= 0.0f ? quot_fp8(min_nan(u[j], k.lim_p), x[j], k.r7p, k.m128p) : 0.0f;
+    vm[j] = x[j] < 0.0f ? quot_fp8(max_nan(u[j], -k.lim_m), x[j], k.r7m, k.m128m) : 0.0f;
   }
   plus = make_uint2(e4m3x4(vp[0], vp[1], vp[2], vp[3]), e4m3x4(vp[4], vp[5], vp[6], vp[7]));
   minus = make_uint2(e4m3x4(vm[0], vm[1], vm[2], vm[3]), e4m3x4(vm[4], vm[5], vm[6], vm[7]));
@@ -170,39 +263,56 @@ __device__ __forceinline__ void dualscale8_fp8(const float (&x)[8], const float 
 // Work unit = one activation group g and one tile of 32 rows x 256 channels.
 // Units are numbered group-major, then column block, then row tile, and every
 // block takes one contiguous range of them: the grid is balanced to within one
-// unit, and a block changes (group, column block) -- and recomputes its eight
-// channels' folded multipliers m+- = 1/(d*s+-), kept in registers as m+/128 and
-// -m-/128 (see dualscale8) -- at most a few times.  With G > 1 every group
+// unit, and a block changes (group, column block) -- and recomputes its
+// constants (StepConsts) -- at most a few times.  With G > 1 every group
 // re-reads the same X tiles, which stay resident in L2 between the passes.
 // Thread 0 keeps kQStages tiles in flight with 2D TMA copies into shared
 // memory; every warp then takes whole rows of the staged tile (lane = 8
 // channels, one conflict-free 16-byte shared load) and writes 8 bytes per plane
 // per row, 256 contiguous bytes per warp.
-// FP8 keeps m+ and m- unscaled in p7 and n7.  fetch_scales reads the inputs
-// of one (group, column block) into registers (s+, s- in sc[0..1], the eight
-// divisors in p7) and fold_multipliers turns them into the multipliers, so
-// that the reads can be issued ahead of the first tile copies.
+// fetch_scales reads the inputs of one (group, column block) into registers
+// (s+, s- in sc[0..1], the eight divisors in dv) and fold_consts turns them
+// into StepConsts, so that the reads can be issued ahead of the first tile
+// copies.
+template <bool HAS_D>
 __device__ __forceinline__ void fetch_scales(int g, int64_t c0, int64_t K, const float *d,
                                              const float *s_act, const SegParams &seg,
-                                             float (&sc)[2], float (&p7)[8]) {
+                                             float (&sc)[2], float (&dv)[8]) {
   if (c0 >= K) return;
   const int i = (seg.mode == SQ_SEG_INPUT) ? seg_index(seg.off, seg.n_seg, c0) : 0;
   sc[0] = s_act[(g * seg.S + i) * 2 + 0];
   sc[1] = s_act[(g * seg.S + i) * 2 + 1];
+  if constexpr (HAS_D) {
 #pragma unroll
-  for (int j = 0; j < 8; ++j) p7[j] = d ? d[g * K + c0 + j] : 1.0f;
+    for (int j = 0; j < 8; ++j) dv[j] = d[g * K + c0 + j];
+  }
 }
-template <bool FP8>
-__device__ __forceinline__ void fold_multipliers(int64_t c0, int64_t K, const float (&sc)[2],
-                                                 float (&p7)[8], float (&n7)[8]) {
+template <bool FP8, bool HAS_D>
+__device__ __forceinline__ void fold_consts(int64_t c0, int64_t K, const float (&sc)[2],
+                                            const float (&dv)[8], StepConsts &k) {
   if (c0 >= K) return;
+  const float rp = __frcp_rn(sc[0]), rm = __frcp_rn(sc[1]);
+  if constexpr (FP8) {
+    k.r7p = rp;
+    k.m128p = -sc[0];
+    k.r7m = rm;
+    k.m128m = -sc[1];
+    k.lim_p = 1024.0f * sc[0];
+    k.lim_m = 1024.0f * sc[1];
+  } else {
+    k.r7p = rp * 0.0078125f;
+    k.m128p = -128.0f * sc[0];
+    k.r7m = rm * -0.0078125f;
+    k.m128m = 128.0f * sc[1];
+  }
+  if constexpr (HAS_D) {
 #pragma unroll
-  for (int j = 0; j < 8; ++j) {
-    const float dv = p7[j];
-    const float mp = __fdiv_rn(1.0f, __fmul_rn(dv, sc[0]));
-    const float mm = __fdiv_rn(1.0f, __fmul_rn(dv, sc[1]));
-    p7[j] = FP8 ? mp : mp * 0.0078125f;
-    n7[j] = FP8 ? mm : mm * -0.0078125f;
+    for (int j = 0; j < 8; ++j) {
+      k.nd[j] = -dv[j];
+      k.rd[j] = __frcp_rn(dv[j]);
+      // min(FLT_MAX / 2 * d, FLT_MAX): no overflow in x fl(1/d), +-inf clamped
+      k.ld[j] = fminf(__fmul_rn(1.7014117e38f, dv[j]), 3.4028235e38f);
+    }
   }
 }
 
@@ -227,7 +337,7 @@ struct UnitCursor {
   }
 };
 
-template <bool FP8>
+template <bool FP8, bool HAS_D>
 __global__ void __launch_bounds__(256, 3) quant_act_kernel(const __grid_constant__ CUtensorMap tmX,
                                                            int64_t M, int64_t K,
                                                            const float *__restrict__ d,
@@ -256,10 +366,11 @@ __global__ void __launch_bounds__(256, 3) quant_act_kernel(const __grid_constant
   // these small reads do not queue behind the whole grid's tile traffic.
   UnitCursor cur;
   cur.set(u_begin, n_cb, n_rt);
-  float sc[2], p7[8], n7[8];
+  float sc[2], dv[8];
+  StepConsts kc;
   if (n_mine > 0)
-    fetch_scales(cur.g, static_cast<int64_t>(cur.cb) * kWarpCols + lane * kColsPerThread, K, d,
-                 s_act, seg, sc, p7);
+    fetch_scales<HAS_D>(cur.g, static_cast<int64_t>(cur.cb) * kWarpCols + lane * kColsPerThread,
+                        K, d, s_act, seg, sc, dv);
   if (tid == 0) {
     fetch.set(u_begin, n_cb, n_rt);
     for (int st = 0; st < kQStages && st < n_mine; ++st) {
@@ -271,17 +382,17 @@ __global__ void __launch_bounds__(256, 3) quant_act_kernel(const __grid_constant
   }
   __syncthreads();  // barriers initialised
   if (n_mine > 0)
-    fold_multipliers<FP8>(static_cast<int64_t>(cur.cb) * kWarpCols + lane * kColsPerThread, K, sc,
-                          p7, n7);
-  int key_g = cur.g, key_cb = cur.cb;  // (group, column block) of the multipliers held
+    fold_consts<FP8, HAS_D>(static_cast<int64_t>(cur.cb) * kWarpCols + lane * kColsPerThread, K,
+                            sc, dv, kc);
+  int key_g = cur.g, key_cb = cur.cb;  // (group, column block) of the constants held
   const int64_t plane_stride = M * K;
   for (int it = 0; it < n_mine; ++it, cur.next(n_cb, n_rt)) {
     const int64_t c0 = static_cast<int64_t>(cur.cb) * kWarpCols + lane * kColsPerThread;
     if (cur.g != key_g || cur.cb != key_cb) {
       key_g = cur.g;
       key_cb = cur.cb;
-      fetch_scales(cur.g, c0, K, d, s_act, seg, sc, p7);
-      fold_multipliers<FP8>(c0, K, sc, p7, n7);
+      fetch_scales<HAS_D>(cur.g, c0, K, d, s_act, seg, sc, dv);
+      fold_consts<FP8, HAS_D>(c0, K, sc, dv, kc);
     }
     const int st = it % kQStages;
     if (!mbar_wait(&full[st], (it / kQStages) & 1, kQuantWaitNs)) {
@@ -300,10 +411,16 @@ __global__ void __launch_bounds__(256, 3) quant_act_kernel(const __grid_constant
         float xv[8];
         unpack8(v, xv);
         uint2 pk, nk;
-        if constexpr (FP8)
-          dualscale8_fp8(xv, p7, n7, pk, nk);
-        else
-          dualscale8(xv, p7, n7, pk, nk);
+        if constexpr (FP8) {
+          float uv[8];
+#pragma unroll
+          for (int j = 0; j < 8; ++j) uv[j] = xv[j];
+          if constexpr (HAS_D) smooth8(uv, kc);
+          dualscale8_fp8(xv, uv, kc, pk, nk);
+        } else {
+          if constexpr (HAS_D) smooth8(xv, kc);  // the sign of x survives in u
+          dualscale8(xv, kc, pk, nk);
+        }
         if (seg.P == 2) {
           *reinterpret_cast<uint2 *>(plus + r * K) = pk;
           *reinterpret_cast<uint2 *>(plus + plane_stride + r * K) = nk;
@@ -463,7 +580,8 @@ sq_status launch_quantize_act(const uint16_t *x, int64_t M, int64_t K, int64_t l
   int64_t nblk = static_cast<int64_t>(num_sms()) * 3;
   if (nblk > n_units) nblk = n_units;
   const size_t smem = kQStages * kQTileBytes + kQStages * sizeof(uint64_t);
-  auto kernel = seg.fp8 ? quant_act_kernel<true> : quant_act_kernel<false>;
+  auto kernel = seg.fp8 ? (d ? quant_act_kernel<true, true> : quant_act_kernel<true, false>)
+                        : (d ? quant_act_kernel<false, true> : quant_act_kernel<false, false>);
   if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(smem)) != cudaSuccess)
     return SQ_ERR_CUDA;

@@ -245,6 +245,8 @@ CONFIGS = {
     "c3_sd35_attn_out": "SD3.5-medium attention out-projection [8858x1536] x W [1536x1536], 24 input segments",
     "c4_sd35_ffn": "SD3.5-medium FFN pair [8858x1536]->[6144]->[1536], one segment each",
     "c5_flux_block": "FLUX DiT block linears at M=9216: AdaNorm, QKV, out-proj, fc1, fc2",
+    "c5_flux_adanorm_m2": "FLUX AdaNorm at its real batch M=2: SiLU(t_emb) [2x3072] x W "
+                          "[3072x18432], 6 output segments (a latency point)",
 }
 
 
@@ -265,4 +267,6 @@ def config_layers(name: str, seed: int = 0, G_output: Optional[int] = None) -> L
                 qkv_layer("c5_qkv", M, 3072, 9216, 3, seed + 1, G=G_output),
                 outproj_layer("c5_attn_out", M, 3072, 3072, 128, seed + 2),
                 *ffn_pair("c5_", M, 3072, 12288, seed + 3)]
+    if name == "c5_flux_adanorm_m2":
+        return [adanorm_layer("c5_adanorm_m2", 2, 3072, 18432, 6, seed, G=G_output)]
     raise KeyError(f"unknown configuration {name!r}; known: {sorted(CONFIGS)}")
