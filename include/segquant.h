@@ -431,12 +431,43 @@ SQ_API sq_status sq_dualscale_seglinear_host_noalloc(const void *x_host, int64_t
 SQ_API sq_status sq_debug_timeout_probe(uint32_t limit_us, sq_stream_t stream);
 
 /*
- * sq_get_device_status -- synchronises the current device, then returns and
- * clears the library's device-side error word: SQ_OK, or
+ * sq_get_device_status -- waits for the work enqueued on `stream`, then
+ * returns the library's device-side error word and clears it: SQ_OK, or
  * SQ_ERR_DEVICE_TIMEOUT if a kernel's bounded wait on a barrier ran out (the
  * kernel then abandoned its tile and left its outputs incomplete).
+ * The word is one per device, shared by every stream and every caller of the
+ * library in the process: a report set by a kernel on another stream is seen
+ * (and cleared) by whichever caller reads first, and a report set between
+ * this call's read and its clear is lost.  Callers that launch on several
+ * streams should synchronise those streams, or serialise their status checks,
+ * before relying on the result.  Synchronises only `stream` (0: the legacy
+ * default stream, which also waits for the other blocking streams).
  */
-SQ_API sq_status sq_get_device_status(void);
+SQ_API sq_status sq_get_device_status(sq_stream_t stream);
+
+/*
+ * sq_choose_single_scale -- the adaptive DualScale policy, on the host: decides
+ * whether a layer should use the single-scale path (SQ_FLAG_SINGLE_SCALE).
+ * Pages: papernotes.org "SegQuant", section "Limitations" (DualScale doubles
+ * the integer work; enable it only where activations are strongly
+ * polarity-asymmetric).  The pages fix no test; the reading taken: for every
+ * group and K-segment recover the calibrated max = s+ * 127 and
+ * |min| = s- * 128 (FP8: both * 448) from the DualScale steps; the layer
+ * switches to single scale when, in every group and K-segment, the larger side
+ * is below threshold times the smaller (fp32 arithmetic).  A side that was
+ * empty in calibration has step 1 and so counts as a large side: such layers
+ * keep DualScale.  After a decision of 1 the caller re-runs sq_calibrate_act
+ * with SQ_FLAG_SINGLE_SCALE and uses that flag on every call of the layer.
+ *   s_act    HOST fp32 [n_steps][2] {s+, s-}: the steps of sq_calibrate_act
+ *            without SQ_FLAG_SINGLE_SCALE, copied to the host; positive, finite
+ *   n_steps  G * S, 1..SQ_MAX_SEGMENTS^2
+ *   flags    0 or SQ_FLAG_FP8 (which code range the steps belong to)
+ *   threshold > 1 (2 in the library's own layer helper)
+ *   single   HOST int32 output: 1 (use single scale) or 0 (keep DualScale)
+ * Touches no device and launches nothing.
+ */
+SQ_API sq_status sq_choose_single_scale(const float *s_act, int32_t n_steps, int32_t flags,
+                                        float threshold, int32_t *single);
 
 /* Static, human-readable name of a status code (never NULL). */
 SQ_API const char *sq_status_string(sq_status status);

@@ -5,6 +5,8 @@ import ctypes
 import os
 import re
 
+import numpy as np
+
 import pytest
 
 from w8a8_gemm_b200 import binding as B
@@ -41,9 +43,9 @@ def test_library_exports_every_declared_symbol(L):
 
 def test_status_strings(L):
     assert B.status_string(0) == "SQ_OK"
-    for code in range(-7, 0):
+    for code in range(-8, 0):
         assert B.status_string(code).startswith("SQ_ERR_")
-    assert B.lib().sq_version() == 103
+    assert B.lib().sq_version() == 200
 
 
 def _seg(mode, offsets, groups=1):
@@ -232,3 +234,55 @@ def test_gelu_quant_validation(L):
     assert f(p(FAKE), p(FAKE), p(FAKE), p(FAKE), None, 0, 64, 64, ctypes.byref(none), p(FAKE), 0,
              p(FAKE), None) == 0
 
+
+
+def _choose(L, steps, flags=0, threshold=2.0):
+    arr = np.ascontiguousarray(np.asarray(steps, np.float32).reshape(-1, 2))
+    out = ctypes.c_int32(-1)
+    rc = L.sq_choose_single_scale(arr.ctypes.data_as(ctypes.c_void_p), arr.shape[0], flags,
+                                  ctypes.c_float(threshold), ctypes.byref(out))
+    return rc, out.value
+
+
+def test_choose_single_scale_policy(L):
+    """The adaptive policy on the host: max = s+ * 127 and |min| = s- * 128
+    (448 for FP8); single scale only where every group and K-segment has
+    max(max, |min|) < threshold * min(max, |min|)."""
+    # max 1.0, |min| 0.9: close -> single
+    assert _choose(L, [[1.0 / 127, 0.9 / 128]]) == (0, 1)
+    # max 1.0, |min| 0.3: ratio 3.3 -> keep DualScale
+    assert _choose(L, [[1.0 / 127, 0.3 / 128]]) == (0, 0)
+    # one asymmetric (group, segment) among symmetric ones keeps the layer DualScale
+    steps = [[1.0 / 127, 1.0 / 128]] * 23 + [[4.0 / 127, 1.0 / 128]]
+    assert _choose(L, steps) == (0, 0)
+    assert _choose(L, steps[:23]) == (0, 1)
+    # the threshold is strict, and it is the caller's
+    assert _choose(L, [[2.0 / 127, 1.0 / 128]], threshold=2.0) == (0, 0)
+    assert _choose(L, [[2.0 / 127, 1.0 / 128]], threshold=2.5) == (0, 1)
+    # an empty side has step 1 and counts as large: a one-sided layer keeps DualScale
+    assert _choose(L, [[0.5 / 127, 1.0]]) == (0, 0)
+    # FP8 steps are max / 448 on both sides
+    assert _choose(L, [[1.0 / 448, 0.6 / 448]], flags=B.SQ_FLAG_FP8) == (0, 1)
+    assert _choose(L, [[1.0 / 448, 0.4 / 448]], flags=B.SQ_FLAG_FP8) == (0, 0)
+
+
+def test_choose_single_scale_rejects_bad_arguments(L):
+    INVALID = -1
+    assert _choose(L, [[0.0, 0.01]])[0] == INVALID          # a step of 0
+    assert _choose(L, [[-0.01, 0.01]])[0] == INVALID        # negative
+    assert _choose(L, [[float("nan"), 0.01]])[0] == INVALID
+    assert _choose(L, [[float("inf"), 0.01]])[0] == INVALID
+    assert _choose(L, [[0.01, 0.01]], threshold=1.0)[0] == INVALID
+    assert _choose(L, [[0.01, 0.01]], flags=B.SQ_FLAG_W4)[0] == INVALID
+    out = ctypes.c_int32(0)
+    arr = np.ones(2, np.float32)
+    assert L.sq_choose_single_scale(arr.ctypes.data_as(ctypes.c_void_p), 0, 0,
+                                    ctypes.c_float(2.0), ctypes.byref(out)) == INVALID
+    assert L.sq_choose_single_scale(None, 1, 0, ctypes.c_float(2.0), ctypes.byref(out)) == INVALID
+
+
+def test_binding_choose_single_scale_takes_any_device_tensor():
+    import torch
+    s = torch.tensor([[[1.0 / 127, 0.9 / 128]], [[1.0 / 127, 0.95 / 128]]])
+    assert B.sq_choose_single_scale(s) is True
+    assert B.sq_choose_single_scale(s, threshold=1.05) is False

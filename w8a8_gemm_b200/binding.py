@@ -33,7 +33,7 @@ EXPORTED = ("sq_calibrate_act", "sq_quantize_act", "sq_quantize_weight_seg",
             "sq_status_string", "sq_version", "sq_debug_timeout_probe",
             "sq_host_pipeline_workspace_bytes", "sq_host_pipeline_create",
             "sq_host_pipeline_destroy", "sq_dualscale_seglinear_host",
-            "sq_dualscale_seglinear_host_noalloc")
+            "sq_dualscale_seglinear_host_noalloc", "sq_choose_single_scale")
 SQ_NOALLOC_SCRATCH_BYTES = 32 * 1024 * 1024
 
 
@@ -109,7 +109,9 @@ def lib() -> ctypes.CDLL:
         L.sq_dualscale_seglinear_gemm_gelu_quant.argtypes = [p, p, p, p, p, i64, i64, i64, seg,
                                                              p, ctypes.c_int32, p, p]
         L.sq_debug_gemm_s32.argtypes = [p, p, i64, i64, i64, seg, p, p]
-        L.sq_get_device_status.argtypes = []
+        L.sq_get_device_status.argtypes = [p]
+        L.sq_choose_single_scale.argtypes = [p, ctypes.c_int32, ctypes.c_int32, ctypes.c_float,
+                                             ctypes.POINTER(ctypes.c_int32)]
         L.sq_debug_timeout_probe.argtypes = [ctypes.c_uint32, p]
         L.sq_host_pipeline_workspace_bytes.argtypes = [i64, i64, i64, ctypes.c_int32,
                                                        ctypes.c_int32]
@@ -129,7 +131,7 @@ def lib() -> ctypes.CDLL:
                   L.sq_host_pipeline_destroy, L.sq_dualscale_seglinear_host,
                   L.sq_dualscale_seglinear_host_noalloc,
                   L.sq_dualscale_seglinear_gemm, L.sq_dualscale_seglinear_gemm_gelu_quant,
-                  L.sq_debug_gemm_s32, L.sq_get_device_status,
+                  L.sq_debug_gemm_s32, L.sq_get_device_status, L.sq_choose_single_scale,
                   L.sq_version, L.sq_debug_timeout_probe):
             f.restype = ctypes.c_int
         _lib = L
@@ -408,8 +410,24 @@ def sq_dualscale_seglinear_host_noalloc(x_host: torch.Tensor, d: Optional[torch.
 
 
 def sq_get_device_status() -> int:
-    """Synchronise and return (and clear) the device error word."""
-    return lib().sq_get_device_status()
+    """Wait for torch's current stream, then return (and clear) the device
+    error word (one per device, shared by all streams and callers)."""
+    return lib().sq_get_device_status(_stream())
+
+
+def sq_choose_single_scale(s_act: torch.Tensor, fp8: bool = False,
+                           threshold: float = 2.0) -> bool:
+    """The adaptive DualScale policy on a layer's calibrated DualScale steps
+    (fp32 [G][S][2], any device; copied to the host): True where every group
+    and K-segment has its larger side below threshold times the smaller."""
+    s = s_act.detach().to("cpu", torch.float32).contiguous()
+    if s.dim() < 1 or s.shape[-1] != 2:
+        raise ValueError("s_act must end in a dimension of 2 ({s+, s-})")
+    out = ctypes.c_int32(0)
+    _check(lib().sq_choose_single_scale(ctypes.c_void_p(s.data_ptr()), s.numel() // 2,
+                                        SQ_FLAG_FP8 if fp8 else 0, float(threshold),
+                                        ctypes.byref(out)), "sq_choose_single_scale")
+    return bool(out.value)
 
 
 def sq_debug_timeout_probe(limit_us: int) -> None:

@@ -347,17 +347,42 @@ sq_status sq_debug_timeout_probe(uint32_t limit_us, sq_stream_t stream) {
   return from_cuda(launch_timeout_probe(limit_us, status, reinterpret_cast<cudaStream_t>(stream)));
 }
 
-sq_status sq_get_device_status(void) {
+sq_status sq_get_device_status(sq_stream_t stream) {
   SQ_TRY(check_device());
-  if (cudaDeviceSynchronize() != cudaSuccess) return SQ_ERR_CUDA;
   int *word = device_status_word();
   if (word == nullptr) return SQ_ERR_CUDA;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  // Everything enqueued on `stream` before this call finishes first; the word
+  // is then read, and cleared only if it was set.
   int v = 0;
-  if (cudaMemcpy(&v, word, sizeof v, cudaMemcpyDeviceToHost) != cudaSuccess) return SQ_ERR_CUDA;
-  const int zero = 0;
-  if (cudaMemcpy(word, &zero, sizeof zero, cudaMemcpyHostToDevice) != cudaSuccess)
+  if (cudaMemcpyAsync(&v, word, sizeof v, cudaMemcpyDeviceToHost, st) != cudaSuccess ||
+      cudaStreamSynchronize(st) != cudaSuccess)
+    return SQ_ERR_CUDA;
+  if (v != 0 && (cudaMemsetAsync(word, 0, sizeof v, st) != cudaSuccess ||
+                 cudaStreamSynchronize(st) != cudaSuccess))
     return SQ_ERR_CUDA;
   return v == 0 ? SQ_OK : static_cast<sq_status>(v);
+}
+
+sq_status sq_choose_single_scale(const float *s_act, int32_t n_steps, int32_t flags,
+                                 float threshold, int32_t *single) {
+  if (s_act == nullptr || single == nullptr) return SQ_ERR_INVALID_ARG;
+  if (n_steps < 1 || n_steps > SQ_MAX_SEGMENTS * SQ_MAX_SEGMENTS) return SQ_ERR_INVALID_ARG;
+  if ((flags & ~SQ_FLAG_FP8) != 0) return SQ_ERR_INVALID_ARG;
+  if (!(threshold > 1.0f) || !(threshold < 3.4e38f)) return SQ_ERR_INVALID_ARG;
+  const float qp = (flags & SQ_FLAG_FP8) ? 448.0f : 127.0f;
+  const float qm = (flags & SQ_FLAG_FP8) ? 448.0f : 128.0f;
+  int32_t all_close = 1;
+  for (int32_t t = 0; t < n_steps; ++t) {
+    const float sp = s_act[2 * t], sm = s_act[2 * t + 1];
+    if (!(sp > 0.0f) || !(sm > 0.0f) || !(sp < 3.4e38f) || !(sm < 3.4e38f))
+      return SQ_ERR_INVALID_ARG;
+    const float hi = sp * qp, lo = sm * qm;  // the calibrated max and |min|
+    const float big = hi > lo ? hi : lo, small = hi > lo ? lo : hi;
+    if (!(big < threshold * small)) all_close = 0;
+  }
+  *single = all_close;
+  return SQ_OK;
 }
 
 const char *sq_status_string(sq_status s) {
@@ -375,6 +400,6 @@ const char *sq_status_string(sq_status s) {
   return "unknown sq_status";
 }
 
-int32_t sq_version(void) { return 103; }
+int32_t sq_version(void) { return 200; }
 
 }  // extern "C"

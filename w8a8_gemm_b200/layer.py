@@ -65,13 +65,11 @@ class DualScaleSegLinear:
         self.s_act = torch.empty(self.G, self.S, 2, dtype=torch.float32, device=dev)
         B.sq_calibrate_act(x_cal, d, seg, self.s_act)
         if adaptive and not seg.flags & B.SQ_FLAG_SINGLE_SCALE:
-            # Adaptive DualScale: keep the two steps only where the calibrated
-            # sides differ by at least `asymmetry_threshold` in some group and
-            # K-segment; otherwise switch the layer to one symmetric step.
-            hi = self.s_act[..., 0] * (448.0 if fp8 else 127.0)
-            lo = self.s_act[..., 1] * (448.0 if fp8 else 128.0)
-            ratio = torch.maximum(hi, lo) / torch.minimum(hi, lo).clamp_min(1e-30)
-            if float(ratio.max()) < asymmetry_threshold:
+            # Adaptive DualScale (the library's policy call): keep the two steps
+            # only where the calibrated sides differ by at least
+            # `asymmetry_threshold` in some group and K-segment; otherwise
+            # switch the layer to one symmetric step.
+            if B.sq_choose_single_scale(self.s_act, fp8=fp8, threshold=asymmetry_threshold):
                 self.seg = B.Segments(seg.mode, seg.offsets, seg.n_groups,
                                       seg.flags | B.SQ_FLAG_SINGLE_SCALE)
                 B.sq_calibrate_act(x_cal, d, self.seg, self.s_act)
