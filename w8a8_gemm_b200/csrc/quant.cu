@@ -403,7 +403,7 @@ __global__ void __launch_bounds__(256, 3) quant_act_kernel(const __grid_constant
     const int64_t r_base = static_cast<int64_t>(cur.rt) * kQRows;
     if (c0 < K) {
       int8_t *plus = planes + static_cast<int64_t>(cur.g) * seg.P * plane_stride + c0;
-#pragma unroll 2
+#pragma unroll 4
       for (int rr = warp; rr < kQRows; rr += 8) {
         const int64_t r = r_base + rr;
         if (r >= M) break;
