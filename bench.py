@@ -188,7 +188,8 @@ def traffic_from_profile():
 
 # ------------------------------------------------------------- our path
 class GpuLayer:
-    def __init__(self, L, dev, adaptive=False, weight_bits=8, w_operand=None, fp8=False):
+    def __init__(self, L, dev, adaptive=False, weight_bits=8, w_operand=None, fp8=False,
+                 workspace=None):
         from w8a8_gemm_b200 import binding as B
         from w8a8_gemm_b200.layer import DualScaleSegLinear
         self.L = L
@@ -198,7 +199,7 @@ class GpuLayer:
         bias = None if L.bias is None else L.bias.to(dev)
         self.lin = DualScaleSegLinear(L.w.to(dev), bias, d, seg, L.x_cal.to(dev),
                                       adaptive=adaptive, weight_bits=weight_bits,
-                                      w_operand=w_operand, fp8=fp8)
+                                      w_operand=w_operand, fp8=fp8, workspace=workspace)
         self.x = L.x.to(dev)
         self.planes = torch.empty(L.G, self.lin.seg.P, L.M, L.K, dtype=torch.int8, device=dev)
         self.y = torch.empty(L.M, L.N, dtype=torch.bfloat16, device=dev)
@@ -240,8 +241,12 @@ def run_ours(args, ws, rank, local):
     # int8 operand buffer before its GEMM (inside the timed GEMM region).
     w_operand = (torch.empty(max(L.N * L.K for L in layers_cpu), dtype=torch.int8, device=dev)
                  if args.weight_bits == 4 else None)
+    # --split-tail: one workspace for every layer's GEMM (they run one after
+    # another on one stream), so the last wave of tiles is shared over all SMs.
+    workspace = B.gemm_workspace(dev) if args.split_tail else None
     glayers = [GpuLayer(L, dev, adaptive=args.adaptive, weight_bits=args.weight_bits,
-                        w_operand=w_operand, fp8=args.fp8) for L in layers_cpu]
+                        w_operand=w_operand, fp8=args.fp8, workspace=workspace)
+               for L in layers_cpu]
     if args.fused_gelu:
         # FFN pairs: fc1's GEMM writes fc2's planes of bf16(gelu(bf16(y1)))
         for a, b in ffn_pairs(layers_cpu):
@@ -469,6 +474,9 @@ def main(argv=None):
     ap.add_argument("--g-output", type=int, default=None, choices=[1],
                     help="1: output-segmented layers share one activation group (one X^, the "
                          "pages' output-segmented formula) instead of one group per segment")
+    ap.add_argument("--split-tail", action="store_true",
+                    help="GEMMs with the workspace (sq_dualscale_seglinear_gemm_ws): the k-blocks "
+                         "of the last, partial wave's tiles are shared over all SMs")
     ap.add_argument("--fused-gelu", action="store_true",
                     help="FFN pairs: fc1's GEMM applies the GELU and writes fc2's activation "
                          "planes (the fused producer); fc2 runs no quantize kernel")
@@ -559,6 +567,9 @@ def main(argv=None):
                    "producer": ("fused: fc1's epilogue writes fc2's planes of "
                                 "bf16(gelu(bf16(y1))), no fc2 quantize kernel"
                                 if args.fused_gelu else "separate activation-quantize kernels"),
+                   "gemm_schedule": ("last wave's k-blocks shared over all SMs "
+                                     "(sq_dualscale_seglinear_gemm_ws)" if args.split_tail
+                                     else "whole tiles, one persistent CTA per SM"),
                    "l2": "flushed between steps, untimed: 512 MiB written, then 256 MiB read",
                    "parallelism": f"replicas x{n_gpus}"},
         "executed_tops": round(n_gpus * exe_tops_step, 2),

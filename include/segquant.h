@@ -259,6 +259,45 @@ SQ_API sq_status sq_dualscale_seglinear_gemm(const int8_t *planes, const int8_t 
                                       sq_stream_t stream);
 
 /*
+ * sq_dualscale_seglinear_gemm_ws -- sq_dualscale_seglinear_gemm with a
+ * workspace that lets one-segment layers (SQ_SEG_NONE and SQ_SEG_OUTPUT)
+ * balance their last wave of tiles.  The GEMM runs one persistent CTA per SM
+ * over 128-row tiles; when the tile count is not a multiple of the SM count,
+ * the last, partial wave would leave SMs idle.  With the workspace, every SM
+ * takes whole tiles for the full waves and an equal share of the k-blocks of
+ * the last wave's tiles: an SM whose share starts inside a tile writes its
+ * int32 partial products to the workspace, and the SM holding the tile's
+ * first k-block adds them (exact integer addition) before the same fp32
+ * epilogue, so every output is bit for bit that of sq_dualscale_seglinear_gemm.
+ * Arguments as sq_dualscale_seglinear_gemm, plus:
+ *   workspace        device memory of at least sq_gemm_workspace_bytes()
+ *                    bytes, 256-byte aligned, owned by the caller; zero-filled
+ *                    once before its first use (every call that completes
+ *                    leaves it as it must be for the next).  NULL, or fewer
+ *                    bytes, gives the whole-tile schedule.
+ *   workspace_bytes  its size.
+ * Calls that use one workspace must not overlap on the GPU (order them on one
+ * stream).  After an SQ_ERR_DEVICE_TIMEOUT report, zero-fill it again.
+ * Input-segmented layers and the fused producer take whole tiles.
+ * Cost: a split tile's partial sums are 128 KB per accumulator plane and SM,
+ * written and read back through memory; on the SD3.5 FFN layers that traffic
+ * costs more than the idle SMs of the last wave, so the plain entry point
+ * (whole tiles) is the faster one there.
+ */
+SQ_API sq_status sq_dualscale_seglinear_gemm_ws(const int8_t *planes, const int8_t *wq,
+                                                const float *s_w, const float *s_act,
+                                                const void *bias, void *y,
+                                                sq_out_dtype out_dtype, int64_t M, int64_t N,
+                                                int64_t K, int64_t ldy, const sq_segments *seg,
+                                                void *workspace, size_t workspace_bytes,
+                                                sq_stream_t stream);
+
+/* Workspace bytes for sq_dualscale_seglinear_gemm_ws and sq_debug_gemm_s32_ws
+ * on the current device (one slot of partial sums per SM, plus flags); 0 if
+ * no sm_100 device is current. */
+SQ_API size_t sq_gemm_workspace_bytes(void);
+
+/*
  * sq_dualscale_seglinear_gemm_gelu_quant -- the fused producer of an FFN's
  * second linear: the same GEMM and epilogue as sq_dualscale_seglinear_gemm,
  * but instead of y it writes the next layer's DualScale activation planes of
@@ -302,6 +341,13 @@ SQ_API sq_status sq_dualscale_seglinear_gemm_gelu_quant(const int8_t *planes, co
 SQ_API sq_status sq_debug_gemm_s32(const int8_t *planes, const int8_t *wq, int64_t M,
                             int64_t N, int64_t K, const sq_segments *seg,
                             int32_t *acc, sq_stream_t stream);
+
+/* sq_debug_gemm_s32 with the workspace of sq_dualscale_seglinear_gemm_ws: the
+ * accumulators of split last-wave tiles are the sums of their pieces. */
+SQ_API sq_status sq_debug_gemm_s32_ws(const int8_t *planes, const int8_t *wq, int64_t M,
+                                      int64_t N, int64_t K, const sq_segments *seg,
+                                      int32_t *acc, void *workspace, size_t workspace_bytes,
+                                      sq_stream_t stream);
 
 /*
  * Host-to-host execution of one layer with overlapped transfers.
@@ -442,6 +488,11 @@ SQ_API sq_status sq_debug_timeout_probe(uint32_t limit_us, sq_stream_t stream);
  * streams should synchronise those streams, or serialise their status checks,
  * before relying on the result.  Synchronises only `stream` (0: the legacy
  * default stream, which also waits for the other blocking streams).
+ * After a timeout a kernel waits, again with a limit, for its own copies and
+ * tensor-core operations to finish before it releases its tensor memory and
+ * exits.  If that wait runs out too, those operations were still pending when
+ * the memory was released: treat the CUDA context as unusable and end the
+ * process (a healthy GPU completes them in microseconds).
  */
 SQ_API sq_status sq_get_device_status(sq_stream_t stream);
 

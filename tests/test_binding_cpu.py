@@ -39,5 +39,9 @@ def test_segment_table_packing():
 def test_every_exported_name_has_a_wrapper_or_is_internal():
     wrapped = {n for n in B.EXPORTED if hasattr(B, n)}
     internal = {"sq_status_string", "sq_host_pipeline_workspace_bytes",
-                "sq_host_pipeline_create", "sq_host_pipeline_destroy"}
+                "sq_host_pipeline_create", "sq_host_pipeline_destroy",
+                # reached through sq_dualscale_seglinear_gemm / sq_debug_gemm_s32
+                # with workspace=, and through gemm_workspace()
+                "sq_dualscale_seglinear_gemm_ws", "sq_debug_gemm_s32_ws",
+                "sq_gemm_workspace_bytes"}
     assert set(B.EXPORTED) - wrapped <= internal

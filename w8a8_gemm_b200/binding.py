@@ -33,7 +33,8 @@ EXPORTED = ("sq_calibrate_act", "sq_quantize_act", "sq_quantize_weight_seg",
             "sq_status_string", "sq_version", "sq_debug_timeout_probe",
             "sq_host_pipeline_workspace_bytes", "sq_host_pipeline_create",
             "sq_host_pipeline_destroy", "sq_dualscale_seglinear_host",
-            "sq_dualscale_seglinear_host_noalloc", "sq_choose_single_scale")
+            "sq_dualscale_seglinear_host_noalloc", "sq_choose_single_scale",
+            "sq_dualscale_seglinear_gemm_ws", "sq_gemm_workspace_bytes", "sq_debug_gemm_s32_ws")
 SQ_NOALLOC_SCRATCH_BYTES = 32 * 1024 * 1024
 
 
@@ -109,6 +110,11 @@ def lib() -> ctypes.CDLL:
         L.sq_dualscale_seglinear_gemm_gelu_quant.argtypes = [p, p, p, p, p, i64, i64, i64, seg,
                                                              p, ctypes.c_int32, p, p]
         L.sq_debug_gemm_s32.argtypes = [p, p, i64, i64, i64, seg, p, p]
+        L.sq_debug_gemm_s32_ws.argtypes = [p, p, i64, i64, i64, seg, p, p, ctypes.c_size_t, p]
+        L.sq_dualscale_seglinear_gemm_ws.argtypes = [p, p, p, p, p, p, ctypes.c_int, i64, i64,
+                                                     i64, i64, seg, p, ctypes.c_size_t, p]
+        L.sq_gemm_workspace_bytes.argtypes = []
+        L.sq_gemm_workspace_bytes.restype = ctypes.c_size_t
         L.sq_get_device_status.argtypes = [p]
         L.sq_choose_single_scale.argtypes = [p, ctypes.c_int32, ctypes.c_int32, ctypes.c_float,
                                              ctypes.POINTER(ctypes.c_int32)]
@@ -132,6 +138,7 @@ def lib() -> ctypes.CDLL:
                   L.sq_dualscale_seglinear_host_noalloc,
                   L.sq_dualscale_seglinear_gemm, L.sq_dualscale_seglinear_gemm_gelu_quant,
                   L.sq_debug_gemm_s32, L.sq_get_device_status, L.sq_choose_single_scale,
+                  L.sq_dualscale_seglinear_gemm_ws, L.sq_debug_gemm_s32_ws,
                   L.sq_version, L.sq_debug_timeout_probe):
             f.restype = ctypes.c_int
         _lib = L
@@ -248,10 +255,23 @@ def sq_unpack_weight_w4(wq4: torch.Tensor, wq: torch.Tensor) -> torch.Tensor:
     return wq
 
 
+def gemm_workspace(device=None) -> torch.Tensor:
+    """A zero-filled workspace for sq_dualscale_seglinear_gemm_ws /
+    sq_debug_gemm_s32_ws on the current device (reuse it for every call on one
+    stream)."""
+    nbytes = lib().sq_gemm_workspace_bytes()
+    if nbytes == 0:
+        raise SegQuantError(-7, "sq_gemm_workspace_bytes")
+    return torch.zeros(nbytes, dtype=torch.uint8, device=device or torch.device("cuda"))
+
+
 def sq_dualscale_seglinear_gemm(planes: torch.Tensor, wq: torch.Tensor, s_w: torch.Tensor,
                                 s_act: torch.Tensor, bias: Optional[torch.Tensor],
-                                y: torch.Tensor, seg: Segments) -> torch.Tensor:
-    """Y = sum_i s_w (s+ X^+_i W^_i + s- X^-_i W^_i) + bias into y (bf16 or fp32 [M][N])."""
+                                y: torch.Tensor, seg: Segments,
+                                workspace: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """Y = sum_i s_w (s+ X^+_i W^_i + s- X^-_i W^_i) + bias into y (bf16 or fp32 [M][N]).
+    With `workspace` (gemm_workspace()), the _ws entry point balances the last
+    wave of tiles; the result is the same bit for bit."""
     _need(planes, torch.int8, "planes")
     _need(wq, torch.int8, "wq")
     _need(s_w, torch.float32, "s_w")
@@ -265,10 +285,19 @@ def sq_dualscale_seglinear_gemm(planes: torch.Tensor, wq: torch.Tensor, s_w: tor
         raise ValueError("shape mismatch between planes [G,P,M,K], wq [N,K] and y [M,N]")
     out = SQ_OUT_BF16 if y.dtype == torch.bfloat16 else SQ_OUT_F32
     cs, keep = seg._c()
-    _check(lib().sq_dualscale_seglinear_gemm(_ptr(planes), _ptr(wq), _ptr(s_w), _ptr(s_act),
-                                             _ptr(bias), _ptr(y), out, M, N, K, y.stride(0),
-                                             ctypes.byref(cs), _stream()),
-           "sq_dualscale_seglinear_gemm")
+    if workspace is None:
+        _check(lib().sq_dualscale_seglinear_gemm(_ptr(planes), _ptr(wq), _ptr(s_w), _ptr(s_act),
+                                                 _ptr(bias), _ptr(y), out, M, N, K, y.stride(0),
+                                                 ctypes.byref(cs), _stream()),
+               "sq_dualscale_seglinear_gemm")
+    else:
+        _need(workspace, torch.uint8, "workspace")
+        _check(lib().sq_dualscale_seglinear_gemm_ws(_ptr(planes), _ptr(wq), _ptr(s_w),
+                                                    _ptr(s_act), _ptr(bias), _ptr(y), out, M, N,
+                                                    K, y.stride(0), ctypes.byref(cs),
+                                                    _ptr(workspace), workspace.numel(),
+                                                    _stream()),
+               "sq_dualscale_seglinear_gemm_ws")
     return y
 
 
@@ -303,8 +332,9 @@ def sq_dualscale_seglinear_gemm_gelu_quant(planes: torch.Tensor, wq: torch.Tenso
 
 
 def sq_debug_gemm_s32(planes: torch.Tensor, wq: torch.Tensor, seg: Segments,
-                      acc: torch.Tensor) -> torch.Tensor:
-    """Raw int32 accumulators [S][P][M][N] of the same tensor-core kernel."""
+                      acc: torch.Tensor, workspace: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """Raw int32 accumulators [S][P][M][N] of the same tensor-core kernel (with
+    `workspace`: the balanced last wave of sq_debug_gemm_s32_ws)."""
     _need(planes, torch.int8, "planes")
     _need(wq, torch.int8, "wq")
     _need(acc, torch.int32, "acc")
@@ -313,8 +343,14 @@ def sq_debug_gemm_s32(planes: torch.Tensor, wq: torch.Tensor, seg: Segments,
     if tuple(acc.shape) != (seg.S, seg.P, M, N) or not acc.is_contiguous():
         raise ValueError(f"acc must be contiguous [{seg.S}, {seg.P}, {M}, {N}]")
     cs, keep = seg._c()
-    _check(lib().sq_debug_gemm_s32(_ptr(planes), _ptr(wq), M, N, K, ctypes.byref(cs), _ptr(acc),
-                                   _stream()), "sq_debug_gemm_s32")
+    if workspace is None:
+        _check(lib().sq_debug_gemm_s32(_ptr(planes), _ptr(wq), M, N, K, ctypes.byref(cs),
+                                       _ptr(acc), _stream()), "sq_debug_gemm_s32")
+    else:
+        _need(workspace, torch.uint8, "workspace")
+        _check(lib().sq_debug_gemm_s32_ws(_ptr(planes), _ptr(wq), M, N, K, ctypes.byref(cs),
+                                          _ptr(acc), _ptr(workspace), workspace.numel(),
+                                          _stream()), "sq_debug_gemm_s32_ws")
     return acc
 
 

@@ -131,7 +131,7 @@ sq_status gemm_common(const int8_t *planes, const int8_t *wq, const float *s_w,
                       const float *s_act, const void *bias, void *y, int out_kind, int64_t M,
                       int64_t N, int64_t K, int64_t ldy, const sq_segments *seg,
                       cudaStream_t stream, bool launch = true, const float *s_next = nullptr,
-                      int p_next = 0) {
+                      int p_next = 0, void *workspace = nullptr, size_t workspace_bytes = 0) {
   if (M < 0 || M > INT32_MAX || N < 1 || N > INT32_MAX) return SQ_ERR_INVALID_ARG;
   // An output of more than 2^44 elements fits no device; the bound keeps the
   // kernel's tile count (at most 2^30 tiles of 128 x 128) inside int32.
@@ -159,6 +159,7 @@ sq_status gemm_common(const int8_t *planes, const int8_t *wq, const float *s_w,
     if (ldy < N) return SQ_ERR_INVALID_ARG;
     if ((ldy * elem) % 16 != 0) return SQ_ERR_ALIGNMENT;
   }
+  if (workspace != nullptr && !aligned(workspace, 256)) return SQ_ERR_ALIGNMENT;
   SQ_TRY(check_device());
   if (!launch) return SQ_OK;
   GemmRequest r;
@@ -176,6 +177,8 @@ sq_status gemm_common(const int8_t *planes, const int8_t *wq, const float *s_w,
   r.seg = sp;
   r.s_next = s_next;
   r.p_next = p_next;
+  r.workspace = workspace;
+  r.workspace_bytes = workspace_bytes;
   r.status = device_status_word();
   if (r.status == nullptr) return SQ_ERR_CUDA;
   return launch_gemm(r, stream);
@@ -320,6 +323,24 @@ sq_status sq_dualscale_seglinear_gemm(const int8_t *planes, const int8_t *wq, co
                      reinterpret_cast<cudaStream_t>(stream));
 }
 
+sq_status sq_dualscale_seglinear_gemm_ws(const int8_t *planes, const int8_t *wq,
+                                         const float *s_w, const float *s_act, const void *bias,
+                                         void *y, sq_out_dtype out_dtype, int64_t M, int64_t N,
+                                         int64_t K, int64_t ldy, const sq_segments *seg,
+                                         void *workspace, size_t workspace_bytes,
+                                         sq_stream_t stream) {
+  if (out_dtype != SQ_OUT_BF16 && out_dtype != SQ_OUT_F32) return SQ_ERR_INVALID_ARG;
+  return gemm_common(planes, wq, s_w, s_act, bias, y,
+                     out_dtype == SQ_OUT_BF16 ? OUT_BF16 : OUT_F32, M, N, K, ldy, seg,
+                     reinterpret_cast<cudaStream_t>(stream), true, nullptr, 0, workspace,
+                     workspace_bytes);
+}
+
+size_t sq_gemm_workspace_bytes(void) {
+  if (check_device() != SQ_OK) return 0;
+  return gemm_workspace_bytes();
+}
+
 sq_status sq_dualscale_seglinear_gemm_gelu_quant(const int8_t *planes, const int8_t *wq,
                                                 const float *s_w, const float *s_act,
                                                 const void *bias, int64_t M, int64_t N, int64_t K,
@@ -337,6 +358,14 @@ sq_status sq_debug_gemm_s32(const int8_t *planes, const int8_t *wq, int64_t M, i
                             sq_stream_t stream) {
   return gemm_common(planes, wq, nullptr, nullptr, nullptr, acc, OUT_S32, M, N, K, N, seg,
                      reinterpret_cast<cudaStream_t>(stream));
+}
+
+sq_status sq_debug_gemm_s32_ws(const int8_t *planes, const int8_t *wq, int64_t M, int64_t N,
+                               int64_t K, const sq_segments *seg, int32_t *acc, void *workspace,
+                               size_t workspace_bytes, sq_stream_t stream) {
+  return gemm_common(planes, wq, nullptr, nullptr, nullptr, acc, OUT_S32, M, N, K, N, seg,
+                     reinterpret_cast<cudaStream_t>(stream), true, nullptr, 0, workspace,
+                     workspace_bytes);
 }
 
 sq_status sq_debug_timeout_probe(uint32_t limit_us, sq_stream_t stream) {

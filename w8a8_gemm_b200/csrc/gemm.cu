@@ -70,7 +70,133 @@ struct GemmParams {
   int *status;
   const float *s_next;  // OUT_PLANES: the next layer's {s+, s-}
   int32_t p_next;       // OUT_PLANES: its planes (2, or 1 single scale)
+  // Split tail (one K-segment only): the first sk_W waves of gridDim.x tiles
+  // run whole, one tile per CTA and wave; the k-blocks of the last sk_R tiles
+  // are shared out evenly over all CTAs.  A CTA whose share starts inside a
+  // tile writes its int32 partial sums to its slot of sk_ws and raises its
+  // epilogue warps' flags; the CTA holding the tile's first k-block adds the
+  // partials before the epilogue.  sk_R == 0: every CTA takes whole tiles.
+  int32_t sk_W, sk_R;
+  int32_t *sk_ws;       // [gridDim.x][slot_words] int32 partial sums
+  int32_t *sk_flags;    // [gridDim.x][EPI_WARPS], zero between calls
+  int64_t sk_slot_words;
 };
+
+// A CTA's work, as pieces (tile, k-blocks [kb0, kb1), role), enumerated in the
+// same order by the producer, the MMA issuer and the epilogue.
+enum PieceRole { PIECE_FULL = 0, PIECE_PARTIAL = 1, PIECE_FINAL = 2 };
+template <bool TAIL>  // false: whole tiles only (input-segmented and fused layers)
+struct Pieces {
+  int c, G, W, KB, num_tiles, j;
+  int64_t U, u, u_end;
+  __device__ void init(const GemmParams &p) {
+    c = blockIdx.x;
+    G = gridDim.x;
+    KB = p.num_kb;
+    num_tiles = p.num_tiles;
+    j = 0;
+    if (TAIL && p.sk_R > 0) {
+      W = p.sk_W;
+      U = static_cast<int64_t>(p.sk_R) * KB;
+      u = U * c / G;
+      u_end = U * (c + 1) / G;
+    } else {
+      W = (num_tiles + G - 1) / G;
+      U = u = u_end = 0;
+    }
+  }
+  __device__ bool next(int &tile, int &kb0, int &kb1, int &role) {
+    if (j < W) {
+      tile = c + j * G;
+      ++j;
+      if (tile >= num_tiles) return false;
+      kb0 = 0;
+      kb1 = KB;
+      role = PIECE_FULL;
+      return true;
+    }
+    if (!TAIL || u >= u_end) return false;
+    const int tt = static_cast<int>(u / KB);
+    kb0 = static_cast<int>(u - static_cast<int64_t>(tt) * KB);
+    const int64_t left = u_end - u;
+    kb1 = (left < KB - kb0) ? kb0 + static_cast<int>(left) : KB;
+    tile = W * G + tt;
+    role = kb0 > 0 ? PIECE_PARTIAL : (kb1 == KB ? PIECE_FULL : PIECE_FINAL);
+    u += kb1 - kb0;
+    return true;
+  }
+  // The CTA holding the last k-block of split tile `tile`: the contributors
+  // of a PIECE_FINAL piece of CTA c are CTAs c + 1 .. that one.
+  __device__ int last_holder(int tile) const {
+    const int64_t v = static_cast<int64_t>(tile - W * G) * KB + KB - 1;
+    int cc = static_cast<int>(v * G / U);
+    while (cc + 1 < G && U * (cc + 1) / G <= v) ++cc;
+    while (cc > 0 && U * cc / G > v) --cc;
+    return cc;
+  }
+};
+
+// Whole tiles only: tile = blockIdx.x, blockIdx.x + gridDim.x, ...
+template <>
+struct Pieces<false> {
+  int tile_, num_tiles, KB;
+  int64_t U = 1;
+  int G = 1;
+  __device__ void init(const GemmParams &p) {
+    tile_ = static_cast<int>(blockIdx.x) - static_cast<int>(gridDim.x);
+    num_tiles = p.num_tiles;
+    KB = p.num_kb;
+  }
+  __device__ bool next(int &tile, int &kb0, int &kb1, int &role) {
+    tile_ += gridDim.x;
+    tile = tile_;
+    kb0 = 0;
+    kb1 = KB;
+    role = PIECE_FULL;
+    return tile_ < num_tiles;
+  }
+  __device__ int last_holder(int) const { return -1; }
+};
+
+// Partial sums: one 32-word run per thread, chunk and polarity.
+// A run holds 32 words per lane of one warp, laid out [v4 group][lane][4]: each
+// store or load instruction of the warp covers 512 contiguous bytes.  `run`
+// points at the run's first word plus 4 * lane; g0 is the first v4 group.
+template <int N>
+__device__ __forceinline__ void sk_store(int32_t *run, int g0, const uint32_t *v) {
+#pragma unroll
+  for (int i = 0; i < N; i += 4)
+    __stcg(reinterpret_cast<uint4 *>(run + (g0 + i / 4) * 128),
+           make_uint4(v[i], v[i + 1], v[i + 2], v[i + 3]));
+}
+// Adds partial sums: int32 (exact) for integer codes, fp32 for FP8 codes.  The
+// loads are plain L2 loads (after the flag's acquire), so the compiler can
+// issue them all before the first add.
+template <int N, bool F8>
+__device__ __forceinline__ void sk_add(const int32_t *run, int g0, uint32_t *v) {
+  uint4 a[N / 4];
+#pragma unroll
+  for (int i = 0; i < N / 4; ++i) a[i] = __ldcg(reinterpret_cast<const uint4 *>(run + (g0 + i) * 128));
+#pragma unroll
+  for (int i = 0; i < N / 4; ++i) {
+    const uint32_t w[4] = {a[i].x, a[i].y, a[i].z, a[i].w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      if constexpr (F8)
+        v[4 * i + e] = __float_as_uint(__fadd_rn(__uint_as_float(v[4 * i + e]), __uint_as_float(w[e])));
+      else
+        v[4 * i + e] += w[e];
+    }
+  }
+}
+__device__ __forceinline__ int ld_acquire(const int32_t *f) {
+  int v;
+  asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(f) : "memory");
+  return v;
+}
+__device__ __forceinline__ void st_release(int32_t *f, int v) {
+  asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(f), "r"(v) : "memory");
+}
 
 // POL = activation planes per group: 2 for DualScale (X^+ and X^-), 1 for the
 // single-scale path (one merged plane).
@@ -256,6 +382,8 @@ __global__ void __launch_bounds__(threads_for(EPI_WARPS), 1)
   // One-segment bf16 output (and the next layer's planes) leave through
   // shared memory and TMA stores.
   constexpr bool TMA_STORE = (OUT == OUT_BF16 || OUT == OUT_PLANES) && !SEGK;
+  // Split tail of the last wave: one-segment layers with a plain output.
+  constexpr bool TAIL = !SEGK && OUT != OUT_PLANES;
   static_assert(OUT != OUT_PLANES || (!SEGK && !F8), "planes output: one K-segment, int8");
   using L = Smem<BN, STAGES, EPI_WARPS, POL, SEGK, TMA_STORE>;
   constexpr int NBUF = L::NBUF;
@@ -312,10 +440,13 @@ __global__ void __launch_bounds__(threads_for(EPI_WARPS), 1)
       int stage = 0;
       uint32_t phase = 0;
       uint32_t armed = 0, armed_parity = 0;  // per stage: has a load, its phase
-      for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x) {
+      Pieces<TAIL> pc;
+      pc.init(p);
+      int tile, kb0, kb1, role;
+      while (pc.next(tile, kb0, kb1, role)) {
         const int mt = tile / p.num_n_tiles, nt = tile % p.num_n_tiles;
         const int g = group_of_tile(p, nt, BN);
-        for (int kb = 0; kb < p.num_kb; ++kb) {
+        for (int kb = kb0; kb < kb1; ++kb) {
           if (!wait_bar(&empty[stage], phase ^ 1, abort_flag, p.status)) goto producer_done;
           uint8_t *sa = smem + stage * L::STAGE_BYTES;
           mbar_arrive_expect_tx(&full[stage], L::STAGE_BYTES);
@@ -341,7 +472,10 @@ __global__ void __launch_bounds__(threads_for(EPI_WARPS), 1)
       int stage = 0;
       uint32_t phase = 0;
       uint32_t acc_iter = 0;
-      for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x) {
+      Pieces<TAIL> pc;
+      pc.init(p);
+      int tile, kb0, kb1, role;
+      while (pc.next(tile, kb0, kb1, role)) {
         int seg = 0;
         int seg_end = SEGK ? p.k_off[1] : p.K;
         uint32_t buf = acc_iter % NBUF;
@@ -350,7 +484,7 @@ __global__ void __launch_bounds__(threads_for(EPI_WARPS), 1)
         tc_fence_after();
         uint32_t d_plus = tmem_base + buf * ACC_COLS;
         uint32_t accumulate = 0;
-        for (int kb = 0; kb < p.num_kb; ++kb) {
+        for (int kb = kb0; kb < kb1; ++kb) {
           if (!wait_bar(&full[stage], phase, abort_flag, p.status)) goto mma_exit;
           tc_fence_after();
           const uint32_t sa = smem_u32(smem + stage * L::STAGE_BYTES);
@@ -423,12 +557,54 @@ __global__ void __launch_bounds__(threads_for(EPI_WARPS), 1)
       rp_nx = __frcp_rn(sp_nx);
       rm_nx = __frcp_rn(sm_nx);
     }
-    for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x) {
+    Pieces<TAIL> pc;
+    pc.init(p);
+    int tile, kb0, kb1, role;
+    while (pc.next(tile, kb0, kb1, role)) {
       const int mt = tile / p.num_n_tiles, nt = tile % p.num_n_tiles;
       const int g = group_of_tile(p, nt, BN);
       const int64_t m = static_cast<int64_t>(mt) * BM + row;
       const int64_t nb = static_cast<int64_t>(nt) * BN + half * HALF;
-      if constexpr (!SEGK && OUT != OUT_S32) {
+      (void)kb0;
+      (void)kb1;
+      // Split tail: the partial sums of a PIECE_PARTIAL go to this CTA's slot;
+      // a PIECE_FINAL adds those of CTAs blockIdx.x + 1 .. sk_last first.
+      int sk_last = -1;
+      if (TAIL && role == PIECE_FINAL) sk_last = pc.last_holder(tile);
+      const auto slot_run = [&](int cta, int c, int pol) {
+        return p.sk_ws + cta * p.sk_slot_words +
+               ((static_cast<int64_t>(ew) * (HALF / 32) + c) * POL + pol) * 1024 + lane * 4;
+      };
+      if (TAIL && role == PIECE_FINAL) {
+        // Wait (bounded) until every contributor has written its partials.
+        bool ok = true;
+        if (lane == 0) {
+          const uint64_t t0 = globaltimer_ns();
+          for (int cc = blockIdx.x + 1; cc <= sk_last && ok; ++cc) {
+            if (pc.U * cc / pc.G == pc.U * (cc + 1) / pc.G) continue;  // holds no k-block
+            const int32_t *f = p.sk_flags + cc * EPI_WARPS + ew;
+            while (ld_acquire(f) == 0) {
+              if (*abort_flag) {
+                ok = false;
+                break;
+              }
+              if (globaltimer_ns() - t0 > kWaitLimitNs) {
+                *abort_flag = 1;
+                atomicExch(p.status, static_cast<int>(SQ_ERR_DEVICE_TIMEOUT));
+                ok = false;
+                break;
+              }
+              __nanosleep(64);
+            }
+          }
+        }
+        ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+        if (!ok) goto epilogue_exit;
+        for (int cc = blockIdx.x + 1; cc <= sk_last; ++cc)  // every lane acquires
+          if (pc.U * cc / pc.G != pc.U * (cc + 1) / pc.G)
+            (void)ld_acquire(p.sk_flags + cc * EPI_WARPS + ew);
+      }
+      if (!SEGK && OUT != OUT_S32 && !(TAIL && role == PIECE_PARTIAL)) {
         // The folded c+- = fl(s_w s+-) and the bias of this warp's columns,
         // staged while the MMAs run (one K-segment: s_act[g][0]).
         const float sp0 = __fmul_rn(p.s_act[g * 2 + 0], p.act_mul);
@@ -502,6 +678,17 @@ __global__ void __launch_bounds__(threads_for(EPI_WARPS), 1)
             tmem_ld_cols<CW>(t_plus + c * CW, ap);
             if constexpr (POL == 2) tmem_ld_cols<CW>(t_plus + BN + c * CW, am);
             tmem_ld_wait();
+            if (TAIL && role == PIECE_PARTIAL) {
+              sk_store<CW>(slot_run(blockIdx.x, c, 0), 0, ap);
+              if constexpr (POL == 2) sk_store<CW>(slot_run(blockIdx.x, c, 1), 0, am);
+              continue;
+            }
+            if (TAIL && role == PIECE_FINAL)
+              for (int cc = blockIdx.x + 1; cc <= sk_last; ++cc)
+                if (pc.U * cc / pc.G != pc.U * (cc + 1) / pc.G) {
+                  sk_add<CW, F8>(slot_run(cc, c, 0), 0, ap);
+                  if constexpr (POL == 2) sk_add<CW, F8>(slot_run(cc, c, 1), 0, am);
+                }
             if (m < p.M) {
               int32_t *accp = reinterpret_cast<int32_t *>(p.y) +
                               ((static_cast<int64_t>(u) * POL) * p.M + m) * p.N;
@@ -531,6 +718,25 @@ __global__ void __launch_bounds__(threads_for(EPI_WARPS), 1)
               tmem_ld_16x256b_x4(t_plus + BN + c * 32 + kLanes16, mh);
             }
             tmem_ld_wait();
+            if (TAIL && role == PIECE_PARTIAL) {
+              sk_store<16>(slot_run(blockIdx.x, c, 0), 0, pl);
+              sk_store<16>(slot_run(blockIdx.x, c, 0), 4, ph);
+              if constexpr (POL == 2) {
+                sk_store<16>(slot_run(blockIdx.x, c, 1), 0, ml);
+                sk_store<16>(slot_run(blockIdx.x, c, 1), 4, mh);
+              }
+              continue;
+            }
+            if (TAIL && role == PIECE_FINAL)
+              for (int cc = blockIdx.x + 1; cc <= sk_last; ++cc)
+                if (pc.U * cc / pc.G != pc.U * (cc + 1) / pc.G) {
+                  sk_add<16, F8>(slot_run(cc, c, 0), 0, pl);
+                  sk_add<16, F8>(slot_run(cc, c, 0), 4, ph);
+                  if constexpr (POL == 2) {
+                    sk_add<16, F8>(slot_run(cc, c, 1), 0, ml);
+                    sk_add<16, F8>(slot_run(cc, c, 1), 4, mh);
+                  }
+                }
             const int q = lane & 3;
             const float *cpc = cst + c * 32 + 2 * q;
             const float *cmc = cst + HALF + c * 32 + 2 * q;
@@ -653,6 +859,20 @@ __global__ void __launch_bounds__(threads_for(EPI_WARPS), 1)
           if (lane == 0) mbar_arrive(&acc_empty[buf]);
           fold(lo, hi, POL == 2 ? cst + HALF : cst);
         } else {
+          if (TAIL && role == PIECE_PARTIAL) {
+            // every lane's partials are visible before the flag is raised
+            __threadfence();
+            __syncwarp();
+            if (lane == 0) st_release(p.sk_flags + blockIdx.x * EPI_WARPS + ew, 1);
+          }
+          if (TAIL && role == PIECE_FINAL) {
+            // consumed: leave the flags at zero for the next call
+            __syncwarp();
+            if (lane == 0)
+              for (int cc = blockIdx.x + 1; cc <= sk_last; ++cc)
+                if (pc.U * cc / pc.G != pc.U * (cc + 1) / pc.G)
+                  p.sk_flags[cc * EPI_WARPS + ew] = 0;
+          }
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(&acc_empty[buf]);
@@ -807,6 +1027,30 @@ sq_status run_gemm(const GemmRequest &r, const GemmParams &p, cudaStream_t strea
       return SQ_ERR_CUDA;
   }
   static_assert(L::BYTES <= 232448, "dynamic shared memory above the per-block limit");
+  // Split tail of the last wave (one-segment layers, plain outputs): with a
+  // workspace large enough, all SMs take a CTA and the k-blocks of the last,
+  // partial wave's tiles are shared out evenly among them.
+  GemmParams q = p;
+  q.sk_W = q.sk_R = 0;
+  q.sk_ws = nullptr;
+  q.sk_flags = nullptr;
+  q.sk_slot_words = 0;
+  const int sms = device_sm_count();
+  int grid = p.num_tiles < sms ? p.num_tiles : sms;
+  if constexpr (!SEGK && OUT != OUT_PLANES) {
+    const int64_t slot_words = static_cast<int64_t>(EPI_WARPS) * (L::COLS / 32) * POL * 1024;
+    const size_t need = ((static_cast<size_t>(sms) * EPI_WARPS + 63) / 64) * 64 * 4 +
+                        static_cast<size_t>(sms) * slot_words * 4;
+    if (r.workspace != nullptr && r.workspace_bytes >= need && p.num_tiles > sms &&
+        p.num_tiles % sms != 0) {
+      q.sk_W = p.num_tiles / sms;
+      q.sk_R = p.num_tiles % sms;
+      q.sk_flags = static_cast<int32_t *>(r.workspace);
+      q.sk_ws = q.sk_flags + ((static_cast<int64_t>(sms) * EPI_WARPS + 63) / 64) * 64;
+      q.sk_slot_words = slot_words;
+      grid = sms;
+    }
+  }
   auto kernel = dualscale_gemm_kernel<BN, STAGES, OUT, SEGK, EPI_WARPS, POL, F8>;
   static bool attr_set[64] = {};  // per instantiation and device
   int dev = 0;
@@ -818,7 +1062,6 @@ sq_status run_gemm(const GemmRequest &r, const GemmParams &p, cudaStream_t strea
       return SQ_ERR_CUDA;
     attr_set[dev] = true;
   }
-  const int grid = p.num_tiles < device_sm_count() ? p.num_tiles : device_sm_count();
   // Programmatic dependent launch: CTAs may run their prologue (barriers,
   // TMEM allocation) while the preceding kernel finishes.
   cudaLaunchConfig_t cfg = {};
@@ -831,7 +1074,7 @@ sq_status run_gemm(const GemmRequest &r, const GemmParams &p, cudaStream_t strea
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  if (cudaLaunchKernelEx(&cfg, kernel, tmA, tmB, tmY, p) != cudaSuccess) return SQ_ERR_CUDA;
+  if (cudaLaunchKernelEx(&cfg, kernel, tmA, tmB, tmY, q) != cudaSuccess) return SQ_ERR_CUDA;
   return cudaGetLastError() == cudaSuccess ? SQ_OK : SQ_ERR_CUDA;
 }
 
@@ -865,6 +1108,13 @@ sq_status dispatch_kind(const GemmRequest &r, const GemmParams &p, bool segk, in
 }
 
 }  // namespace
+
+size_t gemm_workspace_bytes() {
+  // flags (rounded up to 64 words) and one slot of partial sums per SM, for
+  // the widest configuration: 8 epilogue warps x 128 columns x 2 planes
+  const size_t sms = static_cast<size_t>(device_sm_count());
+  return ((sms * 8 + 63) / 64) * 64 * 4 + sms * (8 * 4 * 2 * 1024 * 4);
+}
 
 sq_status launch_gemm(const GemmRequest &r, cudaStream_t stream) {
   if (r.M == 0) return SQ_OK;

@@ -65,9 +65,16 @@ struct GemmRequest {
   // planes per group (2 DualScale, 1 single scale); y is int8 [p_next][M][N].
   const float *s_next = nullptr;
   int p_next = 0;
+  // Optional workspace for the split last wave (zero-filled before its first
+  // use; every call leaves its flags at zero): nullptr = whole tiles only.
+  void *workspace = nullptr;
+  size_t workspace_bytes = 0;
 };
 
 sq_status launch_gemm(const GemmRequest &req, cudaStream_t stream);
+// Workspace bytes that let any one-segment GEMM split its last wave on the
+// current device.
+size_t gemm_workspace_bytes();
 
 // ---- test-only probe (probe.cu) --------------------------------------------
 cudaError_t launch_timeout_probe(uint32_t limit_us, int *status, cudaStream_t stream);

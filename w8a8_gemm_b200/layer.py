@@ -25,19 +25,23 @@ class DualScaleSegLinear:
            and expanded into the int8 GEMM operand before every GEMM; several
            layers may share one operand buffer, `w_operand`, int8 [>= N*K])
     fp8    FP8 E4M3 codes for activations and weights (SQ_FLAG_FP8) instead of int8
+    workspace  optional uint8 CUDA tensor from binding.gemm_workspace(): the GEMM
+           then balances its last wave of tiles over all SMs (same results); layers
+           run one after another on one stream may share one
     """
 
     def __init__(self, w: torch.Tensor, bias: Optional[torch.Tensor], d: Optional[torch.Tensor],
                  seg: B.Segments, x_cal: torch.Tensor, out_dtype=torch.bfloat16,
                  adaptive: bool = False, asymmetry_threshold: float = 2.0,
                  weight_bits: int = 8, w_operand: Optional[torch.Tensor] = None,
-                 fp8: bool = False):
+                 fp8: bool = False, workspace: Optional[torch.Tensor] = None):
         if weight_bits not in (8, 4):
             raise ValueError("weight_bits must be 8 or 4")
         if fp8 and weight_bits == 4:
             raise ValueError("FP8 codes and W4 weights do not combine")
         self.N, self.K = w.shape
         self.weight_bits = weight_bits
+        self.workspace = workspace
         self.fp8 = fp8
         if weight_bits == 4:
             seg = B.Segments(seg.mode, seg.offsets, seg.n_groups, seg.flags | B.SQ_FLAG_W4)
@@ -94,7 +98,7 @@ class DualScaleSegLinear:
         if self.wq4 is not None:
             B.sq_unpack_weight_w4(self.wq4, self.wq)
         return B.sq_dualscale_seglinear_gemm(planes, self.wq, self.s_w, self.s_act, self.bias,
-                                             y, self.seg)
+                                             y, self.seg, workspace=self.workspace)
 
     def gemm_gelu_quant(self, planes: torch.Tensor, nxt: "DualScaleSegLinear",
                         planes_next: Optional[torch.Tensor] = None) -> torch.Tensor:
