@@ -1,0 +1,63 @@
+"""The activation quantizer forms int8 codes without the quotient's correction
+(one product u * fl(1/s)) when a block-wide test on a few hundred inputs says
+that this gives the exact codes rne(fl(u/s)) for every bf16 input.  These CPU
+tests check that argument on a numpy model of both forms: the test passes
+exactly when the forms agree on all 65,536 bf16 values, over random steps and
+over steps constructed so that the forms differ."""
+import numpy as np
+import pytest
+
+from correction_free import (codes, forms_agree_everywhere, passes_candidate_test,
+                             steps_where_forms_differ)
+
+
+def test_worked_counterexample_is_caught():
+    """s = 0x1.fd0eb8p-8, x = 0x1.5ap-2: x/s = 43.4999980..., fl(x/s) rounds to
+    43, fl(x * fl(1/s)) = 43.5 rounds to 44 (either polarity)."""
+    s = np.float32(float.fromhex("0x1.fd0eb8p-8"))
+    x = np.array([0x3EAD, 0xBEAD], np.uint16)          # +-0x1.5ap-2
+    exact = codes(x, s, s, False)
+    fast = codes(x, s, s, True)
+    assert (exact[0][0], exact[1][1]) == (43, -43)
+    assert (fast[0][0], fast[1][1]) == (44, -44)
+    assert not passes_candidate_test(s, np.float32(1 / 64))
+    assert not passes_candidate_test(np.float32(1 / 64), s)
+    assert passes_candidate_test(np.float32(1 / 64), np.float32(1 / 512))
+
+
+@pytest.mark.parametrize("seed", range(4))
+def test_candidate_test_is_exact_on_random_steps(seed):
+    """Log-uniform steps over 2^-30 .. 2^20: the candidate test passes iff the
+    two forms agree on every bf16 input of both polarities."""
+    rng = np.random.default_rng(100 + seed)
+    n_fast = 0
+    for _ in range(60):
+        sp, sm = np.exp2(rng.uniform(-30, 20, 2)).astype(np.float32)
+        ok = passes_candidate_test(sp, sm)
+        assert ok == forms_agree_everywhere(sp, sm), (float(sp), float(sm))
+        n_fast += ok
+    assert n_fast > 40            # the uncorrected form is the common case
+
+
+def test_candidate_test_rejects_every_constructed_step():
+    """Steps where some bf16 input's codes differ between the forms, on either
+    side: the test must reject each of them."""
+    bad = steps_where_forms_differ(12, seed=7)
+    one = np.float32(1 / 64)
+    for s in bad:
+        s = np.float32(s)
+        assert not forms_agree_everywhere(s, one)
+        assert not passes_candidate_test(s, one), float(s)
+        assert not passes_candidate_test(one, s), float(s)
+
+
+def test_powers_of_two_and_calibrated_steps_pass():
+    """Steps that are powers of two make both forms exact; AMax steps m/127 and
+    m/128 of bf16 maxima are the common case of calibrated layers."""
+    for e in range(-20, 10):
+        assert passes_candidate_test(np.float32(2.0 ** e), np.float32(2.0 ** (e - 3)))
+    rng = np.random.default_rng(3)
+    agree = [forms_agree_everywhere(np.float32(m) / np.float32(127), np.float32(m) / np.float32(128))
+             == passes_candidate_test(np.float32(m) / np.float32(127), np.float32(m) / np.float32(128))
+             for m in rng.uniform(0.1, 40, 40)]
+    assert all(agree)

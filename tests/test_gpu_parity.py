@@ -115,6 +115,34 @@ def test_every_bf16_value_at_non_power_of_two_steps(with_d, single, fp8):
         assert np.array_equal(planes.cpu().numpy(), ref), (sp, sm)
 
 
+@pytest.mark.parametrize("single", [False, True])
+def test_uncorrected_codes_only_where_exact(single):
+    """The quantizer skips the quotient's correction for a column block only
+    after a block-wide test of its step pair.  Four 256-wide input segments,
+    each holding every bf16 value, with step pairs under which the uncorrected
+    codes would differ from rne(fl(x/s)) for some input (segments 0 and 2,
+    constructed by a search) beside ordinary ones: every plane equals the
+    oracle's."""
+    from correction_free import forms_agree_everywhere, steps_where_forms_differ
+    bad = steps_where_forms_differ(2, seed=11)
+    pairs = [(bad[0], 1 / 512), (1 / 64, 1 / 128), (0.0123457, bad[1]), (0.2718, 0.0031416)]
+    if single:
+        pairs = [(a, a) for a, _ in pairs]
+    assert not forms_agree_everywhere(np.float32(pairs[0][0]), np.float32(pairs[0][1]))
+    allbits = np.arange(65536, dtype=np.uint32).astype(np.uint16).reshape(256, 256)
+    xb = np.ascontiguousarray(np.tile(allbits, (1, 4)))
+    offsets = [0, 256, 512, 768, 1024]
+    s_act = np.array([pairs], np.float32)
+    ref = oracle.quantize_act(xb, s_act, mode=oracle.MODE_INPUT, offsets=offsets, G=1,
+                              single=single)
+    x = torch.from_numpy(xb.view(np.int16)).view(torch.bfloat16).cuda()
+    flags = B.SQ_FLAG_SINGLE_SCALE if single else 0
+    seg = B.Segments(B.SQ_SEG_INPUT, offsets, 1, flags=flags)
+    planes = torch.empty(1, seg.P, 256, 1024, dtype=torch.int8, device="cuda")
+    B.sq_quantize_act(x, None, torch.from_numpy(s_act).cuda(), seg, planes)
+    assert np.array_equal(planes.cpu().numpy(), ref)
+
+
 @pytest.mark.parametrize("kind", ["positive", "negative", "zero", "nan_and_inf", "mixed"])
 def test_calibration_degenerate_slices_on_gpu(kind):
     """AMax calibration on the GPU equals the oracle's, bit for bit, including

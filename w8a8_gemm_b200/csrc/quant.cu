@@ -11,6 +11,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <type_traits>
+
 #include "sm100.cuh"
 #include "sq_internal.h"
 
@@ -229,6 +231,55 @@ __device__ __forceinline__ void dualscale8(const float (&u)[8], const StepConsts
   minus = make_uint2(pack4_lo(qm[0], qm[1], qm[2], qm[3]), pack4_lo(qm[4], qm[5], qm[6], qm[7]));
 }
 
+// The same codes without the quotient's correction, for step pairs where that
+// provably changes none: q+ = rne(128 sat(RN(u fl(1/s+)) / 128)), and q- the
+// same with s-.  RN(u fl(1/s)) and fl(u / s) both lie within 2^-23 relative of
+// u / s, so their integer roundings can differ only for u next to a rounding
+// boundary (h + 1/2) s, h = 0 .. 127; step_pair_exact_without_correction()
+// tests exactly those inputs before a block uses this form.  NaN, overflow
+// and the other polarity saturate as in dualscale8.
+__device__ __forceinline__ void dualscale8_fast(const float (&u)[8], const StepConsts &k,
+                                                uint2 &plus, uint2 &minus) {
+  uint32_t qp[8], qm[8];
+#pragma unroll
+  for (int j = 0; j < 8; j += 2) {
+    round2(mul_sat(u[j], k.r7p), mul_sat(u[j + 1], k.r7p), 128.0f, qp[j], qp[j + 1]);
+    round2(mul_sat(u[j], k.r7m), mul_sat(u[j + 1], k.r7m), -128.0f, qm[j], qm[j + 1]);
+  }
+  plus = make_uint2(__vminu4(pack4_lo(qp[0], qp[1], qp[2], qp[3]), 0x7F7F7F7Fu),
+                    __vminu4(pack4_lo(qp[4], qp[5], qp[6], qp[7]), 0x7F7F7F7Fu));
+  minus = make_uint2(pack4_lo(qm[0], qm[1], qm[2], qm[3]), pack4_lo(qm[4], qm[5], qm[6], qm[7]));
+}
+
+// Block-wide test (every thread of the block calls it with the same step
+// pair): true if dualscale8_fast gives dualscale8's codes for every bf16
+// input (int8 codes, no divisor).  The two roundings of u / s are within
+// 2^-23 relative of it, so a difference needs a boundary b = h + 1/2 within
+// 2^-23 relative of u / s, i.e. u within that distance of b s.  bf16 values
+// are 2^-8 relative apart, so such a u is a bf16 neighbour of fl(b s) (itself
+// within 2^-24 of b s): the candidates are fl(b s) truncated to bf16 and the
+// bf16 values just below and above it, for b = 1/2 .. 127 + 1/2 and both
+// polarities (768 inputs).  Beyond 127.5 both forms saturate alike.
+__device__ bool step_pair_exact_without_correction(const StepConsts &k, float s_plus,
+                                                   float s_minus) {
+  int bad = 0;
+  for (int j = threadIdx.x; j < 768; j += blockDim.x) {
+    const int pol = j / 384, rem = j - pol * 384;
+    const float b = static_cast<float>(rem / 3) + 0.5f;
+    const uint32_t t = __float_as_uint(__fmul_rn(b, pol ? s_minus : s_plus)) & 0xFFFF0000u;
+    float x = __uint_as_float(t + static_cast<uint32_t>(rem % 3 - 1) * 0x10000u);
+    if (pol) x = -x;
+    float u[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) u[e] = x;
+    uint2 p0, m0, p1, m1;
+    dualscale8(u, k, p0, m0);
+    dualscale8_fast(u, k, p1, m1);
+    bad |= (p0.x != p1.x) | (m0.x != m1.x);
+  }
+  return __syncthreads_or(bad) == 0;
+}
+
 // FP8 (E4M3) codes of eight channels: v = fl(u / s) by the same correction
 // (unscaled), code = e4m3(v), round half to even with saturation to +-448 (the
 // CUDA conversion intrinsics).  u is clamped to 1024 s on its own side first
@@ -384,6 +435,28 @@ __global__ void __launch_bounds__(256, 3) quant_act_kernel(const __grid_constant
   if (n_mine > 0)
     fold_consts<FP8, HAS_D>(static_cast<int64_t>(cur.cb) * kWarpCols + lane * kColsPerThread, K,
                             sc, dv, kc);
+  // Whether the block's current (group, column block) may take the codes
+  // without the quotient's correction (block-uniform): int8 codes, no
+  // divisor, one K-segment across the column block, and the block-wide test
+  // of its step pair passed.
+  const auto correction_free = [&](int g, int cb) -> bool {
+    if constexpr (FP8 || HAS_D) {
+      return false;
+    } else {
+      const int64_t first = static_cast<int64_t>(cb) * kWarpCols;
+      const int64_t last = (first + kWarpCols < K ? first + kWarpCols : K) - 1;
+      int i = 0;
+      if (seg.mode == SQ_SEG_INPUT) {
+        i = seg_index(seg.off, seg.n_seg, first);
+        if (seg_index(seg.off, seg.n_seg, last) != i) return false;
+      }
+      const float pair[2] = {s_act[(g * seg.S + i) * 2 + 0], s_act[(g * seg.S + i) * 2 + 1]};
+      StepConsts k;
+      fold_consts<false, false>(0, 1, pair, dv, k);
+      return step_pair_exact_without_correction(k, pair[0], pair[1]);
+    }
+  };
+  bool fast = n_mine > 0 ? correction_free(cur.g, cur.cb) : false;
   int key_g = cur.g, key_cb = cur.cb;  // (group, column block) of the constants held
   const int64_t plane_stride = M * K;
   for (int it = 0; it < n_mine; ++it, cur.next(n_cb, n_rt)) {
@@ -393,6 +466,7 @@ __global__ void __launch_bounds__(256, 3) quant_act_kernel(const __grid_constant
       key_cb = cur.cb;
       fetch_scales<HAS_D>(cur.g, c0, K, d, s_act, seg, sc, dv);
       fold_consts<FP8, HAS_D>(c0, K, sc, dv, kc);
+      fast = correction_free(cur.g, cur.cb);
     }
     const int st = it % kQStages;
     if (!mbar_wait(&full[st], (it / kQStages) & 1, kQuantWaitNs)) {
@@ -401,7 +475,9 @@ __global__ void __launch_bounds__(256, 3) quant_act_kernel(const __grid_constant
     }
     const uint16_t *tile = reinterpret_cast<const uint16_t *>(qsmem + st * kQTileBytes);
     const int64_t r_base = static_cast<int64_t>(cur.rt) * kQRows;
-    if (c0 < K) {
+    const auto rows = [&](auto fast_form) {
+      // (the uncorrected codes exist for int8 codes without a divisor only)
+      constexpr bool FAST = decltype(fast_form)::value && !FP8 && !HAS_D;
       int8_t *plus = planes + static_cast<int64_t>(cur.g) * seg.P * plane_stride + c0;
 #pragma unroll 4
       for (int rr = warp; rr < kQRows; rr += 8) {
@@ -411,7 +487,9 @@ __global__ void __launch_bounds__(256, 3) quant_act_kernel(const __grid_constant
         float xv[8];
         unpack8(v, xv);
         uint2 pk, nk;
-        if constexpr (FP8) {
+        if constexpr (FAST) {
+          dualscale8_fast(xv, kc, pk, nk);
+        } else if constexpr (FP8) {
           float uv[8];
 #pragma unroll
           for (int j = 0; j < 8; ++j) uv[j] = xv[j];
@@ -430,6 +508,12 @@ __global__ void __launch_bounds__(256, 3) quant_act_kernel(const __grid_constant
           *reinterpret_cast<uint2 *>(plus + r * K) = make_uint2(pk.x | nk.x, pk.y | nk.y);
         }
       }
+    };
+    if (c0 < K) {
+      if (!FP8 && !HAS_D && fast)
+        rows(std::true_type{});
+      else
+        rows(std::false_type{});
     }
     __syncthreads();  // every warp is done with stage st
     if (tid == 0 && it + kQStages < n_mine) {
