@@ -116,29 +116,44 @@ def test_every_bf16_value_at_non_power_of_two_steps(with_d, single, fp8):
 
 
 @pytest.mark.parametrize("single", [False, True])
-def test_uncorrected_codes_only_where_exact(single):
-    """The quantizer skips the quotient's correction for a column block only
-    after a block-wide test of its step pair.  Four 256-wide input segments,
-    each holding every bf16 value, with step pairs under which the uncorrected
-    codes would differ from rne(fl(x/s)) for some input (segments 0 and 2,
-    constructed by a search) beside ordinary ones: every plane equals the
-    oracle's."""
+@pytest.mark.parametrize("layout", ["wide", "narrow"])
+def test_uncorrected_codes_only_where_exact(layout, single):
+    """The quantizer skips the quotient's correction for a 256-channel column
+    block only after a block-wide test of the step pair of every K-segment in
+    it.  Every segment holds every bf16 value; some step pairs are ones under
+    which the uncorrected codes would differ from rne(fl(x/s)) for some input
+    (constructed by a search), beside ordinary ones.  "wide": four 256-wide
+    segments (one per column block, segments 0 and 2 with such steps);
+    "narrow": eight 64-wide segments, the first column block with one such
+    step among four, the second with none.  Every plane equals the oracle's."""
     from correction_free import forms_agree_everywhere, steps_where_forms_differ
     bad = steps_where_forms_differ(2, seed=11)
-    pairs = [(bad[0], 1 / 512), (1 / 64, 1 / 128), (0.0123457, bad[1]), (0.2718, 0.0031416)]
+    allbits = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    if layout == "wide":
+        pairs = [(bad[0], 1 / 512), (1 / 64, 1 / 128), (0.0123457, bad[1]), (0.2718, 0.0031416)]
+        xb = np.tile(allbits.reshape(256, 256), (1, 4))
+        offsets = [0, 256, 512, 768, 1024]
+    else:
+        pairs = [(1 / 64, 1 / 128), (0.0123457, bad[1]), (0.2718, 0.0031416), (1 / 32, 0.75),
+                 (0.00057, 0.0419), (1 / 64, 1 / 512), (0.5, 0.25), (0.0123457, 0.000731)]
+        xb = np.tile(allbits.reshape(1024, 64), (1, 8))
+        offsets = list(range(0, 513, 64))
     if single:
         pairs = [(a, a) for a, _ in pairs]
-    assert not forms_agree_everywhere(np.float32(pairs[0][0]), np.float32(pairs[0][1]))
-    allbits = np.arange(65536, dtype=np.uint32).astype(np.uint16).reshape(256, 256)
-    xb = np.ascontiguousarray(np.tile(allbits, (1, 4)))
-    offsets = [0, 256, 512, 768, 1024]
+        if layout == "narrow":
+            pairs[1] = (bad[1], bad[1])
+    dangerous = [(a, b) for a, b in pairs if a in bad or b in bad]
+    assert dangerous
+    assert not any(forms_agree_everywhere(np.float32(a), np.float32(b)) for a, b in dangerous)
+    xb = np.ascontiguousarray(xb)
+    M, K = xb.shape
     s_act = np.array([pairs], np.float32)
     ref = oracle.quantize_act(xb, s_act, mode=oracle.MODE_INPUT, offsets=offsets, G=1,
                               single=single)
     x = torch.from_numpy(xb.view(np.int16)).view(torch.bfloat16).cuda()
     flags = B.SQ_FLAG_SINGLE_SCALE if single else 0
     seg = B.Segments(B.SQ_SEG_INPUT, offsets, 1, flags=flags)
-    planes = torch.empty(1, seg.P, 256, 1024, dtype=torch.int8, device="cuda")
+    planes = torch.empty(1, seg.P, M, K, dtype=torch.int8, device="cuda")
     B.sq_quantize_act(x, None, torch.from_numpy(s_act).cuda(), seg, planes)
     assert np.array_equal(planes.cpu().numpy(), ref)
 

@@ -235,8 +235,9 @@ __device__ __forceinline__ void dualscale8(const float (&u)[8], const StepConsts
 // provably changes none: q+ = rne(128 sat(RN(u fl(1/s+)) / 128)), and q- the
 // same with s-.  RN(u fl(1/s)) and fl(u / s) both lie within 2^-23 relative of
 // u / s, so their integer roundings can differ only for u next to a rounding
-// boundary (h + 1/2) s, h = 0 .. 127; step_pair_exact_without_correction()
-// tests exactly those inputs before a block uses this form.  NaN, overflow
+// boundary (h + 1/2) s, h = 0 .. 127; correction_changes_a_code() tests
+// exactly those inputs (for every step pair of a column block) before a block
+// uses this form.  NaN, overflow
 // and the other polarity saturate as in dualscale8.
 __device__ __forceinline__ void dualscale8_fast(const float (&u)[8], const StepConsts &k,
                                                 uint2 &plus, uint2 &minus) {
@@ -251,33 +252,39 @@ __device__ __forceinline__ void dualscale8_fast(const float (&u)[8], const StepC
   minus = make_uint2(pack4_lo(qm[0], qm[1], qm[2], qm[3]), pack4_lo(qm[4], qm[5], qm[6], qm[7]));
 }
 
-// Block-wide test (every thread of the block calls it with the same step
-// pair): true if dualscale8_fast gives dualscale8's codes for every bf16
-// input (int8 codes, no divisor).  The two roundings of u / s are within
+// This thread's share of the test whether dualscale8_fast gives dualscale8's
+// codes for every bf16 input at the step pair of `k` (int8 codes, no
+// divisor); returns true if one of its inputs differs, and the block combines
+// the threads' answers.  The two roundings of u / s are within
 // 2^-23 relative of it, so a difference needs a boundary b = h + 1/2 within
 // 2^-23 relative of u / s, i.e. u within that distance of b s.  bf16 values
 // are 2^-8 relative apart, so such a u is a bf16 neighbour of fl(b s) (itself
 // within 2^-24 of b s): the candidates are fl(b s) truncated to bf16 and the
 // bf16 values just below and above it, for b = 1/2 .. 127 + 1/2 and both
 // polarities (768 inputs).  Beyond 127.5 both forms saturate alike.
-__device__ bool step_pair_exact_without_correction(const StepConsts &k, float s_plus,
-                                                   float s_minus) {
+__device__ bool correction_changes_a_code(const StepConsts &k, float s_plus, float s_minus) {
   int bad = 0;
   for (int j = threadIdx.x; j < 768; j += blockDim.x) {
     const int pol = j / 384, rem = j - pol * 384;
     const float b = static_cast<float>(rem / 3) + 0.5f;
     const uint32_t t = __float_as_uint(__fmul_rn(b, pol ? s_minus : s_plus)) & 0xFFFF0000u;
-    float x = __uint_as_float(t + static_cast<uint32_t>(rem % 3 - 1) * 0x10000u);
-    if (pol) x = -x;
-    float u[8];
-#pragma unroll
-    for (int e = 0; e < 8; ++e) u[e] = x;
-    uint2 p0, m0, p1, m1;
-    dualscale8(u, k, p0, m0);
-    dualscale8_fast(u, k, p1, m1);
-    bad |= (p0.x != p1.x) | (m0.x != m1.x);
+    const float x = __uint_as_float(t + static_cast<uint32_t>(rem % 3 - 1) * 0x10000u);
+    // One element of dualscale8 and of dualscale8_fast, on the candidate's
+    // own plane (the other plane's code is 0 in both forms).
+    const float u = pol ? -x : x;
+    const float r7 = pol ? k.r7m : k.r7p, m128 = pol ? k.m128m : k.m128p;
+    const float scale = pol ? -128.0f : 128.0f;
+    const float a = mul_sat(u, r7);
+    const float v = fma_sat(__fmaf_rn(a, m128, u), r7, a);
+    uint32_t q_exact = __float_as_uint(__fmaf_rn(v, scale, 12582912.0f)) & 0xFFu;
+    uint32_t q_fast = __float_as_uint(__fmaf_rn(a, scale, 12582912.0f)) & 0xFFu;
+    if (!pol) {  // the + plane's codes are lowered to 127
+      q_exact = min(q_exact, 127u);
+      q_fast = min(q_fast, 127u);
+    }
+    bad |= q_exact != q_fast;
   }
-  return __syncthreads_or(bad) == 0;
+  return bad != 0;
 }
 
 // FP8 (E4M3) codes of eight channels: v = fl(u / s) by the same correction
@@ -437,23 +444,27 @@ __global__ void __launch_bounds__(256, 3) quant_act_kernel(const __grid_constant
                             sc, dv, kc);
   // Whether the block's current (group, column block) may take the codes
   // without the quotient's correction (block-uniform): int8 codes, no
-  // divisor, one K-segment across the column block, and the block-wide test
-  // of its step pair passed.
+  // divisor, and the block-wide test passed for the step pair of every
+  // K-segment that meets the column block.
   const auto correction_free = [&](int g, int cb) -> bool {
     if constexpr (FP8 || HAS_D) {
       return false;
     } else {
       const int64_t first = static_cast<int64_t>(cb) * kWarpCols;
       const int64_t last = (first + kWarpCols < K ? first + kWarpCols : K) - 1;
-      int i = 0;
+      int i0 = 0, i1 = 0;
       if (seg.mode == SQ_SEG_INPUT) {
-        i = seg_index(seg.off, seg.n_seg, first);
-        if (seg_index(seg.off, seg.n_seg, last) != i) return false;
+        i0 = seg_index(seg.off, seg.n_seg, first);
+        i1 = seg_index(seg.off, seg.n_seg, last);
       }
-      const float pair[2] = {s_act[(g * seg.S + i) * 2 + 0], s_act[(g * seg.S + i) * 2 + 1]};
-      StepConsts k;
-      fold_consts<false, false>(0, 1, pair, dv, k);
-      return step_pair_exact_without_correction(k, pair[0], pair[1]);
+      bool bad = false;
+      for (int i = i0; i <= i1; ++i) {
+        const float pair[2] = {s_act[(g * seg.S + i) * 2 + 0], s_act[(g * seg.S + i) * 2 + 1]};
+        StepConsts k;
+        fold_consts<false, false>(0, 1, pair, dv, k);
+        bad |= correction_changes_a_code(k, pair[0], pair[1]);
+      }
+      return __syncthreads_or(bad) == 0;
     }
   };
   bool fast = n_mine > 0 ? correction_free(cur.g, cur.cb) : false;
