@@ -1124,6 +1124,16 @@ sq_status launch_gemm(const GemmRequest &r, cudaStream_t stream) {
     for (int j = 0; j < r.seg.n_seg; ++j)
       if ((r.seg.off[j + 1] - r.seg.off[j]) % 256 != 0) BN = 128;
   }
+  // A layer with at most half as many 256-wide tiles as SMs (a few rows) is
+  // bound by streaming its weights, not by the MMAs: 128-wide tiles put twice
+  // as many SMs on that stream.  Measured: 256 x 1536 x 1536 GEMM 18.0 ->
+  // 16.0 us, two rows x 3072 -> 18432 in six groups 27.0 -> 23.2 us; but with
+  // one row tile and one activation group (every CTA reading the same two
+  // activation rows) 26.8 -> 29.2 us, so that case keeps 256-wide tiles.
+  const int64_t m_tiles = (r.M + BM - 1) / BM;
+  if (!segk && BN == 256 && r.out_kind != OUT_PLANES && (m_tiles > 1 || r.seg.G > 1) &&
+      2 * m_tiles * ((r.N + 255) / 256) <= device_sm_count())
+    BN = 128;
   GemmParams p;
   p.M = static_cast<int32_t>(r.M);
   p.N = static_cast<int32_t>(r.N);
