@@ -153,6 +153,11 @@ __device__ __forceinline__ float max_nan(float a, float b) {
   return r;
 }
 
+// Lowers every byte equal to 128 to 127 in a word of + codes (bytes 0 .. 128):
+// bit 7 of a byte moved to its bit 0 and subtracted, with no borrow between
+// bytes.
+__device__ __forceinline__ uint32_t cap127(uint32_t w) { return w - ((w >> 7) & 0x01010101u); }
+
 // Packs the low bytes of four words into one word (byte j = low byte of word j).
 __device__ __forceinline__ uint32_t pack4_lo(uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
   return __byte_perm(__byte_perm(a, b, 0x0040), __byte_perm(c, d, 0x0040), 0x5410);
@@ -226,8 +231,8 @@ __device__ __forceinline__ void dualscale8(const float (&u)[8], const StepConsts
     round2(vp0, vp1, 128.0f, qp[j], qp[j + 1]);
     round2(vm0, vm1, -128.0f, qm[j], qm[j + 1]);
   }
-  plus = make_uint2(__vminu4(pack4_lo(qp[0], qp[1], qp[2], qp[3]), 0x7F7F7F7Fu),
-                    __vminu4(pack4_lo(qp[4], qp[5], qp[6], qp[7]), 0x7F7F7F7Fu));
+  plus = make_uint2(cap127(pack4_lo(qp[0], qp[1], qp[2], qp[3])),
+                    cap127(pack4_lo(qp[4], qp[5], qp[6], qp[7])));
   minus = make_uint2(pack4_lo(qm[0], qm[1], qm[2], qm[3]), pack4_lo(qm[4], qm[5], qm[6], qm[7]));
 }
 
@@ -247,8 +252,8 @@ __device__ __forceinline__ void dualscale8_fast(const float (&u)[8], const StepC
     round2(mul_sat(u[j], k.r7p), mul_sat(u[j + 1], k.r7p), 128.0f, qp[j], qp[j + 1]);
     round2(mul_sat(u[j], k.r7m), mul_sat(u[j + 1], k.r7m), -128.0f, qm[j], qm[j + 1]);
   }
-  plus = make_uint2(__vminu4(pack4_lo(qp[0], qp[1], qp[2], qp[3]), 0x7F7F7F7Fu),
-                    __vminu4(pack4_lo(qp[4], qp[5], qp[6], qp[7]), 0x7F7F7F7Fu));
+  plus = make_uint2(cap127(pack4_lo(qp[0], qp[1], qp[2], qp[3])),
+                    cap127(pack4_lo(qp[4], qp[5], qp[6], qp[7])));
   minus = make_uint2(pack4_lo(qm[0], qm[1], qm[2], qm[3]), pack4_lo(qm[4], qm[5], qm[6], qm[7]));
 }
 
@@ -486,14 +491,15 @@ __global__ void __launch_bounds__(256, 3) quant_act_kernel(const __grid_constant
     }
     const uint16_t *tile = reinterpret_cast<const uint16_t *>(qsmem + st * kQTileBytes);
     const int64_t r_base = static_cast<int64_t>(cur.rt) * kQRows;
-    const auto rows = [&](auto fast_form) {
+    const int rows_here = static_cast<int>(M - r_base < kQRows ? M - r_base : kQRows);
+    const auto rows = [&](auto fast_form, auto two_planes) {
       // (the uncorrected codes exist for int8 codes without a divisor only)
       constexpr bool FAST = decltype(fast_form)::value && !FP8 && !HAS_D;
-      int8_t *plus = planes + static_cast<int64_t>(cur.g) * seg.P * plane_stride + c0;
+      constexpr bool P2 = decltype(two_planes)::value;
+      int8_t *plus = planes + static_cast<int64_t>(cur.g) * (P2 ? 2 : 1) * plane_stride + c0;
 #pragma unroll 4
-      for (int rr = warp; rr < kQRows; rr += 8) {
+      for (int rr = warp; rr < rows_here; rr += 8) {
         const int64_t r = r_base + rr;
-        if (r >= M) break;
         const uint4 v = *reinterpret_cast<const uint4 *>(tile + rr * kWarpCols + lane * kColsPerThread);
         float xv[8];
         unpack8(v, xv);
@@ -510,7 +516,7 @@ __global__ void __launch_bounds__(256, 3) quant_act_kernel(const __grid_constant
           if constexpr (HAS_D) smooth8(xv, kc);  // the sign of x survives in u
           dualscale8(xv, kc, pk, nk);
         }
-        if (seg.P == 2) {
+        if constexpr (P2) {
           *reinterpret_cast<uint2 *>(plus + r * K) = pk;
           *reinterpret_cast<uint2 *>(plus + plane_stride + r * K) = nk;
         } else {
@@ -521,10 +527,17 @@ __global__ void __launch_bounds__(256, 3) quant_act_kernel(const __grid_constant
       }
     };
     if (c0 < K) {
-      if (!FP8 && !HAS_D && fast)
-        rows(std::true_type{});
-      else
-        rows(std::false_type{});
+      if (seg.P == 2) {
+        if (!FP8 && !HAS_D && fast)
+          rows(std::true_type{}, std::true_type{});
+        else
+          rows(std::false_type{}, std::true_type{});
+      } else {
+        if (!FP8 && !HAS_D && fast)
+          rows(std::true_type{}, std::false_type{});
+        else
+          rows(std::false_type{}, std::false_type{});
+      }
     }
     __syncthreads();  // every warp is done with stage st
     if (tid == 0 && it + kQStages < n_mine) {
