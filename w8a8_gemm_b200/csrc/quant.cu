@@ -216,7 +216,7 @@ __device__ __forceinline__ void quot2_sat(float u0, float u1, float r7, float m1
 // Eight channels u of one row -> X^+ and X^- codes, 8 bytes each:
 //   q+ = rne(128 v+), v+ = sat(fl(u / s+) / 128): the FP add of 1.5 * 2^23
 //        rounds to nearest even and the code is the low byte of the sum's
-//        bits; 128 is then lowered to 127 with a byte-wise unsigned min;
+//        bits; 128 is then lowered to 127 (cap127, four codes at a time);
 //   q- = -rne(128 v-), v- = sat(fl(-u / s-) / 128), codes in [-128, 0].
 // This is the case-wise Q_dual with the reference's clamps: u >= 0 (including
 // -0.0) gives a code in [0, 127] and none in X^-, u < 0 the reverse, NaN 0.
