@@ -66,7 +66,9 @@ typedef enum {
   SQ_ERR_CUDA = -5,          /* a CUDA runtime call failed                    */
   SQ_ERR_DEVICE_TIMEOUT = -6,/* a kernel gave up waiting (see status call)    */
   SQ_ERR_NO_DEVICE = -7,     /* no sm_100 device is current                   */
-  SQ_ERR_TOO_LARGE = -8      /* one row does not fit a fixed-size scratch     */
+  SQ_ERR_TOO_LARGE = -8,     /* one row does not fit a fixed-size scratch     */
+  SQ_ERR_DEVICE_BOUNDS = -9  /* debug build: a kernel skipped a store outside
+                                its buffer (see sq_debug_bounds_checks)      */
 } sq_status;
 
 typedef enum {
@@ -477,10 +479,35 @@ SQ_API sq_status sq_dualscale_seglinear_host_noalloc(const void *x_host, int64_t
 SQ_API sq_status sq_debug_timeout_probe(uint32_t limit_us, sq_stream_t stream);
 
 /*
+ * sq_debug_bounds_checks -- 1 if this library is the bounds-checked debug
+ * build (libsegquant_debug.so, compiled with SQ_DEBUG_BOUNDS), 0 for the
+ * release build.  In the debug build every plain global store of every kernel
+ * first tests its index against its buffer's logical extent (the sizes and
+ * leading dimensions of the call); a store that fails the test is skipped and
+ * the kernel records SQ_ERR_DEVICE_BOUNDS in the device error word (the first
+ * report of a launch wins), read with sq_get_device_status().  Tensor stores
+ * (TMA) are clipped to their tensor maps by the hardware and need no test.
+ * The debug build computes the same results as the release build; it exists
+ * to run the test suite with the checks in place.
+ */
+SQ_API int32_t sq_debug_bounds_checks(void);
+
+/*
+ * sq_debug_bounds_probe -- test only: launches one thread that stores through
+ * the checked path into element n of `buf` while telling the check that the
+ * buffer holds n elements.  buf: device int32 [n + 1] (the extra element is a
+ * guard, so that even an unchecked store stays inside the allocation);
+ * n >= 1.  The debug build skips the store and records SQ_ERR_DEVICE_BOUNDS;
+ * the release build launches nothing and returns SQ_ERR_UNSUPPORTED.
+ */
+SQ_API sq_status sq_debug_bounds_probe(int32_t *buf, int64_t n, sq_stream_t stream);
+
+/*
  * sq_get_device_status -- waits for the work enqueued on `stream`, then
  * returns the library's device-side error word and clears it: SQ_OK, or
  * SQ_ERR_DEVICE_TIMEOUT if a kernel's bounded wait on a barrier ran out (the
- * kernel then abandoned its tile and left its outputs incomplete).
+ * kernel then abandoned its tile and left its outputs incomplete), or, in the
+ * debug build only, SQ_ERR_DEVICE_BOUNDS.
  * The word is one per device, shared by every stream and every caller of the
  * library in the process: a report set by a kernel on another stream is seen
  * (and cleared) by whichever caller reads first, and a report set between

@@ -43,9 +43,9 @@ def test_library_exports_every_declared_symbol(L):
 
 def test_status_strings(L):
     assert B.status_string(0) == "SQ_OK"
-    for code in range(-8, 0):
+    for code in range(-9, 0):
         assert B.status_string(code).startswith("SQ_ERR_")
-    assert B.lib().sq_version() == 200
+    assert B.lib().sq_version() == 201
 
 
 def _seg(mode, offsets, groups=1):
@@ -286,3 +286,29 @@ def test_binding_choose_single_scale_takes_any_device_tensor():
     s = torch.tensor([[[1.0 / 127, 0.9 / 128]], [[1.0 / 127, 0.95 / 128]]])
     assert B.sq_choose_single_scale(s) is True
     assert B.sq_choose_single_scale(s, threshold=1.05) is False
+
+
+def test_debug_build_exports_the_same_calls_and_reports_its_checks(L):
+    """The bounds-checked debug build is a second build of the same sources:
+    it exports every declared call, and sq_debug_bounds_checks() tells the two
+    builds apart (no device is touched)."""
+    debug = ctypes.CDLL(sqbuild.build(debug=True))
+    for name in declared_entry_points():
+        assert hasattr(debug, name), name
+    debug.sq_debug_bounds_checks.restype = ctypes.c_int32
+    L.sq_debug_bounds_checks.restype = ctypes.c_int32
+    assert debug.sq_debug_bounds_checks() == 1
+    assert L.sq_debug_bounds_checks() == 0
+    debug.sq_version.restype = ctypes.c_int32
+    assert debug.sq_version() == L.sq_version()
+
+
+def test_bounds_probe_rejects_bad_arguments_on_the_host(L):
+    f = L.sq_debug_bounds_probe
+    f.argtypes = [ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p]
+    f.restype = ctypes.c_int
+    assert f(None, 8, None) == SQ_ERR_INVALID_ARG
+    assert f(ctypes.c_void_p(256), 0, None) == SQ_ERR_INVALID_ARG
+    assert f(ctypes.c_void_p(258), 8, None) == SQ_ERR_ALIGNMENT
+    # the release build launches nothing for a valid request
+    assert f(ctypes.c_void_p(256), 8, None) == SQ_ERR_UNSUPPORTED

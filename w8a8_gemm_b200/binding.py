@@ -16,9 +16,14 @@ from typing import Optional, Sequence
 
 import torch
 
-LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libsegquant.so")
+# The library: the release build, or another build of it named by the
+# environment variable SQ_LIBRARY (the test suite runs some cases against the
+# bounds-checked debug build, libsegquant_debug.so).
+LIB_PATH = os.environ.get("SQ_LIBRARY") or os.path.join(
+    os.path.dirname(os.path.abspath(__file__)), "libsegquant.so")
 
 SQ_OK = 0
+SQ_ERR_UNSUPPORTED = -2
 SQ_SEG_NONE, SQ_SEG_OUTPUT, SQ_SEG_INPUT = 0, 1, 2
 SQ_OUT_BF16, SQ_OUT_F32 = 0, 1
 SQ_MAX_SEGMENTS = 64
@@ -34,7 +39,9 @@ EXPORTED = ("sq_calibrate_act", "sq_quantize_act", "sq_quantize_weight_seg",
             "sq_host_pipeline_workspace_bytes", "sq_host_pipeline_create",
             "sq_host_pipeline_destroy", "sq_dualscale_seglinear_host",
             "sq_dualscale_seglinear_host_noalloc", "sq_choose_single_scale",
-            "sq_dualscale_seglinear_gemm_ws", "sq_gemm_workspace_bytes", "sq_debug_gemm_s32_ws")
+            "sq_dualscale_seglinear_gemm_ws", "sq_gemm_workspace_bytes", "sq_debug_gemm_s32_ws",
+            "sq_debug_bounds_checks", "sq_debug_bounds_probe")
+SQ_ERR_DEVICE_BOUNDS = -9
 SQ_NOALLOC_SCRATCH_BYTES = 32 * 1024 * 1024
 
 
@@ -119,6 +126,8 @@ def lib() -> ctypes.CDLL:
         L.sq_choose_single_scale.argtypes = [p, ctypes.c_int32, ctypes.c_int32, ctypes.c_float,
                                              ctypes.POINTER(ctypes.c_int32)]
         L.sq_debug_timeout_probe.argtypes = [ctypes.c_uint32, p]
+        L.sq_debug_bounds_checks.argtypes = []
+        L.sq_debug_bounds_probe.argtypes = [p, i64, p]
         L.sq_host_pipeline_workspace_bytes.argtypes = [i64, i64, i64, ctypes.c_int32,
                                                        ctypes.c_int32]
         L.sq_host_pipeline_workspace_bytes.restype = ctypes.c_size_t
@@ -139,7 +148,8 @@ def lib() -> ctypes.CDLL:
                   L.sq_dualscale_seglinear_gemm, L.sq_dualscale_seglinear_gemm_gelu_quant,
                   L.sq_debug_gemm_s32, L.sq_get_device_status, L.sq_choose_single_scale,
                   L.sq_dualscale_seglinear_gemm_ws, L.sq_debug_gemm_s32_ws,
-                  L.sq_version, L.sq_debug_timeout_probe):
+                  L.sq_version, L.sq_debug_timeout_probe, L.sq_debug_bounds_checks,
+                  L.sq_debug_bounds_probe):
             f.restype = ctypes.c_int
         _lib = L
     return _lib
@@ -470,6 +480,21 @@ def sq_debug_timeout_probe(limit_us: int) -> None:
     """Test only: a kernel whose bounded barrier wait runs out after limit_us;
     the timeout lands in the device error word (see sq_get_device_status)."""
     _check(lib().sq_debug_timeout_probe(int(limit_us), _stream()), "sq_debug_timeout_probe")
+
+
+def sq_debug_bounds_checks() -> bool:
+    """True if the loaded library is the bounds-checked debug build."""
+    return lib().sq_debug_bounds_checks() == 1
+
+
+def sq_debug_bounds_probe(buf: torch.Tensor, n: int) -> None:
+    """Test only (debug build): one checked store to buf[n] while the check is
+    told the buffer holds n elements; buf must hold n + 1 int32 (a guard).
+    The debug build skips the store and records SQ_ERR_DEVICE_BOUNDS."""
+    _need(buf, torch.int32, "buf")
+    if buf.numel() < n + 1:
+        raise ValueError("buf must hold n + 1 elements")
+    _check(lib().sq_debug_bounds_probe(_ptr(buf), int(n), _stream()), "sq_debug_bounds_probe")
 
 
 def sq_version() -> int:

@@ -262,8 +262,10 @@ sq_status sq_calibrate_act(const void *x, int64_t M, int64_t K, int64_t ldx, con
   if (s_act == nullptr || !aligned(s_act, 4)) return SQ_ERR_INVALID_ARG;
   if (d && !aligned(d, 4)) return SQ_ERR_ALIGNMENT;
   SQ_TRY(check_device());
+  int *status = device_status_word();
+  if (status == nullptr) return SQ_ERR_CUDA;
   return from_cuda(launch_calibrate_act(static_cast<const uint16_t *>(x), M, K, ldx, d, sp,
-                                        s_act, reinterpret_cast<cudaStream_t>(stream)));
+                                        s_act, status, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 sq_status sq_quantize_act(const void *x, int64_t M, int64_t K, int64_t ldx, const float *d,
@@ -284,8 +286,10 @@ sq_status sq_quantize_weight_seg(const void *w, int64_t N, int64_t K, const floa
   if (!aligned(w, 16) || !aligned(wq, 16) || !aligned(s_w, 4) || (d && !aligned(d, 4)))
     return SQ_ERR_ALIGNMENT;
   SQ_TRY(check_device());
+  int *status = device_status_word();
+  if (status == nullptr) return SQ_ERR_CUDA;
   return from_cuda(launch_quantize_weight(static_cast<const uint16_t *>(w), N, K, d, sp, wq, s_w,
-                                          reinterpret_cast<cudaStream_t>(stream)));
+                                          status, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 sq_status sq_quantize_weight_w4(const void *w, int64_t N, int64_t K, const float *d,
@@ -299,8 +303,10 @@ sq_status sq_quantize_weight_w4(const void *w, int64_t N, int64_t K, const float
   if (!aligned(w, 16) || !aligned(wq4, 16) || !aligned(s_w, 4) || (d && !aligned(d, 4)))
     return SQ_ERR_ALIGNMENT;
   SQ_TRY(check_device());
+  int *status = device_status_word();
+  if (status == nullptr) return SQ_ERR_CUDA;
   return from_cuda(launch_quantize_weight_w4(static_cast<const uint16_t *>(w), N, K, d, sp, wq4,
-                                             s_w, reinterpret_cast<cudaStream_t>(stream)));
+                                             s_w, status, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 sq_status sq_unpack_weight_w4(const uint8_t *wq4, int64_t N, int64_t K, int8_t *wq,
@@ -310,7 +316,10 @@ sq_status sq_unpack_weight_w4(const uint8_t *wq4, int64_t N, int64_t K, int8_t *
   if (wq4 == nullptr || wq == nullptr) return SQ_ERR_INVALID_ARG;
   if (!aligned(wq4, 16) || !aligned(wq, 16)) return SQ_ERR_ALIGNMENT;
   SQ_TRY(check_device());
-  return from_cuda(launch_unpack_w4(wq4, N, K, wq, reinterpret_cast<cudaStream_t>(stream)));
+  int *status = device_status_word();
+  if (status == nullptr) return SQ_ERR_CUDA;
+  return from_cuda(
+      launch_unpack_w4(wq4, N, K, wq, status, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 sq_status sq_dualscale_seglinear_gemm(const int8_t *planes, const int8_t *wq, const float *s_w,
@@ -376,6 +385,24 @@ sq_status sq_debug_timeout_probe(uint32_t limit_us, sq_stream_t stream) {
   return from_cuda(launch_timeout_probe(limit_us, status, reinterpret_cast<cudaStream_t>(stream)));
 }
 
+int32_t sq_debug_bounds_checks(void) {
+#ifdef SQ_DEBUG_BOUNDS
+  return 1;
+#else
+  return 0;
+#endif
+}
+
+sq_status sq_debug_bounds_probe(int32_t *buf, int64_t n, sq_stream_t stream) {
+  if (buf == nullptr || n < 1) return SQ_ERR_INVALID_ARG;
+  if (!aligned(buf, 4)) return SQ_ERR_ALIGNMENT;
+  if (!sq_debug_bounds_checks()) return SQ_ERR_UNSUPPORTED;
+  SQ_TRY(check_device());
+  int *status = device_status_word();
+  if (status == nullptr) return SQ_ERR_CUDA;
+  return from_cuda(launch_bounds_probe(buf, n, status, reinterpret_cast<cudaStream_t>(stream)));
+}
+
 sq_status sq_get_device_status(sq_stream_t stream) {
   SQ_TRY(check_device());
   int *word = device_status_word();
@@ -425,10 +452,12 @@ const char *sq_status_string(sq_status s) {
     case SQ_ERR_DEVICE_TIMEOUT: return "SQ_ERR_DEVICE_TIMEOUT: a kernel gave up waiting on a barrier";
     case SQ_ERR_NO_DEVICE: return "SQ_ERR_NO_DEVICE: no sm_100 device is current";
     case SQ_ERR_TOO_LARGE: return "SQ_ERR_TOO_LARGE: one row does not fit the fixed scratch";
+    case SQ_ERR_DEVICE_BOUNDS:
+      return "SQ_ERR_DEVICE_BOUNDS: a kernel skipped a store outside its buffer (debug build)";
   }
   return "unknown sq_status";
 }
 
-int32_t sq_version(void) { return 200; }
+int32_t sq_version(void) { return 201; }
 
 }  // extern "C"

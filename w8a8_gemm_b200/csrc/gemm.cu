@@ -162,12 +162,17 @@ struct Pieces<false> {
 // A run holds 32 words per lane of one warp, laid out [v4 group][lane][4]: each
 // store or load instruction of the warp covers 512 contiguous bytes.  `run`
 // points at the run's first word plus 4 * lane; g0 is the first v4 group.
+// (p: the workspace's extent, gridDim.x slots of sk_slot_words, for the
+// debug build's bound test)
 template <int N>
-__device__ __forceinline__ void sk_store(int32_t *run, int g0, const uint32_t *v) {
+__device__ __forceinline__ void sk_store(const GemmParams &p, int32_t *run, int g0,
+                                         const uint32_t *v) {
 #pragma unroll
-  for (int i = 0; i < N; i += 4)
-    __stcg(reinterpret_cast<uint4 *>(run + (g0 + i / 4) * 128),
-           make_uint4(v[i], v[i + 1], v[i + 2], v[i + 3]));
+  for (int i = 0; i < N; i += 4) {
+    int32_t *at = run + (g0 + i / 4) * 128;
+    if (store_ok(p.status, at >= p.sk_ws && at + 4 <= p.sk_ws + gridDim.x * p.sk_slot_words))
+      __stcg(reinterpret_cast<uint4 *>(at), make_uint4(v[i], v[i + 1], v[i + 2], v[i + 3]));
+  }
 }
 // Adds partial sums: int32 (exact) for integer codes, fp32 for FP8 codes.  The
 // loads are plain L2 loads (after the flag's acquire), so the compiler can
@@ -333,6 +338,8 @@ template <int OUT>
 __device__ __forceinline__ void store_pair(const GemmParams &p, int64_t m, int64_t n, float y0,
                                            float y1) {
   if (n >= p.N) return;
+  // y: [M][ldy], columns < N <= ldy
+  if (!store_ok(p.status, m >= 0 && m < p.M && n >= 0 && n < p.ldy)) return;
   if (OUT == OUT_BF16) {
     uint16_t *row = reinterpret_cast<uint16_t *>(p.y) + m * p.ldy;
     if (n + 1 < p.N) {
@@ -679,8 +686,8 @@ __global__ void __launch_bounds__(threads_for(EPI_WARPS), 1)
             if constexpr (POL == 2) tmem_ld_cols<CW>(t_plus + BN + c * CW, am);
             tmem_ld_wait();
             if (TAIL && role == PIECE_PARTIAL) {
-              sk_store<CW>(slot_run(blockIdx.x, c, 0), 0, ap);
-              if constexpr (POL == 2) sk_store<CW>(slot_run(blockIdx.x, c, 1), 0, am);
+              sk_store<CW>(p, slot_run(blockIdx.x, c, 0), 0, ap);
+              if constexpr (POL == 2) sk_store<CW>(p, slot_run(blockIdx.x, c, 1), 0, am);
               continue;
             }
             if (TAIL && role == PIECE_FINAL)
@@ -695,7 +702,9 @@ __global__ void __launch_bounds__(threads_for(EPI_WARPS), 1)
               int32_t *accm = accp + static_cast<int64_t>(p.M) * p.N;
 #pragma unroll
               for (int j = 0; j < CW; ++j)
-                if (n0 + j < p.N) {
+                // acc: [units][POL][M][N]
+                if (n0 + j < p.N &&
+                    store_ok(p.status, u < (SEGK ? p.S : 1) && m < p.M && n0 + j >= 0)) {
                   accp[n0 + j] = static_cast<int32_t>(ap[j]);
                   if constexpr (POL == 2) accm[n0 + j] = static_cast<int32_t>(am[j]);
                 }
@@ -719,11 +728,11 @@ __global__ void __launch_bounds__(threads_for(EPI_WARPS), 1)
             }
             tmem_ld_wait();
             if (TAIL && role == PIECE_PARTIAL) {
-              sk_store<16>(slot_run(blockIdx.x, c, 0), 0, pl);
-              sk_store<16>(slot_run(blockIdx.x, c, 0), 4, ph);
+              sk_store<16>(p, slot_run(blockIdx.x, c, 0), 0, pl);
+              sk_store<16>(p, slot_run(blockIdx.x, c, 0), 4, ph);
               if constexpr (POL == 2) {
-                sk_store<16>(slot_run(blockIdx.x, c, 1), 0, ml);
-                sk_store<16>(slot_run(blockIdx.x, c, 1), 4, mh);
+                sk_store<16>(p, slot_run(blockIdx.x, c, 1), 0, ml);
+                sk_store<16>(p, slot_run(blockIdx.x, c, 1), 4, mh);
               }
               continue;
             }
@@ -863,7 +872,8 @@ __global__ void __launch_bounds__(threads_for(EPI_WARPS), 1)
             // every lane's partials are visible before the flag is raised
             __threadfence();
             __syncwarp();
-            if (lane == 0) st_release(p.sk_flags + blockIdx.x * EPI_WARPS + ew, 1);
+            if (lane == 0 && store_ok(p.status, ew < EPI_WARPS))  // flags: [gridDim.x][EPI_WARPS]
+              st_release(p.sk_flags + blockIdx.x * EPI_WARPS + ew, 1);
           }
           if (TAIL && role == PIECE_FINAL) {
             // consumed: leave the flags at zero for the next call
@@ -871,7 +881,8 @@ __global__ void __launch_bounds__(threads_for(EPI_WARPS), 1)
             if (lane == 0)
               for (int cc = blockIdx.x + 1; cc <= sk_last; ++cc)
                 if (pc.U * cc / pc.G != pc.U * (cc + 1) / pc.G)
-                  p.sk_flags[cc * EPI_WARPS + ew] = 0;
+                  if (store_ok(p.status, cc < static_cast<int>(gridDim.x)))
+                    p.sk_flags[cc * EPI_WARPS + ew] = 0;
           }
           tc_fence_before();
           __syncwarp();
@@ -923,7 +934,8 @@ __global__ void __launch_bounds__(threads_for(EPI_WARPS), 1)
                 if (odd) { w[0] = s0; w[2] = s1; } else { w[1] = s0; w[3] = s1; }
               }
               const int64_t n0 = nb + 8 * q;
-              if (mr < p.M && n0 < p.N) {
+              // y: [M][ldy], columns < N <= ldy
+              if (mr < p.M && n0 < p.N && store_ok(p.status, mr >= 0 && n0 >= 0 && n0 < p.ldy)) {
                 uint16_t *row = reinterpret_cast<uint16_t *>(p.y) + mr * p.ldy;
                 if (n0 + 8 <= p.N) {
                   *reinterpret_cast<uint4 *>(row + n0) = make_uint4(w[0], w[1], w[2], w[3]);

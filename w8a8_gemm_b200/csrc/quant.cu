@@ -47,7 +47,8 @@ __device__ __forceinline__ void unpack8(const uint4 &v, float (&x)[8]) {
 __global__ void __launch_bounds__(256) calib_reduce_kernel(const uint16_t *__restrict__ x,
                                                            int64_t M, int64_t K, int64_t ldx,
                                                            const float *__restrict__ d,
-                                                           SegParams seg, float *s_act) {
+                                                           SegParams seg, float *s_act,
+                                                           int *status) {
   const int g = blockIdx.z;
   const int64_t c0 = (static_cast<int64_t>(blockIdx.x) * 32 + threadIdx.x) * kColsPerThread;
   if (c0 >= K) return;
@@ -73,7 +74,8 @@ __global__ void __launch_bounds__(256) calib_reduce_kernel(const uint16_t *__res
   const unsigned group = __match_any_sync(__activemask(), i);
   const unsigned hib = __reduce_max_sync(group, __float_as_uint(hi));
   const unsigned nlob = __reduce_max_sync(group, __float_as_uint(nlo));
-  if ((threadIdx.x & 31) == __ffs(group) - 1) {
+  if ((threadIdx.x & 31) == __ffs(group) - 1 &&
+      store_ok(status, g < seg.G && i < seg.S)) {  // s_act: [G][S][2]
     unsigned int *slot = reinterpret_cast<unsigned int *>(s_act + (g * seg.S + i) * 2);
     if (hib) atomicMax(slot, hib);
     if (nlob) atomicMax(slot + 1, nlob);
@@ -83,9 +85,10 @@ __global__ void __launch_bounds__(256) calib_reduce_kernel(const uint16_t *__res
 // Pass 2: s+ = max / 127, s- = |min| / 128; an empty side gets step 1.  In
 // single-scale mode both take max(max, |min|) / 127.  FP8 (E4M3): both
 // divisors are 448.
-__global__ void calib_finalize_kernel(float *s_act, int n, int single, int fp8) {
+__global__ void calib_finalize_kernel(float *s_act, int n, int single, int fp8, int *status) {
   const float qp = fp8 ? 448.0f : 127.0f, qm = fp8 ? 448.0f : 128.0f;
   for (int t = threadIdx.x; t < n; t += blockDim.x) {
+    if (!store_ok(status, 2 * t + 1 < 2 * n)) continue;
     const float hi = s_act[2 * t], nlo = s_act[2 * t + 1];
     if (single) {
       const float amax = hi > nlo ? hi : nlo;
@@ -516,6 +519,12 @@ __global__ void __launch_bounds__(256, 3) quant_act_kernel(const __grid_constant
           if constexpr (HAS_D) smooth8(xv, kc);  // the sign of x survives in u
           dualscale8(xv, kc, pk, nk);
         }
+        // planes: [G][P][M][K]; this row's 8 codes of each plane
+        const int64_t at = (plus - planes) + r * K;
+        if (!store_ok(status, at >= 0 && r < M && c0 + 8 <= K &&
+                                  at + (P2 ? plane_stride : 0) + 8 <=
+                                      static_cast<int64_t>(seg.G) * seg.P * plane_stride))
+          continue;
         if constexpr (P2) {
           *reinterpret_cast<uint2 *>(plus + r * K) = pk;
           *reinterpret_cast<uint2 *>(plus + plane_stride + r * K) = nk;
@@ -579,7 +588,8 @@ __global__ void __launch_bounds__(256) quant_weight_kernel(const uint16_t *__res
                                                            const float *__restrict__ d,
                                                            SegParams seg,
                                                            int8_t *__restrict__ wq,
-                                                           float *__restrict__ s_w) {
+                                                           float *__restrict__ s_w,
+                                                           int *status) {
   constexpr float kQ = static_cast<float>(QMAX);
   __shared__ float red[32];
   const int64_t n = blockIdx.x;
@@ -596,23 +606,27 @@ __global__ void __launch_bounds__(256) quant_weight_kernel(const uint16_t *__res
     }
     amax = block_max(amax, red);
     const float s = amax > 0.0f ? __fdiv_rn(amax, kQ) : 1.0f;
-    if (threadIdx.x == 0) s_w[i * N + n] = s;
+    if (threadIdx.x == 0 && store_ok(status, i < seg.S && n < N)) s_w[i * N + n] = s;  // [S][N]
     const auto wval = [&](int64_t k) {
       return dg ? __fmul_rn(bf16_bits_to_f32(row[k]), dg[k]) : bf16_bits_to_f32(row[k]);
     };
+    // wq: [N][K] (int8 and FP8 codes) or [N][K / 2] (packed W4 pairs)
     if constexpr (QMAX == 127) {
       for (int64_t k = k0 + threadIdx.x; k < k1; k += blockDim.x)
-        wq[n * K + k] = static_cast<int8_t>(weight_code(wval(k), s, kQ));
+        if (store_ok(status, n < N && k < K))
+          wq[n * K + k] = static_cast<int8_t>(weight_code(wval(k), s, kQ));
     } else if constexpr (QMAX == 448) {
       for (int64_t k = k0 + threadIdx.x; k < k1; k += blockDim.x)
-        wq[n * K + k] = static_cast<int8_t>(
-            __nv_cvt_float_to_fp8(__fdiv_rn(wval(k), s), __NV_SATFINITE, __NV_E4M3));
+        if (store_ok(status, n < N && k < K))
+          wq[n * K + k] = static_cast<int8_t>(
+              __nv_cvt_float_to_fp8(__fdiv_rn(wval(k), s), __NV_SATFINITE, __NV_E4M3));
     } else {
       // segment bounds are even (multiples of 32), so pairs never straddle one
       uint8_t *packed = reinterpret_cast<uint8_t *>(wq) + n * (K / 2);
       for (int64_t j = k0 / 2 + threadIdx.x; j < k1 / 2; j += blockDim.x) {
         const int lo = weight_code(wval(2 * j), s, kQ), hi = weight_code(wval(2 * j + 1), s, kQ);
-        packed[j] = static_cast<uint8_t>((lo & 0xF) | ((hi & 0xF) << 4));
+        if (store_ok(status, n < N && 2 * j + 1 < K))
+          packed[j] = static_cast<uint8_t>((lo & 0xF) | ((hi & 0xF) << 4));
       }
     }
   }
@@ -622,9 +636,11 @@ __global__ void __launch_bounds__(256) quant_weight_kernel(const uint16_t *__res
 // nibble of its own byte (low nibble 0), so no sign extension is needed.  One
 // thread per 8 packed bytes (16 codes); a grid-stride loop over N*K/16 units.
 __global__ void __launch_bounds__(256) unpack_w4_kernel(const uint2 *__restrict__ src,
-                                                        uint4 *__restrict__ dst, int64_t units) {
+                                                        uint4 *__restrict__ dst, int64_t units,
+                                                        int *status) {
   for (int64_t u = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; u < units;
        u += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    if (!store_ok(status, u >= 0 && u < units)) continue;  // dst: [N * K / 16] uint4
     const uint2 v = src[u];
     const uint32_t e0 = (v.x & 0x0F0F0F0Fu) << 4, o0 = v.x & 0xF0F0F0F0u;  // channels 2j, 2j+1
     const uint32_t e1 = (v.y & 0x0F0F0F0Fu) << 4, o1 = v.y & 0xF0F0F0F0u;
@@ -648,7 +664,7 @@ int num_sms() {
 
 cudaError_t launch_calibrate_act(const uint16_t *x, int64_t M, int64_t K, int64_t ldx,
                                  const float *d, const SegParams &seg, float *s_act,
-                                 cudaStream_t stream) {
+                                 int *status, cudaStream_t stream) {
   const int n = seg.G * seg.S;
   cudaError_t e = cudaMemsetAsync(s_act, 0, sizeof(float) * 2 * n, stream);
   if (e != cudaSuccess) return e;
@@ -658,11 +674,11 @@ cudaError_t launch_calibrate_act(const uint16_t *x, int64_t M, int64_t K, int64_
     const int cap = (num_sms() * 4 + gx * seg.G - 1) / (gx * seg.G);
     if (gy > cap) gy = cap < 1 ? 1 : cap;
     calib_reduce_kernel<<<dim3(gx, gy, seg.G), dim3(32, kRowsPerBlock), 0, stream>>>(
-        x, M, K, ldx, d, seg, s_act);
+        x, M, K, ldx, d, seg, s_act, status);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
-  calib_finalize_kernel<<<1, 256, 0, stream>>>(s_act, n, seg.P == 1 ? 1 : 0, seg.fp8);
+  calib_finalize_kernel<<<1, 256, 0, stream>>>(s_act, n, seg.P == 1 ? 1 : 0, seg.fp8, status);
   return cudaGetLastError();
 }
 
@@ -711,28 +727,28 @@ sq_status launch_quantize_act(const uint16_t *x, int64_t M, int64_t K, int64_t l
 }
 
 cudaError_t launch_quantize_weight(const uint16_t *w, int64_t N, int64_t K, const float *d,
-                                   const SegParams &seg, int8_t *wq, float *s_w,
+                                   const SegParams &seg, int8_t *wq, float *s_w, int *status,
                                    cudaStream_t stream) {
   if (N == 0) return cudaSuccess;
   if (seg.fp8)
     quant_weight_kernel<448><<<static_cast<unsigned>(N), 256, 0, stream>>>(w, N, K, d, seg, wq,
-                                                                          s_w);
+                                                                          s_w, status);
   else
     quant_weight_kernel<127><<<static_cast<unsigned>(N), 256, 0, stream>>>(w, N, K, d, seg, wq,
-                                                                          s_w);
+                                                                          s_w, status);
   return cudaGetLastError();
 }
 
 cudaError_t launch_quantize_weight_w4(const uint16_t *w, int64_t N, int64_t K, const float *d,
                                       const SegParams &seg, uint8_t *wq4, float *s_w,
-                                      cudaStream_t stream) {
+                                      int *status, cudaStream_t stream) {
   if (N == 0) return cudaSuccess;
   quant_weight_kernel<7><<<static_cast<unsigned>(N), 256, 0, stream>>>(
-      w, N, K, d, seg, reinterpret_cast<int8_t *>(wq4), s_w);
+      w, N, K, d, seg, reinterpret_cast<int8_t *>(wq4), s_w, status);
   return cudaGetLastError();
 }
 
-cudaError_t launch_unpack_w4(const uint8_t *wq4, int64_t N, int64_t K, int8_t *wq,
+cudaError_t launch_unpack_w4(const uint8_t *wq4, int64_t N, int64_t K, int8_t *wq, int *status,
                              cudaStream_t stream) {
   const int64_t units = N * K / 16;  // K % 16 == 0
   if (units == 0) return cudaSuccess;
@@ -740,7 +756,7 @@ cudaError_t launch_unpack_w4(const uint8_t *wq4, int64_t N, int64_t K, int8_t *w
   const int64_t cap = static_cast<int64_t>(num_sms()) * 8;
   if (blocks > cap) blocks = cap;
   unpack_w4_kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(
-      reinterpret_cast<const uint2 *>(wq4), reinterpret_cast<uint4 *>(wq), units);
+      reinterpret_cast<const uint2 *>(wq4), reinterpret_cast<uint4 *>(wq), units, status);
   return cudaGetLastError();
 }
 

@@ -21,6 +21,22 @@ struct SegParams {
   int32_t off[SQ_MAX_SEGMENTS + 1];
 };
 
+// Guard of a plain global store: `ok` is the test of the store's index against
+// its buffer's logical extent.  In the bounds-checked debug build
+// (SQ_DEBUG_BOUNDS) a failed test records SQ_ERR_DEVICE_BOUNDS in `status`
+// (first report wins) and the caller skips the store; in the release build the
+// guard is always true and costs nothing.
+__device__ __forceinline__ bool store_ok(int *status, bool ok) {
+#ifdef SQ_DEBUG_BOUNDS
+  if (!ok) atomicCAS(status, 0, static_cast<int>(SQ_ERR_DEVICE_BOUNDS));
+  return ok;
+#else
+  (void)status;
+  (void)ok;
+  return true;
+#endif
+}
+
 // Index i with off[i] <= p < off[i + 1] (tables are short: a linear scan).
 __host__ __device__ inline int seg_index(const int32_t *off, int n_seg, int64_t p) {
   int i = 0;
@@ -31,17 +47,17 @@ __host__ __device__ inline int seg_index(const int32_t *off, int n_seg, int64_t 
 // ---- launchers (quant.cu) --------------------------------------------------
 cudaError_t launch_calibrate_act(const uint16_t *x, int64_t M, int64_t K, int64_t ldx,
                                  const float *d, const SegParams &seg, float *s_act,
-                                 cudaStream_t stream);
+                                 int *status, cudaStream_t stream);
 sq_status launch_quantize_act(const uint16_t *x, int64_t M, int64_t K, int64_t ldx,
                               const float *d, const float *s_act, const SegParams &seg,
                               int8_t *planes, int *status, cudaStream_t stream);
 cudaError_t launch_quantize_weight(const uint16_t *w, int64_t N, int64_t K, const float *d,
-                                   const SegParams &seg, int8_t *wq, float *s_w,
+                                   const SegParams &seg, int8_t *wq, float *s_w, int *status,
                                    cudaStream_t stream);
 cudaError_t launch_quantize_weight_w4(const uint16_t *w, int64_t N, int64_t K, const float *d,
                                       const SegParams &seg, uint8_t *wq4, float *s_w,
-                                      cudaStream_t stream);
-cudaError_t launch_unpack_w4(const uint8_t *wq4, int64_t N, int64_t K, int8_t *wq,
+                                      int *status, cudaStream_t stream);
+cudaError_t launch_unpack_w4(const uint8_t *wq4, int64_t N, int64_t K, int8_t *wq, int *status,
                              cudaStream_t stream);
 
 // ---- launcher (gemm.cu) ----------------------------------------------------
@@ -76,8 +92,10 @@ sq_status launch_gemm(const GemmRequest &req, cudaStream_t stream);
 // current device.
 size_t gemm_workspace_bytes();
 
-// ---- test-only probe (probe.cu) --------------------------------------------
+// ---- test-only probes (probe.cu) -------------------------------------------
 cudaError_t launch_timeout_probe(uint32_t limit_us, int *status, cudaStream_t stream);
+// Debug build only: one checked store to element n of a buffer said to hold n.
+cudaError_t launch_bounds_probe(int32_t *buf, int64_t n, int *status, cudaStream_t stream);
 
 // Host-side validation of a quantize / GEMM call without launching anything
 // (the checks of sq_quantize_act and sq_dualscale_seglinear_gemm).
