@@ -189,6 +189,41 @@ SQ_API sq_status sq_quantize_act(const void *x, int64_t M, int64_t K, int64_t ld
                           sq_stream_t stream);
 
 /*
+ * sq_quantize_act_plan -- for layers with SmoothQuant divisors: decides, per
+ * activation group and channel, whether the quantizer may form that channel's
+ * codes without either quotient's correction (u = RN(x * fl(1/d)), then the
+ * code of RN(u * fl(1/s)) -- one product each) and still produce exactly the
+ * codes of sq_quantize_act for every bf16 input.  (A speed-up of the same
+ * Q_dual; the pages define only the codes.)  Both forms lie within 2^-22 of
+ * x / (d s), so they can differ only for x next to a rounding boundary
+ * (h + 1/2) s d, h = 0 .. 127; the plan evaluates both forms on the bf16
+ * neighbours of each boundary (768 inputs per channel) with the kernels' own
+ * operations.  Call it once per layer after sq_calibrate_act (it depends on
+ * d, the steps and the segment table only).
+ *   d      fp32 [G][K] device (required);  s_act fp32 [G][S][2] device
+ *   plan   uint32 [G][ceil(K / 32)] device output, 4-byte aligned: bit c % 32
+ *          of word [g][c / 32] set when channel c of group g qualifies
+ *          (also set for the padding channels past K)
+ * int8 codes only: SQ_FLAG_FP8 gives SQ_ERR_UNSUPPORTED.
+ */
+SQ_API sq_status sq_quantize_act_plan(const float *d, int64_t K, const float *s_act,
+                                      const sq_segments *seg, uint32_t *plan,
+                                      sq_stream_t stream);
+
+/*
+ * sq_quantize_act_planned -- sq_quantize_act with a plan of
+ * sq_quantize_act_plan made from the same d, s_act and segment table: every
+ * 256-channel block whose channels all qualify takes the codes without the
+ * corrections; the others, as sq_quantize_act.  The planes are bit for bit
+ * those of sq_quantize_act.  plan NULL: exactly sq_quantize_act.  A plan
+ * without d is SQ_ERR_INVALID_ARG; with SQ_FLAG_FP8, SQ_ERR_UNSUPPORTED.
+ */
+SQ_API sq_status sq_quantize_act_planned(const void *x, int64_t M, int64_t K, int64_t ldx,
+                                         const float *d, const float *s_act,
+                                         const sq_segments *seg, const uint32_t *plan,
+                                         int8_t *planes, sq_stream_t stream);
+
+/*
  * sq_quantize_weight_seg -- segment-wise symmetric AMax weight quantization
  * (offline, once per layer).  Pages: papernotes.org section SegLinear (each
  * segment of W quantized independently) and AMax calibrator.

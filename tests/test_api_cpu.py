@@ -312,3 +312,30 @@ def test_bounds_probe_rejects_bad_arguments_on_the_host(L):
     assert f(ctypes.c_void_p(258), 8, None) == SQ_ERR_ALIGNMENT
     # the release build launches nothing for a valid request
     assert f(ctypes.c_void_p(256), 8, None) == SQ_ERR_UNSUPPORTED
+
+
+def test_quantize_plan_rejects_bad_arguments_on_the_host(L):
+    """The plan and the planned quantize check their arguments before touching
+    a device: a plan needs divisors, covers int8 codes only, and is 4-byte
+    aligned."""
+    plan_f = L.sq_quantize_act_plan
+    plan_f.argtypes = [ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p, ctypes.c_void_p,
+                       ctypes.c_void_p, ctypes.c_void_p]
+    plan_f.restype = ctypes.c_int
+    seg = B.Segments()
+    cs, keep = seg._c()
+    ok = ctypes.c_void_p(256)
+    assert plan_f(None, 256, ok, ctypes.byref(cs), ok, None) == SQ_ERR_INVALID_ARG
+    assert plan_f(ok, 256, ok, ctypes.byref(cs), None, None) == SQ_ERR_INVALID_ARG
+    assert plan_f(ok, 256, ok, ctypes.byref(cs), ctypes.c_void_p(258), None) == SQ_ERR_ALIGNMENT
+    assert plan_f(ok, 100, ok, ctypes.byref(cs), ok, None) != 0     # K must be a multiple of 16
+    cs8, keep8 = B.Segments(flags=B.SQ_FLAG_FP8)._c()
+    assert plan_f(ok, 256, ok, ctypes.byref(cs8), ok, None) == SQ_ERR_UNSUPPORTED
+    q = L.sq_quantize_act_planned
+    q.argtypes = [ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64, ctypes.c_void_p,
+                  ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+                  ctypes.c_void_p]
+    q.restype = ctypes.c_int
+    # a plan without divisors
+    assert q(ok, 4, 256, 256, None, ok, ctypes.byref(cs), ok, ok, None) == SQ_ERR_INVALID_ARG
+    assert q(ok, 4, 256, 256, ok, ok, ctypes.byref(cs8), ok, ok, None) == SQ_ERR_UNSUPPORTED

@@ -43,5 +43,7 @@ def test_every_exported_name_has_a_wrapper_or_is_internal():
                 # reached through sq_dualscale_seglinear_gemm / sq_debug_gemm_s32
                 # with workspace=, and through gemm_workspace()
                 "sq_dualscale_seglinear_gemm_ws", "sq_debug_gemm_s32_ws",
-                "sq_gemm_workspace_bytes"}
+                "sq_gemm_workspace_bytes",
+                # reached through sq_quantize_act(..., plan=)
+                "sq_quantize_act_planned"}
     assert set(B.EXPORTED) - wrapped <= internal

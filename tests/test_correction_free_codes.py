@@ -61,3 +61,42 @@ def test_powers_of_two_and_calibrated_steps_pass():
              == passes_candidate_test(np.float32(m) / np.float32(127), np.float32(m) / np.float32(128))
              for m in rng.uniform(0.1, 40, 40)]
     assert all(agree)
+
+
+# ---------------------------------------------- with SmoothQuant divisors
+from correction_free import (channel_forms_agree_everywhere_d, channel_passes_test_d,  # noqa: E402
+                             codes_d, divisors_where_forms_differ)
+
+
+@pytest.mark.parametrize("seed", range(3))
+def test_channel_test_is_exact_with_divisors(seed):
+    """With a divisor d, the per-channel test (the bf16 neighbours of
+    fl(fl((h + 1/2) s) d)) passes iff the doubly uncorrected codes equal the
+    exact ones on every bf16 input, over log-uniform d and steps."""
+    rng = np.random.default_rng(300 + seed)
+    n_fast = 0
+    for _ in range(40):
+        d = np.float32(np.exp2(rng.uniform(-6, 6)))
+        sp, sm = np.exp2(rng.uniform(-20, 8, 2)).astype(np.float32)
+        ok = channel_passes_test_d(d, sp, sm)
+        assert ok == channel_forms_agree_everywhere_d(d, sp, sm), (float(d), float(sp), float(sm))
+        n_fast += ok
+    assert n_fast > 10
+
+
+def test_channel_test_rejects_constructed_divisors():
+    s = np.float32(float.fromhex("0x1.0adc5p-7"))
+    for d in divisors_where_forms_differ(8, s, seed=17):
+        d = np.float32(d)
+        assert not channel_forms_agree_everywhere_d(d, s, s)
+        assert not channel_passes_test_d(d, s, s), float(d)
+        assert not channel_passes_test_d(d, s, np.float32(1 / 64)), float(d)
+
+
+def test_divisor_one_reduces_to_the_plain_forms():
+    s = np.float32(float.fromhex("0x1.fd0eb8p-8"))
+    x = np.array([0x3EAD, 0xBEAD], np.uint16)
+    exact = codes_d(x, np.float32(1), s, s, False)
+    fast = codes_d(x, np.float32(1), s, s, True)
+    assert (exact[0][0], exact[1][1]) == (43, -43)
+    assert (fast[0][0], fast[1][1]) == (44, -44)

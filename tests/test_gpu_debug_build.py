@@ -38,7 +38,7 @@ def test_suites_pass_under_the_debug_build():
     env = dict(os.environ, SQ_LIBRARY=lib)
     files = ["debug_build_cases.py", "test_gpu_parity.py", "test_gpu_fuzz.py",
              "test_gpu_split_tail.py", "test_gpu_w4.py", "test_gpu_single_scale.py",
-             "test_gpu_fp8.py", "test_gpu_host.py"]
+             "test_gpu_fp8.py", "test_gpu_host.py", "test_gpu_quantize_plan.py"]
     cmd = [sys.executable, "-m", "pytest", "-q", "-x", "-m", "gpu", "-p", "no:cacheprovider",
            "-k", "not full_size and not ffn_workload",
            *[os.path.join(HERE, f) for f in files]]

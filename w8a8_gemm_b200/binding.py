@@ -40,7 +40,8 @@ EXPORTED = ("sq_calibrate_act", "sq_quantize_act", "sq_quantize_weight_seg",
             "sq_host_pipeline_destroy", "sq_dualscale_seglinear_host",
             "sq_dualscale_seglinear_host_noalloc", "sq_choose_single_scale",
             "sq_dualscale_seglinear_gemm_ws", "sq_gemm_workspace_bytes", "sq_debug_gemm_s32_ws",
-            "sq_debug_bounds_checks", "sq_debug_bounds_probe")
+            "sq_debug_bounds_checks", "sq_debug_bounds_probe",
+            "sq_quantize_act_plan", "sq_quantize_act_planned")
 SQ_ERR_DEVICE_BOUNDS = -9
 SQ_NOALLOC_SCRATCH_BYTES = 32 * 1024 * 1024
 
@@ -109,6 +110,8 @@ def lib() -> ctypes.CDLL:
         seg = ctypes.POINTER(_Segments)
         L.sq_calibrate_act.argtypes = [p, i64, i64, i64, p, seg, p, p]
         L.sq_quantize_act.argtypes = [p, i64, i64, i64, p, p, seg, p, p]
+        L.sq_quantize_act_plan.argtypes = [p, i64, p, seg, p, p]
+        L.sq_quantize_act_planned.argtypes = [p, i64, i64, i64, p, p, seg, p, p, p]
         L.sq_quantize_weight_seg.argtypes = [p, i64, i64, p, seg, p, p, p]
         L.sq_quantize_weight_w4.argtypes = [p, i64, i64, p, seg, p, p, p]
         L.sq_unpack_weight_w4.argtypes = [p, i64, i64, p, p]
@@ -149,7 +152,7 @@ def lib() -> ctypes.CDLL:
                   L.sq_debug_gemm_s32, L.sq_get_device_status, L.sq_choose_single_scale,
                   L.sq_dualscale_seglinear_gemm_ws, L.sq_debug_gemm_s32_ws,
                   L.sq_version, L.sq_debug_timeout_probe, L.sq_debug_bounds_checks,
-                  L.sq_debug_bounds_probe):
+                  L.sq_debug_bounds_probe, L.sq_quantize_act_plan, L.sq_quantize_act_planned):
             f.restype = ctypes.c_int
         _lib = L
     return _lib
@@ -204,19 +207,46 @@ def sq_calibrate_act(x: torch.Tensor, d: Optional[torch.Tensor], seg: Segments,
 
 
 def sq_quantize_act(x: torch.Tensor, d: Optional[torch.Tensor], s_act: torch.Tensor,
-                    seg: Segments, planes: torch.Tensor) -> torch.Tensor:
-    """DualScale quantization of X / d into planes int8 [G][P][M][K]."""
+                    seg: Segments, planes: torch.Tensor,
+                    plan: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """DualScale quantization of X / d into planes int8 [G][P][M][K]; with a
+    plan from sq_quantize_act_plan (same d, s_act, seg), sq_quantize_act_planned."""
     _need(x, torch.bfloat16, "x")
     _need(d, torch.float32, "d", optional=True)
     _need(s_act, torch.float32, "s_act")
     _need(planes, torch.int8, "planes")
+    _need(plan, torch.int32, "plan", optional=True)
     M, K, ldx = _rows(x)
     if tuple(planes.shape) != (seg.n_groups, seg.P, M, K) or not planes.is_contiguous():
         raise ValueError(f"planes must be contiguous [{seg.n_groups}, {seg.P}, {M}, {K}]")
     cs, keep = seg._c()
-    _check(lib().sq_quantize_act(_ptr(x), M, K, ldx, _ptr(d), _ptr(s_act), ctypes.byref(cs),
-                                 _ptr(planes), _stream()), "sq_quantize_act")
+    if plan is None:
+        _check(lib().sq_quantize_act(_ptr(x), M, K, ldx, _ptr(d), _ptr(s_act), ctypes.byref(cs),
+                                     _ptr(planes), _stream()), "sq_quantize_act")
+    else:
+        _check(lib().sq_quantize_act_planned(_ptr(x), M, K, ldx, _ptr(d), _ptr(s_act),
+                                             ctypes.byref(cs), _ptr(plan), _ptr(planes),
+                                             _stream()), "sq_quantize_act_planned")
     return planes
+
+
+def sq_quantize_act_plan(d: torch.Tensor, s_act: torch.Tensor, seg: Segments,
+                         plan: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """Per (group, channel) bits [G][ceil(K/32)] (int32 storage of the uint32
+    words): channels whose codes may skip both quotient corrections."""
+    _need(d, torch.float32, "d")
+    _need(s_act, torch.float32, "s_act")
+    K = d.shape[-1]
+    words = (K + 31) // 32
+    if plan is None:
+        plan = torch.empty(seg.n_groups, words, dtype=torch.int32, device=d.device)
+    _need(plan, torch.int32, "plan")
+    if tuple(plan.shape) != (seg.n_groups, words) or not plan.is_contiguous():
+        raise ValueError(f"plan must be contiguous int32 [{seg.n_groups}, {words}]")
+    cs, keep = seg._c()
+    _check(lib().sq_quantize_act_plan(_ptr(d), K, _ptr(s_act), ctypes.byref(cs), _ptr(plan),
+                                      _stream()), "sq_quantize_act_plan")
+    return plan
 
 
 def sq_quantize_weight_seg(w: torch.Tensor, d: Optional[torch.Tensor], seg: Segments,

@@ -186,20 +186,24 @@ sq_status gemm_common(const int8_t *planes, const int8_t *wq, const float *s_w,
 
 sq_status quantize_common(const void *x, int64_t M, int64_t K, int64_t ldx, const float *d,
                           const float *s_act, const sq_segments *seg, int8_t *planes,
-                          cudaStream_t stream, bool launch = true) {
+                          cudaStream_t stream, bool launch = true,
+                          const uint32_t *plan = nullptr) {
   SQ_TRY(check_act(x, M, K, ldx));
   SegParams sp;
   SQ_TRY(parse_segments(seg, K, -1, &sp));
+  if (plan != nullptr && d == nullptr) return SQ_ERR_INVALID_ARG;  // a plan is per divisor
+  if (plan != nullptr && sp.fp8) return SQ_ERR_UNSUPPORTED;      // it covers int8 codes
   if (M == 0) return SQ_OK;
   if (s_act == nullptr || planes == nullptr) return SQ_ERR_INVALID_ARG;
-  if (!aligned(s_act, 4) || (d && !aligned(d, 4)) || !aligned(planes, 16))
+  if (!aligned(s_act, 4) || (d && !aligned(d, 4)) || !aligned(planes, 16) ||
+      (plan && !aligned(plan, 4)))
     return SQ_ERR_ALIGNMENT;
   SQ_TRY(check_device());
   if (!launch) return SQ_OK;
   int *status = device_status_word();
   if (status == nullptr) return SQ_ERR_CUDA;
   return launch_quantize_act(static_cast<const uint16_t *>(x), M, K, ldx, d, s_act, sp, planes,
-                             status, stream);
+                             plan, status, stream);
 }
 
 }  // namespace
@@ -273,6 +277,28 @@ sq_status sq_quantize_act(const void *x, int64_t M, int64_t K, int64_t ldx, cons
                           sq_stream_t stream) {
   return quantize_common(x, M, K, ldx, d, s_act, seg, planes,
                          reinterpret_cast<cudaStream_t>(stream));
+}
+
+sq_status sq_quantize_act_plan(const float *d, int64_t K, const float *s_act,
+                               const sq_segments *seg, uint32_t *plan, sq_stream_t stream) {
+  SQ_TRY(check_k(K));
+  SegParams sp;
+  SQ_TRY(parse_segments(seg, K, -1, &sp));
+  if (d == nullptr || s_act == nullptr || plan == nullptr) return SQ_ERR_INVALID_ARG;
+  if (sp.fp8) return SQ_ERR_UNSUPPORTED;
+  if (!aligned(d, 4) || !aligned(s_act, 4) || !aligned(plan, 4)) return SQ_ERR_ALIGNMENT;
+  SQ_TRY(check_device());
+  int *status = device_status_word();
+  if (status == nullptr) return SQ_ERR_CUDA;
+  return from_cuda(
+      launch_quantize_plan(d, K, s_act, sp, plan, status, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+sq_status sq_quantize_act_planned(const void *x, int64_t M, int64_t K, int64_t ldx,
+                                  const float *d, const float *s_act, const sq_segments *seg,
+                                  const uint32_t *plan, int8_t *planes, sq_stream_t stream) {
+  return quantize_common(x, M, K, ldx, d, s_act, seg, planes,
+                         reinterpret_cast<cudaStream_t>(stream), true, plan);
 }
 
 sq_status sq_quantize_weight_seg(const void *w, int64_t N, int64_t K, const float *d,

@@ -25,6 +25,8 @@ constexpr int kRowsPerBlock = 8;                      // warps per block
 constexpr int kQRows = 32;                            // rows per staged tile
 constexpr int kQStages = 4;                           // tiles in flight per block
 constexpr int kQTileBytes = kQRows * kWarpCols * 2;   // 16 KB of bf16
+constexpr int kFixMax = 16;                           // channels a column block may patch
+constexpr int kFixOffset = kQStages * kQTileBytes + 64;  // the warps' lists, after the barriers
 constexpr uint64_t kQuantWaitNs = 2000000000ull;      // bounded wait on a tile: 2 s
 
 __device__ __forceinline__ float bf16_bits_to_f32(uint32_t h) {
@@ -201,6 +203,16 @@ __device__ __forceinline__ void smooth8(float (&x)[8], const StepConsts &k) {
   }
 }
 
+// u = RN(x fl(1/d)) for eight channels, without the correction and the clamp:
+// for channels whose codes a quantize plan shows to be the same as with both
+// corrections (an overflowing product saturates its code like the clamped
+// quotient, and NaN stays NaN).
+__device__ __forceinline__ void scale8(float (&x)[8], const StepConsts &k) {
+#pragma unroll
+  for (int j = 0; j < 8; j += 2)
+    unpack2(fmul2(pack2(x[j], x[j + 1]), pack2(k.rd[j], k.rd[j + 1])), x[j], x[j + 1]);
+}
+
 // sat(fl(u / s) / 128) for two channels of one polarity, everything scaled by
 // 2^-7 (exact) so that .sat clamps to the code range: q0 = sat(u fl(1/s)/128)
 // (x on the other side of zero, NaN and overflow all clamp), the residual
@@ -353,6 +365,16 @@ __device__ __forceinline__ void fetch_scales(int g, int64_t c0, int64_t K, const
     for (int j = 0; j < 8; ++j) dv[j] = d[g * K + c0 + j];
   }
 }
+// The quantize plan's bits for one thread's eight channels c0 .. c0 + 7 of
+// group g (0xFF when all may skip the corrections; channels past K count as
+// set; 0 without a plan), read beside the scales for the same reason.
+__device__ __forceinline__ uint32_t plan_bits8(const uint32_t *plan, int g, int64_t c0,
+                                               int64_t K) {
+  if (plan == nullptr) return 0u;
+  if (c0 >= K) return 0xFFu;
+  const int64_t words = (K + 31) / 32;
+  return (plan[g * words + c0 / 32] >> (c0 & 31)) & 0xFFu;
+}
 template <bool FP8, bool HAS_D>
 __device__ __forceinline__ void fold_consts(int64_t c0, int64_t K, const float (&sc)[2],
                                             const float (&dv)[8], StepConsts &k) {
@@ -403,6 +425,92 @@ struct UnitCursor {
   }
 };
 
+// With divisors and a quantize plan, a column block whose plan leaves out a
+// few channels still takes the uncorrected codes, and each warp then rewrites
+// the codes of those channels in its rows with the exact form (patch_codes).
+// build_fix_list puts the left-out channels of this thread's column block --
+// enumerated by bit of the lanes' eight plan bits, then by lane -- with their
+// constants (folded exactly as fold_consts does) into the warp's list: entry i
+// = {channel offset in the block, fl(1/d), -d, the clamp} and {r7p, m128p,
+// r7m, m128m}.  Returns the number of channels, which exceeds kFixMax (and
+// leaves the list unused) when there are more than the list holds.
+__device__ __noinline__ int build_fix_list(uint32_t pbits, const float (&sc)[2], const float (&dv)[8],
+                              int lane, float4 *list) {
+  const uint32_t out = ~pbits & 0xFFu;
+  int total = 0, my_bit = 0, my_src = 0;
+  for (int b = 0; b < 8; ++b) {
+    const uint32_t m = __ballot_sync(0xFFFFFFFFu, (out >> b) & 1u);
+    const int n = __popc(m);
+    if (lane >= total && lane < total + n) {
+      uint32_t mm = m;
+      for (int i = 0; i < lane - total; ++i) mm &= mm - 1;  // drop the lower set bits
+      my_bit = b;
+      my_src = __ffs(mm) - 1;
+    }
+    total += n;
+  }
+  if (total > kFixMax) return total;
+  const float s2[2] = {__shfl_sync(0xFFFFFFFFu, sc[0], my_src),
+                       __shfl_sync(0xFFFFFFFFu, sc[1], my_src)};
+  float d1 = 1.0f;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    const float t = __shfl_sync(0xFFFFFFFFu, dv[j], my_src);
+    if (j == my_bit) d1 = t;
+  }
+  if (lane < total) {
+    float d8[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) d8[j] = d1;
+    StepConsts k;
+    fold_consts<false, true>(0, 1, s2, d8, k);
+    list[2 * lane] = make_float4(__int_as_float(my_src * kColsPerThread + my_bit), k.rd[0],
+                                 k.nd[0], k.ld[0]);
+    list[2 * lane + 1] = make_float4(k.r7p, k.m128p, k.r7m, k.m128m);
+  }
+  __syncwarp();
+  return total;
+}
+
+// The exact codes (smooth8, then dualscale8, on one element) of the listed
+// channels in this warp's rows of the staged tile (rows warp, warp + 8, ...),
+// written over the uncorrected ones.  blk = the group's first plane at the
+// column block's first channel c_blk.
+template <bool P2>
+__device__ __noinline__ void patch_codes(const uint16_t *tile, const float4 *list, int nfix, int warp,
+                            int lane, int rows_here, int64_t r_base, int8_t *blk,
+                            int8_t *planes, int64_t plane_stride, int64_t K, int64_t c_blk,
+                            const SegParams &seg, int *status) {
+  const int n_rows = (rows_here - warp + 7) / 8;
+  for (int e = lane; e < n_rows * nfix; e += 32) {
+    const int t = e / nfix, f = e - t * nfix;
+    const int rr = warp + 8 * t;
+    const float4 a = list[2 * f], b = list[2 * f + 1];
+    const int co = __float_as_int(a.x);
+    const float x = __uint_as_float(static_cast<uint32_t>(tile[rr * kWarpCols + co]) << 16);
+    const float xc = max_nan(min_nan(x, a.w), -a.w);
+    const float q0 = __fmul_rn(xc, a.y);
+    const float u = __fmaf_rn(__fmaf_rn(q0, a.z, xc), a.y, q0);
+    const float ap = mul_sat(u, b.x), am = mul_sat(u, b.z);
+    const float vp = fma_sat(__fmaf_rn(ap, b.y, u), b.x, ap);
+    const float vm = fma_sat(__fmaf_rn(am, b.w, u), b.z, am);
+    const uint32_t qp = min(__float_as_uint(__fmaf_rn(vp, 128.0f, 12582912.0f)) & 0xFFu, 127u);
+    const uint32_t qm = __float_as_uint(__fmaf_rn(vm, -128.0f, 12582912.0f)) & 0xFFu;
+    const int64_t r = r_base + rr;
+    const int64_t at = (blk - planes) + r * K + co;
+    if (!store_ok(status, at >= 0 && c_blk + co < K &&
+                              at + (P2 ? plane_stride : 0) <
+                                  static_cast<int64_t>(seg.G) * seg.P * plane_stride))
+      continue;
+    if constexpr (P2) {
+      blk[r * K + co] = static_cast<int8_t>(qp);
+      blk[plane_stride + r * K + co] = static_cast<int8_t>(qm);
+    } else {
+      blk[r * K + co] = static_cast<int8_t>(qp | qm);
+    }
+  }
+}
+
 template <bool FP8, bool HAS_D>
 __global__ void __launch_bounds__(256, 3) quant_act_kernel(const __grid_constant__ CUtensorMap tmX,
                                                            int64_t M, int64_t K,
@@ -410,6 +518,7 @@ __global__ void __launch_bounds__(256, 3) quant_act_kernel(const __grid_constant
                                                            const float *__restrict__ s_act,
                                                            SegParams seg,
                                                            int8_t *__restrict__ planes,
+                                                           const uint32_t *__restrict__ plan,
                                                            int *status) {
   extern __shared__ __align__(128) uint8_t qsmem[];
   uint64_t *full = reinterpret_cast<uint64_t *>(qsmem + kQStages * kQTileBytes);
@@ -432,11 +541,16 @@ __global__ void __launch_bounds__(256, 3) quant_act_kernel(const __grid_constant
   // these small reads do not queue behind the whole grid's tile traffic.
   UnitCursor cur;
   cur.set(u_begin, n_cb, n_rt);
-  float sc[2], dv[8];
+  float sc[2] = {1.0f, 1.0f}, dv[8] = {1.0f, 1.0f, 1.0f, 1.0f, 1.0f, 1.0f, 1.0f, 1.0f};
   StepConsts kc;
-  if (n_mine > 0)
-    fetch_scales<HAS_D>(cur.g, static_cast<int64_t>(cur.cb) * kWarpCols + lane * kColsPerThread,
-                        K, d, s_act, seg, sc, dv);
+  uint32_t pbits = 0;  // plan bits of this thread's channels (with divisors)
+  int nfix = 0;        // channels the current column block patches
+  float4 *fix_list = reinterpret_cast<float4 *>(qsmem + kFixOffset) + warp * 2 * kFixMax;
+  if (n_mine > 0) {
+    const int64_t c0 = static_cast<int64_t>(cur.cb) * kWarpCols + lane * kColsPerThread;
+    fetch_scales<HAS_D>(cur.g, c0, K, d, s_act, seg, sc, dv);
+    if constexpr (HAS_D && !FP8) pbits = plan_bits8(plan, cur.g, c0, K);
+  }
   if (tid == 0) {
     fetch.set(u_begin, n_cb, n_rt);
     for (int st = 0; st < kQStages && st < n_mine; ++st) {
@@ -451,12 +565,18 @@ __global__ void __launch_bounds__(256, 3) quant_act_kernel(const __grid_constant
     fold_consts<FP8, HAS_D>(static_cast<int64_t>(cur.cb) * kWarpCols + lane * kColsPerThread, K,
                             sc, dv, kc);
   // Whether the block's current (group, column block) may take the codes
-  // without the quotient's correction (block-uniform): int8 codes, no
-  // divisor, and the block-wide test passed for the step pair of every
-  // K-segment that meets the column block.
+  // without the quotients' corrections (block-uniform), for int8 codes:
+  // without a divisor, when the block-wide test passed for the step pair of
+  // every K-segment that meets the column block; with divisors, when a
+  // quantize plan is given and leaves out at most kFixMax of the 256 channels
+  // (each warp sees the same 256 and lists them for patch_codes).
   const auto correction_free = [&](int g, int cb) -> bool {
-    if constexpr (FP8 || HAS_D) {
+    if constexpr (FP8) {
       return false;
+    } else if constexpr (HAS_D) {
+      if (plan == nullptr) return false;
+      nfix = build_fix_list(pbits, sc, dv, lane, fix_list);
+      return nfix <= kFixMax;
     } else {
       const int64_t first = static_cast<int64_t>(cb) * kWarpCols;
       const int64_t last = (first + kWarpCols < K ? first + kWarpCols : K) - 1;
@@ -484,6 +604,7 @@ __global__ void __launch_bounds__(256, 3) quant_act_kernel(const __grid_constant
       key_g = cur.g;
       key_cb = cur.cb;
       fetch_scales<HAS_D>(cur.g, c0, K, d, s_act, seg, sc, dv);
+      if constexpr (HAS_D && !FP8) pbits = plan_bits8(plan, cur.g, c0, K);
       fold_consts<FP8, HAS_D>(c0, K, sc, dv, kc);
       fast = correction_free(cur.g, cur.cb);
     }
@@ -496,8 +617,8 @@ __global__ void __launch_bounds__(256, 3) quant_act_kernel(const __grid_constant
     const int64_t r_base = static_cast<int64_t>(cur.rt) * kQRows;
     const int rows_here = static_cast<int>(M - r_base < kQRows ? M - r_base : kQRows);
     const auto rows = [&](auto fast_form, auto two_planes) {
-      // (the uncorrected codes exist for int8 codes without a divisor only)
-      constexpr bool FAST = decltype(fast_form)::value && !FP8 && !HAS_D;
+      // (the uncorrected codes exist for int8 codes only)
+      constexpr bool FAST = decltype(fast_form)::value && !FP8;
       constexpr bool P2 = decltype(two_planes)::value;
       int8_t *plus = planes + static_cast<int64_t>(cur.g) * (P2 ? 2 : 1) * plane_stride + c0;
 #pragma unroll 4
@@ -508,6 +629,7 @@ __global__ void __launch_bounds__(256, 3) quant_act_kernel(const __grid_constant
         unpack8(v, xv);
         uint2 pk, nk;
         if constexpr (FAST) {
+          if constexpr (HAS_D) scale8(xv, kc);  // u = RN(x fl(1/d)), the sign of x kept
           dualscale8_fast(xv, kc, pk, nk);
         } else if constexpr (FP8) {
           float uv[8];
@@ -537,15 +659,32 @@ __global__ void __launch_bounds__(256, 3) quant_act_kernel(const __grid_constant
     };
     if (c0 < K) {
       if (seg.P == 2) {
-        if (!FP8 && !HAS_D && fast)
+        if (!FP8 && fast)
           rows(std::true_type{}, std::true_type{});
         else
           rows(std::false_type{}, std::true_type{});
       } else {
-        if (!FP8 && !HAS_D && fast)
+        if (!FP8 && fast)
           rows(std::true_type{}, std::false_type{});
         else
           rows(std::false_type{}, std::false_type{});
+      }
+    }
+    if constexpr (HAS_D && !FP8) {
+      // every lane, including those past K in a ragged block (fast and nfix
+      // are block-uniform)
+      if (fast && nfix > 0) {
+        __syncwarp();  // the warp's row stores come before the patches
+        int8_t *blk = planes + static_cast<int64_t>(cur.g) * seg.P * plane_stride +
+                      static_cast<int64_t>(cur.cb) * kWarpCols;
+        if (seg.P == 2)
+          patch_codes<true>(tile, fix_list, nfix, warp, lane, rows_here, r_base, blk, planes,
+                            plane_stride, K, static_cast<int64_t>(cur.cb) * kWarpCols, seg,
+                            status);
+        else
+          patch_codes<false>(tile, fix_list, nfix, warp, lane, rows_here, r_base, blk, planes,
+                             plane_stride, K, static_cast<int64_t>(cur.cb) * kWarpCols, seg,
+                             status);
       }
     }
     __syncthreads();  // every warp is done with stage st
@@ -556,6 +695,72 @@ __global__ void __launch_bounds__(256, 3) quant_act_kernel(const __grid_constant
       fetch.next(n_cb, n_rt);
     }
   }
+}
+
+// ------------------------------------------------------------ quantize plan
+// For every activation group g and channel c (with a divisor d[g][c]): whether
+// the codes formed without either correction -- u = RN(x fl(1/d)), then
+// q = rne(128 sat(RN(u fl(1/s)) / 128)) -- equal the quantizer's exact codes
+// (u = fl(x/d), then fl(u/s)) for every bf16 input x, at the calibrated step
+// pair of c's K-segment.  Both forms lie within 2^-22 (relative) of
+// x / (d s), so they can differ only for x within that distance of a rounding
+// boundary (h + 1/2) s d; bf16 inputs are 2^-8 apart, so such an x is a bf16
+// neighbour of fl(fl((h + 1/2) s) d) (itself within 2^-23 of the boundary).
+// One thread per channel evaluates both forms on those neighbours -- the
+// truncation to bf16 and the values just below and above, h = 0 .. 127, both
+// polarities: 768 inputs -- with exactly the kernels' operations.  Bit c % 32
+// of word [g][c / 32] is set when all agree (and for channels past K).
+__global__ void __launch_bounds__(256) quant_plan_kernel(const float *__restrict__ d, int64_t K,
+                                                         const float *__restrict__ s_act,
+                                                         SegParams seg, uint32_t *plan,
+                                                         int *status) {
+  const int g = blockIdx.y;
+  const int64_t c = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  bool ok = true;
+  if (c < K) {
+    const int i = (seg.mode == SQ_SEG_INPUT) ? seg_index(seg.off, seg.n_seg, c) : 0;
+    const float sc[2] = {s_act[(g * seg.S + i) * 2 + 0], s_act[(g * seg.S + i) * 2 + 1]};
+    const float dc = d[g * K + c];
+    StepConsts k;
+    float dv[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) dv[j] = dc;
+    fold_consts<false, true>(0, 1, sc, dv, k);
+    for (int pol = 0; pol < 2; ++pol) {
+      const float s = sc[pol];
+      const float r7 = pol ? k.r7m : k.r7p, m128 = pol ? k.m128m : k.m128p;
+      const float scale = pol ? -128.0f : 128.0f;
+      for (int h = 0; h < 128; ++h) {
+        const float b = static_cast<float>(h) + 0.5f;
+        const uint32_t t = __float_as_uint(__fmul_rn(__fmul_rn(b, s), dc)) & 0xFFFF0000u;
+        for (int e = -1; e <= 1; ++e) {
+          const float xm = __uint_as_float(t + static_cast<uint32_t>(e) * 0x10000u);
+          const float x = pol ? -xm : xm;
+          // exact: smooth8's quotient, then dualscale8's
+          const float xc = max_nan(min_nan(x, k.ld[0]), -k.ld[0]);
+          const float q0 = __fmul_rn(xc, k.rd[0]);
+          const float u = __fmaf_rn(__fmaf_rn(q0, k.nd[0], xc), k.rd[0], q0);
+          const float a = mul_sat(u, r7);
+          const float v = fma_sat(__fmaf_rn(a, m128, u), r7, a);
+          uint32_t q_exact = __float_as_uint(__fmaf_rn(v, scale, 12582912.0f)) & 0xFFu;
+          // uncorrected: scale8, then dualscale8_fast
+          const float uf = __fmul_rn(x, k.rd[0]);
+          uint32_t q_fast =
+              __float_as_uint(__fmaf_rn(mul_sat(uf, r7), scale, 12582912.0f)) & 0xFFu;
+          if (!pol) {  // the + plane's codes are lowered to 127
+            q_exact = min(q_exact, 127u);
+            q_fast = min(q_fast, 127u);
+          }
+          ok = ok && q_exact == q_fast;
+        }
+      }
+    }
+  }
+  const unsigned bits = __ballot_sync(0xFFFFFFFFu, ok);
+  const int64_t words = (K + 31) / 32;
+  // plan: [G][words]
+  if ((threadIdx.x & 31) == 0 && c / 32 < words && store_ok(status, g < seg.G))
+    plan[g * words + c / 32] = bits;
 }
 
 // -------------------------------------------------------- weight quantize
@@ -684,7 +889,8 @@ cudaError_t launch_calibrate_act(const uint16_t *x, int64_t M, int64_t K, int64_
 
 sq_status launch_quantize_act(const uint16_t *x, int64_t M, int64_t K, int64_t ldx,
                               const float *d, const float *s_act, const SegParams &seg,
-                              int8_t *planes, int *status, cudaStream_t stream) {
+                              int8_t *planes, const uint32_t *plan, int *status,
+                              cudaStream_t stream) {
   if (M == 0) return SQ_OK;
   EncodeTiledFn enc = tensor_map_encoder();
   if (enc == nullptr) return SQ_ERR_CUDA;
@@ -703,7 +909,9 @@ sq_status launch_quantize_act(const uint16_t *x, int64_t M, int64_t K, int64_t l
   // units are split evenly over exactly that many blocks.
   int64_t nblk = static_cast<int64_t>(num_sms()) * 3;
   if (nblk > n_units) nblk = n_units;
-  const size_t smem = kQStages * kQTileBytes + kQStages * sizeof(uint64_t);
+  const size_t smem = kFixOffset + (d != nullptr && plan != nullptr && !seg.fp8
+                                         ? 8 * 2 * kFixMax * sizeof(float4)
+                                         : 0);
   auto kernel = seg.fp8 ? (d ? quant_act_kernel<true, true> : quant_act_kernel<true, false>)
                         : (d ? quant_act_kernel<false, true> : quant_act_kernel<false, false>);
   if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -721,9 +929,18 @@ sq_status launch_quantize_act(const uint16_t *x, int64_t M, int64_t K, int64_t l
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  if (cudaLaunchKernelEx(&cfg, kernel, tmX, M, K, d, s_act, seg, planes, status) != cudaSuccess)
+  if (cudaLaunchKernelEx(&cfg, kernel, tmX, M, K, d, s_act, seg, planes, plan, status) !=
+      cudaSuccess)
     return SQ_ERR_CUDA;
   return cudaGetLastError() == cudaSuccess ? SQ_OK : SQ_ERR_CUDA;
+}
+
+cudaError_t launch_quantize_plan(const float *d, int64_t K, const float *s_act,
+                                 const SegParams &seg, uint32_t *plan, int *status,
+                                 cudaStream_t stream) {
+  const dim3 grid(static_cast<unsigned>((K + 255) / 256), static_cast<unsigned>(seg.G));
+  quant_plan_kernel<<<grid, 256, 0, stream>>>(d, K, s_act, seg, plan, status);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_quantize_weight(const uint16_t *w, int64_t N, int64_t K, const float *d,

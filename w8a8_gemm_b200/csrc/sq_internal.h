@@ -50,7 +50,12 @@ cudaError_t launch_calibrate_act(const uint16_t *x, int64_t M, int64_t K, int64_
                                  int *status, cudaStream_t stream);
 sq_status launch_quantize_act(const uint16_t *x, int64_t M, int64_t K, int64_t ldx,
                               const float *d, const float *s_act, const SegParams &seg,
-                              int8_t *planes, int *status, cudaStream_t stream);
+                              int8_t *planes, const uint32_t *plan, int *status,
+                              cudaStream_t stream);
+// Quantize plan: bits [G][ceil(K/32)] (see quant_plan_kernel).
+cudaError_t launch_quantize_plan(const float *d, int64_t K, const float *s_act,
+                                 const SegParams &seg, uint32_t *plan, int *status,
+                                 cudaStream_t stream);
 cudaError_t launch_quantize_weight(const uint16_t *w, int64_t N, int64_t K, const float *d,
                                    const SegParams &seg, int8_t *wq, float *s_w, int *status,
                                    cudaStream_t stream);

@@ -78,6 +78,10 @@ class DualScaleSegLinear:
                                       seg.flags | B.SQ_FLAG_SINGLE_SCALE)
                 B.sq_calibrate_act(x_cal, d, self.seg, self.s_act)
         self.single_scale = bool(self.seg.flags & B.SQ_FLAG_SINGLE_SCALE)
+        # With SmoothQuant divisors: the channels whose codes may skip both
+        # quotient corrections (same codes; sq_quantize_act_plan).
+        self.plan = (B.sq_quantize_act_plan(d, self.s_act, self.seg)
+                     if d is not None and not fp8 else None)
         self._planes = None
 
     def planes_for(self, M: int, device) -> torch.Tensor:
@@ -89,7 +93,7 @@ class DualScaleSegLinear:
     def quantize(self, x: torch.Tensor, planes: Optional[torch.Tensor] = None) -> torch.Tensor:
         if planes is None:
             planes = self.planes_for(x.shape[0], x.device)
-        return B.sq_quantize_act(x, self.d, self.s_act, self.seg, planes)
+        return B.sq_quantize_act(x, self.d, self.s_act, self.seg, planes, plan=self.plan)
 
     def gemm(self, planes: torch.Tensor, y: Optional[torch.Tensor] = None) -> torch.Tensor:
         M = planes.shape[2]
