@@ -100,3 +100,48 @@ def test_divisor_one_reduces_to_the_plain_forms():
     fast = codes_d(x, np.float32(1), s, s, True)
     assert (exact[0][0], exact[1][1]) == (43, -43)
     assert (fast[0][0], fast[1][1]) == (44, -44)
+
+
+# ------------------------------------------- the model against the oracle
+from correction_free import ALL_BF16  # noqa: E402
+
+
+@pytest.mark.parametrize("seed", range(2))
+def test_exact_form_is_the_oracles_quantizer(seed):
+    """The model's exact form (IEEE quotients, x/s or x/d then u/s) gives the
+    oracle's planes on every bf16 input, with and without a divisor, at steps
+    and divisors that are not powers of two: the verdicts of the block test
+    and of the plan are statements about the oracle's codes."""
+    import oracle
+    rng = np.random.default_rng(500 + seed)
+    xb = np.ascontiguousarray(ALL_BF16.reshape(4096, 16))
+    for _ in range(3):
+        sp, sm = np.exp2(rng.uniform(-12, 4, 2)).astype(np.float32)
+        s_act = np.array([[[sp, sm]]], np.float32)
+        planes = oracle.quantize_act(xb, s_act)
+        qp, qm = codes(xb.ravel(), sp, sm, False)
+        assert np.array_equal(planes[0, 0].ravel(), qp), (float(sp), float(sm))
+        assert np.array_equal(planes[0, 1].ravel(), qm), (float(sp), float(sm))
+        dv = np.float32(np.exp2(rng.uniform(-4, 4)))
+        planes = oracle.quantize_act(xb, s_act, d=np.full((1, 16), dv, np.float32))
+        qp, qm = codes_d(xb.ravel(), dv, sp, sm, False)
+        assert np.array_equal(planes[0, 0].ravel(), qp), (float(dv), float(sp), float(sm))
+        assert np.array_equal(planes[0, 1].ravel(), qm), (float(dv), float(sp), float(sm))
+
+
+def test_uncorrected_form_departs_from_the_oracle_where_the_plan_says():
+    """At a divisor the plan rejects, the uncorrected codes differ from the
+    oracle's for some bf16 input; at one it accepts, they agree everywhere."""
+    import oracle
+    s = np.float32(float.fromhex("0x1.0adc5p-7"))
+    s_act = np.array([[[s, s]]], np.float32)
+    xb = np.ascontiguousarray(ALL_BF16.reshape(4096, 16))
+    bad = np.float32(divisors_where_forms_differ(1, s, seed=29)[0])
+    good = np.float32(1.5)
+    assert not channel_passes_test_d(bad, s, s) and channel_passes_test_d(good, s, s)
+    for dv, agree in ((bad, False), (good, True)):
+        planes = oracle.quantize_act(xb, s_act, d=np.full((1, 16), dv, np.float32))
+        qp, qm = codes_d(xb.ravel(), dv, s, s, True)
+        same = (np.array_equal(planes[0, 0].ravel(), qp)
+                and np.array_equal(planes[0, 1].ravel(), qm))
+        assert same == agree, float(dv)
