@@ -204,7 +204,10 @@ SQ_API sq_status sq_quantize_act(const void *x, int64_t M, int64_t K, int64_t ld
  *   plan   uint32 [G][ceil(K / 32)] device output, 4-byte aligned: bit c % 32
  *          of word [g][c / 32] set when channel c of group g qualifies
  *          (also set for the padding channels past K)
- * int8 codes only: SQ_FLAG_FP8 gives SQ_ERR_UNSUPPORTED.
+ * All buffers are the caller's; the call is asynchronous on `stream` and
+ * allocates nothing.  Errors: SQ_ERR_INVALID_ARG (a NULL buffer, K < 16 or
+ * K % 16 != 0, a bad segment table), SQ_ERR_ALIGNMENT, SQ_ERR_UNSUPPORTED
+ * with SQ_FLAG_FP8 (int8 codes only), SQ_ERR_CUDA.
  */
 SQ_API sq_status sq_quantize_act_plan(const float *d, int64_t K, const float *s_act,
                                       const sq_segments *seg, uint32_t *plan,
@@ -212,11 +215,15 @@ SQ_API sq_status sq_quantize_act_plan(const float *d, int64_t K, const float *s_
 
 /*
  * sq_quantize_act_planned -- sq_quantize_act with a plan of
- * sq_quantize_act_plan made from the same d, s_act and segment table: every
- * 256-channel block whose channels all qualify takes the codes without the
- * corrections; the others, as sq_quantize_act.  The planes are bit for bit
- * those of sq_quantize_act.  plan NULL: exactly sq_quantize_act.  A plan
- * without d is SQ_ERR_INVALID_ARG; with SQ_FLAG_FP8, SQ_ERR_UNSUPPORTED.
+ * sq_quantize_act_plan made from the same d, s_act and segment table (a plan
+ * made from other steps or divisors gives wrong codes; nothing checks it).
+ * A 256-channel block in which at most 16 channels do not qualify takes the
+ * codes without the corrections and then rewrites those channels' codes with
+ * the exact form; a block with more is quantized as by sq_quantize_act.  The
+ * planes are bit for bit those of sq_quantize_act.  plan NULL: exactly
+ * sq_quantize_act.  Arguments and errors as sq_quantize_act's, and: a plan
+ * without d is SQ_ERR_INVALID_ARG, a plan with SQ_FLAG_FP8 SQ_ERR_UNSUPPORTED,
+ * a plan not 4-byte aligned SQ_ERR_ALIGNMENT.
  */
 SQ_API sq_status sq_quantize_act_planned(const void *x, int64_t M, int64_t K, int64_t ldx,
                                          const float *d, const float *s_act,
